@@ -18,8 +18,9 @@ bumped by the Weyl constants (0x9E3779B9, 0xBB67AE85).
 
 Normals: for counter block c of stream ``kind`` the generator is called on
 counter (c mod 2^32, c div 2^32, kind, 0) and key (seed mod 2^32, seed div
-2^32). Each 32-bit output x becomes u = ((x >> 8) + 0.5) / 2^24, which lies in
-(0, 1) and is exact in both fp32 and fp64. Box-Muller (G. E. P. Box and M. E.
+2^32). Each 32-bit output x becomes u = ((x >> 9) + 0.5) / 2^23, which lies in
+(0, 1) and is exact in both fp32 and fp64 (the top 23 bits plus a half need
+24 significant bits, the fp32 significand). Box-Muller (G. E. P. Box and M. E.
 Muller, Ann. Math. Statist. 29 (1958)) turns (u0, u1) into
 r cos(2 pi u1), r sin(2 pi u1) with r = sqrt(-2 ln u0), and likewise (u2, u3);
 element 4c + j of the stream takes the j-th of these four normals.
@@ -58,8 +59,8 @@ def philox4x32_10(c0, c1, c2, c3, k0, k1):
 
 
 def uniform_from_bits(x: np.ndarray) -> np.ndarray:
-    """Map 32 random bits to (0, 1): ((x >> 8) + 0.5) / 2^24, exact in fp32."""
-    return ((x >> np.uint32(8)).astype(np.float64) + 0.5) * (1.0 / 16777216.0)
+    """Map 32 random bits to (0, 1): ((x >> 9) + 0.5) / 2^23, exact in fp32."""
+    return ((x >> np.uint32(9)).astype(np.float64) + 0.5) * (1.0 / 8388608.0)
 
 
 def normals(kind: int, n: int, seed: int) -> np.ndarray:

@@ -92,7 +92,11 @@ def test_normals_are_standard_normal():
 
 def test_uniform_mapping_endpoints():
     u = philox.uniform_from_bits(np.array([0, 0xFFFFFFFF], dtype=np.uint32))
-    assert u[0] == 0.5 / 2 ** 24 and u[1] == 1.0 - 0.5 / 2 ** 24
+    assert u[0] == 0.5 / 2 ** 23 and u[1] == 1.0 - 0.5 / 2 ** 23
+    # every value is exactly representable in fp32 (the CUDA side computes it in fp32)
+    x = np.random.default_rng(0).integers(0, 2 ** 32, 10000, dtype=np.uint64).astype(np.uint32)
+    uu = philox.uniform_from_bits(x)
+    assert np.array_equal(uu.astype(np.float32).astype(np.float64), uu)
 
 
 def test_init_statistics():
