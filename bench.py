@@ -1,0 +1,331 @@
+"""GPT-2 124M training throughput on B200 (fwd + bwd + clip + AdamW), one JSON line.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: GPT-2 124M (12 blocks, 12 heads, 768 channels, context 1,024,
+vocabulary 50,257 padded to 50,304, tied embeddings), micro-batch 19 x 9
+accumulation steps = 175,104 tokens per optimizer step, bf16 activations with
+fp32 master weights, gradients and Adam state, AdamW with global-norm clip 1.0
+and the warmup + cosine schedule ("Pretraining and adapting a language model
+on a dependency-free stack", §4.1, §4.3, §4.4). Tokens are a synthetic
+Zipf(1.1) stream with end-of-text ids at geometric(mean 1000) document
+boundaries, seed 1337 (+ rank), resident in HBM before timing starts.
+
+A step is 9 x gpt2_fwd_bwd + gpt2_clip_adamw. `value` is whole-job tokens/s
+from CUDA events over exactly K steps (max over ranks). `e2e` repeats the
+measurement through gpt2_train_step_host with pinned host token buffers (the
+host->device copies and the loss/norm readback inside the timed region).
+With --gpus N each rank trains an independent replica on its own token stream
+(no gradient exchange), so scaling is weak.
+
+--impl reference times the CPU oracle (the fp64 numpy definition of the same
+step) on the host cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "gpt2_124m"
+PAGES_TOKENS_PER_S = 43374.0  # the pages' own stack, one card of their 3-card box (numbat §5.4, Table 3)
+N_PARAMS = 124_439_808
+FLOPS_PER_TOKEN = 6 * N_PARAMS + 6 * 12 * 768 * 1024  # 6N + causal attention
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def workload_desc(w, n_gpus):
+    return {
+        "workload": (f"GPT-2 124M training step: L{w['n_layer']} H{w['n_head']} C{w['n_embd']} "
+                     f"T{w['seq_len']} V{w['vocab_real']}->50304, micro-batch {w['micro_batch']} x "
+                     f"{w['grad_accum']} accumulation"),
+        "global_batch": w["micro_batch"] * w["grad_accum"] * n_gpus,
+        "seq_len": w["seq_len"],
+        "tokens_per_step": w["micro_batch"] * w["grad_accum"] * w["seq_len"] * n_gpus,
+        "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
+        "l2": "inputs larger than L2 (each micro-step touches ~8 GB of activations and logits)",
+        "inputs": "synthetic Zipf(1.1) token stream, geometric(1000) documents, seed 1337+rank",
+    }
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        busy = [s for s in sm if s > 0.5 * (mx or 1)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    """Time the CPU oracle on a bounded sample of the workload (rank 0 only)."""
+    if rank != 0:
+        return
+    res = cpu_baseline(target_seconds=max(10.0, 4.0 * args.steps), steps=args.steps, warmup=args.warmup)
+    w = __import__("gpt_step_b200.workloads", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
+    line = {
+        "metric": "GPT-2 124M train tokens/s on 1 B200 (fwd+bwd+AdamW); MFU vs bf16 dense peak",
+        "impl": "reference",
+        "value": res["value"], "unit": "tokens/s", "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000.0 * w["micro_batch"] * w["grad_accum"] * 1024 / res["value"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_desc(w, 1),
+        "cpu_baseline": res,
+        "e2e": {"value": res["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline(target_seconds=15.0, steps=1, warmup=0):
+    """Oracle tokens/s: fwd+bwd of 1 x 1024 tokens plus AdamW amortised over a full step."""
+    from gpt_step_b200 import synth, workloads
+    from oracle import gpt2 as G
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+    except Exception:
+        cores = os.cpu_count()
+    args = workloads.model_args(WORKLOAD, micro_batch=1)
+    cfg = G.Config(**args)
+    w = workloads.WORKLOADS[WORKLOAD]
+    p = G.init_params(cfg, 1337)
+    src = synth.TokenSource(1, cfg.T, cfg.V, 1337, w["mean_doc_len"], 8)
+    t_micro = []
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        x, y = src.get()
+        a = time.perf_counter()
+        _, g = G.fwd_bwd(cfg, p, x, y)
+        t_micro.append(time.perf_counter() - a)
+        n += 1
+        if n >= max(1, steps) and time.perf_counter() - t0 > 0.6 * target_seconds:
+            break
+        if n >= 4:
+            break
+    m, v = G.zeros_like_params(cfg), G.zeros_like_params(cfg)
+    a = time.perf_counter()
+    G.clip_adamw(cfg, p, g, m, v, 0)
+    t_adam = time.perf_counter() - a
+    seqs_per_step = w["micro_batch"] * w["grad_accum"]
+    t_seq = statistics.median(t_micro)
+    sec_per_token = (t_seq + t_adam / seqs_per_step) / cfg.T
+    return {"value": 1.0 / sec_per_token, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": (f"{n} oracle micro-steps of 1 x 1024 tokens (fwd+bwd, fp64 numpy; median "
+                       f"{t_seq:.2f} s) + one clip+AdamW over all 124.5M parameters "
+                       f"({t_adam:.2f} s) amortised over the {seqs_per_step} sequences of a step")}
+
+
+# --------------------------------------------------------------------------- our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import gpt_step_b200 as gs
+    from gpt_step_b200 import build, synth, workloads
+
+    torch.cuda.set_device(local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    build.build()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+
+    w = workloads.WORKLOADS[WORKLOAD]
+    B, T, A = w["micro_batch"], w["seq_len"], w["grad_accum"]
+    cfg = gs.Config.make(**workloads.model_args(WORKLOAD))
+    model = gs.GPT2(cfg, 1337 + rank)
+    n_steps = args.warmup + args.steps
+    n_win = n_steps * A * B
+    src = synth.TokenSource(B, T, cfg.vocab_real, 1337 + rank, w["mean_doc_len"], n_win)
+    xs, ys = [], []
+    for _ in range(n_steps * A):
+        x, y = src.get()
+        xs.append(x)
+        ys.append(y)
+    tok = torch.tensor(np.stack(xs), device="cuda")     # [steps*A, B, T] resident in HBM
+    tgt = torch.tensor(np.stack(ys), device="cuda")
+    stream = model.stream
+
+    def step(i):
+        for a in range(A):
+            j = i * A + a
+            model.fwd_bwd(tok[j], tgt[j])
+        model.clip_adamw(i)
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        step(i)
+    l0, _ = model.last_step_stats() if args.warmup else (float("nan"), 0)
+    barrier()
+    launches0 = model.kernel_launches()
+    model.profile(True)
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for i in range(args.warmup, n_steps):
+        step(i)
+    ev1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = ev0.elapsed_time(ev1)
+    prof = model.profile_read()
+    model.profile(False)
+    launches = model.kernel_launches() - launches0
+    loss, norm = model.last_step_stats()
+    t_max = ms
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_max = float(t.item())
+    tokens = args.steps * A * B * T * world
+    value = tokens / (t_max / 1000.0)
+
+    # end to end through the host-buffer C-ABI call
+    e2e = None
+    if not args.no_e2e:
+        htok = torch.empty((A, B, T), dtype=torch.int32, pin_memory=True)
+        htgt = torch.empty((A, B, T), dtype=torch.int32, pin_memory=True)
+        host_batches = [(np.stack(xs[i * A:(i + 1) * A]), np.stack(ys[i * A:(i + 1) * A]))
+                        for i in range(args.warmup, n_steps)]
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for k, (hx, hy) in enumerate(host_batches):
+            htok.numpy()[...] = hx
+            htgt.numpy()[...] = hy
+            model.train_step_host_ptr(htok.data_ptr(), htgt.data_ptr(), A, n_steps + k)
+        e1.record(stream)
+        barrier()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ems], device="cuda")
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": tokens / (ems / 1000.0), "unit": "tokens/s",
+               "h2d_bytes_per_step": 2 * A * B * T * 4, "d2h_bytes_per_step": 8,
+               "api": "gpt2_train_step_host (pinned host tokens/targets)"}
+
+    peaks = load_peaks()
+    roof = None
+    if prof and prof.get("gemm", {}).get("ms", 0) > 0:
+        g = prof["gemm"]
+        ach = g["flops"] / (g["ms"] / 1000.0) / 1e12
+        pk = peaks["bf16_tflops_sustained"]
+        roof = {"bound": "tensor", "kernel": "gemm_tc_kernel (all tcgen05 GEMM launches)",
+                "achieved": round(ach, 1), "peak": pk, "unit": "TFLOP/s", "frac": round(ach / pk, 4),
+                "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
+                "traffic": None, "launches": g["launches"], "share_of_step": round(g["ms"] / ms, 4)}
+
+    if rank == 0:
+        mfu = value / world * FLOPS_PER_TOKEN / (peaks["bf16_tflops"] * 1e12)
+        line = {
+            "metric": "GPT-2 124M train tokens/s on 1 B200 (fwd+bwd+AdamW); MFU vs bf16 dense peak",
+            "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": round(value / PAGES_TOKENS_PER_S, 3),
+            "dtype": "bf16", "data": "synthetic", "config": workload_desc(w, world),
+            "mfu": round(mfu, 4), "mfu_peak": f"{peaks['bf16_tflops']} TFLOP/s bf16 dense ({peaks['source']})",
+            "loss": round(loss, 4), "grad_norm": round(norm, 4),
+            "gpu_launches": int(launches), "clocks": clk, "roofline": roof, "e2e": e2e,
+            "kernels": prof,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            line["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(line), flush=True)
+    model.close()
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,451 @@
+// tcgen05 GEMM for the dense contractions of the GPT-2 step (sm_100a).
+//
+//   D[M, N] = sum_k A(m, k) * B(n, k)          bf16 inputs, fp32 accumulation
+//
+// Operands are staged by TMA into 128-byte-swizzled shared memory and fed to
+// tcgen05.mma (cta_group::1, M = 128, N = BN, K = 16 per instruction) with the
+// accumulator in tensor memory. Either operand may be K-major (row-major with
+// the reduction contiguous) or MN-major (the reduction is the strided index),
+// which covers the three products of a linear layer without transposes:
+//   forward   out  = inp . W^T    A = inp  [M, K] K-major,  B = W    [N, K] K-major
+//   dgrad     din  = dout . W     A = dout [M, K] K-major,  B = W^T: W [K, N] MN-major
+//   wgrad     dW  += dout^T . inp A = dout^T: dout [K, M] MN-major, B = inp [K, N] MN-major
+//
+// Kernel organisation (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: fills a ring of STAGES shared-memory stages
+//   warp 1      allocates 2*BN tensor-memory columns; lane 0 issues the MMAs
+//   warps 2..5  epilogue: tcgen05.ld the accumulator, fuse bias / residual /
+//               GELU / GELU' / fp32 accumulation, store to global memory
+// Two accumulator buffers in tensor memory let the epilogue of tile i overlap
+// the main loop of tile i+1. No cluster multicast is used anywhere.
+#pragma once
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+
+namespace gemm {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // bf16 elements per 128-byte swizzle row
+constexpr int UMMA_K = 16;
+constexpr int kThreads = 192;
+
+enum Epi : int {
+  EPI_STORE = 0,    // out = bf16(acc [+ bias])
+  EPI_RESID = 1,    // out = bf16(acc + bias + aux)            (residual add)
+  EPI_GELU = 2,     // out = bf16(acc + bias); out2 = bf16(GELU(acc + bias))
+  EPI_DGELU = 3,    // out = bf16(acc * GELU'(aux))
+  EPI_ACC_F32 = 4,  // outf += acc (fp32; atomic when the reduction is split)
+};
+
+struct Params {
+  int M, N, K;
+  int num_m, num_n, splits, kb_per_split, nkb, num_tiles;
+  bf16* out;
+  bf16* out2;
+  int ldo;
+  const bf16* aux;
+  int ld_aux;
+  const float* bias;
+  float* outf;
+  int ldf;
+  int* err;
+};
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = BN >= 256 ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int BAR_BYTES = 1024;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr int TMEM_COLS = 2 * BN;
+};
+
+GPT2_DEV void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const Params p) {
+  using C = Cfg<BN>;
+  constexpr int S = C::STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* done = bars + 2 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 4 * 32);
+    }
+    mbar_init(smem_u32(done), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+        const int mb = t % p.num_m;
+        const int rest = t / p.num_m;
+        const int nb = rest % p.num_n;
+        const int sp = rest / p.num_n;
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.nkb, kb0 + p.kb_per_split);
+        const int m0 = mb * BM, n0 = nb * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err)) { ok = false; break; }
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+          const int k0 = kb * BK;
+          if (A_MN) {
+#pragma unroll
+            for (int j = 0; j < BM / 64; ++j) tma_load_2d(sa + j * 8192, &tmA, fb, m0 + 64 * j, k0);
+          } else {
+            tma_load_2d(sa, &tmA, fb, k0, m0);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j) tma_load_2d(sb + j * 8192, &tmB, fb, n0 + 64 * j, k0);
+          } else {
+            tma_load_2d(sb, &tmB, fb, k0, n0);
+          }
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x, ++it) {
+        const int rest = t / p.num_m;
+        const int sp = rest / p.num_n;
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.nkb, kb0 + p.kb_per_split);
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sb + kk * 32, 16, 1024);
+            tc_mma_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(smem_u32(&empty[stage]));
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        tc_commit(smem_u32(&tfull[acc]));
+      }
+      // every MMA of this CTA has completed once `done` flips
+      tc_commit(smem_u32(done));
+      mbar_wait(smem_u32(done), 0, p.err);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int it = 0;
+    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++it) {
+      const int mb = t % p.num_m;
+      const int rest = t / p.num_m;
+      const int nb = rest % p.num_n;
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err)) break;
+      tc_fence_after();
+      const int row = mb * BM + q * 32 + lane;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        const int n = nb * BN + c;
+        float v[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c, v);
+        if (!row_ok || n >= p.N) continue;
+        if (EPI == EPI_ACC_F32) {
+          float* dst = p.outf + (size_t)row * p.ldf + n;
+          if (p.splits > 1) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              float4 o = *reinterpret_cast<float4*>(dst + i);
+              o.x += v[i]; o.y += v[i + 1]; o.z += v[i + 2]; o.w += v[i + 3];
+              *reinterpret_cast<float4*>(dst + i) = o;
+            }
+          }
+          continue;
+        }
+        if (EPI == EPI_STORE || EPI == EPI_RESID || EPI == EPI_GELU) {
+          if (p.bias != nullptr) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 b = __ldg(reinterpret_cast<const float4*>(p.bias + n + i));
+              v[i] += b.x; v[i + 1] += b.y; v[i + 2] += b.z; v[i + 3] += b.w;
+            }
+          }
+        }
+        if (EPI == EPI_RESID || EPI == EPI_DGELU) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.aux + (size_t)row * p.ld_aux + n);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 u = src[j];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float2 f = unpack_bf16x2(w[h]);
+              const int i = j * 8 + h * 2;
+              if (EPI == EPI_RESID) {
+                v[i] += f.x; v[i + 1] += f.y;
+              } else {
+                v[i] *= gelu_grad_f(f.x); v[i + 1] *= gelu_grad_f(f.y);
+              }
+            }
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.ldo + n);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int i = j * 8;
+          dst[j] = make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
+                              pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
+        }
+        if (EPI == EPI_GELU) {
+          uint4* dst2 = reinterpret_cast<uint4*>(p.out2 + (size_t)row * p.ldo + n);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int i = j * 8;
+            dst2[j] = make_uint4(pack_bf16x2(gelu_f(v[i]), gelu_f(v[i + 1])),
+                                 pack_bf16x2(gelu_f(v[i + 2]), gelu_f(v[i + 3])),
+                                 pack_bf16x2(gelu_f(v[i + 4]), gelu_f(v[i + 5])),
+                                 pack_bf16x2(gelu_f(v[i + 6]), gelu_f(v[i + 7])));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tempty[acc]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+static bool encode_fn_ready() {
+  if (g_encode) return true;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr)
+    return false;
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return true;
+}
+
+// Row-major bf16 matrix [outer][inner] with row stride `ld` elements; boxes of
+// box_inner x box_outer with 128-byte swizzle (box_inner * 2 bytes == 128).
+static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+                     uint32_t box_inner, uint32_t box_outer) {
+  if (!encode_fn_ready()) return false;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((ld * 2) & 15)) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int g_num_sms = 0;
+
+static int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, Params p, cudaStream_t s) {
+  using C = Cfg<BN>;
+  auto kern = gemm_tc_kernel<BN, A_MN, B_MN, EPI>;
+  static bool attr_set = false;  // per template instance
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
+  kern<<<grid, kThreads, C::SMEM, s>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+// Which operand arrangement a call uses.
+enum Kind { FWD = 0, DGRAD = 1, WGRAD = 2 };
+
+// One GEMM with fused epilogue.
+//   FWD:   out[M,N] = A[M,K] . B[N,K]^T   A = a (ld lda), B = b (ld ldb)
+//   DGRAD: out[M,N] = A[M,K] . B[K,N]     A = a [M,K], B = b stored [K,N]
+//   WGRAD: outf[M,N] += A[K,M]^T . B[K,N] A = a stored [K,M], B = b stored [K,N]
+// Shapes: N % 32 == 0, K % 64 == 0, MN-major extents % 64 == 0, rows 16-byte aligned.
+struct Call {
+  Kind kind;
+  int epi;
+  int M, N, K;
+  const bf16* a;
+  int lda;
+  const bf16* b;
+  int ldb;
+  bf16* out;
+  bf16* out2;
+  int ldo;
+  const bf16* aux;
+  int ld_aux;
+  const float* bias;
+  float* outf;
+  int ldf;
+  int* err;
+  int force_bn;      // 0: automatic
+  int force_splits;  // 0: automatic
+};
+
+static int choose_bn(const Call& c) {
+  if (c.force_bn) return c.force_bn;
+  if (c.N % 256 != 0 && c.N % 128 == 0 && c.N <= 1024) return 128;
+  // whole waves: compare the padded tile work of 128- and 256-wide tiles
+  const long m_t = (c.M + BM - 1) / BM;
+  const long t256 = m_t * ((c.N + 255) / 256), t128 = m_t * ((c.N + 127) / 128);
+  const long sms = num_sms();
+  const double w256 = (double)((t256 + sms - 1) / sms) * 256.0;
+  const double w128 = (double)((t128 + sms - 1) / sms) * 128.0 * 1.06;  // narrower tiles cost more per flop
+  return w256 <= w128 ? 256 : 128;
+}
+
+static int run(const Call& c, cudaStream_t s) {
+  if (c.M <= 0 || c.N <= 0 || c.K <= 0) return GPT2_ERR_ARG;
+  if (c.N % 32 || c.K % BK) return GPT2_ERR_ARG;
+  const int BN = choose_bn(c);
+  if (BN != 128 && BN != 256) return GPT2_ERR_ARG;
+  Params p{};
+  p.M = c.M; p.N = c.N; p.K = c.K;
+  p.num_m = (c.M + BM - 1) / BM;
+  p.num_n = (c.N + BN - 1) / BN;
+  p.nkb = c.K / BK;
+  int splits = 1;
+  if (c.kind == WGRAD) {
+    if (c.force_splits) {
+      splits = c.force_splits;
+    } else {
+      const int tiles = p.num_m * p.num_n;
+      const int sms = num_sms();
+      while (tiles * splits < sms && p.nkb / (splits * 2) >= 8) splits *= 2;
+    }
+  } else if (c.force_splits > 1) {
+    return GPT2_ERR_ARG;
+  }
+  p.kb_per_split = (p.nkb + splits - 1) / splits;
+  p.splits = (p.nkb + p.kb_per_split - 1) / p.kb_per_split;
+  p.num_tiles = p.num_m * p.num_n * p.splits;
+  p.out = c.out; p.out2 = c.out2; p.ldo = c.ldo;
+  p.aux = c.aux; p.ld_aux = c.ld_aux; p.bias = c.bias;
+  p.outf = c.outf; p.ldf = c.ldf; p.err = c.err;
+
+  CUtensorMap ta, tb;
+  bool ok;
+  if (c.kind == WGRAD) {
+    if (c.M % 64 || c.N % 64) return GPT2_ERR_ARG;
+    ok = make_map(&ta, c.a, c.M, c.K, c.lda, 64, 64) && make_map(&tb, c.b, c.N, c.K, c.ldb, 64, 64);
+  } else if (c.kind == DGRAD) {
+    if (c.N % 64) return GPT2_ERR_ARG;
+    ok = make_map(&ta, c.a, c.K, c.M, c.lda, 64, BM) && make_map(&tb, c.b, c.N, c.K, c.ldb, 64, 64);
+  } else {
+    ok = make_map(&ta, c.a, c.K, c.M, c.lda, 64, BM) && make_map(&tb, c.b, c.K, c.N, c.ldb, 64, BN);
+  }
+  if (!ok) return GPT2_ERR_ARG;
+
+  cudaError_t e = cudaErrorInvalidValue;
+#define GPT2_GEMM_CASE(BNV, AMN, BMN, EPIV) \
+  e = launch_tc<BNV, AMN, BMN, EPIV>(ta, tb, p, s)
+  if (c.kind == FWD) {
+    switch (c.epi) {
+      case EPI_STORE: if (BN == 256) GPT2_GEMM_CASE(256, false, false, EPI_STORE); else GPT2_GEMM_CASE(128, false, false, EPI_STORE); break;
+      case EPI_RESID: if (BN == 256) GPT2_GEMM_CASE(256, false, false, EPI_RESID); else GPT2_GEMM_CASE(128, false, false, EPI_RESID); break;
+      case EPI_GELU:  if (BN == 256) GPT2_GEMM_CASE(256, false, false, EPI_GELU);  else GPT2_GEMM_CASE(128, false, false, EPI_GELU);  break;
+      default: return GPT2_ERR_ARG;
+    }
+  } else if (c.kind == DGRAD) {
+    switch (c.epi) {
+      case EPI_STORE: if (BN == 256) GPT2_GEMM_CASE(256, false, true, EPI_STORE); else GPT2_GEMM_CASE(128, false, true, EPI_STORE); break;
+      case EPI_DGELU: if (BN == 256) GPT2_GEMM_CASE(256, false, true, EPI_DGELU); else GPT2_GEMM_CASE(128, false, true, EPI_DGELU); break;
+      default: return GPT2_ERR_ARG;
+    }
+  } else {
+    if (c.epi != EPI_ACC_F32) return GPT2_ERR_ARG;
+    if (BN == 256) GPT2_GEMM_CASE(256, true, true, EPI_ACC_F32); else GPT2_GEMM_CASE(128, true, true, EPI_ACC_F32);
+  }
+#undef GPT2_GEMM_CASE
+  return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
+}
+
+}  // namespace gemm

@@ -1,0 +1,625 @@
+// Bandwidth-bound kernels of the GPT-2 step: initialisation, embeddings,
+// LayerNorm, vocabulary-masked softmax cross-entropy, bias gradients, the
+// global gradient norm and the clipped AdamW update.
+//
+// All of them stream bf16 activations or fp32 state with 16-byte vector loads
+// and reduce with warp shuffles; statistics, losses and optimizer math are fp32
+// (fp64 for the global sum of squares).
+#pragma once
+#include "common.cuh"
+
+namespace k {
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., SC'11) and Box-Muller normals for the
+// initialisation ("Pretraining and adapting a language model on a
+// dependency-free stack", §4.1: N(0, 0.02), residual projections / sqrt(2L)).
+// Counter (c mod 2^32, c div 2^32, kind, 0), key (seed lo, seed hi); each 32-bit
+// output x maps to u = ((x >> 9) + 0.5) / 2^23, exact in fp32.
+// ---------------------------------------------------------------------------
+GPT2_DEV void philox4x32_10(uint32_t c[4], uint32_t k0, uint32_t k1) {
+  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) { k0 += 0x9E3779B9u; k1 += 0xBB67AE85u; }
+    const uint32_t hi0 = __umulhi(M0, c[0]), lo0 = M0 * c[0];
+    const uint32_t hi1 = __umulhi(M1, c[2]), lo1 = M1 * c[2];
+    const uint32_t n0 = hi1 ^ c[1] ^ k0, n2 = hi0 ^ c[3] ^ k1;
+    c[0] = n0; c[1] = lo1; c[2] = n2; c[3] = lo0;
+  }
+}
+
+GPT2_DEV float u01(uint32_t x) { return ((float)(x >> 9) + 0.5f) * (1.0f / 8388608.0f); }
+
+// Init one parameter kind: mode 0 = N(0, std) (rows >= zero_row_from are 0),
+// 1 = ones, 2 = zeros. Writes the fp32 master and the bf16 copy.
+__global__ void init_kind_kernel(float* __restrict__ p, bf16* __restrict__ pb, long n, int mode, float stddev,
+                                 uint32_t kind, uint64_t seed, long zero_from) {
+  const long nblk = (n + 3) / 4;
+  for (long c = blockIdx.x * (long)blockDim.x + threadIdx.x; c < nblk; c += (long)gridDim.x * blockDim.x) {
+    float z[4];
+    if (mode == 0) {
+      uint32_t ctr[4] = {(uint32_t)(c & 0xFFFFFFFFu), (uint32_t)((uint64_t)c >> 32), kind, 0u};
+      philox4x32_10(ctr, (uint32_t)(seed & 0xFFFFFFFFu), (uint32_t)(seed >> 32));
+      const float r01 = sqrtf(-2.0f * logf(u01(ctr[0])));
+      const float r23 = sqrtf(-2.0f * logf(u01(ctr[2])));
+      float s1, c1, s3, c3;
+      sincospif(2.0f * u01(ctr[1]), &s1, &c1);
+      sincospif(2.0f * u01(ctr[3]), &s3, &c3);
+      z[0] = r01 * c1; z[1] = r01 * s1; z[2] = r23 * c3; z[3] = r23 * s3;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) z[j] *= stddev;
+    } else {
+      const float v = mode == 1 ? 1.0f : 0.0f;
+      z[0] = z[1] = z[2] = z[3] = v;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const long e = 4 * c + j;
+      if (e < n) {
+        const float v = (e >= zero_from) ? 0.0f : z[j];
+        p[e] = v;
+        pb[e] = __float2bfloat16_rn(v);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a1  embedding: x[n, :] = wte[tok[n], :] + wpe[n % T, :]   (bf16 copies)
+// ---------------------------------------------------------------------------
+__global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const bf16* __restrict__ wte,
+                                 const bf16* __restrict__ wpe, bf16* __restrict__ x, int N, int T, int C, int V,
+                                 int* err) {
+  const int vpr = C / 8;
+  const long total = (long)N * vpr;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / vpr), c = (int)(i % vpr) * 8;
+    int t = tok[n];
+    if (t < 0 || t >= V) {
+      if (c == 0) atomicOr(err, DEVERR_TOKEN_RANGE);
+      t = 0;
+    }
+    const uint4 a = *reinterpret_cast<const uint4*>(wte + (size_t)t * C + c);
+    const uint4 b = *reinterpret_cast<const uint4*>(wpe + (size_t)(n % T) * C + c);
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, bw[4] = {b.x, b.y, b.z, b.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 fa = unpack_bf16x2(aw[j]), fb = unpack_bf16x2(bw[j]);
+      o[j] = pack_bf16x2(fa.x + fb.x, fa.y + fb.y);
+    }
+    *reinterpret_cast<uint4*>(x + (size_t)n * C + c) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// a1 backward, position part: dwpe[t, :] += sum_b dx[b, t, :]   (deterministic)
+__global__ void embed_bwd_wpe_kernel(const bf16* __restrict__ dx, float* __restrict__ dwpe, int B, int T, int C) {
+  const int vpr = C / 8;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= T * vpr) return;
+  const int t = i / vpr, c = (i % vpr) * 8;
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int b = 0; b < B; ++b) {
+    const uint4 u = *reinterpret_cast<const uint4*>(dx + ((size_t)b * T + t) * C + c);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack_bf16x2(w[j]);
+      acc[2 * j] += f.x;
+      acc[2 * j + 1] += f.y;
+    }
+  }
+  float4* d = reinterpret_cast<float4*>(dwpe + (size_t)t * C + c);
+  float4 d0 = d[0], d1 = d[1];
+  d0.x += acc[0]; d0.y += acc[1]; d0.z += acc[2]; d0.w += acc[3];
+  d1.x += acc[4]; d1.y += acc[5]; d1.z += acc[6]; d1.w += acc[7];
+  d[0] = d0;
+  d[1] = d1;
+}
+
+// a1 backward, token part: dwte[tok[n], :] += dx[n, :]   (fp32 vector atomics)
+__global__ void embed_bwd_wte_kernel(const int32_t* __restrict__ tok, const bf16* __restrict__ dx,
+                                     float* __restrict__ dwte, int N, int C, int V) {
+  const int vpr = C / 8;
+  const long total = (long)N * vpr;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
+    const int n = (int)(i / vpr), c = (int)(i % vpr) * 8;
+    const int t = tok[n];
+    if (t < 0 || t >= V) continue;
+    const uint4 u = *reinterpret_cast<const uint4*>(dx + (size_t)n * C + c);
+    const float2 f0 = unpack_bf16x2(u.x), f1 = unpack_bf16x2(u.y), f2 = unpack_bf16x2(u.z), f3 = unpack_bf16x2(u.w);
+    float* d = dwte + (size_t)t * C + c;
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(d), "f"(f0.x), "f"(f0.y), "f"(f1.x), "f"(f1.y)
+                 : "memory");
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(d + 4), "f"(f2.x), "f"(f2.y), "f"(f3.x),
+                 "f"(f3.y)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a2/a6/a9  LayerNorm forward: one warp per row, fp32 statistics (eps 1e-5,
+// biased variance), y = (x - mean) * rstd * w + b in bf16.
+// ---------------------------------------------------------------------------
+template <int C>
+__global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restrict__ x, const float* __restrict__ w,
+                                                            const float* __restrict__ b, bf16* __restrict__ y,
+                                                            float* __restrict__ mean, float* __restrict__ rstd,
+                                                            int rows) {
+  constexpr int NV = C / 8;                 // 16-byte vectors per row
+  constexpr int VPL = (NV + 31) / 32;       // vectors per lane
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int l = lane_id();
+  if (row >= rows) return;
+  const bf16* xr = x + (size_t)row * C;
+  float v[VPL][8];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = l + 32 * i;
+    if (vi < NV) {
+      const uint4 u = *reinterpret_cast<const uint4*>(xr + vi * 8);
+      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(wv[j]);
+        v[i][2 * j] = f.x;
+        v[i][2 * j + 1] = f.y;
+        s += f.x + f.y;
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[i][j] = 0.f;
+    }
+  }
+  const float mu = warp_sum(s) * (1.0f / C);
+  float ss = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    if (l + 32 * i < NV) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float d = v[i][j] - mu;
+        ss += d * d;
+      }
+    }
+  }
+  const float rs = rsqrtf(warp_sum(ss) * (1.0f / C) + 1e-5f);
+  bf16* yr = y + (size_t)row * C;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = l + 32 * i;
+    if (vi < NV) {
+      const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + vi * 8));
+      const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + vi * 8 + 4));
+      const float4 b0 = __ldg(reinterpret_cast<const float4*>(b + vi * 8));
+      const float4 b1 = __ldg(reinterpret_cast<const float4*>(b + vi * 8 + 4));
+      const float ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        o[j] = pack_bf16x2((v[i][2 * j] - mu) * rs * ww[2 * j] + bb[2 * j],
+                           (v[i][2 * j + 1] - mu) * rs * ww[2 * j + 1] + bb[2 * j + 1]);
+      *reinterpret_cast<uint4*>(yr + vi * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  if (l == 0) {
+    mean[row] = mu;
+    rstd[row] = rs;
+  }
+}
+
+// LayerNorm backward: dx = rstd * (dy*w - mean(dy*w) - xhat * mean(dy*w*xhat))
+// (+ dresid, the gradient flowing along the residual stream), written in bf16;
+// per-block partial column sums of dy*xhat and dy go to `part` ([grid][2][C]).
+template <int C>
+__global__ void __launch_bounds__(256) layernorm_bwd_kernel(const bf16* __restrict__ dy, const bf16* __restrict__ x,
+                                                            const float* __restrict__ mean,
+                                                            const float* __restrict__ rstd,
+                                                            const float* __restrict__ w,
+                                                            const bf16* dresid, bf16* dx,
+                                                            float* __restrict__ part, int rows) {
+  constexpr int NV = C / 8;
+  constexpr int VPL = (NV + 31) / 32;
+  __shared__ float red[2][C];
+  const int warp = threadIdx.x >> 5, l = lane_id();
+  float adw[VPL][8], adb[VPL][8];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) adw[i][j] = adb[i][j] = 0.f;
+  float wv[VPL][8];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = l + 32 * i;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wv[i][j] = (vi < NV) ? w[vi * 8 + j] : 0.f;
+  }
+  for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
+    const float mu = mean[row], rs = rstd[row];
+    float xh[VPL][8], g[VPL][8];
+    float s1 = 0.f, s2 = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = l + 32 * i;
+      if (vi < NV) {
+        const uint4 ux = *reinterpret_cast<const uint4*>(x + (size_t)row * C + vi * 8);
+        const uint4 ud = *reinterpret_cast<const uint4*>(dy + (size_t)row * C + vi * 8);
+        const uint32_t xw[4] = {ux.x, ux.y, ux.z, ux.w}, dw4[4] = {ud.x, ud.y, ud.z, ud.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 fx = unpack_bf16x2(xw[j]), fd = unpack_bf16x2(dw4[j]);
+          xh[i][2 * j] = (fx.x - mu) * rs;
+          xh[i][2 * j + 1] = (fx.y - mu) * rs;
+          adw[i][2 * j] += fd.x * xh[i][2 * j];
+          adw[i][2 * j + 1] += fd.y * xh[i][2 * j + 1];
+          adb[i][2 * j] += fd.x;
+          adb[i][2 * j + 1] += fd.y;
+          g[i][2 * j] = fd.x * wv[i][2 * j];
+          g[i][2 * j + 1] = fd.y * wv[i][2 * j + 1];
+          s1 += g[i][2 * j] + g[i][2 * j + 1];
+          s2 += g[i][2 * j] * xh[i][2 * j] + g[i][2 * j + 1] * xh[i][2 * j + 1];
+        }
+      }
+    }
+    const float m1 = warp_sum(s1) * (1.0f / C), m2 = warp_sum(s2) * (1.0f / C);
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = l + 32 * i;
+      if (vi < NV) {
+        float r[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) r[j] = (g[i][j] - m1 - xh[i][j] * m2) * rs;
+        if (dresid != nullptr) {
+          const uint4 u = *reinterpret_cast<const uint4*>(dresid + (size_t)row * C + vi * 8);
+          const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = unpack_bf16x2(uw[j]);
+            r[2 * j] += f.x;
+            r[2 * j + 1] += f.y;
+          }
+        }
+        *reinterpret_cast<uint4*>(dx + (size_t)row * C + vi * 8) =
+            make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
+                       pack_bf16x2(r[6], r[7]));
+      }
+    }
+  }
+  // combine the 8 warps' column sums in a fixed order (deterministic)
+  for (int wi = 0; wi < 8; ++wi) {
+    if (warp == wi) {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int vi = l + 32 * i;
+        if (vi < NV) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (wi == 0) {
+              red[0][vi * 8 + j] = adw[i][j];
+              red[1][vi * 8 + j] = adb[i][j];
+            } else {
+              red[0][vi * 8 + j] += adw[i][j];
+              red[1][vi * 8 + j] += adb[i][j];
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+  for (int c = threadIdx.x; c < 2 * C; c += blockDim.x)
+    part[(size_t)blockIdx.x * 2 * C + c] = red[c / C][c % C];
+}
+
+// Sum nblk partial rows ([nblk][2][C]) in order and add into dw, db (fp32 grads).
+__global__ void layernorm_bwd_reduce_kernel(const float* __restrict__ part, float* __restrict__ dw,
+                                            float* __restrict__ db, int nblk, int C) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= 2 * C) return;
+  const int which = c / C, col = c % C;
+  float s = 0.f;
+  for (int i = 0; i < nblk; ++i) s += part[((size_t)i * 2 + which) * C + col];
+  if (which == 0) dw[col] += s;
+  else db[col] += s;
+}
+
+// ---------------------------------------------------------------------------
+// bias gradient: db[n] += sum_m dout[m, n] (bf16 input, two deterministic passes)
+// Pass 1: block (32 x 8 threads) covers 256 columns over a strip of rows.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) colsum_partial_kernel(const bf16* __restrict__ a, float* __restrict__ part,
+                                                             int M, int N, int rows_per_strip) {
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int c = (blockIdx.x * 32 + tx) * 8;
+  const int r0 = blockIdx.y * rows_per_strip;
+  const int r1 = min(M, r0 + rows_per_strip);
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  if (c < N) {
+    for (int r = r0 + ty; r < r1; r += 8) {
+      const uint4 u = *reinterpret_cast<const uint4*>(a + (size_t)r * N + c);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(w[j]);
+        acc[2 * j] += f.x;
+        acc[2 * j + 1] += f.y;
+      }
+    }
+  }
+  __shared__ float red[8][32][9];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) red[ty][tx][j] = acc[j];
+  __syncthreads();
+  if (ty == 0 && c < N) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float s = 0.f;
+#pragma unroll
+      for (int y = 0; y < 8; ++y) s += red[y][tx][j];
+      part[(size_t)blockIdx.y * N + c + j] = s;
+    }
+  }
+}
+
+__global__ void colsum_final_kernel(const float* __restrict__ part, float* __restrict__ db, int strips, int N) {
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= N) return;
+  float s = 0.f;
+  for (int i = 0; i < strips; ++i) s += part[(size_t)i * N + c];
+  db[c] += s;
+}
+
+// ---------------------------------------------------------------------------
+// a11  vocabulary-masked softmax cross-entropy, forward and backward fused.
+// One CTA per row: the bf16 logits row is read once into shared memory while a
+// running (max, sum of exp) is kept over the REAL columns j < V only; the row is
+// then overwritten in place with dz = (softmax_j - [j == target]) * dscale for
+// j < V and exactly 0 for the padded columns j >= V ("Pretraining and adapting
+// a language model on a dependency-free stack", §4.1). loss = lse - z[target].
+// ---------------------------------------------------------------------------
+constexpr int kCeThreads = 512;
+
+__global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict__ logits,
+                                                                const int32_t* __restrict__ targets,
+                                                                float* __restrict__ losses, int V, int Vp,
+                                                                float dscale, int write_grad, int* err) {
+  extern __shared__ __align__(16) uint8_t smem_ce[];
+  uint4* row_s = reinterpret_cast<uint4*>(smem_ce);
+  __shared__ float red_m[kCeThreads / 32], red_s[kCeThreads / 32];
+  __shared__ float bc[2];
+  const int row = blockIdx.x;
+  uint4* zr = reinterpret_cast<uint4*>(logits + (size_t)row * Vp);
+  const int nv = Vp / 8;
+  float m = -INFINITY, s = 0.f;
+  for (int i = threadIdx.x; i < nv; i += kCeThreads) {
+    const uint4 u = zr[i];
+    row_s[i] = u;
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    float f[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 t = unpack_bf16x2(w[j]);
+      f[2 * j] = t.x;
+      f[2 * j + 1] = t.y;
+    }
+    float lm = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (i * 8 + j < V) lm = fmaxf(lm, f[j]);
+    if (lm > -INFINITY) {
+      const float nm = fmaxf(m, lm);
+      s *= __expf(m - nm);
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        if (i * 8 + j < V) s += __expf(f[j] - nm);
+      m = nm;
+    }
+  }
+  // combine (m, s) across the CTA
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, m, o), os = __shfl_xor_sync(0xffffffffu, s, o);
+    const float nm = fmaxf(m, om);
+    s = (nm == -INFINITY) ? 0.f : s * __expf(m - nm) + os * __expf(om - nm);
+    m = nm;
+  }
+  const int warp = threadIdx.x >> 5, l = lane_id();
+  if (l == 0) { red_m[warp] = m; red_s[warp] = s; }
+  __syncthreads();
+  if (warp == 0) {
+    m = l < kCeThreads / 32 ? red_m[l] : -INFINITY;
+    s = l < kCeThreads / 32 ? red_s[l] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float om = __shfl_xor_sync(0xffffffffu, m, o), os = __shfl_xor_sync(0xffffffffu, s, o);
+      const float nm = fmaxf(m, om);
+      s = (nm == -INFINITY) ? 0.f : s * __expf(m - nm) + os * __expf(om - nm);
+      m = nm;
+    }
+    if (l == 0) { bc[0] = m; bc[1] = s; }
+  }
+  __syncthreads();
+  const float M = bc[0], inv = 1.0f / bc[1];
+  int t = targets[row];
+  const bool tok_ok = (t >= 0 && t < V);
+  if (!tok_ok) {
+    if (threadIdx.x == 0) atomicOr(err, DEVERR_TOKEN_RANGE);
+    t = -1;
+  }
+  if (threadIdx.x == 0) {
+    float zt = 0.f;
+    if (tok_ok) {
+      const bf16* zs = reinterpret_cast<const bf16*>(row_s);
+      zt = __bfloat162float(zs[t]);
+    }
+    losses[row] = tok_ok ? (M + logf(bc[1]) - zt) : 0.f;
+  }
+  if (!write_grad) return;
+  for (int i = threadIdx.x; i < nv; i += kCeThreads) {
+    const uint4 u = row_s[i];
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = unpack_bf16x2(w[j]);
+      const int c0 = i * 8 + 2 * j;
+      float g0 = 0.f, g1 = 0.f;
+      if (c0 < V) g0 = (__expf(f.x - M) * inv - (c0 == t ? 1.f : 0.f)) * dscale;
+      if (c0 + 1 < V) g1 = (__expf(f.y - M) * inv - (c0 + 1 == t ? 1.f : 0.f)) * dscale;
+      o[j] = pack_bf16x2(g0, g1);
+    }
+    zr[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// Sum n per-row losses (fp64 accumulation) into acc[0] and store the micro-batch
+// mean in *mean_out.
+__global__ void loss_reduce_kernel(const float* __restrict__ losses, int n, double* __restrict__ acc,
+                                   float* __restrict__ mean_out) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += (double)losses[i];
+  s = warp_sum_d(s);
+  if (lane_id() == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    s = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.0;
+    s = warp_sum_d(s);
+    if (threadIdx.x == 0) {
+      acc[0] += s;
+      *mean_out = (float)(s / n);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a12  global gradient norm. Pass 1: per-block fp64 partial sums of g^2 over
+// the flat fp32 gradient array (float4 loads).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(512) sumsq_partial_kernel(const float* __restrict__ g, long n4,
+                                                            double* __restrict__ part) {
+  __shared__ double red[16];
+  double s = 0.0;
+  const float4* g4 = reinterpret_cast<const float4*>(g);
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+    const float4 v = g4[i];
+    s += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+  }
+  s = warp_sum_d(s);
+  if (lane_id() == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    s = threadIdx.x < 16 ? red[threadIdx.x] : 0.0;
+    s = warp_sum_d(s);
+    if (threadIdx.x == 0) part[blockIdx.x] = s;
+  }
+}
+
+// Optimizer scalars shared by the norm and AdamW kernels (device memory).
+struct StepScalars {
+  double loss_sum;      // sum of micro-batch losses x rows since the last step
+  float norm;           // pre-clip norm of g / n_micro
+  float gscale;         // multiplier applied to raw g: min(1, clip/norm) / n_micro
+  int skip;             // 1: non-finite loss or norm, update not applied
+  int n_micro;          // micro-steps accumulated (device copy)
+  float last_loss;      // mean loss of the last completed step
+  float last_norm;      // pre-clip norm of the last completed step
+  float micro_loss;     // mean loss of the last micro-batch
+  int pad;
+};
+
+// Pass 2: combine partials; derive the clip multiplier; flag non-finite steps.
+__global__ void norm_finalize_kernel(const double* __restrict__ part, int nparts, StepScalars* sc, int n_micro,
+                                     long rows_per_micro, float clip, int* err) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) s += part[i];
+  s = warp_sum_d(s);
+  if (lane_id() == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+    const double norm = sqrt(t) / (double)n_micro;
+    const double mean_loss = sc->loss_sum / ((double)rows_per_micro * n_micro);
+    const bool finite = isfinite(norm) && isfinite(mean_loss);
+    const double k = (norm > clip) ? (double)clip / norm : 1.0;
+    sc->norm = (float)norm;
+    sc->gscale = (float)(k / (double)n_micro);
+    sc->skip = finite ? 0 : 1;
+    sc->last_loss = (float)mean_loss;
+    sc->last_norm = (float)norm;
+    sc->loss_sum = 0.0;
+    if (!finite) atomicOr(err, DEVERR_NONFINITE);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// a13  clipped AdamW over the flat parameter arrays (float4 per thread).
+// Kinds are contiguous and 64-element aligned; `bound[k]` is the first element
+// of kind k (bound[nk] = end) and bit k of `decay_mask` says whether kind k is a
+// 2-D weight that takes decoupled weight decay. Writes p, m, v, the bf16 copy
+// and clears g. If the step is flagged non-finite only g is cleared.
+// ---------------------------------------------------------------------------
+struct KindTable {
+  long bound[17];
+  int nk;
+  unsigned decay_mask;
+};
+
+__global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, float* __restrict__ g,
+                                                    float* __restrict__ m, float* __restrict__ v,
+                                                    bf16* __restrict__ pb, long n4, const KindTable kt,
+                                                    const StepScalars* __restrict__ sc, float lr, float beta1,
+                                                    float beta2, float eps, float wd, float bc1, float bc2) {
+  const float gs = sc->gscale;
+  const int skip = sc->skip;
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+    const long e = i * 4;
+    float4* g4 = reinterpret_cast<float4*>(g) + i;
+    if (skip) {
+      *g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      continue;
+    }
+    int kind = 0;
+#pragma unroll 1
+    while (kind + 1 < kt.nk && e >= kt.bound[kind + 1]) ++kind;
+    const float lam = ((kt.decay_mask >> kind) & 1u) ? wd : 0.f;
+    float4 gv = *g4;
+    float4 pv = reinterpret_cast<float4*>(p)[i];
+    float4 mv = reinterpret_cast<float4*>(m)[i];
+    float4 vv = reinterpret_cast<float4*>(v)[i];
+    float* gp = &gv.x;
+    float* pp = &pv.x;
+    float* mp = &mv.x;
+    float* vp = &vv.x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float gg = gp[j] * gs;
+      mp[j] = beta1 * mp[j] + (1.0f - beta1) * gg;
+      vp[j] = beta2 * vp[j] + (1.0f - beta2) * gg * gg;
+      const float mh = mp[j] / bc1;
+      const float vh = vp[j] / bc2;
+      pp[j] = pp[j] - lr * (mh / (sqrtf(vh) + eps) + lam * pp[j]);
+    }
+    reinterpret_cast<float4*>(p)[i] = pv;
+    reinterpret_cast<float4*>(m)[i] = mv;
+    reinterpret_cast<float4*>(v)[i] = vv;
+    *g4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    uint2 pk;
+    pk.x = pack_bf16x2(pv.x, pv.y);
+    pk.y = pack_bf16x2(pv.z, pv.w);
+    *reinterpret_cast<uint2*>(pb + e) = pk;
+  }
+}
+
+// fp32 -> bf16 copy (used after host writes of parameters).
+__global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, long n) {
+  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
+    dst[i] = __float2bfloat16_rn(src[i]);
+}
+
+}  // namespace k

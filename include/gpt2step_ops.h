@@ -1,0 +1,106 @@
+/*
+ * gpt2step_ops -- the individual steps of the GPT-2 training step, one call
+ * each, on caller-owned device buffers. They are the kernels gpt2_fwd_bwd and
+ * gpt2_clip_adamw run, exposed so that each step can be checked on its own.
+ *
+ * Common conventions:
+ *   - "bf16" buffers hold IEEE bfloat16 values (2 bytes), row-major, with the
+ *     row stride equal to the row length and 16-byte aligned base pointers.
+ *   - fp32 buffers are float, row-major.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream); every call only
+ *     enqueues work and returns GPT2_OK, GPT2_ERR_ARG (unsupported shape or NULL
+ *     pointer, nothing enqueued) or GPT2_ERR_CUDA (launch failure).
+ *   - `dev_err` is a device int the caller zeroes; kernels OR flags into it
+ *     (1 = token id out of range, 4 = a bounded device wait timed out).
+ *   - Workspaces are caller-owned device memory of at least the size the
+ *     matching *_workspace query returns; their contents on entry do not matter.
+ *
+ * Section references are to "Pretraining and adapting a language model on a
+ * dependency-free stack" (arXiv 2609.28568) unless noted.
+ */
+#ifndef GPT2STEP_OPS_H
+#define GPT2STEP_OPS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Linear layer forward (§4.1 Fig. 1: QKV, attention and MLP projections, tied
+ * head). out[M,N] = inp[M,K] . w[N,K]^T (+ bias[N]) (+ resid[M,N]); all bf16
+ * except bias (fp32, may be NULL unless resid is given). Requires N % 32 == 0,
+ * K % 64 == 0. Runs on the tcgen05 tensor cores with fp32 accumulation. */
+int gpt2op_linear_fwd(const void* inp, const void* w, const float* bias, const void* resid, void* out, int M,
+                      int N, int K, int* dev_err, void* stream);
+
+/* MLP fc + GELU (tanh approximation): pre = inp . w^T + bias, gelu = GELU(pre);
+ * both written as bf16 [M,N]. */
+int gpt2op_linear_fwd_gelu(const void* inp, const void* w, const float* bias, void* pre_out, void* gelu_out, int M,
+                           int N, int K, int* dev_err, void* stream);
+
+/* Input gradient of a linear layer: din[M,K] = dout[M,N] . w[N,K], optionally
+ * multiplied elementwise by GELU'(gelu_pre[M,K]) (gelu_pre may be NULL).
+ * Requires K % 64 == 0 and N % 64 == 0. */
+int gpt2op_linear_dgrad(const void* dout, const void* w, const void* gelu_pre, void* din, int M, int N, int K,
+                        int* dev_err, void* stream);
+
+/* Weight gradient: dw[N,K] (fp32) += dout[M,N]^T . inp[M,K]. `splits` > 1
+ * divides the M reduction across CTAs (fp32 atomic accumulation); 0 chooses
+ * automatically. Requires N % 64 == 0, K % 64 == 0, M % 64 == 0. */
+int gpt2op_linear_wgrad(const void* dout, const void* inp, float* dw, int M, int N, int K, int splits, int* dev_err,
+                        void* stream);
+
+/* Bias gradient: db[N] (fp32) += sum over rows of dout[M,N] (bf16),
+ * deterministic two-pass column sum. N % 8 == 0. */
+size_t gpt2op_bias_grad_workspace(int M, int N);
+int gpt2op_bias_grad(const void* dout, float* db, int M, int N, void* workspace, size_t ws_bytes, void* stream);
+
+/* LayerNorm forward over rows of C (§4.1 pre-LN blocks, §4.3 fp32 statistics):
+ * y = (x - mean) * rstd * w + b with eps 1e-5 and biased variance; x, y bf16
+ * [rows, C]; w, b fp32 [C]; mean, rstd fp32 [rows]. C in {128, 256, 384, 512,
+ * 768, 1024, 1536, 2048}. */
+int gpt2op_layernorm_fwd(const void* x, const float* w, const float* b, void* y, float* mean, float* rstd, int rows,
+                         int C, void* stream);
+
+/* LayerNorm backward: dx = LN'(dy) (+ dresid, the residual-stream gradient, may
+ * be NULL; dx may alias dresid); dw, db (fp32 [C]) += column sums of dy * xhat
+ * and dy (deterministic). */
+size_t gpt2op_layernorm_bwd_workspace(int rows, int C);
+int gpt2op_layernorm_bwd(const void* dy, const void* x, const float* mean, const float* rstd, const float* w,
+                         const void* dresid, void* dx, float* dw, float* db, int rows, int C, void* workspace,
+                         size_t ws_bytes, void* stream);
+
+/* Causal multi-head attention forward (grow_a_language_model_intro, activities
+ * 5-6: softmax(Q K^T / sqrt(hd)) V with a causal mask). qkv bf16 [B,T,3C]
+ * (q | k | v, heads contiguous), out bf16 [B,T,C], lse fp32 [B,H,T] (natural
+ * log-sum-exp of the scaled scores). hd in {32, 64}, T % 64 == 0. */
+int gpt2op_attention_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int hd, void* stream);
+
+/* Attention backward from the saved output and lse: dqkv bf16 [B,T,3C]. */
+size_t gpt2op_attention_bwd_workspace(int B, int T, int H, int hd);
+int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv, int B,
+                         int T, int H, int hd, void* workspace, size_t ws_bytes, void* stream);
+
+/* Vocabulary-masked softmax cross-entropy, forward and backward fused (§4.1:
+ * softmax over the V real ids only). logits bf16 [N,Vp] are overwritten in
+ * place with dz = (softmax - onehot(target)) * dscale for columns < V and
+ * exactly 0 for columns >= V; losses fp32 [N] = lse - z[target]. A target
+ * outside [0, V) gives loss 0, no one-hot term, and flag 1 in dev_err. */
+int gpt2op_softmax_ce(void* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,
+                      int* dev_err, void* stream);
+
+/* Token + position embedding: out[b,t,:] = wte[tok[b,t],:] + wpe[t,:] (bf16).
+ * Ids outside [0, V) read row 0 and set flag 1 in dev_err. */
+int gpt2op_embedding_fwd(const int32_t* tokens, const void* wte, const void* wpe, void* out, int B, int T, int C,
+                         int V, int* dev_err, void* stream);
+
+/* Embedding backward: dwte[tok,:] += dx (fp32 atomics), dwpe[t,:] += sum_b dx. */
+int gpt2op_embedding_bwd(const int32_t* tokens, const void* dx, float* dwte, float* dwpe, int B, int T, int C, int V,
+                         void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GPT2STEP_OPS_H */

@@ -1,0 +1,65 @@
+"""The C-ABI library builds, loads and exports every declared symbol (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gpt_step_b200 as gs
+from gpt_step_b200 import build, workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b(gpt2\w*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return gs.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 30
+    raw = ctypes.CDLL(gs.LIB_PATH)
+    for n in names:
+        assert hasattr(raw, n), n
+        assert n in gs._SIGNATURES, f"binding lacks {n}"
+
+
+def test_param_count_through_the_library(lib):
+    cfg = gs.Config.make(**workloads.model_args("gpt2_124m"))
+    assert gs.num_params(cfg) == 124_439_808          # numbat §4.1
+    assert gs.num_params(cfg, padded=True) == 124_439_808 + 47 * 768
+
+
+def test_arena_sizes(lib):
+    for name in workloads.WORKLOADS:
+        cfg = gs.Config.make(**workloads.model_args(name))
+        n = gs.arena_bytes(cfg)
+        assert n > gs.num_params(cfg, padded=True) * 18, name
+        assert n < 40 * 2 ** 30, name     # fits easily in 180 GB
+    bad = gs.Config.make(n_layer=2, n_head=3, n_embd=144, seq_len=64, vocab_real=100)
+    assert gs.arena_bytes(bad) == 0      # head size 48 is not supported
+
+
+def test_status_strings(lib):
+    for st in range(7):
+        assert len(lib.gpt2_status_string(st)) > 0
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(gs, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(gs, "_lib_handle", None)
+    with pytest.raises(RuntimeError, match="no fallback"):
+        gs.lib()

@@ -1,0 +1,253 @@
+"""Whole-step parity: gpt2_create / gpt2_fwd_bwd / gpt2_clip_adamw against the oracle.
+
+Both sides draw the initial weights from the same Philox stream (the oracle in
+fp64, the device in fp32) and see the same seeded tokens. Tolerances are the
+ones the target fixes for a bf16-activation / fp32-master step against an fp32
+definition: |loss diff| <= 2e-2, per-tensor gradient relative L2 <= 3e-2,
+post-step weights relative L2 (whole parameter vector) <= 1e-3, and the AdamW
+update on identical fp32 gradients within 1e-6 relative.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import gpt_step_b200 as gs
+from gpt_step_b200 import synth, workloads
+from oracle import gpt2 as G
+
+from gpu_util import i32, rel_l2, require_gpu, torch
+
+pytestmark = pytest.mark.gpu
+
+LOSS_TOL, GRAD_TOL, STEP_TOL, ADAM_TOL = 2e-2, 3e-2, 1e-3, 1e-6
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def pair(name, seed=1337, **over):
+    args = workloads.model_args(name, **over)
+    m = gs.GPT2(gs.Config.make(**args), seed)
+    return m, G.Config(**args)
+
+
+def oracle_named(ocfg, arrays):
+    return G.split_named(ocfg, arrays)
+
+
+def flat(named, names):
+    return np.concatenate([np.asarray(named[n], np.float64).ravel() for n in names])
+
+
+def batch_for(name, ocfg, seed=1337, n=1):
+    w = workloads.WORKLOADS[name]
+    if w["input"] == "uniform":
+        return [synth.uniform_next_token_batch(ocfg.micro_batch, ocfg.T, ocfg.V, seed + i) for i in range(n)]
+    src = synth.TokenSource(ocfg.micro_batch, ocfg.T, ocfg.V, seed, w["mean_doc_len"], n * ocfg.micro_batch)
+    return [src.get() for _ in range(n)]
+
+
+# --- initialisation ([numbat] §4.1) ----------------------------------------------------------
+
+def test_initial_weights_match_oracle():
+    m, ocfg = pair("tiny")
+    got = m.read_all(gs.GPT2_PARAMS)
+    ref = oracle_named(ocfg, G.init_params(ocfg, 1337))
+    assert len(got) == len(G.tensor_names(ocfg))
+    for name, a in got.items():
+        assert a.shape == ref[name].shape, name
+        assert np.max(np.abs(a - ref[name])) <= 2e-7 * max(1.0, np.max(np.abs(ref[name]))), name
+    assert np.all(got["wte.weight"][ocfg.V:] == 0.0)
+
+
+# --- one full step on the tiny configuration -------------------------------------------------
+
+def test_tiny_step_parity():
+    m, ocfg = pair("tiny")
+    (x, y), = batch_for("tiny", ocfg)
+    loss = m.fwd_bwd(i32(x), i32(y), want_loss=True)
+    grads = m.read_all(gs.GPT2_GRADS)
+    p = G.init_params(ocfg, 1337)
+    oloss, og = G.fwd_bwd(ocfg, p, x, y)
+    assert abs(loss - oloss) <= LOSS_TOL
+    assert abs(oloss - math.log(ocfg.V)) < 0.1
+    ogn = oracle_named(ocfg, og)
+    for name, a in grads.items():
+        assert rel_l2(a, ogn[name]) <= GRAD_TOL, (name, rel_l2(a, ogn[name]))
+    assert np.all(grads["wte.weight"][ocfg.V:] == 0.0)
+    norm = m.clip_adamw(0, want_norm=True)
+    m_, v_ = G.zeros_like_params(ocfg), G.zeros_like_params(ocfg)
+    onorm = G.clip_adamw(ocfg, p, og, m_, v_, 0)
+    assert abs(norm - onorm) <= GRAD_TOL * onorm
+    got = m.read_all(gs.GPT2_PARAMS)
+    names = list(got)
+    on = oracle_named(ocfg, p)
+    assert rel_l2(flat(got, names), flat(on, names)) <= STEP_TOL
+    assert np.all(got["wte.weight"][ocfg.V:] == 0.0)
+    # gradients are cleared by the step
+    assert all(np.all(g == 0) for g in m.read_all(gs.GPT2_GRADS).values())
+    ml, mn = m.last_step_stats()
+    assert ml == pytest.approx(loss, rel=1e-6) and mn == pytest.approx(norm, rel=1e-6)
+
+
+def test_eval_loss_and_token_losses_match_forward():
+    m, ocfg = pair("tiny")
+    (x, y), = batch_for("tiny", ocfg, seed=5)
+    ev = m.eval_loss(i32(x), i32(y))
+    loss = m.fwd_bwd(i32(x), i32(y), want_loss=True)
+    tl = m.token_losses()
+    assert ev == pytest.approx(loss, abs=1e-5)
+    assert float(tl.mean()) == pytest.approx(loss, abs=1e-5)
+    ref = G.token_losses(ocfg, G.init_params(ocfg, 1337), x, y)
+    assert np.max(np.abs(tl - ref)) < 5e-2
+    # eval over more rows than the micro-batch is chunked
+    x2 = np.concatenate([x, x[::-1]])
+    y2 = np.concatenate([y, y[::-1]])
+    assert m.eval_loss(i32(x2), i32(y2)) == pytest.approx(loss, abs=1e-5)
+
+
+def test_adamw_on_identical_fp32_gradients():
+    m, ocfg = pair("tiny")
+    (x, y), = batch_for("tiny", ocfg)
+    m.fwd_bwd(i32(x), i32(y))      # one micro-step pending
+    rng = np.random.default_rng(99)
+    names = [t.name for t in m.tensors()]
+    P, Gd, M, V = {}, {}, {}, {}
+    for i, t in enumerate(m.tensors()):
+        P[t.name] = (rng.standard_normal(t.shape) * 0.05).astype(np.float32)
+        Gd[t.name] = (rng.standard_normal(t.shape) * 0.02).astype(np.float32)
+        M[t.name] = (rng.standard_normal(t.shape) * 1e-3).astype(np.float32)
+        V[t.name] = (rng.random(t.shape) * 1e-4).astype(np.float32)
+        m.write(gs.GPT2_PARAMS, i, P[t.name])
+        m.write(gs.GPT2_GRADS, i, Gd[t.name])
+        m.write(gs.GPT2_ADAM_M, i, M[t.name])
+        m.write(gs.GPT2_ADAM_V, i, V[t.name])
+    step = 1000
+    norm = m.clip_adamw(step, want_norm=True)
+    # oracle on the same fp32 values, per kind arrays assembled from named tensors
+    def kinds(named):
+        out = {}
+        for kind, shape, _ in G.param_shapes(ocfg):
+            out[kind] = np.zeros(shape)
+        for name, kind, layer, _ in G.tensor_names(ocfg):
+            if layer < 0:
+                out[kind][...] = named[name]
+            else:
+                out[kind][layer] = named[name]
+        return out
+    op, og, om, ov = kinds(P), kinds(Gd), kinds(M), kinds(V)
+    onorm = G.clip_adamw(ocfg, op, og, om, ov, step)
+    assert norm == pytest.approx(onorm, rel=ADAM_TOL)
+    for what, ref in ((gs.GPT2_PARAMS, op), (gs.GPT2_ADAM_M, om), (gs.GPT2_ADAM_V, ov)):
+        got = m.read_all(what)
+        refn = oracle_named(ocfg, ref)
+        for n in names:
+            assert rel_l2(got[n], refn[n]) <= ADAM_TOL, (what, n, rel_l2(got[n], refn[n]))
+
+
+def test_bad_token_and_nonfinite_are_reported():
+    m, ocfg = pair("tiny")
+    (x, y), = batch_for("tiny", ocfg)
+    bad = x.copy()
+    bad[1, 3] = ocfg.V
+    with pytest.raises(gs.GPT2Error) as e:
+        m.fwd_bwd(i32(bad), i32(y), want_loss=True)
+    assert e.value.status == 3
+    with pytest.raises(gs.GPT2Error) as e:
+        m.clip_adamw(0)
+        m.clip_adamw(0)
+    assert e.value.status == 5        # second step with no micro-step in between
+    # a non-finite parameter: the step is refused and the weights stay as they were
+    before = m.read_all(gs.GPT2_PARAMS)
+    idx = [t.name for t in m.tensors()].index("ln_f.weight")
+    w = before["ln_f.weight"].copy()
+    w[0] = np.nan
+    m.write(gs.GPT2_PARAMS, idx, w)
+    m.fwd_bwd(i32(x), i32(y))
+    with pytest.raises(gs.GPT2Error) as e:
+        m.clip_adamw(1, want_norm=True)
+    assert e.value.status == 4
+    after = m.read_all(gs.GPT2_PARAMS)
+    for n in before:
+        if n != "ln_f.weight":
+            np.testing.assert_array_equal(after[n], before[n])
+    # still usable after restoring the weight
+    m.write(gs.GPT2_PARAMS, idx, before["ln_f.weight"])
+    assert np.isfinite(m.fwd_bwd(i32(x), i32(y), want_loss=True))
+
+
+def test_host_train_step_matches_device_calls():
+    m1, ocfg = pair("tiny")
+    m2, _ = pair("tiny")
+    bs = batch_for("tiny", ocfg, n=2)
+    for x, y in bs:
+        m1.fwd_bwd(i32(x), i32(y))
+    m1.clip_adamw(0)
+    l1, n1 = m1.last_step_stats()
+    toks = np.stack([b[0] for b in bs]).astype(np.int32)
+    tgts = np.stack([b[1] for b in bs]).astype(np.int32)
+    l2, n2 = m2.train_step_host(toks, tgts, 0)
+    assert l1 == pytest.approx(l2, abs=1e-6) and n1 == pytest.approx(n2, rel=1e-3)
+
+
+# --- the small configuration: full context length, many tiles --------------------------------
+
+def test_small_config_step_parity():
+    m, ocfg = pair("small", micro_batch=2)
+    (x, y), = batch_for("small", ocfg)
+    loss = m.fwd_bwd(i32(x), i32(y), want_loss=True)
+    grads = m.read_all(gs.GPT2_GRADS)
+    p = G.init_params(ocfg, 1337)
+    oloss, og = G.fwd_bwd(ocfg, p, x, y)
+    assert abs(loss - oloss) <= LOSS_TOL
+    ogn = oracle_named(ocfg, og)
+    worst = max(rel_l2(a, ogn[n]) for n, a in grads.items())
+    assert worst <= GRAD_TOL, worst
+    m.clip_adamw(0)
+    G.clip_adamw(ocfg, p, og, G.zeros_like_params(ocfg), G.zeros_like_params(ocfg), 0)
+    got = m.read_all(gs.GPT2_PARAMS)
+    names = list(got)
+    assert rel_l2(flat(got, names), flat(oracle_named(ocfg, p), names)) <= STEP_TOL
+
+
+def test_small_config_accumulated_steps_track_oracle():
+    m, ocfg = pair("small", micro_batch=1)
+    p = G.init_params(ocfg, 1337)
+    om, ov = G.zeros_like_params(ocfg), G.zeros_like_params(ocfg)
+    src = synth.TokenSource(1, ocfg.T, ocfg.V, 1337, 800, 8)
+    for step in range(3):
+        bs = [src.get(), src.get()]
+        for x, y in bs:
+            m.fwd_bwd(i32(x), i32(y))
+        m.clip_adamw(step)
+        gl, gn = m.last_step_stats()
+        ol, on = G.train_step(ocfg, p, om, ov, step, bs)
+        assert abs(gl - ol) <= LOSS_TOL, (step, gl, ol)
+        assert abs(gn - on) <= GRAD_TOL * on, (step, gn, on)
+    got = m.read_all(gs.GPT2_PARAMS)
+    names = list(got)
+    assert rel_l2(flat(got, names), flat(oracle_named(ocfg, p), names)) <= STEP_TOL
+
+
+# --- GPT-2 124M in the launch configuration the benchmark times (B = 19) ---------------------
+
+def test_gpt2_124m_bench_configuration_sampled():
+    m, ocfg = pair("gpt2_124m")
+    (x, y), = batch_for("gpt2_124m", ocfg)
+    loss = m.fwd_bwd(i32(x), i32(y), want_loss=True)
+    tl = m.token_losses()
+    assert float(tl.mean()) == pytest.approx(loss, abs=1e-4)
+    p = G.init_params(ocfg, 1337)
+    for b in (0, 18):                                   # sequences the oracle computes one by one
+        ref = G.token_losses(ocfg, p, x[b:b + 1], y[b:b + 1])[0]
+        assert abs(float(tl[b].mean()) - float(ref.mean())) <= LOSS_TOL
+        assert np.max(np.abs(tl[b] - ref)) < 0.15
+    g = m.read_all(gs.GPT2_GRADS)
+    assert np.all(g["wte.weight"][ocfg.V:] == 0.0)
+    assert all(np.all(np.isfinite(a)) for a in g.values())
+    norm = m.clip_adamw(0, want_norm=True)
+    assert np.isfinite(norm) and norm > 0
+    assert np.all(m.read(gs.GPT2_PARAMS, 0)[ocfg.V:] == 0.0)
