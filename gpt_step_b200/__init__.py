@@ -89,6 +89,8 @@ _SIGNATURES = {
     "gpt2op_layernorm_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P]),
     "gpt2op_layernorm_bwd_workspace": (_SZ, [_I, _I]),
     "gpt2op_layernorm_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _SZ, _P]),
+    "gpt2op_layernorm_bwd_noalloc_max_bytes": (_SZ, []),
+    "gpt2op_layernorm_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P]),
     "gpt2op_attention_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "gpt2op_attention_bwd_workspace": (_SZ, [_I, _I, _I, _I]),
     "gpt2op_attention_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
@@ -347,6 +349,14 @@ def layernorm_bwd(dy, x, mean, rstd, w, dresid, dx, dw, db, workspace, stream=No
     check(lib().gpt2op_layernorm_bwd(_ptr(dy), _ptr(x), _ptr(mean), _ptr(rstd), _ptr(w), _ptr(dresid),
                                      _ptr(dx), _ptr(dw), _ptr(db), rows, C, _ptr(workspace),
                                      workspace.numel(), _s(stream)), "gpt2op_layernorm_bwd")
+
+
+def layernorm_bwd_noalloc(dy, x, mean, rstd, w, dresid, dx, dw, db, stream=None):
+    """LayerNorm backward with the library's own fixed scratch (no workspace argument)."""
+    rows, C = x.shape
+    check(lib().gpt2op_layernorm_bwd_noalloc(_ptr(dy), _ptr(x), _ptr(mean), _ptr(rstd), _ptr(w),
+                                             _ptr(dresid), _ptr(dx), _ptr(dw), _ptr(db), rows, C,
+                                             _s(stream)), "gpt2op_layernorm_bwd_noalloc")
 
 
 def attention_fwd(qkv, out, lse, n_head, stream=None):

@@ -17,6 +17,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -984,6 +985,55 @@ int gpt2op_layernorm_bwd(const void* dy, const void* x, const float* mean, const
   return launch::ln_bwd(static_cast<const bf16*>(dy), static_cast<const bf16*>(x), mean, rstd, w,
                         static_cast<const bf16*>(dresid), static_cast<bf16*>(dx), dw, db, rows, C,
                         static_cast<float*>(workspace), ws_bytes, static_cast<cudaStream_t>(stream));
+}
+
+// LayerNorm backward that allocates nothing and takes no workspace.
+//
+// Its per-block partial column sums live in one library-wide device array,
+// g_ln_bwd_noalloc_scratch, of kLnNoallocScratchFloats floats (2,424,832 bytes).
+// Every GPU that loads this library holds that array until the process exits.
+// Host code cannot use the array's name as a device address, so the first call
+// on each device looks the address up with cudaGetSymbolAddress (with that
+// device current) and keeps it; that first call should therefore happen before
+// any stream capture. All calls share the array, so calls that overlap on the
+// GPU (different streams, or different host threads without ordering) race on
+// it. Nothing in it has to start at zero: every launch writes each partial it
+// later reads.
+namespace noalloc {
+constexpr size_t kLnNoallocScratchFloats = (size_t)kLnBwdBlocks * 2 * 1024;
+__device__ __align__(256) static float g_ln_bwd_noalloc_scratch[kLnNoallocScratchFloats];
+constexpr int kMaxDevices = 64;
+static float* g_scratch_addr[kMaxDevices] = {};
+static std::mutex g_scratch_mu;
+
+// Device address of the scratch array on the current device (set up once per device).
+static int scratch_for_current_device(float** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GPT2_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_ln_bwd_noalloc_scratch) != cudaSuccess || p == nullptr) return GPT2_ERR_CUDA;
+    g_scratch_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_scratch_addr[dev];
+  return GPT2_OK;
+}
+}  // namespace noalloc
+
+size_t gpt2op_layernorm_bwd_noalloc_max_bytes(void) { return noalloc::kLnNoallocScratchFloats * sizeof(float); }
+
+int gpt2op_layernorm_bwd_noalloc(const void* dy, const void* x, const float* mean, const float* rstd, const float* w,
+                                 const void* dresid, void* dx, float* dw, float* db, int rows, int C, void* stream) {
+  if (!dy || !x || !mean || !rstd || !w || !dx || !dw || !db || rows <= 0) return GPT2_ERR_ARG;
+  // the partial sums this launch needs must fit the fixed scratch; refuse before touching the GPU
+  if (launch::ln_bwd_workspace(rows, C) > gpt2op_layernorm_bwd_noalloc_max_bytes()) return GPT2_ERR_ARG;
+  float* scratch = nullptr;
+  const int st = noalloc::scratch_for_current_device(&scratch);
+  if (st != GPT2_OK) return st;
+  return launch::ln_bwd(static_cast<const bf16*>(dy), static_cast<const bf16*>(x), mean, rstd, w,
+                        static_cast<const bf16*>(dresid), static_cast<bf16*>(dx), dw, db, rows, C, scratch,
+                        gpt2op_layernorm_bwd_noalloc_max_bytes(), static_cast<cudaStream_t>(stream));
 }
 
 int gpt2op_attention_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int hd, void* stream) {

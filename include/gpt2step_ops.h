@@ -72,6 +72,23 @@ int gpt2op_layernorm_bwd(const void* dy, const void* x, const float* mean, const
                          const void* dresid, void* dx, float* dw, float* db, int rows, int C, void* workspace,
                          size_t ws_bytes, void* stream);
 
+/* LayerNorm backward for callers that cannot allocate device memory: the same
+ * operation, arguments and results as gpt2op_layernorm_bwd, without the
+ * workspace. The pages have no counterpart; it exists for code that must not
+ * call cudaMalloc, e.g. a plugin whose host application owns every device
+ * allocation through its own budgeted pool, or a thread that may not block on
+ * the implicit device synchronisation an allocation can cause.
+ * Its scratch is one fixed array inside the library, of
+ * gpt2op_layernorm_bwd_noalloc_max_bytes() = 2,424,832 bytes, that every GPU
+ * which loads the library keeps until the process exits. A call needing more
+ * (min(296, ceil(rows / 8)) * 2 * C * 4 bytes; any row count fits for
+ * C <= 1024) returns GPT2_ERR_ARG before touching the GPU. The first call on a
+ * device looks up the array's device address and should come before any stream
+ * capture. All calls share the array: calls that overlap on the GPU race. */
+size_t gpt2op_layernorm_bwd_noalloc_max_bytes(void);
+int gpt2op_layernorm_bwd_noalloc(const void* dy, const void* x, const float* mean, const float* rstd, const float* w,
+                                 const void* dresid, void* dx, float* dw, float* db, int rows, int C, void* stream);
+
 /* Causal multi-head attention forward (grow_a_language_model_intro, activities
  * 5-6: softmax(Q K^T / sqrt(hd)) V with a causal mask). qkv bf16 [B,T,3C]
  * (q | k | v, heads contiguous), out bf16 [B,T,C], lse fp32 [B,H,T] (natural

@@ -63,3 +63,12 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(gs, "_lib_handle", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         gs.lib()
+
+
+def test_noalloc_layernorm_bwd_rejects_oversized_calls_before_touching_the_gpu(lib):
+    cap = lib.gpt2op_layernorm_bwd_noalloc_max_bytes()
+    assert cap == 296 * 2 * 1024 * 4
+    dummy = ctypes.c_void_p(16)   # never dereferenced: the size check comes first
+    st = lib.gpt2op_layernorm_bwd_noalloc(dummy, dummy, dummy, dummy, dummy, None, dummy, dummy, dummy,
+                                          100000, 1536, None)
+    assert st == 1                # GPT2_ERR_ARG
