@@ -277,14 +277,28 @@ __global__ void attn_bwd_dot_kernel(const bf16* __restrict__ out, const bf16* __
   Dv[((size_t)b * H + h) * T + t] = acc;
 }
 
+// Per-warp dQ staging for the bulk reduce: HD/32 boxes of 16 rows x 32 fp32
+// (128 bytes per row, 128-byte swizzle), double buffered.
+template <int HD>
+struct DqStage {
+  static constexpr int BOX_BYTES = 16 * 32 * 4;               // 2 KB
+  static constexpr int BUF_BYTES = (HD / 32) * BOX_BYTES;     // one iteration of one warp
+  static constexpr int BYTES = 4 * 2 * BUF_BYTES;             // 4 warps x 2 buffers
+};
+
 template <int HD>
 __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ qkv, const bf16* __restrict__ dout,
                                                        const float* __restrict__ lse,
-                                                       const float* __restrict__ Dv, float* __restrict__ dq_acc,
+                                                       const float* __restrict__ Dv,
+                                                       const __grid_constant__ CUtensorMap tm_dq,
                                                        bf16* __restrict__ dqkv, int T, int H, float scale) {
   constexpr int LD = Tile<HD>::LD;
   constexpr int LDS = BLK + 8;  // dS^T tile [key][query]
-  extern __shared__ __align__(16) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem_raw_bwd[];
+  // dQ staging first (1024-byte aligned for the swizzle), then the tiles
+  uint8_t* smem_al = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_bwd) + 1023) & ~uintptr_t(1023));
+  uint8_t* dq_stage = smem_al;
+  uint8_t* smem = smem_al + DqStage<HD>::BYTES;
   bf16* Ks = reinterpret_cast<bf16*>(smem);
   bf16* Vs = Ks + BLK * LD;
   bf16* Qs = Vs + BLK * LD;             // two buffers
@@ -430,20 +444,37 @@ __global__ void __launch_bounds__(128) attn_bwd_kernel(const bf16* __restrict__ 
           mma16816(dqa[2 * dq + 1], a, bb[2], bb[3]);
         }
       }
-      const int qrow = qi * BLK + warp * 16 + (l >> 2);
-      float* d0 = dq_acc + ((size_t)b * T + qrow) * C + h * HD;
-      float* d1 = d0 + (size_t)8 * C;
+      // stage scale * dQ (16 x HD fp32) in swizzled shared memory, then one bulk
+      // reduce-add per 32-column box into the fp32 accumulator
+      uint8_t* buf = dq_stage + (warp * 2 + ((qi - kb) & 1)) * DqStage<HD>::BUF_BYTES;
+      if (l == 0) bulk_wait_group_read<1>();  // this buffer's reduce from two iterations ago has read it
+      __syncwarp();
+      const int r0 = l >> 2;
 #pragma unroll
       for (int dt = 0; dt < HD / 8; ++dt) {
         const int c = dt * 8 + 2 * (l & 3);
-        atomicAdd(d0 + c, dqa[dt][0] * scale);
-        atomicAdd(d0 + c + 1, dqa[dt][1] * scale);
-        atomicAdd(d1 + c, dqa[dt][2] * scale);
-        atomicAdd(d1 + c + 1, dqa[dt][3] * scale);
+        const int half = c >> 5, cc = c & 31, j = cc >> 2;
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int r = r0 + 8 * rr;
+          float2* dst = reinterpret_cast<float2*>(buf + half * DqStage<HD>::BOX_BYTES + r * 128 + ((j ^ (r & 7)) << 4) +
+                                                  (cc & 3) * 4);
+          *dst = make_float2(dqa[dt][2 * rr] * scale, dqa[dt][2 * rr + 1] * scale);
+        }
+      }
+      fence_async_smem();
+      __syncwarp();
+      if (l == 0) {
+        const int qrow0 = b * T + qi * BLK + warp * 16;
+#pragma unroll
+        for (int half = 0; half < HD / 32; ++half)
+          tma_reduce_add_2d(&tm_dq, smem_u32(buf + half * DqStage<HD>::BOX_BYTES), h * HD + 32 * half, qrow0);
+        bulk_commit_group();
       }
     }
     __syncthreads();
   }
+  if (l == 0) bulk_wait_group<0>();
   // write dK (scaled) and dV for this warp's 16 keys
   bf16* k0p = dqkv + ((size_t)b * T + key0) * C3 + C + h * HD;
   bf16* v0p = k0p + C;
@@ -476,7 +507,7 @@ template <int HD>
 constexpr int fwd_smem() { return 5 * Tile<HD>::BYTES; }
 template <int HD>
 constexpr int bwd_smem() {
-  return 6 * Tile<HD>::BYTES + BLK * (BLK + 8) * 2 + 4 * BLK * 4;
+  return 1024 + DqStage<HD>::BYTES + 6 * Tile<HD>::BYTES + BLK * (BLK + 8) * 2 + 4 * BLK * 4;
 }
 
 template <int HD>
@@ -504,9 +535,13 @@ static cudaError_t bwd(const bf16* qkv, const bf16* out, const bf16* dout, const
   }
   const int rows = B * T * H;
   attn_bwd_dot_kernel<HD><<<(rows + 255) / 256, 256, 0, s>>>(out, dout, Dv, B, T, H);
-  dim3 grid(T / BLK, B * H);
-  attn_bwd_kernel<HD><<<grid, 128, bwd_smem<HD>(), s>>>(qkv, dout, lse, Dv, dq_acc, dqkv, T, H, 1.0f / sqrtf((float)HD));
   const int C = H * HD;
+  CUtensorMap tm_dq;
+  if (!encode_map_2d(&tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, C, (uint64_t)B * T, C, 32, 16,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  dim3 grid(T / BLK, B * H);
+  attn_bwd_kernel<HD><<<grid, 128, bwd_smem<HD>(), s>>>(qkv, dout, lse, Dv, tm_dq, dqkv, T, H, 1.0f / sqrtf((float)HD));
   const size_t nvec = (size_t)B * T * C / 8;
   int blocks = (int)((nvec + 255) / 256);
   if (blocks > 148 * 8) blocks = 148 * 8;

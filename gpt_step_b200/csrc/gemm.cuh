@@ -20,6 +20,7 @@
 // the main loop of tile i+1. No cluster multicast is used anywhere.
 #pragma once
 #include <cudaTypedefs.h>
+#include <string.h>
 
 #include "common.cuh"
 
@@ -59,9 +60,37 @@ struct Cfg {
   static constexpr int B_BYTES = BN * BK * 2;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int BAR_BYTES = 1024;
-  static constexpr int SMEM = STAGES * STAGE_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  // per epilogue warp: two 32x32 bf16 staging buffers for each of the (up to) two outputs
+  static constexpr int EPI_BYTES = 4 * 4 * 2048;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 2 * BN;
 };
+
+// TMA store of a 32 x 32 bf16 box (64-byte swizzle) from shared memory.
+GPT2_DEV void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+GPT2_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed bulk groups still read their shared-memory source.
+template <int N>
+GPT2_DEV void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory"); }
+template <int N>
+GPT2_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group %0;" ::"n"(N) : "memory"); }
+GPT2_DEV void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Write one thread's row of 32 bf16 (16 packed words) into a 32 x 32 staging
+// buffer in the 64-byte-swizzled order the TMA store expects: 16-byte chunk j
+// of row r lives at r * 64 + ((j ^ ((r >> 1) & 3)) * 16).
+GPT2_DEV void stage_row(uint8_t* buf, int r, const uint32_t (&w)[16]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int pj = j ^ ((r >> 1) & 3);
+    *reinterpret_cast<uint4*>(buf + r * 64 + pj * 16) = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  }
+}
 
 GPT2_DEV void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
@@ -72,12 +101,14 @@ GPT2_DEV void red_add_v4(float* addr, float a, float b, float c, float d) {
 template <int BN, bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                    const Params p) {
   using C = Cfg<BN>;
   constexpr int S = C::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES);
+  uint8_t* epi_smem = smem + S * C::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::STAGE_BYTES + C::EPI_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* tfull = bars + 2 * S;
@@ -101,6 +132,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (EPI != EPI_ACC_F32) tma_prefetch_desc(&tmO);
+    if (EPI == EPI_GELU) tma_prefetch_desc(&tmO2);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -191,6 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
+    uint8_t* wbuf = epi_smem + q * 8192;  // [out b0 | out b1 | out2 b0 | out2 b1], 2 KB each
+    uint32_t nstore = 0;                  // chunks this warp has staged (selects the buffer)
     int it = 0;
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x, ++it) {
       const int mb = t % p.num_m;
@@ -200,15 +235,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t acc_phase = (it >> 1) & 1;
       if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err)) break;
       tc_fence_after();
-      const int row = mb * BM + q * 32 + lane;
+      const int row0 = mb * BM + q * 32;
+      const int row = row0 + lane;
       const bool row_ok = row < p.M;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         const int n = nb * BN + c;
         float v[32];
         tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c, v);
-        if (!row_ok || n >= p.N) continue;
+        if (n >= p.N) continue;  // uniform across the warp
         if (EPI == EPI_ACC_F32) {
+          if (!row_ok) continue;
           float* dst = p.outf + (size_t)row * p.ldf + n;
           if (p.splits > 1) {
 #pragma unroll
@@ -232,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (EPI == EPI_RESID || EPI == EPI_DGELU) {
+        if ((EPI == EPI_RESID || EPI == EPI_DGELU) && row_ok) {
           const uint4* src = reinterpret_cast<const uint4*>(p.aux + (size_t)row * p.ld_aux + n);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -250,28 +287,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        uint4* dst = reinterpret_cast<uint4*>(p.out + (size_t)row * p.ldo + n);
+        uint32_t pk[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int i = j * 8;
-          dst[j] = make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
-                              pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
-        }
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        const uint32_t b = nstore & 1;
+        // the store issued from this buffer two chunks ago must have read it
+        if (lane == 0) bulk_wait_read<1>();
+        __syncwarp();
+        stage_row(wbuf + b * 2048, lane, pk);
         if (EPI == EPI_GELU) {
-          uint4* dst2 = reinterpret_cast<uint4*>(p.out2 + (size_t)row * p.ldo + n);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int i = j * 8;
-            dst2[j] = make_uint4(pack_bf16x2(gelu_f(v[i]), gelu_f(v[i + 1])),
-                                 pack_bf16x2(gelu_f(v[i + 2]), gelu_f(v[i + 3])),
-                                 pack_bf16x2(gelu_f(v[i + 4]), gelu_f(v[i + 5])),
-                                 pack_bf16x2(gelu_f(v[i + 6]), gelu_f(v[i + 7])));
-          }
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(gelu_f(v[2 * i]), gelu_f(v[2 * i + 1]));
+          stage_row(wbuf + 4096 + b * 2048, lane, pk);
         }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmO, smem_u32(wbuf + b * 2048), n, row0);
+          if (EPI == EPI_GELU) tma_store_2d(&tmO2, smem_u32(wbuf + 4096 + b * 2048), n, row0);
+          bulk_commit();
+        }
+        ++nstore;
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty[acc]));
     }
+    if (EPI != EPI_ACC_F32 && lane == 0) bulk_wait_all<0>();
   }
 
   tc_fence_before();
@@ -285,33 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-static PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-
-static bool encode_fn_ready() {
-  if (g_encode) return true;
-  void* fn = nullptr;
-  cudaDriverEntryPointQueryResult q;
-  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-      q != cudaDriverEntryPointSuccess || fn == nullptr)
-    return false;
-  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-  return true;
-}
-
-// Row-major bf16 matrix [outer][inner] with row stride `ld` elements; boxes of
-// box_inner x box_outer with 128-byte swizzle (box_inner * 2 bytes == 128).
+// Row-major bf16 matrix [outer][inner] with row stride `ld` elements.
 static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-                     uint32_t box_inner, uint32_t box_outer) {
-  if (!encode_fn_ready()) return false;
-  if ((reinterpret_cast<uintptr_t>(base) & 15) || ((ld * 2) & 15)) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 2};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t es[2] = {1, 1};
-  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                        box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+                     uint32_t box_inner, uint32_t box_outer,
+                     CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+  return encode_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, ld, box_inner, box_outer, swz);
 }
 
 static int g_num_sms = 0;
@@ -327,7 +346,8 @@ static int num_sms() {
 }
 
 template <int BN, bool A_MN, bool B_MN, int EPI>
-static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, Params p, cudaStream_t s) {
+static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                             const CUtensorMap& to2, Params p, cudaStream_t s) {
   using C = Cfg<BN>;
   auto kern = gemm_tc_kernel<BN, A_MN, B_MN, EPI>;
   static bool attr_set = false;  // per template instance
@@ -337,7 +357,7 @@ static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, Param
     attr_set = true;
   }
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
-  kern<<<grid, kThreads, C::SMEM, s>>>(ta, tb, p);
+  kern<<<grid, kThreads, C::SMEM, s>>>(ta, tb, to, to2, p);
   return cudaGetLastError();
 }
 
@@ -370,22 +390,38 @@ struct Call {
   int force_splits;  // 0: automatic
 };
 
+// Tile width: whole waves of 148 SMs, with 128-wide tiles charged 1.3x because a
+// single-CTA 128 x 128 x 16 MMA needs ~120 B/clk of shared-memory operand
+// bandwidth (near the SM's limit) against ~90 B/clk for 128 x 256 x 16.
 static int choose_bn(const Call& c) {
   if (c.force_bn) return c.force_bn;
-  if (c.N % 256 != 0 && c.N % 128 == 0 && c.N <= 1024) return 128;
-  // whole waves: compare the padded tile work of 128- and 256-wide tiles
   const long m_t = (c.M + BM - 1) / BM;
-  const long t256 = m_t * ((c.N + 255) / 256), t128 = m_t * ((c.N + 127) / 128);
   const long sms = num_sms();
+  const long t256 = m_t * ((c.N + 255) / 256), t128 = m_t * ((c.N + 127) / 128);
   const double w256 = (double)((t256 + sms - 1) / sms) * 256.0;
-  const double w128 = (double)((t128 + sms - 1) / sms) * 128.0 * 1.06;  // narrower tiles cost more per flop
+  const double w128 = (double)((t128 + sms - 1) / sms) * 128.0 * 1.3;
   return w256 <= w128 ? 256 : 128;
+}
+
+// Split of the reduction for weight gradients (fp32 atomic accumulation): the
+// smallest split that fills the waves best, keeping >= 8 k-blocks per split.
+static int choose_splits(long tiles, int nkb) {
+  const long sms = num_sms();
+  int best = 1;
+  double best_eff = 0.0;
+  for (int sp = 1; sp <= 32 && nkb >= 8 * sp; ++sp) {
+    const long t = tiles * sp;
+    const double eff = (double)t / (double)(sms * ((t + sms - 1) / sms));
+    if (eff > best_eff + 0.03) { best_eff = eff; best = sp; }
+  }
+  return best;
 }
 
 static int run(const Call& c, cudaStream_t s) {
   if (c.M <= 0 || c.N <= 0 || c.K <= 0) return GPT2_ERR_ARG;
   if (c.N % 32 || c.K % BK) return GPT2_ERR_ARG;
-  const int BN = choose_bn(c);
+  // weight gradients take full-width tiles; the split of the reduction fills the waves
+  const int BN = (c.kind == WGRAD && !c.force_bn && c.N % 256 == 0) ? 256 : choose_bn(c);
   if (BN != 128 && BN != 256) return GPT2_ERR_ARG;
   Params p{};
   p.M = c.M; p.N = c.N; p.K = c.K;
@@ -394,13 +430,7 @@ static int run(const Call& c, cudaStream_t s) {
   p.nkb = c.K / BK;
   int splits = 1;
   if (c.kind == WGRAD) {
-    if (c.force_splits) {
-      splits = c.force_splits;
-    } else {
-      const int tiles = p.num_m * p.num_n;
-      const int sms = num_sms();
-      while (tiles * splits < sms && p.nkb / (splits * 2) >= 8) splits *= 2;
-    }
+    splits = c.force_splits ? c.force_splits : choose_splits((long)p.num_m * p.num_n, p.nkb);
   } else if (c.force_splits > 1) {
     return GPT2_ERR_ARG;
   }
@@ -423,10 +453,19 @@ static int run(const Call& c, cudaStream_t s) {
     ok = make_map(&ta, c.a, c.K, c.M, c.lda, 64, BM) && make_map(&tb, c.b, c.K, c.N, c.ldb, 64, BN);
   }
   if (!ok) return GPT2_ERR_ARG;
+  // bf16 outputs leave through TMA stores of 32 x 32 boxes (64-byte swizzle)
+  CUtensorMap to, to2;
+  memset(&to, 0, sizeof(to));
+  memset(&to2, 0, sizeof(to2));
+  if (c.epi != EPI_ACC_F32) {
+    if (!make_map(&to, c.out, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return GPT2_ERR_ARG;
+    if (c.epi == EPI_GELU && !make_map(&to2, c.out2, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      return GPT2_ERR_ARG;
+  }
 
   cudaError_t e = cudaErrorInvalidValue;
 #define GPT2_GEMM_CASE(BNV, AMN, BMN, EPIV) \
-  e = launch_tc<BNV, AMN, BMN, EPIV>(ta, tb, p, s)
+  e = launch_tc<BNV, AMN, BMN, EPIV>(ta, tb, to, to2, p, s)
   if (c.kind == FWD) {
     switch (c.epi) {
       case EPI_STORE: if (BN == 256) GPT2_GEMM_CASE(256, false, false, EPI_STORE); else GPT2_GEMM_CASE(128, false, false, EPI_STORE); break;

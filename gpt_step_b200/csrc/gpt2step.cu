@@ -131,7 +131,7 @@ void make_layout(const Dims& d, Layout* lay) {
   lay->datty = take(N * C * 2);
   lay->dq_acc = take(N * C * 4);
   lay->attD = take(N * d.H * 4);
-  lay->ln_part = take((size_t)kLnBwdBlocks * 2 * C * 4);
+  lay->ln_part = take((size_t)kLnBwdBlocks * 3 * C * 4);
   lay->col_part = take((size_t)kMaxStrips * 4 * C * 4);
   lay->norm_part = take(kNormBlocks * 8);
   lay->losses = take(N * 4);
@@ -241,33 +241,49 @@ int ln_fwd(const bf16* x, const float* w, const float* b, bf16* y, float* mean, 
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
-size_t ln_bwd_workspace(int rows, int C) {
-  const int blocks = std::min(kLnBwdBlocks, (rows + 7) / 8);
-  return (size_t)blocks * 2 * C * 4;
+int ln_bwd_blocks(int rows, int C) {
+  const int warps = C <= 768 ? 8 : 4;
+  return std::min(kLnBwdBlocks, (rows + warps - 1) / warps);
 }
+
+// Workspace of the LayerNorm backward: one partial row of nq * C floats per CTA
+// (nq = 2: dw, db; nq = 3 adds the column sum of dx).
+size_t ln_bwd_workspace(int rows, int C, int nq = 2) { return (size_t)ln_bwd_blocks(rows, C) * nq * C * 4; }
 
 template <int C>
 void ln_bwd_c(const bf16* dy, const bf16* x, const float* mean, const float* rstd, const float* w,
-              const bf16* dresid, bf16* dx, float* part, int rows, int blocks, cudaStream_t s) {
-  k::layernorm_bwd_kernel<C><<<blocks, 256, 0, s>>>(dy, x, mean, rstd, w, dresid, dx, part, rows);
+              const bf16* dresid, bf16* dx, float* part, int rows, int blocks, int with_dxsum, cudaStream_t s) {
+  using Cfg = k::LnBwdCfg<C>;
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(k::layernorm_bwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
+    attr = true;
+  }
+  k::layernorm_bwd_kernel<C><<<blocks, Cfg::WARPS * 32, Cfg::SMEM, s>>>(dy, x, mean, rstd, w, dresid, dx, part, rows,
+                                                                        with_dxsum);
 }
 
+// dbias (may be NULL) receives the column sum of dx: the bias gradient of the
+// projection whose output gradient dx is.
 int ln_bwd(const bf16* dy, const bf16* x, const float* mean, const float* rstd, const float* w, const bf16* dresid,
-           bf16* dx, float* dw, float* db, int rows, int C, float* part, size_t part_bytes, cudaStream_t s) {
-  const int blocks = std::min(kLnBwdBlocks, (rows + 7) / 8);
-  if (part_bytes < (size_t)blocks * 2 * C * 4) return GPT2_ERR_ARG;
+           bf16* dx, float* dw, float* db, float* dbias, int rows, int C, float* part, size_t part_bytes,
+           cudaStream_t s) {
+  const int nq = dbias ? 3 : 2;
+  const int blocks = ln_bwd_blocks(rows, C);
+  if (part_bytes < (size_t)blocks * nq * C * 4) return GPT2_ERR_ARG;
+  const int wd = dbias ? 1 : 0;
   switch (C) {
-    case 128: ln_bwd_c<128>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, s); break;
-    case 256: ln_bwd_c<256>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, s); break;
-    case 384: ln_bwd_c<384>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, s); break;
-    case 512: ln_bwd_c<512>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, s); break;
-    case 768: ln_bwd_c<768>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, s); break;
-    case 1024: ln_bwd_c<1024>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, s); break;
-    case 1536: ln_bwd_c<1536>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, s); break;
-    case 2048: ln_bwd_c<2048>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, s); break;
+    case 128: ln_bwd_c<128>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 256: ln_bwd_c<256>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 384: ln_bwd_c<384>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 512: ln_bwd_c<512>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 768: ln_bwd_c<768>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 1024: ln_bwd_c<1024>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 1536: ln_bwd_c<1536>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 2048: ln_bwd_c<2048>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
     default: return GPT2_ERR_ARG;
   }
-  k::layernorm_bwd_reduce_kernel<<<(2 * C + 255) / 256, 256, 0, s>>>(part, dw, db, blocks, C);
+  k::partial_rows_reduce_kernel<<<(nq * C + 31) / 32, 256, 0, s>>>(part, blocks, nq * C, dw, db, dbias, C);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -299,7 +315,8 @@ int bias_grad(const bf16* dout, float* db, int M, int N, float* part, size_t par
 
 int softmax_ce(bf16* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,
                int write_grad, int* err, cudaStream_t s) {
-  if (Vp % 8 || V > Vp || V <= 0) return GPT2_ERR_ARG;
+  if (Vp % 8 || V > Vp || V <= 0 || Vp * 2 > 200 * 1024) return GPT2_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(logits) & 15) != 0) return GPT2_ERR_ARG;
   const int smem = Vp * 2;
   static int attr_bytes = 0;
   if (smem > 48 * 1024 && smem > attr_bytes) {
@@ -482,11 +499,12 @@ int bias_grad_m(gpt2_model* m, const bf16* dout, float* db, int M, int N) {
 }
 
 int ln_bwd_m(gpt2_model* m, const bf16* dy, const bf16* x, const float* mean, const float* rstd, int kw, int kb,
-             int l, const bf16* dresid, bf16* dx) {
+             int l, const bf16* dresid, bf16* dx, float* dbias) {
   const Dims& d = m->lay.d;
   const size_t p = prof_begin(m);
-  const int st = launch::ln_bwd(dy, x, mean, rstd, m->P(kw, l), dresid, dx, m->G(kw, l), m->G(kb, l), (int)d.N, d.C,
-                                m->at<float>(m->lay.ln_part), (size_t)kLnBwdBlocks * 2 * d.C * 4, m->stream);
+  const int st = launch::ln_bwd(dy, x, mean, rstd, m->P(kw, l), dresid, dx, m->G(kw, l), m->G(kb, l), dbias,
+                                (int)d.N, d.C, m->at<float>(m->lay.ln_part), (size_t)kLnBwdBlocks * 3 * d.C * 4,
+                                m->stream);
   prof_end(m, p, PC_LN_BWD, (double)d.N * ((dresid ? 8.0 : 6.0) * d.C + 8), 2);
   return st;
 }
@@ -519,8 +537,9 @@ int backward(gpt2_model* m, const int32_t* tok) {
     c.a = dlogits; c.lda = d.Vp; c.b = lnf; c.ldb = C; c.outf = m->G(K_WTE); c.ldf = C;
     GPT2_TRY(run_gemm(m, c));
   }
+  // the residual gradient leaving ln_f is the output gradient of the last MLP projection
   GPT2_TRY(ln_bwd_m(m, dln, resid + L * NC, m->at<float>(y.lnf_mean), m->at<float>(y.lnf_rstd), K_LNFW, K_LNFB, 0,
-                    nullptr, dresid));
+                    nullptr, dresid, L > 0 ? m->G(K_FCPROJB, L - 1) : nullptr));
 
   for (int l = L - 1; l >= 0; --l) {
     bf16* x_in = resid + l * NC;
@@ -539,7 +558,6 @@ int backward(gpt2_model* m, const int32_t* tok) {
       c.a = dresid; c.lda = C; c.b = fchg; c.ldb = 4 * C; c.outf = m->G(K_FCPROJW, l); c.ldf = 4 * C;
       GPT2_TRY(run_gemm(m, c));
     }
-    GPT2_TRY(bias_grad_m(m, dresid, m->G(K_FCPROJB, l), N, C));
     {
       gemm::Call c = gemm_call(gemm::DGRAD, gemm::EPI_DGELU, N, 4 * C, C, err);
       c.a = dresid; c.lda = C; c.b = m->W(K_FCPROJW, l); c.ldb = 4 * C; c.out = d4c; c.ldo = 4 * C;
@@ -559,14 +577,13 @@ int backward(gpt2_model* m, const int32_t* tok) {
       GPT2_TRY(run_gemm(m, c));
     }
     GPT2_TRY(ln_bwd_m(m, dln, xmid, m->at<float>(y.ln2_mean) + l * d.N, m->at<float>(y.ln2_rstd) + l * d.N, K_LN2W,
-                      K_LN2B, l, dresid, dresid));
+                      K_LN2B, l, dresid, dresid, m->G(K_ATTPROJB, l)));
     // attention projection
     {
       gemm::Call c = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, C, C, N, err);
       c.a = dresid; c.lda = C; c.b = atty; c.ldb = C; c.outf = m->G(K_ATTPROJW, l); c.ldf = C;
       GPT2_TRY(run_gemm(m, c));
     }
-    GPT2_TRY(bias_grad_m(m, dresid, m->G(K_ATTPROJB, l), N, C));
     {
       gemm::Call c = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, C, err);
       c.a = dresid; c.lda = C; c.b = m->W(K_ATTPROJW, l); c.ldb = C; c.out = datty; c.ldo = C;
@@ -591,7 +608,7 @@ int backward(gpt2_model* m, const int32_t* tok) {
       GPT2_TRY(run_gemm(m, c));
     }
     GPT2_TRY(ln_bwd_m(m, dln, x_in, m->at<float>(y.ln1_mean) + l * d.N, m->at<float>(y.ln1_rstd) + l * d.N, K_LN1W,
-                      K_LN1B, l, dresid, dresid));
+                      K_LN1B, l, dresid, dresid, l > 0 ? m->G(K_FCPROJB, l - 1) : nullptr));
   }
   // embeddings
   {
@@ -983,7 +1000,7 @@ int gpt2op_layernorm_bwd(const void* dy, const void* x, const float* mean, const
                          size_t ws_bytes, void* stream) {
   if (!dy || !x || !mean || !rstd || !w || !dx || !dw || !db || !workspace || rows <= 0) return GPT2_ERR_ARG;
   return launch::ln_bwd(static_cast<const bf16*>(dy), static_cast<const bf16*>(x), mean, rstd, w,
-                        static_cast<const bf16*>(dresid), static_cast<bf16*>(dx), dw, db, rows, C,
+                        static_cast<const bf16*>(dresid), static_cast<bf16*>(dx), dw, db, nullptr, rows, C,
                         static_cast<float*>(workspace), ws_bytes, static_cast<cudaStream_t>(stream));
 }
 
@@ -1032,7 +1049,7 @@ int gpt2op_layernorm_bwd_noalloc(const void* dy, const void* x, const float* mea
   const int st = noalloc::scratch_for_current_device(&scratch);
   if (st != GPT2_OK) return st;
   return launch::ln_bwd(static_cast<const bf16*>(dy), static_cast<const bf16*>(x), mean, rstd, w,
-                        static_cast<const bf16*>(dresid), static_cast<bf16*>(dx), dw, db, rows, C, scratch,
+                        static_cast<const bf16*>(dresid), static_cast<bf16*>(dx), dw, db, nullptr, rows, C, scratch,
                         gpt2op_layernorm_bwd_noalloc_max_bytes(), static_cast<cudaStream_t>(stream));
 }
 

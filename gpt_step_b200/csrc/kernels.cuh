@@ -212,55 +212,67 @@ __global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restri
 }
 
 // LayerNorm backward: dx = rstd * (dy*w - mean(dy*w) - xhat * mean(dy*w*xhat))
-// (+ dresid, the gradient flowing along the residual stream), written in bf16;
-// per-block partial column sums of dy*xhat and dy go to `part` ([grid][2][C]).
+// (+ dresid, the gradient flowing along the residual stream), written in bf16.
+// Each warp keeps private column sums of dy*xhat, dy and (optionally) of its
+// output dx in shared memory; the CTA writes one partial row per quantity to
+// `part` ([grid][NQ][C], NQ = 3 with the dx sum, else 2), summed in a fixed
+// order afterwards. The dx column sum is the gradient of the bias of the
+// projection that wrote the residual stream (its output gradient is dx).
 template <int C>
-__global__ void __launch_bounds__(256) layernorm_bwd_kernel(const bf16* __restrict__ dy, const bf16* __restrict__ x,
-                                                            const float* __restrict__ mean,
-                                                            const float* __restrict__ rstd,
-                                                            const float* __restrict__ w,
-                                                            const bf16* dresid, bf16* dx,
-                                                            float* __restrict__ part, int rows) {
+struct LnBwdCfg {
+  static constexpr int WARPS = C <= 768 ? 8 : 4;
+  static constexpr int SMEM = WARPS * 3 * C * 4;
+};
+
+template <int C>
+__global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, 2)
+    layernorm_bwd_kernel(const bf16* __restrict__ dy, const bf16* __restrict__ x, const float* __restrict__ mean,
+                         const float* __restrict__ rstd, const float* __restrict__ w, const bf16* dresid, bf16* dx,
+                         float* __restrict__ part, int rows, int with_dxsum) {
   constexpr int NV = C / 8;
   constexpr int VPL = (NV + 31) / 32;
-  __shared__ float red[2][C];
+  constexpr int WARPS = LnBwdCfg<C>::WARPS;
+  extern __shared__ __align__(16) float ln_acc[];  // [WARPS][3][C]
   const int warp = threadIdx.x >> 5, l = lane_id();
-  float adw[VPL][8], adb[VPL][8];
-#pragma unroll
-  for (int i = 0; i < VPL; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) adw[i][j] = adb[i][j] = 0.f;
-  float wv[VPL][8];
-#pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int vi = l + 32 * i;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) wv[i][j] = (vi < NV) ? w[vi * 8 + j] : 0.f;
-  }
-  for (int row = blockIdx.x * 8 + warp; row < rows; row += gridDim.x * 8) {
+  float* acc = ln_acc + warp * 3 * C;
+  for (int i = l; i < 3 * C; i += 32) acc[i] = 0.f;
+  __syncwarp();
+  const int nq = with_dxsum ? 3 : 2;
+  for (int row = blockIdx.x * WARPS + warp; row < rows; row += gridDim.x * WARPS) {
     const float mu = mean[row], rs = rstd[row];
-    float xh[VPL][8], g[VPL][8];
+    uint4 ux[VPL], ud[VPL], ur[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = l + 32 * i;
+      ur[i] = make_uint4(0u, 0u, 0u, 0u);
+      if (vi < NV) {
+        ux[i] = *reinterpret_cast<const uint4*>(x + (size_t)row * C + vi * 8);
+        ud[i] = *reinterpret_cast<const uint4*>(dy + (size_t)row * C + vi * 8);
+        if (dresid != nullptr) ur[i] = *reinterpret_cast<const uint4*>(dresid + (size_t)row * C + vi * 8);
+      }
+    }
     float s1 = 0.f, s2 = 0.f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int vi = l + 32 * i;
       if (vi < NV) {
-        const uint4 ux = *reinterpret_cast<const uint4*>(x + (size_t)row * C + vi * 8);
-        const uint4 ud = *reinterpret_cast<const uint4*>(dy + (size_t)row * C + vi * 8);
-        const uint32_t xw[4] = {ux.x, ux.y, ux.z, ux.w}, dw4[4] = {ud.x, ud.y, ud.z, ud.w};
+        const uint32_t xw[4] = {ux[i].x, ux[i].y, ux[i].z, ux[i].w}, dw4[4] = {ud[i].x, ud[i].y, ud[i].z, ud[i].w};
+        const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + vi * 8));
+        const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + vi * 8 + 4));
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        float* a0 = acc + vi * 8;
+        float* a1 = acc + C + vi * 8;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 fx = unpack_bf16x2(xw[j]), fd = unpack_bf16x2(dw4[j]);
-          xh[i][2 * j] = (fx.x - mu) * rs;
-          xh[i][2 * j + 1] = (fx.y - mu) * rs;
-          adw[i][2 * j] += fd.x * xh[i][2 * j];
-          adw[i][2 * j + 1] += fd.y * xh[i][2 * j + 1];
-          adb[i][2 * j] += fd.x;
-          adb[i][2 * j + 1] += fd.y;
-          g[i][2 * j] = fd.x * wv[i][2 * j];
-          g[i][2 * j + 1] = fd.y * wv[i][2 * j + 1];
-          s1 += g[i][2 * j] + g[i][2 * j + 1];
-          s2 += g[i][2 * j] * xh[i][2 * j] + g[i][2 * j + 1] * xh[i][2 * j + 1];
+          const float xh0 = (fx.x - mu) * rs, xh1 = (fx.y - mu) * rs;
+          a0[2 * j] += fd.x * xh0;
+          a0[2 * j + 1] += fd.y * xh1;
+          a1[2 * j] += fd.x;
+          a1[2 * j + 1] += fd.y;
+          const float g0 = fd.x * wv[2 * j], g1 = fd.y * wv[2 * j + 1];
+          s1 += g0 + g1;
+          s2 += g0 * xh0 + g1 * xh1;
         }
       }
     }
@@ -269,61 +281,65 @@ __global__ void __launch_bounds__(256) layernorm_bwd_kernel(const bf16* __restri
     for (int i = 0; i < VPL; ++i) {
       const int vi = l + 32 * i;
       if (vi < NV) {
+        const uint32_t xw[4] = {ux[i].x, ux[i].y, ux[i].z, ux[i].w}, dw4[4] = {ud[i].x, ud[i].y, ud[i].z, ud[i].w};
+        const uint32_t rw[4] = {ur[i].x, ur[i].y, ur[i].z, ur[i].w};
+        const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + vi * 8));
+        const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + vi * 8 + 4));
+        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         float r[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) r[j] = (g[i][j] - m1 - xh[i][j] * m2) * rs;
-        if (dresid != nullptr) {
-          const uint4 u = *reinterpret_cast<const uint4*>(dresid + (size_t)row * C + vi * 8);
-          const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+        for (int j = 0; j < 4; ++j) {
+          const float2 fx = unpack_bf16x2(xw[j]), fd = unpack_bf16x2(dw4[j]), fr = unpack_bf16x2(rw[j]);
+          r[2 * j] = (fd.x * wv[2 * j] - m1 - (fx.x - mu) * rs * m2) * rs + fr.x;
+          r[2 * j + 1] = (fd.y * wv[2 * j + 1] - m1 - (fx.y - mu) * rs * m2) * rs + fr.y;
+        }
+        const uint4 o = make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
+                                   pack_bf16x2(r[6], r[7]));
+        *reinterpret_cast<uint4*>(dx + (size_t)row * C + vi * 8) = o;
+        if (with_dxsum) {
+          // the bias gradient sees the stored (bf16) residual gradient
+          const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
+          float* a2 = acc + 2 * C + vi * 8;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const float2 f = unpack_bf16x2(uw[j]);
-            r[2 * j] += f.x;
-            r[2 * j + 1] += f.y;
-          }
-        }
-        *reinterpret_cast<uint4*>(dx + (size_t)row * C + vi * 8) =
-            make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
-                       pack_bf16x2(r[6], r[7]));
-      }
-    }
-  }
-  // combine the 8 warps' column sums in a fixed order (deterministic)
-  for (int wi = 0; wi < 8; ++wi) {
-    if (warp == wi) {
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        const int vi = l + 32 * i;
-        if (vi < NV) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            if (wi == 0) {
-              red[0][vi * 8 + j] = adw[i][j];
-              red[1][vi * 8 + j] = adb[i][j];
-            } else {
-              red[0][vi * 8 + j] += adw[i][j];
-              red[1][vi * 8 + j] += adb[i][j];
-            }
+            const float2 f = unpack_bf16x2(ow[j]);
+            a2[2 * j] += f.x;
+            a2[2 * j + 1] += f.y;
           }
         }
       }
     }
-    __syncthreads();
   }
-  for (int c = threadIdx.x; c < 2 * C; c += blockDim.x)
-    part[(size_t)blockIdx.x * 2 * C + c] = red[c / C][c % C];
+  __syncthreads();
+  // combine the warps' column sums in a fixed order (deterministic)
+  for (int c = threadIdx.x; c < nq * C; c += WARPS * 32) {
+    float sum = 0.f;
+#pragma unroll
+    for (int wi = 0; wi < WARPS; ++wi) sum += ln_acc[wi * 3 * C + c];
+    part[(size_t)blockIdx.x * nq * C + c] = sum;
+  }
 }
 
-// Sum nblk partial rows ([nblk][2][C]) in order and add into dw, db (fp32 grads).
-__global__ void layernorm_bwd_reduce_kernel(const float* __restrict__ part, float* __restrict__ dw,
-                                            float* __restrict__ db, int nblk, int C) {
-  const int c = blockIdx.x * blockDim.x + threadIdx.x;
-  if (c >= 2 * C) return;
-  const int which = c / C, col = c % C;
+// Sum the nblk partial rows of `part` ([nblk][width], width = nq * C) column by
+// column in a fixed order and add them into out0 (dw), out1 (db) and out2 (bias
+// grad, when nq == 3). Block (32 x 8): 32 columns, 8 row-lanes, then a fold.
+__global__ void __launch_bounds__(256) partial_rows_reduce_kernel(const float* __restrict__ part, int nblk, int width,
+                                                                 float* out0, float* out1, float* out2, int C) {
+  __shared__ float red[8][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  const int col = blockIdx.x * 32 + tx;
   float s = 0.f;
-  for (int i = 0; i < nblk; ++i) s += part[((size_t)i * 2 + which) * C + col];
-  if (which == 0) dw[col] += s;
-  else db[col] += s;
+  if (col < width)
+    for (int i = ty; i < nblk; i += 8) s += part[(size_t)i * width + col];
+  red[ty][tx] = s;
+  __syncthreads();
+  if (ty == 0 && col < width) {
+#pragma unroll
+    for (int y = 1; y < 8; ++y) s += red[y][tx];
+    const int which = col / C, c = col % C;
+    float* dst = which == 0 ? out0 : (which == 1 ? out1 : out2);
+    dst[c] += s;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -338,7 +354,24 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const bf16* __restr
   const int r1 = min(M, r0 + rows_per_strip);
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (c < N) {
-    for (int r = r0 + ty; r < r1; r += 8) {
+    int r = r0 + ty;
+    // four independent rows per iteration keep four 16-byte loads in flight
+    for (; r + 24 < r1; r += 32) {
+      uint4 u[4];
+#pragma unroll
+      for (int k2 = 0; k2 < 4; ++k2) u[k2] = *reinterpret_cast<const uint4*>(a + (size_t)(r + 8 * k2) * N + c);
+#pragma unroll
+      for (int k2 = 0; k2 < 4; ++k2) {
+        const uint32_t w[4] = {u[k2].x, u[k2].y, u[k2].z, u[k2].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack_bf16x2(w[j]);
+          acc[2 * j] += f.x;
+          acc[2 * j + 1] += f.y;
+        }
+      }
+    }
+    for (; r < r1; r += 8) {
       const uint4 u = *reinterpret_cast<const uint4*>(a + (size_t)r * N + c);
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
@@ -349,6 +382,7 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const bf16* __restr
       }
     }
   }
+
   __shared__ float red[8][32][9];
 #pragma unroll
   for (int j = 0; j < 8; ++j) red[ty][tx][j] = acc[j];
@@ -386,17 +420,31 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
                                                                 const int32_t* __restrict__ targets,
                                                                 float* __restrict__ losses, int V, int Vp,
                                                                 float dscale, int write_grad, int* err) {
-  extern __shared__ __align__(16) uint8_t smem_ce[];
+  extern __shared__ __align__(128) uint8_t smem_ce[];
   uint4* row_s = reinterpret_cast<uint4*>(smem_ce);
   __shared__ float red_m[kCeThreads / 32], red_s[kCeThreads / 32];
   __shared__ float bc[2];
+  __shared__ __align__(8) uint64_t bar;
   const int row = blockIdx.x;
   uint4* zr = reinterpret_cast<uint4*>(logits + (size_t)row * Vp);
   const int nv = Vp / 8;
+  // the whole row arrives with one bulk copy (Vp * 2 bytes, a multiple of 16)
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(smem_u32(&bar), (uint32_t)Vp * 2u);
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(row_s)),
+                 "l"(zr), "r"((uint32_t)Vp * 2u), "r"(smem_u32(&bar))
+                 : "memory");
+  }
+  const bool loaded = mbar_wait(smem_u32(&bar), 0, err);
   float m = -INFINITY, s = 0.f;
-  for (int i = threadIdx.x; i < nv; i += kCeThreads) {
-    const uint4 u = zr[i];
-    row_s[i] = u;
+  for (int i = threadIdx.x; i < nv && loaded; i += kCeThreads) {
+    const uint4 u = row_s[i];
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
     float f[8];
 #pragma unroll

@@ -1,0 +1,107 @@
+"""Profiling driver: one training micro-step, or one GEMM shape, in isolation.
+
+  python -m gpt_step_b200.profile_step step --workload gpt2_124m [--micro-batch B]
+      Creates the model, runs one warm-up optimizer step (1 micro-step), then
+      one micro-step (fwd_bwd) plus clip_adamw inside an NVTX range named
+      "profiled" (use `ncu --nvtx --nvtx-include "profiled/"`), and prints the
+      kernel launch count of that range and per-class event timings.
+
+  python -m gpt_step_b200.profile_step gemm --kind fwd|dgrad|wgrad --shape M,N,K [--iters n]
+      Times one tcgen05 GEMM arrangement through the op-level C ABI with CUDA
+      events (bf16 inputs, fp32 accumulation) and prints TFLOP/s. M, N, K are the
+      GEMM's own dimensions: output M x N, reduction K.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import numpy as np
+
+
+def run_step(args):
+    import torch
+
+    import gpt_step_b200 as gs
+    from gpt_step_b200 import build, synth, workloads
+    build.build()
+    over = {}
+    if args.micro_batch:
+        over["micro_batch"] = args.micro_batch
+    margs = workloads.model_args(args.workload, **over)
+    w = workloads.WORKLOADS[args.workload]
+    m = gs.GPT2(gs.Config.make(**margs), 1337)
+    B, T, V = margs["micro_batch"], margs["seq_len"], margs["vocab_real"]
+    src = synth.TokenSource(B, T, V, 1337, w["mean_doc_len"], 4 * B)
+    batches = [src.get() for _ in range(2)]
+    tok = [torch.tensor(x, device="cuda") for x, _ in batches]
+    tgt = [torch.tensor(y, device="cuda") for _, y in batches]
+    m.fwd_bwd(tok[0], tgt[0])
+    m.clip_adamw(0)
+    torch.cuda.synchronize()
+    n0 = m.kernel_launches()
+    m.profile(True)
+    torch.cuda.nvtx.range_push("profiled")
+    m.fwd_bwd(tok[1], tgt[1])
+    m.clip_adamw(1)
+    torch.cuda.nvtx.range_pop()
+    torch.cuda.synchronize()
+    prof = m.profile_read()
+    print(json.dumps({"workload": args.workload, "micro_batch": B,
+                      "launches_in_range": m.kernel_launches() - n0, "classes": prof}))
+
+
+def run_gemm(args):
+    import torch
+
+    import gpt_step_b200 as gs
+    from gpt_step_b200 import build
+    build.build()
+    M, N, K = (int(v) for v in args.shape.split(","))
+    rng = np.random.default_rng(0)
+    bf = lambda *s: torch.tensor(rng.standard_normal(s).astype(np.float32) * 0.1).to(torch.bfloat16).cuda()
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    if args.kind == "fwd":
+        a, b, out = bf(M, K), bf(N, K), torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        fn = lambda: gs.linear_fwd(a, b, None, None, out, err)
+    elif args.kind == "dgrad":
+        # din[M, N] = dout[M, K] . w[K, N]   (the op names the reduction N)
+        a, b, out = bf(M, K), bf(K, N), torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        fn = lambda: gs.linear_dgrad(a, b, None, out, err)
+    else:
+        # dw[M, N] += dout[K, M]^T . inp[K, N]
+        a, b = bf(K, M), bf(K, N)
+        out = torch.zeros(M, N, device="cuda")
+        fn = lambda: gs.linear_wgrad(a, b, out, err, splits=args.splits)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.iters
+    tf = 2.0 * M * N * K / (ms / 1000.0) / 1e12
+    print(json.dumps({"kind": args.kind, "M": M, "N": N, "K": K, "ms": ms, "tflops": tf,
+                      "err": int(err.sum())}))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    sub = ap.add_subparsers(dest="mode", required=True)
+    s = sub.add_parser("step")
+    s.add_argument("--workload", default="gpt2_124m")
+    s.add_argument("--micro-batch", type=int, default=0)
+    g = sub.add_parser("gemm")
+    g.add_argument("--kind", choices=["fwd", "dgrad", "wgrad"], default="fwd")
+    g.add_argument("--shape", default="19456,3072,768")
+    g.add_argument("--iters", type=int, default=20)
+    g.add_argument("--splits", type=int, default=0)
+    args = ap.parse_args()
+    run_step(args) if args.mode == "step" else run_gemm(args)
+
+
+if __name__ == "__main__":
+    main()

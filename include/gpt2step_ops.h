@@ -81,8 +81,8 @@ int gpt2op_layernorm_bwd(const void* dy, const void* x, const float* mean, const
  * Its scratch is one fixed array inside the library, of
  * gpt2op_layernorm_bwd_noalloc_max_bytes() = 2,424,832 bytes, that every GPU
  * which loads the library keeps until the process exits. A call needing more
- * (min(296, ceil(rows / 8)) * 2 * C * 4 bytes; any row count fits for
- * C <= 1024) returns GPT2_ERR_ARG before touching the GPU. The first call on a
+ * (8 * C * min(296, ceil(rows / w)) bytes, w = 8 for C <= 768 and 4 above; any
+ * row count fits for C <= 1024) returns GPT2_ERR_ARG before touching the GPU. The first call on a
  * device looks up the array's device address and should come before any stream
  * capture. All calls share the array: calls that overlap on the GPU race. */
 size_t gpt2op_layernorm_bwd_noalloc_max_bytes(void);
