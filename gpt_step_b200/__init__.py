@@ -91,9 +91,9 @@ _SIGNATURES = {
     "gpt2op_layernorm_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _SZ, _P]),
     "gpt2op_layernorm_bwd_noalloc_max_bytes": (_SZ, []),
     "gpt2op_layernorm_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P]),
-    "gpt2op_attention_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "gpt2op_attention_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "gpt2op_attention_bwd_workspace": (_SZ, [_I, _I, _I, _I]),
-    "gpt2op_attention_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]),
+    "gpt2op_attention_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P]),
     "gpt2op_softmax_ce": (_I, [_P, _P, _P, _I, _I, _I, _F, _P, _P]),
     "gpt2op_embedding_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "gpt2op_embedding_bwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
@@ -359,23 +359,23 @@ def layernorm_bwd_noalloc(dy, x, mean, rstd, w, dresid, dx, dw, db, stream=None)
                                              _s(stream)), "gpt2op_layernorm_bwd_noalloc")
 
 
-def attention_fwd(qkv, out, lse, n_head, stream=None):
+def attention_fwd(qkv, out, lse, n_head, err, stream=None):
     B, T, C3 = qkv.shape
     hd = C3 // 3 // n_head
-    check(lib().gpt2op_attention_fwd(_ptr(qkv), _ptr(out), _ptr(lse), B, T, n_head, hd, _s(stream)),
-          "gpt2op_attention_fwd")
+    check(lib().gpt2op_attention_fwd(_ptr(qkv), _ptr(out), _ptr(lse), B, T, n_head, hd, _ptr(err),
+                                     _s(stream)), "gpt2op_attention_fwd")
 
 
 def attention_bwd_workspace(B, T, H, hd):
     return lib().gpt2op_attention_bwd_workspace(B, T, H, hd)
 
 
-def attention_bwd(qkv, out, dout, lse, dqkv, n_head, workspace, stream=None):
+def attention_bwd(qkv, out, dout, lse, dqkv, n_head, workspace, err, stream=None):
     B, T, C3 = qkv.shape
     hd = C3 // 3 // n_head
     check(lib().gpt2op_attention_bwd(_ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dqkv), B, T,
-                                     n_head, hd, _ptr(workspace), workspace.numel(), _s(stream)),
-          "gpt2op_attention_bwd")
+                                     n_head, hd, _ptr(workspace), workspace.numel(), _ptr(err),
+                                     _s(stream)), "gpt2op_attention_bwd")
 
 
 def softmax_ce(logits, targets, losses, V, dscale, err, stream=None):

@@ -1,0 +1,655 @@
+// Causal flash attention forward on the 5th-generation tensor cores (head size 64).
+//
+// Same operation as attn::attn_fwd_kernel (grow_a_language_model_intro,
+// activities 5-6: softmax(Q K^T / sqrt(d)) V with a causal mask, per head),
+// organised for tcgen05:
+//
+//   CTA     one (batch, head) and 128 query rows; walks key blocks of 128
+//   warp 0  TMA: Q once, then K_j and V_j (double-buffered ring)
+//   warp 1  tensor-memory allocation; lane 0 issues
+//             S_j = Q K_j^T   (M=128, N=128, K=64)  into S[j % 2] (TMEM)
+//             O  += P_j V_j   (M=128, N=64,  K=128) into O (TMEM)
+//   warps 2-5  one query row per thread: read S_j from TMEM, online softmax in
+//             log2 units, write P_j (bf16) to shared memory as the A operand of
+//             the next MMA, rescale O in TMEM when the row maximum grows by more
+//             than 2^8 (otherwise the stale maximum is kept: p <= 256 is exact
+//             enough in fp32 and bf16), finally O / l and the log-sum-exp.
+//
+// Operands: Q, K are K-major (head dimension contiguous); V is used as stored
+// ([key][head dim]) as an MN-major B operand; P is K-major. All tiles use the
+// 128-byte swizzle (rows of 64 bf16). No cluster multicast.
+#pragma once
+#include "common.cuh"
+
+namespace attn_tc {
+
+constexpr int BQ = 128, BKV = 128, HD = 64;
+constexpr int kThreads = 192;
+constexpr int Q_BYTES = BQ * HD * 2;         // 16 KB
+constexpr int KV_BYTES = BKV * HD * 2;       // 16 KB each for K and V
+constexpr int P_BYTES = BQ * BKV * 2;        // 32 KB (two 64-key K blocks)
+constexpr int STAGES = 2;
+constexpr int SMEM_BYTES = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr int TMEM_COLS = 256;               // S [0,128), O [128,192); two CTAs share an SM
+constexpr uint32_t S_COL0 = 0, O_COL = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kRescaleThreshold = 8.0f;    // log2(256)
+
+GPT2_DEV void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]),
+      "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]),
+      "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]),
+      "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 2)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
+                       int T, int H, float scale, int* err) {
+  extern __shared__ __align__(1024) uint8_t smem_raw_af[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_af) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + Q_BYTES;                  // [STAGES][KV_BYTES]
+  uint8_t* sV = sK + STAGES * KV_BYTES;        // [STAGES][KV_BYTES]
+  uint8_t* sP = sV + STAGES * KV_BYTES;        // [P_BYTES]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + P_BYTES);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;     // [2]  K_j landed
+  uint64_t* k_empty = bars + 3;    // [2]  S_j computed: K stage free
+  uint64_t* v_full = bars + 5;     // [2]
+  uint64_t* v_empty = bars + 7;    // [2]  P_j V_j computed: V stage free
+  uint64_t* s_full = bars + 9;
+  uint64_t* s_empty = bars + 10;
+  uint64_t* p_full = bars + 11;
+  uint64_t* p_empty = bars + 12;
+  uint64_t* o_done = bars + 13;
+  uint64_t* done = bars + 14;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nqb = T / BQ;
+  const int qb = nqb - 1 - blockIdx.x;  // heaviest query tiles first
+  const int bh = blockIdx.y;
+  const int b = bh / H, h = bh % H;
+  const int C = H * HD;
+  const int row_base = b * T;           // row of token (b, 0) in the [B*T, 3C] view
+  const int nkv = qb + 1;               // causal: key blocks 0..qb
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(q_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&k_full[i]), 1);
+      mbar_init(smem_u32(&k_empty[i]), 1);
+      mbar_init(smem_u32(&v_full[i]), 1);
+      mbar_init(smem_u32(&v_empty[i]), 1);
+    }
+    mbar_init(smem_u32(s_full), 1);
+    mbar_init(smem_u32(s_empty), 128);
+    mbar_init(smem_u32(p_full), 128);
+    mbar_init(smem_u32(p_empty), 1);
+    mbar_init(smem_u32(o_done), 1);
+    mbar_init(smem_u32(done), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // -------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(smem_u32(q_full), Q_BYTES);
+      tma_load_2d(smem_u32(sQ), &tm_qkv, smem_u32(q_full), h * HD, row_base + qb * BQ);
+      // K and V run as separate two-deep rings: K_j is released once S_j is
+      // computed, V_j once P_j V_j is, so K runs further ahead than V.
+      int nk = 0, nv = 0;
+      const unsigned long long t0 = globaltimer_ns();
+      while (nk < nkv || nv < nkv) {
+        bool progressed = false;
+        if (nk < nkv && (nk < 2 || mbar_try_wait(smem_u32(&k_empty[nk & 1]), ((nk >> 1) & 1) ^ 1))) {
+          const int st = nk & 1;
+          mbar_arrive_expect_tx(smem_u32(&k_full[st]), KV_BYTES);
+          tma_load_2d(smem_u32(sK + st * KV_BYTES), &tm_qkv, smem_u32(&k_full[st]), C + h * HD,
+                      row_base + nk * BKV);
+          ++nk;
+          progressed = true;
+        }
+        if (nv < nkv && nv < nk && (nv < 2 || mbar_try_wait(smem_u32(&v_empty[nv & 1]), ((nv >> 1) & 1) ^ 1))) {
+          const int st = nv & 1;
+          mbar_arrive_expect_tx(smem_u32(&v_full[st]), KV_BYTES);
+          tma_load_2d(smem_u32(sV + st * KV_BYTES), &tm_qkv, smem_u32(&v_full[st]), 2 * C + h * HD,
+                      row_base + nv * BKV);
+          ++nv;
+          progressed = true;
+        }
+        if (!progressed) {
+          if (*(volatile int*)err & DEVERR_TIMEOUT) break;
+          if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(err, DEVERR_TIMEOUT);
+            break;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKV, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(BQ, HD, false, true);
+      bool ok = mbar_wait(smem_u32(q_full), 0, err);
+      const uint32_t q_addr = smem_u32(sQ);
+      auto issue_s = [&](int j) {
+        const int st = j & 1;
+        const uint32_t k_addr = smem_u32(sK + st * KV_BYTES);
+        const uint32_t d = tmem + S_COL0;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          tc_mma_bf16(d, smem_desc_sw128(q_addr + kk * 32, 16, 1024), smem_desc_sw128(k_addr + kk * 32, 16, 1024),
+                      idesc_s, kk > 0 ? 1u : 0u);
+        tc_commit(smem_u32(s_full));
+        tc_commit(smem_u32(&k_empty[st]));
+      };
+      if (ok && mbar_wait(smem_u32(&k_full[0]), 0, err)) {
+        tc_fence_after();
+        issue_s(0);
+      } else {
+        ok = false;
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int st = j & 1;
+        if (j + 1 < nkv) {
+          const int sn = (j + 1) & 1;
+          // K_{j+1} landed, and the softmax has taken S_j out of tensor memory
+          if (!mbar_wait(smem_u32(&k_full[sn]), ((j + 1) >> 1) & 1, err)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(s_empty), j & 1, err)) { ok = false; break; }
+          tc_fence_after();
+          issue_s(j + 1);
+        }
+        // P_j written (and O rescaled if needed)
+        if (!mbar_wait(smem_u32(p_full), j & 1, err)) { ok = false; break; }
+        if (!mbar_wait(smem_u32(&v_full[st]), (j >> 1) & 1, err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t p_addr = smem_u32(sP);
+        const uint32_t v_addr = smem_u32(sV + st * KV_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * (BQ * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, 8192, 1024);
+          tc_mma_bf16(tmem + O_COL, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(smem_u32(p_empty));
+        tc_commit(smem_u32(&v_empty[st]));
+        tc_commit(smem_u32(o_done));
+      }
+      tc_commit(smem_u32(done));
+      mbar_wait(smem_u32(done), 0, err);
+    }
+  } else {
+    // -------------------------------------------------------------- softmax / epilogue
+    const int q4 = warp & 3;                        // TMEM lane quarter
+    const int r = q4 * 32 + lane;                   // query row within the tile
+    const int qrow = qb * BQ + r;                   // query position
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const float sl2 = scale * kLog2e;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nkv; ++j) {
+      if (!mbar_wait(smem_u32(s_full), j & 1, err)) { ok = false; break; }
+      tc_fence_after();
+      const bool diag = (j == qb);
+      const uint32_t s_tm = tmem + lane_off + S_COL0;
+      // the whole score row (128 fp32) in four loads, one wait; S is free again at once
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32_async(s_tm + c * 32, sr[c]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(s_empty));
+      if (diag) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (c * 32 + i > r) sr[c][i] = __float_as_uint(-INFINITY);
+      }
+      float mraw = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mraw = fmaxf(mraw, __uint_as_float(sr[c][i]));
+      const float mx = mraw * sl2;  // scale > 0: max commutes with it
+      // lazy rescale: keep the stale maximum unless the new one exceeds it by > 2^8
+      const bool grow = (mx > m + kRescaleThreshold) || (m == -INFINITY);
+      const float m_new = grow ? mx : m;
+      const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
+      float sum = 0.f;
+      uint32_t pkall[4][16];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i]), sl2, -m_new));
+          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, -m_new));
+          sum += p0 + p1;
+          pkall[c][i] = pack_bf16x2(p0, p1);
+        }
+      // the P buffer was last read by the PV product of block j-1
+      if (j >= 1 && !mbar_wait(smem_u32(p_empty), (j - 1) & 1, err)) { ok = false; break; }
+      uint8_t* pb = sP;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t (&pk)[16] = pkall[c];
+        const int kb = c >> 1;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int ch = (c & 1) * 4 + q;  // 16-byte chunk within the 64-key block
+          *reinterpret_cast<uint4*>(pb + kb * (BQ * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      l = l * alpha + sum;
+      m = m_new;
+      // O rescale (rows whose maximum moved) once the PV product of block j-1 is done
+      if (j > 0 && __any_sync(0xffffffffu, grow)) {
+        if (!mbar_wait(smem_u32(o_done), (j - 1) & 1, err)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          float v[32];
+          tmem_ld32(tmem + lane_off + O_COL + c * 32, v);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] *= alpha;
+          tmem_st32(tmem + lane_off + O_COL + c * 32, v);
+        }
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(p_full));
+    }
+    // epilogue: O / l, log-sum-exp
+    if (ok && mbar_wait(smem_u32(o_done), (nkv - 1) & 1, err)) {
+      tc_fence_after();
+      const float inv = 1.0f / l;
+      bf16* orow = out + ((size_t)(row_base + qrow)) * C + h * HD;
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_off + O_COL + c * 32, v);
+#pragma unroll
+        for (int i = 0; i < 32; i += 8)
+          *reinterpret_cast<uint4*>(orow + c * 32 + i) =
+              make_uint4(pack_bf16x2(v[i] * inv, v[i + 1] * inv), pack_bf16x2(v[i + 2] * inv, v[i + 3] * inv),
+                         pack_bf16x2(v[i + 4] * inv, v[i + 5] * inv), pack_bf16x2(v[i + 6] * inv, v[i + 7] * inv));
+      }
+      lse[(size_t)bh * T + qrow] = (m + log2f(l)) * kLn2;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// qkv bf16 [B*T, 3C] (q | k | v, heads contiguous), out bf16 [B*T, C], lse fp32 [B, H, T].
+static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, int* err, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    // ask for the whole shared-memory carveout so that two CTAs share an SM
+    e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int C = H * HD;
+  CUtensorMap tm;
+  if (!encode_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qkv, 3 * (uint64_t)C, (uint64_t)B * T, 3 * (uint64_t)C,
+                     64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  dim3 grid(T / BQ, B * H);
+  attn_fwd_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(tm, out, lse, T, H, 1.0f / sqrtf((float)HD), err);
+  return cudaGetLastError();
+}
+
+
+// ===========================================================================
+// Backward (head size 64): per CTA one (batch, head) and a block of 128 keys;
+// loop over the query blocks at or after it (causal). With Q_i, dO_i (128
+// queries) and K, V (128 keys) in shared memory:
+//   S^T  = K Q_i^T           dP^T = V dO_i^T        (M=128 keys, N=128 queries, K=64)
+//   P^T  = exp(S^T * scale - lse)  dS^T = P^T * (dP^T - D)   (warps 2-5, one key row each)
+//   dV  += P^T dO_i          dK  += dS^T Q_i         (M=128 keys, N=64, K=128 queries)
+//   dQ_i = dS K                                      (M=128 queries, N=64, K=128 keys)
+// The same Q/dO/K tiles serve as K-major operands of the first products and
+// as MN-major operands of the later ones, and the dS^T tile written for dK is
+// read MN-major for dQ; nothing is transposed. dQ_i leaves TMEM through a
+// staged TMA bulk reduce-add into the fp32 accumulator; dK (times the softmax
+// scale) and dV are written once at the end.
+// TMEM: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384), dQ two buffers [384,512).
+// ===========================================================================
+namespace bwd {
+constexpr int BKEY = 128, BQRY = 128;
+constexpr int T_BYTES = 128 * HD * 2;            // 16 KB: a 128-row tile of K, V, Q or dO
+constexpr int PT_BYTES = BKEY * BQRY * 2;        // 32 KB: P^T or dS^T
+constexpr int DQS_BYTES = BQRY * HD * 4;         // 32 KB: dQ staging (two 32-column boxes)
+constexpr int SMEM_BYTES = 2 * T_BYTES /*K,V*/ + 2 * 2 * T_BYTES /*Q,dO x2*/ + 2 * PT_BYTES + DQS_BYTES +
+                           2 * 2 * BQRY * 4 /*lse, D x2*/ + 1024 /*barriers*/ + 1024 /*align*/;
+constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 320, C_DQ = 384;  // dQ buffer b at C_DQ + 64 b
+}  // namespace bwd
+
+GPT2_DEV void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+constexpr int kThreadsBwd = 320;  // TMA, MMA, 8 softmax-backward warps
+
+__global__ void __launch_bounds__(kThreadsBwd, 1)
+    attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ lse,
+                       const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, float scale, int* err) {
+  using namespace bwd;
+  extern __shared__ __align__(1024) uint8_t smem_raw_ab[];
+  uint8_t* smem =
+      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_ab) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + T_BYTES;
+  uint8_t* sQ = sV + T_BYTES;               // [2]
+  uint8_t* sDO = sQ + 2 * T_BYTES;          // [2]
+  uint8_t* sPT = sDO + 2 * T_BYTES;
+  uint8_t* sDST = sPT + PT_BYTES;
+  uint8_t* sDQ = sDST + PT_BYTES;
+  float* sLse = reinterpret_cast<float*>(sDQ + DQS_BYTES);  // [2][128], in log2 units after load
+  float* sD = sLse + 2 * BQRY;                              // [2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sD + 2 * BQRY);
+  uint64_t* kv_full = bars;
+  uint64_t* qdo_full = bars + 1;    // [2]
+  uint64_t* qdo_empty = bars + 3;   // [2]
+  uint64_t* st_full = bars + 5;
+  uint64_t* st_empty = bars + 6;
+  uint64_t* ds_full = bars + 7;
+  uint64_t* ds_empty = bars + 8;
+  uint64_t* dq_full = bars + 9;     // [2]
+  uint64_t* dq_empty = bars + 11;   // [2]
+  uint64_t* dkdv_full = bars + 13;
+  uint64_t* done = bars + 14;
+  uint64_t* gbar = bars + 15;       // group barrier of the 8 softmax-backward warps
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = T / BKEY;
+  const int kb = blockIdx.x;               // key block; block 0 has the most query blocks
+  const int bh = blockIdx.y;
+  const int b = bh / H, h = bh % H;
+  const int C = H * HD;
+  const int row_base = b * T;
+  const int nit = nb - kb;                 // query blocks kb .. nb-1
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(kv_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&qdo_full[i]), 1);
+      mbar_init(smem_u32(&qdo_empty[i]), 1);
+    }
+    mbar_init(smem_u32(st_full), 1);
+    mbar_init(smem_u32(st_empty), 256);
+    mbar_init(smem_u32(ds_full), 256);
+    mbar_init(smem_u32(ds_empty), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&dq_full[i]), 1);
+      mbar_init(smem_u32(&dq_empty[i]), 256);
+    }
+    mbar_init(smem_u32(dkdv_full), 1);
+    mbar_init(smem_u32(done), 1);
+    mbar_init(smem_u32(gbar), 256);
+    fence_mbar_init();
+    tma_prefetch_desc(&tm_qkv);
+    tma_prefetch_desc(&tm_do);
+    tma_prefetch_desc(&tm_dq);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // -------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      mbar_arrive_expect_tx(smem_u32(kv_full), 2 * T_BYTES);
+      tma_load_2d(smem_u32(sK), &tm_qkv, smem_u32(kv_full), C + h * HD, row_base + kb * BKEY);
+      tma_load_2d(smem_u32(sV), &tm_qkv, smem_u32(kv_full), 2 * C + h * HD, row_base + kb * BKEY);
+      const float* lse_b = lse + (size_t)bh * T;
+      const float* D_b = Dv + (size_t)bh * T;
+      for (int it = 0; it < nit; ++it) {
+        const int s = it & 1, qi = kb + it;
+        if (!mbar_wait(smem_u32(&qdo_empty[s]), ((it >> 1) & 1) ^ 1, err)) break;
+        const uint32_t fb = smem_u32(&qdo_full[s]);
+        mbar_arrive_expect_tx(fb, 2 * T_BYTES + 2 * BQRY * 4);
+        tma_load_2d(smem_u32(sQ + s * T_BYTES), &tm_qkv, fb, h * HD, row_base + qi * BQRY);
+        tma_load_2d(smem_u32(sDO + s * T_BYTES), &tm_do, fb, h * HD, row_base + qi * BQRY);
+        bulk_load_1d(smem_u32(sLse + s * BQRY), lse_b + qi * BQRY, BQRY * 4, fb);
+        bulk_load_1d(smem_u32(sD + s * BQRY), D_b + qi * BQRY, BQRY * 4, fb);
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_st = idesc_bf16_f32(BKEY, BQRY, false, false);  // S^T, dP^T
+      constexpr uint32_t id_kv = idesc_bf16_f32(BKEY, HD, false, true);     // dV, dK
+      constexpr uint32_t id_q = idesc_bf16_f32(BQRY, HD, true, true);       // dQ
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      const uint32_t pt_addr = smem_u32(sPT), dst_addr = smem_u32(sDST);
+      bool ok = mbar_wait(smem_u32(kv_full), 0, err);
+      for (int it = 0; it < nit && ok; ++it) {
+        const int s = it & 1;
+        const uint32_t q_addr = smem_u32(sQ + s * T_BYTES), do_addr = smem_u32(sDO + s * T_BYTES);
+        if (!mbar_wait(smem_u32(&qdo_full[s]), (it >> 1) & 1, err)) { ok = false; break; }
+        if (it > 0 && !mbar_wait(smem_u32(st_empty), (it - 1) & 1, err)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          tc_mma_bf16(tmem + C_S, smem_desc_sw128(k_addr + kk * 32, 16, 1024),
+                      smem_desc_sw128(q_addr + kk * 32, 16, 1024), id_st, kk > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + C_DP, smem_desc_sw128(v_addr + kk * 32, 16, 1024),
+                      smem_desc_sw128(do_addr + kk * 32, 16, 1024), id_st, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(st_full));
+        // P^T and dS^T are in shared memory
+        if (!mbar_wait(smem_u32(ds_full), it & 1, err)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BQRY / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * (BKEY * 128) + (kk & 3) * 32;
+          tc_mma_bf16(tmem + C_DV, smem_desc_sw128(pt_addr + aoff, 16, 1024),
+                      smem_desc_sw128(do_addr + kk * 2048, 8192, 1024), id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_bf16(tmem + C_DK, smem_desc_sw128(dst_addr + aoff, 16, 1024),
+                      smem_desc_sw128(q_addr + kk * 2048, 8192, 1024), id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        // dQ_i = dS K into buffer it % 2 once the dQ of block it-2 has left it
+        const int qb2 = it & 1;
+        if (it > 1 && !mbar_wait(smem_u32(&dq_empty[qb2]), ((it - 2) >> 1) & 1, err)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BKEY / 16; ++kk)
+          tc_mma_bf16(tmem + C_DQ + 64 * qb2, smem_desc_sw128(dst_addr + kk * 2048, BKEY * 128, 1024),
+                      smem_desc_sw128(k_addr + kk * 2048, 8192, 1024), id_q, kk > 0 ? 1u : 0u);
+        tc_commit(smem_u32(&dq_full[qb2]));
+        tc_commit(smem_u32(ds_empty));
+        tc_commit(smem_u32(&qdo_empty[s]));
+      }
+      tc_commit(smem_u32(dkdv_full));
+      tc_commit(smem_u32(done));
+      mbar_wait(smem_u32(done), 0, err);
+    }
+  } else {
+    // -------------------------------------------------------------- softmax-backward warps
+    // warps 2..9: TMEM lane quarter q4 = warp & 3, query-column half hf
+    const int q4 = warp & 3, hf = (warp - 2) >> 2;
+    const int r = q4 * 32 + lane;                  // key row (and query row for dQ)
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const float sl2 = scale * kLog2e;
+    const int tid = threadIdx.x - 64;              // 0..255 within the group
+    // barrier among the 256 threads of this group with a bounded wait (an mbarrier,
+    // so that a thread that gave up on an earlier wait cannot hang the others)
+    uint32_t gphase = 0;
+    auto group_sync = [&]() -> bool {
+      mbar_arrive(smem_u32(gbar));
+      const bool r2 = mbar_wait(smem_u32(gbar), gphase, err);
+      gphase ^= 1;
+      return r2;
+    };
+    // dQ of query block `jt` (TMEM buffer jt % 2; query row r, columns 32 hf ..) ->
+    // staging box hf (128-byte swizzle) -> bulk reduce-add into the accumulator
+    auto drain_dq = [&](int jt) -> bool {
+      const int b2 = jt & 1;
+      if (!mbar_wait(smem_u32(&dq_full[b2]), (jt >> 1) & 1, err)) return false;
+      tc_fence_after();
+      if (tid == 0) bulk_wait_group_read<0>();   // the previous reduce has read the staging buffer
+      if (!group_sync()) return false;
+      float v[32];
+      tmem_ld32(tmem + lane_off + C_DQ + 64 * b2 + hf * 32, v);
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<float4*>(sDQ + hf * (BQRY * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) =
+            make_float4(v[4 * ch] * scale, v[4 * ch + 1] * scale, v[4 * ch + 2] * scale, v[4 * ch + 3] * scale);
+      tc_fence_before();
+      mbar_arrive(smem_u32(&dq_empty[b2]));
+      fence_async_smem();
+      if (!group_sync()) return false;
+      if (tid == 0) {
+        const int qrow0 = row_base + (kb + jt) * BQRY;
+        tma_reduce_add_2d(&tm_dq, smem_u32(sDQ), h * HD, qrow0);
+        tma_reduce_add_2d(&tm_dq, smem_u32(sDQ + BQRY * 128), h * HD + 32, qrow0);
+        bulk_commit_group();
+      }
+      return true;
+    };
+    bool ok = true;
+    for (int it = 0; it < nit && ok; ++it) {
+      const int s = it & 1, qi = kb + it;
+      const bool diag = (qi == kb);
+      if (!mbar_wait(smem_u32(st_full), it & 1, err)) { ok = false; break; }
+      tc_fence_after();
+      // this thread's 64 query columns of S^T and dP^T; tensor memory is free again at once
+      uint32_t sv[2][32], dv[2][32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        tmem_ld32_async(tmem + lane_off + C_S + hf * 64 + c * 32, sv[c]);
+        tmem_ld32_async(tmem + lane_off + C_DP + hf * 64 + c * 32, dv[c]);
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(smem_u32(st_empty));
+      // lse / D of this query block arrived with Q_i (the MMA waited on it before S^T)
+      const float* lq = sLse + s * BQRY + hf * 64;
+      const float* dq = sD + s * BQRY + hf * 64;
+      uint32_t pp[2][16], pd[2][16];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int q0 = c * 32 + 2 * i;           // within this half
+          float p0 = ex2_approx(fmaf(__uint_as_float(sv[c][2 * i]), sl2, -lq[q0] * kLog2e));
+          float p1 = ex2_approx(fmaf(__uint_as_float(sv[c][2 * i + 1]), sl2, -lq[q0 + 1] * kLog2e));
+          if (diag && r > hf * 64 + q0) p0 = 0.f;
+          if (diag && r > hf * 64 + q0 + 1) p1 = 0.f;
+          pp[c][i] = pack_bf16x2(p0, p1);
+          pd[c][i] = pack_bf16x2(p0 * (__uint_as_float(dv[c][2 * i]) - dq[q0]),
+                                 p1 * (__uint_as_float(dv[c][2 * i + 1]) - dq[q0 + 1]));
+        }
+      }
+      // P^T / dS^T were last read by the MMAs of the previous query block
+      if (it > 0 && !mbar_wait(smem_u32(ds_empty), (it - 1) & 1, err)) { ok = false; break; }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+#pragma unroll
+        for (int qq = 0; qq < 4; ++qq) {
+          const int ch = c * 4 + qq;
+          const int off = hf * (BKEY * 128) + r * 128 + ((ch ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(sPT + off) =
+              make_uint4(pp[c][4 * qq], pp[c][4 * qq + 1], pp[c][4 * qq + 2], pp[c][4 * qq + 3]);
+          *reinterpret_cast<uint4*>(sDST + off) =
+              make_uint4(pd[c][4 * qq], pd[c][4 * qq + 1], pd[c][4 * qq + 2], pd[c][4 * qq + 3]);
+        }
+      }
+      fence_async_smem();
+      mbar_arrive(smem_u32(ds_full));
+      // while the MMAs of this block run, move the dQ of the previous block out
+      if (it > 0 && !drain_dq(it - 1)) { ok = false; break; }
+    }
+    if (ok && nit > 0) ok = drain_dq(nit - 1);
+    if (tid == 0) bulk_wait_group<0>();
+    // dK (x scale), dV for key row r, columns 32 hf ..
+    if (ok && mbar_wait(smem_u32(dkdv_full), 0, err)) {
+      tc_fence_after();
+      bf16* krow = dqkv + ((size_t)(row_base + kb * BKEY + r)) * 3 * C + C + h * HD + hf * 32;
+      bf16* vrow = krow + C;
+      float v[32];
+      tmem_ld32(tmem + lane_off + C_DK + hf * 32, v);
+#pragma unroll
+      for (int i = 0; i < 32; i += 8)
+        *reinterpret_cast<uint4*>(krow + i) =
+            make_uint4(pack_bf16x2(v[i] * scale, v[i + 1] * scale), pack_bf16x2(v[i + 2] * scale, v[i + 3] * scale),
+                       pack_bf16x2(v[i + 4] * scale, v[i + 5] * scale), pack_bf16x2(v[i + 6] * scale, v[i + 7] * scale));
+      tmem_ld32(tmem + lane_off + C_DV + hf * 32, v);
+#pragma unroll
+      for (int i = 0; i < 32; i += 8)
+        *reinterpret_cast<uint4*>(vrow + i) =
+            make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]), pack_bf16x2(v[i + 4], v[i + 5]),
+                       pack_bf16x2(v[i + 6], v[i + 7]));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// dq_acc (fp32 [B*T, C]) must be zero on entry; attn::attn_dq_convert_kernel
+// moves it into dqkv and clears it again.
+static cudaError_t bwd_main(const bf16* qkv, const bf16* dout, const float* lse, const float* Dv, float* dq_acc,
+                            bf16* dqkv, int B, int T, int H, int* err, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e =
+        cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int C = H * HD;
+  CUtensorMap tm_qkv, tm_do, tm_dq;
+  if (!encode_map_2d(&tm_qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qkv, 3 * (uint64_t)C, (uint64_t)B * T,
+                     3 * (uint64_t)C, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_map_2d(&tm_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dout, (uint64_t)C, (uint64_t)B * T, (uint64_t)C, 64,
+                     128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_map_2d(&tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, (uint64_t)C, (uint64_t)B * T, (uint64_t)C,
+                     32, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  dim3 grid(T / bwd::BKEY, B * H);
+  attn_bwd_tc_kernel<<<grid, kThreadsBwd, bwd::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, lse, Dv, dqkv, T, H,
+                                                             1.0f / sqrtf((float)HD), err);
+  return cudaGetLastError();
+}
+
+}  // namespace attn_tc

@@ -24,6 +24,7 @@
 #include "../../include/gpt2step.h"
 #include "../../include/gpt2step_ops.h"
 #include "attention.cuh"
+#include "attention_tc.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
 #include "kernels.cuh"
@@ -328,20 +329,35 @@ int softmax_ce(bf16* logits, const int32_t* targets, float* losses, int N, int V
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
-int attention_fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, int hd, cudaStream_t s) {
+// Head size 64 with T a multiple of 128 runs on tcgen05 (S, O in tensor memory);
+// other supported shapes use the mma.sync kernel.
+int attention_fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, int hd, int* err, cudaStream_t s) {
   if (T % 64) return GPT2_ERR_ARG;
   cudaError_t e;
-  if (hd == 64) e = attn::fwd<64>(qkv, out, lse, B, T, H, s);
+  if (hd == 64 && T % attn_tc::BQ == 0 && err != nullptr) e = attn_tc::fwd(qkv, out, lse, B, T, H, err, s);
+  else if (hd == 64) e = attn::fwd<64>(qkv, out, lse, B, T, H, s);
   else if (hd == 32) e = attn::fwd<32>(qkv, out, lse, B, T, H, s);
   else return GPT2_ERR_ARG;
   return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
 int attention_bwd(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dv, float* dq_acc,
-                  bf16* dqkv, int B, int T, int H, int hd, cudaStream_t s) {
+                  bf16* dqkv, int B, int T, int H, int hd, int* err, cudaStream_t s) {
   if (T % 64) return GPT2_ERR_ARG;
   cudaError_t e;
-  if (hd == 64) e = attn::bwd<64>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
+  if (hd == 64 && T % attn_tc::bwd::BKEY == 0 && err != nullptr) {
+    const int rows = B * T * H;
+    attn::attn_bwd_dot_kernel<64><<<(rows + 255) / 256, 256, 0, s>>>(out, dout, Dv, B, T, H);
+    e = attn_tc::bwd_main(qkv, dout, lse, Dv, dq_acc, dqkv, B, T, H, err, s);
+    if (e == cudaSuccess) {
+      const int C = H * 64;
+      const size_t nvec = (size_t)B * T * C / 8;
+      int blocks = (int)((nvec + 255) / 256);
+      if (blocks > 148 * 8) blocks = 148 * 8;
+      attn::attn_dq_convert_kernel<<<blocks, 256, 0, s>>>(dq_acc, dqkv, B * T, C);
+      e = cudaGetLastError();
+    }
+  } else if (hd == 64) e = attn::bwd<64>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
   else if (hd == 32) e = attn::bwd<32>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
   else return GPT2_ERR_ARG;
   return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
@@ -447,7 +463,7 @@ int forward(gpt2_model* m, const int32_t* tok, const int32_t* tgt, int b, bool t
     }
     {
       const size_t p = prof_begin(m);
-      GPT2_TRY(launch::attention_fwd(qkv, atty, lse, b, T, d.H, d.hd, s));
+      GPT2_TRY(launch::attention_fwd(qkv, atty, lse, b, T, d.H, d.hd, err, s));
       prof_end(m, p, PC_ATTN_FWD, 2.0 * b * d.H * (double)T * (T + 64) * d.hd, 1);
     }
     {
@@ -592,7 +608,7 @@ int backward(gpt2_model* m, const int32_t* tok) {
     {
       const size_t p = prof_begin(m);
       GPT2_TRY(launch::attention_bwd(qkv, atty, datty, lse, m->at<float>(y.attD), m->at<float>(y.dq_acc), dqkv, d.B,
-                                     T, d.H, d.hd, s));
+                                     T, d.H, d.hd, err, s));
       prof_end(m, p, PC_ATTN_BWD, 5.0 * d.B * d.H * (double)T * (T + 64) * d.hd, 3);
     }
     // QKV projection
@@ -1053,9 +1069,10 @@ int gpt2op_layernorm_bwd_noalloc(const void* dy, const void* x, const float* mea
                         gpt2op_layernorm_bwd_noalloc_max_bytes(), static_cast<cudaStream_t>(stream));
 }
 
-int gpt2op_attention_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int hd, void* stream) {
-  if (!qkv || !out || !lse) return GPT2_ERR_ARG;
-  return launch::attention_fwd(static_cast<const bf16*>(qkv), static_cast<bf16*>(out), lse, B, T, H, hd,
+int gpt2op_attention_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int hd, int* dev_err,
+                         void* stream) {
+  if (!qkv || !out || !lse || !dev_err) return GPT2_ERR_ARG;
+  return launch::attention_fwd(static_cast<const bf16*>(qkv), static_cast<bf16*>(out), lse, B, T, H, hd, dev_err,
                                static_cast<cudaStream_t>(stream));
 }
 
@@ -1064,8 +1081,8 @@ size_t gpt2op_attention_bwd_workspace(int B, int T, int H, int hd) {
 }
 
 int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv, int B,
-                         int T, int H, int hd, void* workspace, size_t ws_bytes, void* stream) {
-  if (!qkv || !out || !dout || !lse || !dqkv || !workspace) return GPT2_ERR_ARG;
+                         int T, int H, int hd, void* workspace, size_t ws_bytes, int* dev_err, void* stream) {
+  if (!qkv || !out || !dout || !lse || !dqkv || !workspace || !dev_err) return GPT2_ERR_ARG;
   if (ws_bytes < gpt2op_attention_bwd_workspace(B, T, H, hd)) return GPT2_ERR_ARG;
   float* dq_acc = static_cast<float*>(workspace);
   float* Dv = dq_acc + (size_t)B * T * H * hd;
@@ -1073,7 +1090,7 @@ int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, con
   if (cudaMemsetAsync(dq_acc, 0, (size_t)B * T * H * hd * 4, s) != cudaSuccess) return GPT2_ERR_CUDA;
   return launch::attention_bwd(static_cast<const bf16*>(qkv), static_cast<const bf16*>(out),
                                static_cast<const bf16*>(dout), lse, Dv, dq_acc, static_cast<bf16*>(dqkv), B, T, H, hd,
-                               s);
+                               dev_err, s);
 }
 
 int gpt2op_softmax_ce(void* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,

@@ -10,6 +10,10 @@
       Times one tcgen05 GEMM arrangement through the op-level C ABI with CUDA
       events (bf16 inputs, fp32 accumulation) and prints TFLOP/s. M, N, K are the
       GEMM's own dimensions: output M x N, reduction K.
+
+  python -m gpt_step_b200.profile_step attn --dir fwd|bwd --shape B,T,H [--iters n]
+      Times the causal attention forward or backward (head size 64) through the
+      op-level C ABI and prints TFLOP/s (causal FLOPs incl. the diagonal block).
 """
 from __future__ import annotations
 
@@ -88,6 +92,44 @@ def run_gemm(args):
                       "err": int(err.sum())}))
 
 
+def run_attn(args):
+    import torch
+
+    import gpt_step_b200 as gs
+    from gpt_step_b200 import build
+    build.build()
+    B, T, H = (int(v) for v in args.shape.split(","))
+    hd = 64
+    C = H * hd
+    rng = np.random.default_rng(0)
+    qkv = torch.tensor(rng.standard_normal((B, T, 3 * C)).astype(np.float32)).to(torch.bfloat16).cuda()
+    out = torch.empty(B, T, C, dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(B, H, T, device="cuda")
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    gs.attention_fwd(qkv, out, lse, H, err)
+    if args.dir == "fwd":
+        fn = lambda: gs.attention_fwd(qkv, out, lse, H, err)
+        flops = 2.0 * B * H * T * (T + 128) * hd
+    else:
+        dout = torch.tensor(rng.standard_normal((B, T, C)).astype(np.float32)).to(torch.bfloat16).cuda()
+        dqkv = torch.empty_like(qkv)
+        ws = torch.empty(gs.attention_bwd_workspace(B, T, H, hd), dtype=torch.uint8, device="cuda")
+        fn = lambda: gs.attention_bwd(qkv, out, dout, lse, dqkv, H, ws, err)
+        flops = 5.0 * B * H * T * (T + 128) * hd
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.iters
+    print(json.dumps({"dir": args.dir, "B": B, "T": T, "H": H, "ms": ms,
+                      "tflops": flops / (ms / 1000.0) / 1e12, "err": int(err.sum())}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     sub = ap.add_subparsers(dest="mode", required=True)
@@ -99,8 +141,12 @@ def main():
     g.add_argument("--shape", default="19456,3072,768")
     g.add_argument("--iters", type=int, default=20)
     g.add_argument("--splits", type=int, default=0)
+    a = sub.add_parser("attn")
+    a.add_argument("--dir", choices=["fwd", "bwd"], default="fwd")
+    a.add_argument("--shape", default="19,1024,12")
+    a.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
-    run_step(args) if args.mode == "step" else run_gemm(args)
+    {"step": run_step, "gemm": run_gemm, "attn": run_attn}[args.mode](args)
 
 
 if __name__ == "__main__":

@@ -92,13 +92,18 @@ int gpt2op_layernorm_bwd_noalloc(const void* dy, const void* x, const float* mea
 /* Causal multi-head attention forward (grow_a_language_model_intro, activities
  * 5-6: softmax(Q K^T / sqrt(hd)) V with a causal mask). qkv bf16 [B,T,3C]
  * (q | k | v, heads contiguous), out bf16 [B,T,C], lse fp32 [B,H,T] (natural
- * log-sum-exp of the scaled scores). hd in {32, 64}, T % 64 == 0. */
-int gpt2op_attention_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int hd, void* stream);
+ * log-sum-exp of the scaled scores). hd in {32, 64}, T % 64 == 0. Head size 64
+ * with T % 128 == 0 runs on tcgen05 (scores and output accumulated in tensor
+ * memory); other shapes on mma.sync. */
+int gpt2op_attention_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int hd, int* dev_err,
+                         void* stream);
 
-/* Attention backward from the saved output and lse: dqkv bf16 [B,T,3C]. */
+/* Attention backward from the saved output and lse: dqkv bf16 [B,T,3C]. Head
+ * size 64 with T % 128 == 0 runs on tcgen05, other shapes on mma.sync. The
+ * workspace (fp32 dQ accumulator and row dot products) must be 16-byte aligned. */
 size_t gpt2op_attention_bwd_workspace(int B, int T, int H, int hd);
 int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv, int B,
-                         int T, int H, int hd, void* workspace, size_t ws_bytes, void* stream);
+                         int T, int H, int hd, void* workspace, size_t ws_bytes, int* dev_err, void* stream);
 
 /* Vocabulary-masked softmax cross-entropy, forward and backward fused (§4.1:
  * softmax over the V real ids only). logits bf16 [N,Vp] are overwritten in

@@ -122,14 +122,16 @@ def test_layernorm_fwd_bwd(C):
 
 # --- a4: causal attention ------------------------------------------------------------------
 
-@pytest.mark.parametrize("B,T,H,hd", [(2, 64, 2, 32), (2, 192, 3, 64), (1, 1024, 2, 64), (2, 256, 4, 32)])
+@pytest.mark.parametrize("B,T,H,hd", [(2, 64, 2, 32), (2, 192, 3, 64), (1, 1024, 2, 64), (2, 256, 4, 32),
+                                      (2, 256, 2, 64), (1, 512, 3, 64), (3, 128, 1, 64)])
 def test_attention_fwd_bwd(B, T, H, hd):
     C = H * hd
     qkv = rnd((B, T, 3 * C), 23)
     out = torch.empty(B, T, C, dtype=torch.bfloat16, device="cuda")
     lse = torch.empty(B, H, T, device="cuda")
     qd = bf16(qkv)
-    gs.attention_fwd(qd, out, lse, H)
+    err = err_word()
+    gs.attention_fwd(qd, out, lse, H, err)
     qr = rounded(qkv)
     q, k, v = (qr[..., i * C:(i + 1) * C].reshape(B, T, H, hd).transpose(0, 2, 1, 3) for i in range(3))
     o, l = G.attention_fwd(q, k, v)
@@ -138,12 +140,13 @@ def test_attention_fwd_bwd(B, T, H, hd):
     do = rnd((B, T, C), 24)
     dqkv = torch.empty_like(qd)
     ws = torch.empty(gs.attention_bwd_workspace(B, T, H, hd), dtype=torch.uint8, device="cuda")
-    gs.attention_bwd(qd, out, bf16(do), lse, dqkv, H, ws)
+    gs.attention_bwd(qd, out, bf16(do), lse, dqkv, H, ws, err)
     dor = rounded(do).reshape(B, T, H, hd).transpose(0, 2, 1, 3)
     dq, dk, dv = G.attention_bwd(dor, q, k, v)
     got = host(dqkv)
     for i, ref in enumerate((dq, dk, dv)):
         assert rel_l2(got[..., i * C:(i + 1) * C], ref.transpose(0, 2, 1, 3).reshape(B, T, C)) < 2e-2, "qkv"[i]
+    assert int(err.sum()) == 0
 
 
 # --- a11: vocabulary-masked softmax cross-entropy ------------------------------------------
