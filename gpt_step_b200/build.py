@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libgpt2step.so")
 SOURCES = ["gpt2step.cu"]
-DEPS = ["common.cuh", "gemm.cuh", "attention.cuh", "attention_tc.cuh", "kernels.cuh"]
+DEPS = ["common.cuh", "gemm.cuh", "gemm2sm.cuh", "attention.cuh", "attention_tc.cuh", "kernels.cuh"]
 HEADERS = [os.path.join(ROOT, "include", h) for h in ("gpt2step.h", "gpt2step_ops.h")]
 
 NVCC_FLAGS = [

@@ -29,7 +29,10 @@ constexpr int Q_BYTES = BQ * HD * 2;         // 16 KB
 constexpr int KV_BYTES = BKV * HD * 2;       // 16 KB each for K and V
 constexpr int P_BYTES = BQ * BKV * 2;        // 32 KB (two 64-key K blocks)
 constexpr int STAGES = 2;
-constexpr int SMEM_BYTES = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + 1024 /*barriers*/ + 1024 /*align*/;
+// No alignment slack: without static shared memory the dynamic block starts on a
+// 1 KB boundary (checked at run time), and 115,712 bytes is exactly what lets two
+// CTAs (plus the driver's 1 KB each) share an SM's 233,472 bytes.
+constexpr int SMEM_BYTES = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + 1024 /*barriers*/;
 constexpr int TMEM_COLS = 256;               // S [0,128), O [128,192); two CTAs share an SM
 constexpr uint32_t S_COL0 = 0, O_COL = 128;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -52,8 +55,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
                        int T, int H, float scale, int* err) {
   extern __shared__ __align__(1024) uint8_t smem_raw_af[];
-  uint8_t* smem =
-      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_af) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = smem_raw_af;
+  if (smem_u32(smem) & 1023u) {  // the swizzled tiles need a 1 KB-aligned base
+    if (threadIdx.x == 0) atomicOr(err, DEVERR_TIMEOUT);
+    return;
+  }
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + Q_BYTES;                  // [STAGES][KV_BYTES]
   uint8_t* sV = sK + STAGES * KV_BYTES;        // [STAGES][KV_BYTES]
@@ -224,17 +230,24 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i > r) sr[c][i] = __float_as_uint(-INFINITY);
       }
-      float mraw = -INFINITY;
+      // row maximum with eight independent partial maxima (short dependency chains)
+      float mpart[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) mpart[t] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mraw = fmaxf(mraw, __uint_as_float(sr[c][i]));
-      const float mx = mraw * sl2;  // scale > 0: max commutes with it
+        for (int i = 0; i < 32; ++i) mpart[i & 7] = fmaxf(mpart[i & 7], __uint_as_float(sr[c][i]));
+#pragma unroll
+      for (int t = 1; t < 8; ++t) mpart[0] = fmaxf(mpart[0], mpart[t]);
+      const float mx = mpart[0] * sl2;  // scale > 0: max commutes with it
       // lazy rescale: keep the stale maximum unless the new one exceeds it by > 2^8
       const bool grow = (mx > m + kRescaleThreshold) || (m == -INFINITY);
       const float m_new = grow ? mx : m;
       const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
-      float sum = 0.f;
+      float spart[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) spart[t] = 0.f;
       uint32_t pkall[4][16];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -242,9 +255,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int i = 0; i < 16; ++i) {
           const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i]), sl2, -m_new));
           const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, -m_new));
-          sum += p0 + p1;
+          spart[i & 7] += p0 + p1;
           pkall[c][i] = pack_bf16x2(p0, p1);
         }
+      float sum = 0.f;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) sum += spart[t];
       // the P buffer was last read by the PV product of block j-1
       if (j >= 1 && !mbar_wait(smem_u32(p_empty), (j - 1) & 1, err)) { ok = false; break; }
       uint8_t* pb = sP;

@@ -231,14 +231,22 @@ GPT2_DEV double warp_sum_d(double v) {
   return v;
 }
 
-// GPT-2's tanh-approximation GELU and its derivative (fp32).
+// Hardware tanh (MUFU.TANH, max relative error about 2^-11; the GELU results
+// are stored in bf16, whose rounding is 2^-9).
+GPT2_DEV float tanh_hw(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// GPT-2's tanh-approximation GELU and its derivative (fp32 arithmetic).
 GPT2_DEV float gelu_f(float u) {
   const float k = 0.7978845608028654f;  // sqrt(2/pi)
-  return 0.5f * u * (1.0f + tanhf(k * (u + 0.044715f * u * u * u)));
+  return 0.5f * u * (1.0f + tanh_hw(k * (u + 0.044715f * u * u * u)));
 }
 GPT2_DEV float gelu_grad_f(float u) {
   const float k = 0.7978845608028654f;
-  float t = tanhf(k * (u + 0.044715f * u * u * u));
+  const float t = tanh_hw(k * (u + 0.044715f * u * u * u));
   return 0.5f * (1.0f + t) + 0.5f * u * (1.0f - t * t) * k * (1.0f + 3.0f * 0.044715f * u * u);
 }
 

@@ -1,0 +1,426 @@
+// tcgen05 GEMM on CTA pairs (cta_group::2): 256 x BN output tiles.
+//
+// Same contraction and epilogues as gemm::gemm_tc_kernel, but each output tile
+// of 256 rows is computed by a cluster of two CTAs on two SMs: CTA r loads its
+// own 128 rows of A and its half (BN/2 rows) of B, and the even CTA issues
+// tcgen05.mma.cta_group::2 (M = 256, N = BN), which reads A and B from both
+// CTAs' shared memory and leaves rows 128r .. 128r+127 of the accumulator in
+// CTA r's tensor memory. Per SM this moves 32 KB of operands per 4 MMAs of
+// 128 x BN x 16 instead of 48 KB (B is not duplicated).
+//
+// Synchronisation across the pair:
+//   full[s]   on the even CTA only: its producer posts the expected bytes of both
+//             CTAs' loads, and both CTAs' TMA loads complete on it
+//   empty[s]  on both CTAs: the MMA's commit is multicast to the pair
+//   tfull[a]  on both CTAs (multicast commit); tempty[a] on the even CTA only:
+//             all 256 epilogue threads of the pair arrive (the odd CTA remotely)
+// No TMA multicast is used: every load reads global memory into its own CTA.
+#pragma once
+#include "gemm.cuh"
+
+namespace gemm2 {
+
+using gemm::BK;
+using gemm::kThreads;
+using gemm::Params;
+using gemm::UMMA_K;
+
+constexpr int BM_PAIR = 256;  // rows per cluster tile (128 per CTA)
+
+constexpr int kThreads2 = 320;  // TMA, MMA, 8 epilogue warps (two per TMEM lane quarter)
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = 5;
+  static constexpr int A_BYTES = 128 * BK * 2;          // own 128 rows
+  static constexpr int B_BYTES = (BN / 2) * BK * 2;     // own half of B
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int EPI_BYTES = 8 * 4 * 2048;       // per epilogue warp: 2 buffers x 2 outputs
+  static constexpr int BAR_BYTES = 1024;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
+  static constexpr int TMEM_COLS = 2 * BN;
+};
+
+GPT2_DEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// shared::cluster address of the same shared-memory offset in CTA `rank` of the cluster
+GPT2_DEV uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+GPT2_DEV void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+GPT2_DEV void tmem_alloc2(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+GPT2_DEV void tmem_relinquish2() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+GPT2_DEV void tmem_dealloc2(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+GPT2_DEV void tc_mma2_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on `bar` (same offset) in every CTA of `mask` when this thread's MMAs complete.
+GPT2_DEV void tc_commit2_mc(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+// TMA load into this CTA's shared memory completing bytes on an mbarrier that may
+// live in the peer CTA (shared::cluster address `bar`).
+GPT2_DEV void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+GPT2_DEV void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
+                    const Params p) {
+  using C = Cfg<BN>;
+  constexpr int S = C::STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_raw2[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
+  uint8_t* epi_smem = smem + S * C::STAGE_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(epi_smem + C::EPI_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + S;
+  uint64_t* tfull = bars + 2 * S;
+  uint64_t* tempty = bars + 2 * S + 2;
+  uint64_t* done = bars + 2 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * S + 5);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = (rank == 0);
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 2 * 8 * 32);
+    }
+    mbar_init(smem_u32(done), 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (EPI != gemm::EPI_ACC_F32) tma_prefetch_desc(&tmO);
+    if (EPI == gemm::EPI_GELU) tma_prefetch_desc(&tmO2);
+  }
+  if (warp == 1) {
+    tmem_alloc2(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish2();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers exist before anyone signals them
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = cid; t < p.num_tiles && ok; t += ncl) {
+        const int mb = t % p.num_m;
+        const int rest = t / p.num_m;
+        const int nb = rest % p.num_n;
+        const int sp = rest / p.num_n;
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.nkb, kb0 + p.kb_per_split);
+        const int m0 = mb * BM_PAIR + 128 * rank;
+        const int n0 = nb * BN + (BN / 2) * rank;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, p.err)) { ok = false; break; }
+          const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+          if (leader) mbar_arrive_expect_tx(smem_u32(&full[stage]), 2 * C::STAGE_BYTES);
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+          const int k0 = kb * BK;
+          if (A_MN) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j) tma_load_2d_pair(sa + j * 8192, &tmA, fb, m0 + 64 * j, k0);
+          } else {
+            tma_load_2d_pair(sa, &tmA, fb, k0, m0);
+          }
+          if (B_MN) {
+#pragma unroll
+            for (int j = 0; j < BN / 128; ++j) tma_load_2d_pair(sb + j * 8192, &tmB, fb, n0 + 64 * j, k0);
+          } else {
+            tma_load_2d_pair(sb, &tmB, fb, k0, n0);
+          }
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = idesc_bf16_f32(BM_PAIR, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = cid; t < p.num_tiles && ok; t += ncl, ++it) {
+        const int rest = t / p.num_m;
+        const int sp = rest / p.num_n;
+        const int kb0 = sp * p.kb_per_split;
+        const int kb1 = min(p.nkb, kb0 + p.kb_per_split);
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, p.err)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, p.err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sa + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+                                     : smem_desc_sw128(sb + kk * 32, 16, 1024);
+            tc_mma2_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit2_mc(smem_u32(&empty[stage]), 0x3);
+          if (++stage == S) { stage = 0; phase ^= 1; }
+        }
+        tc_commit2_mc(smem_u32(&tfull[acc]), 0x3);
+      }
+      tc_commit2_mc(smem_u32(done), 0x1);
+      mbar_wait(smem_u32(done), 0, p.err);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;              // TMEM lane quarter
+    const int hv = (warp - 2) >> 2;      // column half of the tile this warp drains
+    uint8_t* wbuf = epi_smem + (warp - 2) * 8192;
+    uint32_t nstore = 0;
+    int it = 0;
+    const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
+    const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    for (int t = cid; t < p.num_tiles; t += ncl, ++it) {
+      const int mb = t % p.num_m;
+      const int rest = t / p.num_m;
+      const int nb = rest % p.num_n;
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err)) break;
+      tc_fence_after();
+      const int row0 = mb * BM_PAIR + 128 * rank + q * 32;
+      const int row = row0 + lane;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int c = hv * (BN / 2); c < (hv + 1) * (BN / 2); c += 32) {
+        const int n = nb * BN + c;
+        float v[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c, v);
+        if (n >= p.N) continue;
+        if (EPI == gemm::EPI_ACC_F32) {
+          if (!row_ok) continue;
+          float* dst = p.outf + (size_t)row * p.ldf + n;
+          if (p.splits > 1) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) gemm::red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              float4 o = *reinterpret_cast<float4*>(dst + i);
+              o.x += v[i]; o.y += v[i + 1]; o.z += v[i + 2]; o.w += v[i + 3];
+              *reinterpret_cast<float4*>(dst + i) = o;
+            }
+          }
+          continue;
+        }
+        if (EPI == gemm::EPI_STORE || EPI == gemm::EPI_RESID || EPI == gemm::EPI_GELU) {
+          if (p.bias != nullptr) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              const float4 b = __ldg(reinterpret_cast<const float4*>(p.bias + n + i));
+              v[i] += b.x; v[i + 1] += b.y; v[i + 2] += b.z; v[i + 3] += b.w;
+            }
+          }
+        }
+        if ((EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU) && row_ok) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.aux + (size_t)row * p.ld_aux + n);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint4 u = src[j];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float2 f = unpack_bf16x2(w[h]);
+              const int i = j * 8 + h * 2;
+              if (EPI == gemm::EPI_RESID) {
+                v[i] += f.x; v[i + 1] += f.y;
+              } else {
+                v[i] *= gelu_grad_f(f.x); v[i + 1] *= gelu_grad_f(f.y);
+              }
+            }
+          }
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        const uint32_t b = nstore & 1;
+        if (lane == 0) gemm::bulk_wait_read<1>();
+        __syncwarp();
+        gemm::stage_row(wbuf + b * 2048, lane, pk);
+        if (EPI == gemm::EPI_GELU) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(gelu_f(v[2 * i]), gelu_f(v[2 * i + 1]));
+          gemm::stage_row(wbuf + 4096 + b * 2048, lane, pk);
+        }
+        gemm::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          gemm::tma_store_2d(&tmO, smem_u32(wbuf + b * 2048), n, row0);
+          if (EPI == gemm::EPI_GELU) gemm::tma_store_2d(&tmO2, smem_u32(wbuf + 4096 + b * 2048), n, row0);
+          gemm::bulk_commit();
+        }
+        ++nstore;
+      }
+      tc_fence_before();
+      mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+    }
+    if (EPI != gemm::EPI_ACC_F32 && lane == 0) gemm::bulk_wait_all<0>();
+  }
+
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while its pair may still read its shared memory
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc2(tmem_base, C::TMEM_COLS);
+  }
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+static cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                              const CUtensorMap& to2, Params p, cudaStream_t s) {
+  using C = Cfg<BN>;
+  auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EPI>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int pairs = gemm::num_sms() / 2;
+  const int grid = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
+  kern<<<grid, kThreads2, C::SMEM, s>>>(ta, tb, to, to2, p);
+  return cudaGetLastError();
+}
+
+}  // namespace gemm2
+
+namespace gemm2 {
+
+// Entry point for every GEMM of the step: CTA pairs for tiles of 256 x 256 when
+// the output has at least 256 rows and 256-wide tiles are chosen, otherwise the
+// single-CTA kernel (gemm::run).
+static int run(const gemm::Call& c, cudaStream_t s) {
+  using namespace gemm;
+  if (c.M <= 0 || c.N <= 0 || c.K <= 0) return GPT2_ERR_ARG;
+  if (c.N % 32 || c.K % BK) return GPT2_ERR_ARG;
+  const int BN = (c.kind == WGRAD && !c.force_bn && c.N % 256 == 0) ? 256 : choose_bn(c);
+  const bool pair = (BN == 256) && c.M >= BM_PAIR && c.force_bn != 128;
+  if (!pair) return gemm::run(c, s);
+  Params p{};
+  p.M = c.M; p.N = c.N; p.K = c.K;
+  p.num_m = (c.M + BM_PAIR - 1) / BM_PAIR;
+  p.num_n = (c.N + BN - 1) / BN;
+  p.nkb = c.K / BK;
+  int splits = 1;
+  if (c.kind == WGRAD) {
+    // waves of SM pairs: the split search sees pair tiles against 74 pairs
+    if (c.force_splits) {
+      splits = c.force_splits;
+    } else {
+      const long pairs = num_sms() / 2;
+      double best_eff = 0.0;
+      for (int sp = 1; sp <= 32 && p.nkb >= 8 * sp; ++sp) {
+        const long t = (long)p.num_m * p.num_n * sp;
+        const double eff = (double)t / (double)(pairs * ((t + pairs - 1) / pairs));
+        if (eff > best_eff + 0.03) { best_eff = eff; splits = sp; }
+      }
+    }
+  } else if (c.force_splits > 1) {
+    return GPT2_ERR_ARG;
+  }
+  p.kb_per_split = (p.nkb + splits - 1) / splits;
+  p.splits = (p.nkb + p.kb_per_split - 1) / p.kb_per_split;
+  p.num_tiles = p.num_m * p.num_n * p.splits;
+  p.out = c.out; p.out2 = c.out2; p.ldo = c.ldo;
+  p.aux = c.aux; p.ld_aux = c.ld_aux; p.bias = c.bias;
+  p.outf = c.outf; p.ldf = c.ldf; p.err = c.err;
+
+  CUtensorMap ta, tb, to, to2;
+  memset(&to, 0, sizeof(to));
+  memset(&to2, 0, sizeof(to2));
+  bool ok;
+  if (c.kind == WGRAD) {
+    if (c.M % 64 || c.N % 64) return GPT2_ERR_ARG;
+    ok = make_map(&ta, c.a, c.M, c.K, c.lda, 64, 64) && make_map(&tb, c.b, c.N, c.K, c.ldb, 64, 64);
+  } else if (c.kind == DGRAD) {
+    if (c.N % 64) return GPT2_ERR_ARG;
+    ok = make_map(&ta, c.a, c.K, c.M, c.lda, 64, 128) && make_map(&tb, c.b, c.N, c.K, c.ldb, 64, 64);
+  } else {
+    ok = make_map(&ta, c.a, c.K, c.M, c.lda, 64, 128) && make_map(&tb, c.b, c.K, c.N, c.ldb, 64, BN / 2);
+  }
+  if (!ok) return GPT2_ERR_ARG;
+  if (c.epi != EPI_ACC_F32) {
+    if (!make_map(&to, c.out, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return GPT2_ERR_ARG;
+    if (c.epi == EPI_GELU && !make_map(&to2, c.out2, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+      return GPT2_ERR_ARG;
+  }
+  cudaError_t e = cudaErrorInvalidValue;
+  if (c.kind == FWD) {
+    switch (c.epi) {
+      case EPI_STORE: e = launch_tc2<256, false, false, EPI_STORE>(ta, tb, to, to2, p, s); break;
+      case EPI_RESID: e = launch_tc2<256, false, false, EPI_RESID>(ta, tb, to, to2, p, s); break;
+      case EPI_GELU: e = launch_tc2<256, false, false, EPI_GELU>(ta, tb, to, to2, p, s); break;
+      default: return GPT2_ERR_ARG;
+    }
+  } else if (c.kind == DGRAD) {
+    switch (c.epi) {
+      case EPI_STORE: e = launch_tc2<256, false, true, EPI_STORE>(ta, tb, to, to2, p, s); break;
+      case EPI_DGELU: e = launch_tc2<256, false, true, EPI_DGELU>(ta, tb, to, to2, p, s); break;
+      default: return GPT2_ERR_ARG;
+    }
+  } else {
+    if (c.epi != EPI_ACC_F32) return GPT2_ERR_ARG;
+    e = launch_tc2<256, true, true, EPI_ACC_F32>(ta, tb, to, to2, p, s);
+  }
+  return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
+}
+
+}  // namespace gemm2

@@ -27,6 +27,7 @@
 #include "attention_tc.cuh"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm2sm.cuh"
 #include "kernels.cuh"
 
 namespace {
@@ -316,16 +317,9 @@ int bias_grad(const bf16* dout, float* db, int M, int N, float* part, size_t par
 
 int softmax_ce(bf16* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,
                int write_grad, int* err, cudaStream_t s) {
-  if (Vp % 8 || V > Vp || V <= 0 || Vp * 2 > 200 * 1024) return GPT2_ERR_ARG;
+  if (Vp % 8 || V > Vp || V <= 0) return GPT2_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(logits) & 15) != 0) return GPT2_ERR_ARG;
-  const int smem = Vp * 2;
-  static int attr_bytes = 0;
-  if (smem > 48 * 1024 && smem > attr_bytes) {
-    if (cudaFuncSetAttribute(k::softmax_ce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return GPT2_ERR_ARG;
-    attr_bytes = smem;
-  }
-  k::softmax_ce_kernel<<<N, k::kCeThreads, smem, s>>>(logits, targets, losses, V, Vp, dscale, write_grad, err);
+  k::softmax_ce_kernel<<<N, k::kCeThreads, 0, s>>>(logits, targets, losses, V, Vp, dscale, write_grad, err);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -413,7 +407,7 @@ void prof_end(gpt2_model* m, size_t i, int cls, double work, int nlaunch) {
 
 int run_gemm(gpt2_model* m, const gemm::Call& c) {
   const size_t p = prof_begin(m);
-  const int st = gemm::run(c, m->stream);
+  const int st = gemm2::run(c, m->stream);
   prof_end(m, p, PC_GEMM, 2.0 * c.M * c.N * c.K, 1);
   return st;
 }
@@ -962,7 +956,7 @@ int gpt2op_linear_fwd(const void* inp, const void* w, const float* bias, const v
   c.a = static_cast<const bf16*>(inp); c.lda = K; c.b = static_cast<const bf16*>(w); c.ldb = K;
   c.out = static_cast<bf16*>(out); c.ldo = N; c.bias = bias; c.aux = static_cast<const bf16*>(resid); c.ld_aux = N;
   if (resid && !bias) return GPT2_ERR_ARG;
-  return gemm::run(c, static_cast<cudaStream_t>(stream));
+  return gemm2::run(c, static_cast<cudaStream_t>(stream));
 }
 
 int gpt2op_linear_fwd_gelu(const void* inp, const void* w, const float* bias, void* pre_out, void* gelu_out, int M,
@@ -971,7 +965,7 @@ int gpt2op_linear_fwd_gelu(const void* inp, const void* w, const float* bias, vo
   gemm::Call c = gemm_call(gemm::FWD, gemm::EPI_GELU, M, N, K, dev_err);
   c.a = static_cast<const bf16*>(inp); c.lda = K; c.b = static_cast<const bf16*>(w); c.ldb = K;
   c.out = static_cast<bf16*>(pre_out); c.out2 = static_cast<bf16*>(gelu_out); c.ldo = N; c.bias = bias;
-  return gemm::run(c, static_cast<cudaStream_t>(stream));
+  return gemm2::run(c, static_cast<cudaStream_t>(stream));
 }
 
 int gpt2op_linear_dgrad(const void* dout, const void* w, const void* gelu_pre, void* din, int M, int N, int K,
@@ -981,7 +975,7 @@ int gpt2op_linear_dgrad(const void* dout, const void* w, const void* gelu_pre, v
   gemm::Call c = gemm_call(gemm::DGRAD, gelu_pre ? gemm::EPI_DGELU : gemm::EPI_STORE, M, K, N, dev_err);
   c.a = static_cast<const bf16*>(dout); c.lda = N; c.b = static_cast<const bf16*>(w); c.ldb = K;
   c.out = static_cast<bf16*>(din); c.ldo = K; c.aux = static_cast<const bf16*>(gelu_pre); c.ld_aux = K;
-  return gemm::run(c, static_cast<cudaStream_t>(stream));
+  return gemm2::run(c, static_cast<cudaStream_t>(stream));
 }
 
 int gpt2op_linear_wgrad(const void* dout, const void* inp, float* dw, int M, int N, int K, int splits, int* dev_err,
@@ -991,7 +985,7 @@ int gpt2op_linear_wgrad(const void* dout, const void* inp, float* dw, int M, int
   gemm::Call c = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, N, K, M, dev_err);
   c.a = static_cast<const bf16*>(dout); c.lda = N; c.b = static_cast<const bf16*>(inp); c.ldb = K;
   c.outf = dw; c.ldf = K; c.force_splits = splits;
-  return gemm::run(c, static_cast<cudaStream_t>(stream));
+  return gemm2::run(c, static_cast<cudaStream_t>(stream));
 }
 
 size_t gpt2op_bias_grad_workspace(int M, int N) { return launch::bias_grad_workspace(M, N); }

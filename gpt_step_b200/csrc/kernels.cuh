@@ -414,66 +414,69 @@ __global__ void colsum_final_kernel(const float* __restrict__ part, float* __res
 // j < V and exactly 0 for the padded columns j >= V ("Pretraining and adapting
 // a language model on a dependency-free stack", §4.1). loss = lse - z[target].
 // ---------------------------------------------------------------------------
-constexpr int kCeThreads = 512;
+constexpr int kCeThreads = 256;
+constexpr int kCeUnroll = 4;
 
+// Online (max, sum of exp) update with the real columns of one 8-wide vector.
+GPT2_DEV void ce_accumulate(uint4 u, int col0, int V, float& m, float& s) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  float f[8];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 t = unpack_bf16x2(w[j]);
+    f[2 * j] = t.x;
+    f[2 * j + 1] = t.y;
+  }
+  float lm = -INFINITY;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (col0 + j < V) lm = fmaxf(lm, f[j]);
+  if (lm == -INFINITY) return;
+  const float nm = fmaxf(m, lm);
+  float acc = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (col0 + j < V) acc += __expf(f[j] - nm);
+  s = s * __expf(m - nm) + acc;
+  m = nm;
+}
+
+GPT2_DEV void ce_combine(float& m, float& s, float om, float os) {
+  const float nm = fmaxf(m, om);
+  s = (nm == -INFINITY) ? 0.f : s * __expf(m - nm) + os * __expf(om - nm);
+  m = nm;
+}
+
+// One CTA per row, no shared-memory staging: pass 1 streams the bf16 row
+// (kCeUnroll 16-byte loads in flight per thread) for the running (max, sum of
+// exp) over the real columns; pass 2 reads the row again (from L2) and
+// overwrites it with dz.
 __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict__ logits,
                                                                 const int32_t* __restrict__ targets,
                                                                 float* __restrict__ losses, int V, int Vp,
                                                                 float dscale, int write_grad, int* err) {
-  extern __shared__ __align__(128) uint8_t smem_ce[];
-  uint4* row_s = reinterpret_cast<uint4*>(smem_ce);
   __shared__ float red_m[kCeThreads / 32], red_s[kCeThreads / 32];
   __shared__ float bc[2];
-  __shared__ __align__(8) uint64_t bar;
   const int row = blockIdx.x;
   uint4* zr = reinterpret_cast<uint4*>(logits + (size_t)row * Vp);
   const int nv = Vp / 8;
-  // the whole row arrives with one bulk copy (Vp * 2 bytes, a multiple of 16)
-  if (threadIdx.x == 0) {
-    mbar_init(smem_u32(&bar), 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(smem_u32(&bar), (uint32_t)Vp * 2u);
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(row_s)),
-                 "l"(zr), "r"((uint32_t)Vp * 2u), "r"(smem_u32(&bar))
-                 : "memory");
-  }
-  const bool loaded = mbar_wait(smem_u32(&bar), 0, err);
   float m = -INFINITY, s = 0.f;
-  for (int i = threadIdx.x; i < nv && loaded; i += kCeThreads) {
-    const uint4 u = row_s[i];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    float f[8];
+  for (int i0 = threadIdx.x; i0 < nv; i0 += kCeThreads * kCeUnroll) {
+    uint4 u[kCeUnroll];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 t = unpack_bf16x2(w[j]);
-      f[2 * j] = t.x;
-      f[2 * j + 1] = t.y;
+    for (int k2 = 0; k2 < kCeUnroll; ++k2) {
+      const int i = i0 + k2 * kCeThreads;
+      u[k2] = i < nv ? __ldcg(zr + i) : make_uint4(0u, 0u, 0u, 0u);
     }
-    float lm = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-      if (i * 8 + j < V) lm = fmaxf(lm, f[j]);
-    if (lm > -INFINITY) {
-      const float nm = fmaxf(m, lm);
-      s *= __expf(m - nm);
-#pragma unroll
-      for (int j = 0; j < 8; ++j)
-        if (i * 8 + j < V) s += __expf(f[j] - nm);
-      m = nm;
+    for (int k2 = 0; k2 < kCeUnroll; ++k2) {
+      const int i = i0 + k2 * kCeThreads;
+      if (i < nv) ce_accumulate(u[k2], i * 8, V, m, s);
     }
   }
-  // combine (m, s) across the CTA
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float om = __shfl_xor_sync(0xffffffffu, m, o), os = __shfl_xor_sync(0xffffffffu, s, o);
-    const float nm = fmaxf(m, om);
-    s = (nm == -INFINITY) ? 0.f : s * __expf(m - nm) + os * __expf(om - nm);
-    m = nm;
-  }
+  for (int o = 16; o > 0; o >>= 1)
+    ce_combine(m, s, __shfl_xor_sync(0xffffffffu, m, o), __shfl_xor_sync(0xffffffffu, s, o));
   const int warp = threadIdx.x >> 5, l = lane_id();
   if (l == 0) { red_m[warp] = m; red_s[warp] = s; }
   __syncthreads();
@@ -481,12 +484,8 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
     m = l < kCeThreads / 32 ? red_m[l] : -INFINITY;
     s = l < kCeThreads / 32 ? red_s[l] : 0.f;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float om = __shfl_xor_sync(0xffffffffu, m, o), os = __shfl_xor_sync(0xffffffffu, s, o);
-      const float nm = fmaxf(m, om);
-      s = (nm == -INFINITY) ? 0.f : s * __expf(m - nm) + os * __expf(om - nm);
-      m = nm;
-    }
+    for (int o = 16; o > 0; o >>= 1)
+      ce_combine(m, s, __shfl_xor_sync(0xffffffffu, m, o), __shfl_xor_sync(0xffffffffu, s, o));
     if (l == 0) { bc[0] = m; bc[1] = s; }
   }
   __syncthreads();
@@ -498,28 +497,35 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
     t = -1;
   }
   if (threadIdx.x == 0) {
-    float zt = 0.f;
-    if (tok_ok) {
-      const bf16* zs = reinterpret_cast<const bf16*>(row_s);
-      zt = __bfloat162float(zs[t]);
-    }
+    const float zt = tok_ok ? __bfloat162float(logits[(size_t)row * Vp + t]) : 0.f;
     losses[row] = tok_ok ? (M + logf(bc[1]) - zt) : 0.f;
   }
   if (!write_grad) return;
-  for (int i = threadIdx.x; i < nv; i += kCeThreads) {
-    const uint4 u = row_s[i];
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-    uint32_t o[4];
+  __syncthreads();  // the target logit is read before the row is overwritten
+  for (int i0 = threadIdx.x; i0 < nv; i0 += kCeThreads * kCeUnroll) {
+    uint4 u[kCeUnroll];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float2 f = unpack_bf16x2(w[j]);
-      const int c0 = i * 8 + 2 * j;
-      float g0 = 0.f, g1 = 0.f;
-      if (c0 < V) g0 = (__expf(f.x - M) * inv - (c0 == t ? 1.f : 0.f)) * dscale;
-      if (c0 + 1 < V) g1 = (__expf(f.y - M) * inv - (c0 + 1 == t ? 1.f : 0.f)) * dscale;
-      o[j] = pack_bf16x2(g0, g1);
+    for (int k2 = 0; k2 < kCeUnroll; ++k2) {
+      const int i = i0 + k2 * kCeThreads;
+      u[k2] = i < nv ? __ldcg(zr + i) : make_uint4(0u, 0u, 0u, 0u);
     }
-    zr[i] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+    for (int k2 = 0; k2 < kCeUnroll; ++k2) {
+      const int i = i0 + k2 * kCeThreads;
+      if (i >= nv) continue;
+      const uint32_t w[4] = {u[k2].x, u[k2].y, u[k2].z, u[k2].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = unpack_bf16x2(w[j]);
+        const int c0 = i * 8 + 2 * j;
+        float g0 = 0.f, g1 = 0.f;
+        if (c0 < V) g0 = (__expf(f.x - M) * inv - (c0 == t ? 1.f : 0.f)) * dscale;
+        if (c0 + 1 < V) g1 = (__expf(f.y - M) * inv - (c0 + 1 == t ? 1.f : 0.f)) * dscale;
+        o[j] = pack_bf16x2(g0, g1);
+      }
+      __stcs(zr + i, make_uint4(o[0], o[1], o[2], o[3]));
+    }
   }
 }
 

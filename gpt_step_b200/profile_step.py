@@ -14,6 +14,10 @@
   python -m gpt_step_b200.profile_step attn --dir fwd|bwd --shape B,T,H [--iters n]
       Times the causal attention forward or backward (head size 64) through the
       op-level C ABI and prints TFLOP/s (causal FLOPs incl. the diagonal block).
+
+  python -m gpt_step_b200.profile_step bw --kernel ln_fwd|ln_bwd|ce --shape rows,C [--iters n]
+      Times a bandwidth-bound kernel alone and prints GB/s of algorithmic bytes
+      (for ce, C is the padded vocabulary and the real one is C - 47).
 """
 from __future__ import annotations
 
@@ -130,6 +134,55 @@ def run_attn(args):
                       "tflops": flops / (ms / 1000.0) / 1e12, "err": int(err.sum())}))
 
 
+def run_bw(args):
+    """Bandwidth-bound kernels alone: LayerNorm fwd/bwd, softmax-CE (GB/s of algorithmic bytes)."""
+    import torch
+
+    import gpt_step_b200 as gs
+    from gpt_step_b200 import build
+    build.build()
+    rows, C = (int(v) for v in args.shape.split(","))
+    rng = np.random.default_rng(0)
+    bf = lambda *s: torch.tensor(rng.standard_normal(s).astype(np.float32)).to(torch.bfloat16).cuda()
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    if args.kernel in ("ln_fwd", "ln_bwd"):
+        x, w, b = bf(rows, C), torch.ones(C, device="cuda"), torch.zeros(C, device="cuda")
+        y = torch.empty_like(x)
+        mean, rstd = torch.empty(rows, device="cuda"), torch.empty(rows, device="cuda")
+        gs.layernorm_fwd(x, w, b, y, mean, rstd)
+        if args.kernel == "ln_fwd":
+            fn = lambda: gs.layernorm_fwd(x, w, b, y, mean, rstd)
+            nbytes = rows * (4.0 * C + 8)
+        else:
+            dy, dres = bf(rows, C), bf(rows, C)
+            dx = torch.empty_like(x)
+            dw, db = torch.zeros(C, device="cuda"), torch.zeros(C, device="cuda")
+            ws = torch.empty(gs.layernorm_bwd_workspace(rows, C), dtype=torch.uint8, device="cuda")
+            fn = lambda: gs.layernorm_bwd(dy, x, mean, rstd, w, dres, dx, dw, db, ws)
+            nbytes = rows * (8.0 * C + 8)
+    else:  # ce: rows x C logits (C = padded vocabulary), real vocabulary C - 47
+        z0 = bf(rows, C)
+        z = torch.empty_like(z0)
+        t = torch.tensor(rng.integers(0, C - 47, rows), dtype=torch.int32, device="cuda")
+        losses = torch.empty(rows, device="cuda")
+        def fn():
+            gs.softmax_ce(z, t, losses, C - 47, 1.0 / rows, err)
+        nbytes = rows * C * 4.0
+        z.copy_(z0)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.iters
+    print(json.dumps({"kernel": args.kernel, "rows": rows, "C": C, "us": ms * 1000,
+                      "gbs": nbytes / (ms / 1000.0) / 1e9}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     sub = ap.add_subparsers(dest="mode", required=True)
@@ -145,8 +198,12 @@ def main():
     a.add_argument("--dir", choices=["fwd", "bwd"], default="fwd")
     a.add_argument("--shape", default="19,1024,12")
     a.add_argument("--iters", type=int, default=20)
+    w = sub.add_parser("bw")
+    w.add_argument("--kernel", choices=["ln_fwd", "ln_bwd", "ce"], default="ln_fwd")
+    w.add_argument("--shape", default="19456,768")
+    w.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
-    {"step": run_step, "gemm": run_gemm, "attn": run_attn}[args.mode](args)
+    {"step": run_step, "gemm": run_gemm, "attn": run_attn, "bw": run_bw}[args.mode](args)
 
 
 if __name__ == "__main__":
