@@ -343,28 +343,47 @@ static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int
 
 
 // ===========================================================================
-// Backward (head size 64): per CTA one (batch, head) and a block of 128 keys;
-// loop over the query blocks at or after it (causal). With Q_i, dO_i (128
-// queries) and K, V (128 keys) in shared memory:
-//   S^T  = K Q_i^T           dP^T = V dO_i^T        (M=128 keys, N=128 queries, K=64)
-//   P^T  = exp(S^T * scale - lse)  dS^T = P^T * (dP^T - D)   (warps 2-5, one key row each)
-//   dV  += P^T dO_i          dK  += dS^T Q_i         (M=128 keys, N=64, K=128 queries)
-//   dQ_i = dS K                                      (M=128 queries, N=64, K=128 keys)
-// The same Q/dO/K tiles serve as K-major operands of the first products and
-// as MN-major operands of the later ones, and the dS^T tile written for dK is
-// read MN-major for dQ; nothing is transposed. dQ_i leaves TMEM through a
-// staged TMA bulk reduce-add into the fp32 accumulator; dK (times the softmax
-// scale) and dV are written once at the end.
-// TMEM: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384), dQ two buffers [384,512).
+// Backward (head size 64). Three kernels:
+//
+//   bwd_prep_kernel   per (batch, head, query): D = rowsum(dO o O) (the softmax
+//                     Jacobian term), stored as -D * scale, and -lse * log2(e);
+//                     clears the fp32 dQ accumulator.
+//   attn_bwd_tc_kernel  per CTA one (batch, head) and a block of 128 keys; walks
+//                     the query blocks at or after it (causal). With K, V resident
+//                     and Q_i, dO_i streamed through a three-deep ring:
+//       S^T  = K Q_i^T,  dP^T = V dO_i^T          (M=128 keys, N=128 queries, K=64)
+//       P^T  = exp2(S^T * scale*log2e - lse*log2e)  (warps 2-9, one key row each)
+//       dS^T = P^T * (dP^T - D) * scale
+//       dV  += P^T dO_i   (A = P^T from tensor memory)   (M=128 keys, N=64, K=128)
+//       dK  += dS^T Q_i   (A = dS^T from shared memory)
+//       dQ_i = dS K       (A = dS^T read MN-major)       (M=128 queries, N=64, K=128)
+//     S^T/dP^T of query block i+1 are issued before the dV/dK/dQ products of
+//     block i, so the tensor cores work on block i while the softmax warps turn
+//     block i+1's scores into P and dS. Each softmax warp moves its 32 x 32
+//     quarter of dQ_i out of tensor memory and adds it into the fp32
+//     accumulator with its own TMA bulk reduce (no block-wide barrier).
+//   bwd_post_kernel   dQ accumulator (fp32) -> the q third of dqkv (bf16).
+//
+// The softmax scale 1/8 is a power of two, so folding it into dS (bf16) is
+// exact: dK and dQ need no rescale.
+// TMEM: S^T [0,128), dP^T [128,256), dV [256,320), dK [320,384), dQ [384,448),
+//       P^T as bf16 pairs [448,512).
 // ===========================================================================
 namespace bwd {
 constexpr int BKEY = 128, BQRY = 128;
-constexpr int T_BYTES = 128 * HD * 2;            // 16 KB: a 128-row tile of K, V, Q or dO
-constexpr int PT_BYTES = BKEY * BQRY * 2;        // 32 KB: P^T or dS^T
-constexpr int DQS_BYTES = BQRY * HD * 4;         // 32 KB: dQ staging (two 32-column boxes)
-constexpr int SMEM_BYTES = 2 * T_BYTES /*K,V*/ + 2 * 2 * T_BYTES /*Q,dO x2*/ + 2 * PT_BYTES + DQS_BYTES +
-                           2 * 2 * BQRY * 4 /*lse, D x2*/ + 1024 /*barriers*/ + 1024 /*align*/;
-constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 320, C_DQ = 384;  // dQ buffer b at C_DQ + 64 b
+constexpr int NQS = 3;                              // Q / dO ring depth
+constexpr int T_BYTES = 128 * HD * 2;               // 16 KB: a 128-row tile of K, V, Q or dO
+constexpr int DST_BYTES = BKEY * BQRY * 2;          // 32 KB: dS^T
+constexpr int DQW_BYTES = 32 * 32 * 4;              // 4 KB: one warp's dQ staging box
+constexpr int kSoftmaxWarps = 8;
+constexpr int kThreads = 64 + 32 * kSoftmaxWarps;   // TMA, MMA, softmax-backward warps
+constexpr int SMEM_BYTES = 2 * T_BYTES /*K,V*/ + NQS * 2 * T_BYTES /*Q,dO*/ + DST_BYTES +
+                           kSoftmaxWarps * DQW_BYTES + NQS * 2 * BQRY * 4 /*lse, D*/ + 256 /*barriers*/ +
+                           1024 /*align*/;
+constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 320, C_DQ = 384, C_P = 448;
+constexpr int TMEM_COLS_BWD = 512;
+constexpr int kPrepRows = 32;                       // query rows per prep block
+constexpr int kMaxHeads = 64;
 }  // namespace bwd
 
 GPT2_DEV void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
@@ -373,44 +392,125 @@ GPT2_DEV void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32
                : "memory");
 }
 
-constexpr int kThreadsBwd = 320;  // TMA, MMA, 8 softmax-backward warps
+// D[tmem] (+)= A[tmem] * B[smem]^T (A: M rows in TMEM lanes, K along columns as bf16 pairs).
+GPT2_DEV void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 
-__global__ void __launch_bounds__(kThreadsBwd, 1)
+GPT2_DEV void tmem_st32_u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+GPT2_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// Block: 32 consecutive query rows of one sequence, all heads. Each warp takes
+// four rows; lanes hold 16-byte chunks of O and dO, eight chunks per head.
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
+                                                       const float* __restrict__ lse, float* __restrict__ nl2,
+                                                       float* __restrict__ dsc, float* __restrict__ dq_acc, int T,
+                                                       int H, float scale) {
+  using namespace bwd;
+  __shared__ float sDot[kMaxHeads][kPrepRows];
+  const int C = H * HD;
+  const int NV = C / 8;                      // 16-byte chunks per row
+  const int row0 = blockIdx.x * kPrepRows;   // global row (b*T + t) of the first query
+  const int b = row0 / T, t0 = row0 % T;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int rr = 0; rr < kPrepRows / 8; ++rr) {
+    const int rl = warp * (kPrepRows / 8) + rr;
+    const size_t base = (size_t)(row0 + rl) * C;
+    for (int v0 = 0; v0 < NV; v0 += 32) {
+      const int vi = v0 + lane;
+      float acc = 0.f;
+      if (vi < NV) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(out + base) + vi);
+        const uint4 c = __ldg(reinterpret_cast<const uint4*>(dout + base) + vi);
+        const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float2 fa = unpack_bf16x2(aw[k]), fc = unpack_bf16x2(cw[k]);
+          acc = fmaf(fa.x, fc.x, fmaf(fa.y, fc.y, acc));
+        }
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+      if ((lane & 7) == 0 && vi < NV) sDot[vi >> 3][rl] = acc;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < H * kPrepRows; i += blockDim.x) {
+    const int h = i / kPrepRows, rl = i % kPrepRows;
+    const size_t o = ((size_t)b * H + h) * T + t0 + rl;
+    nl2[o] = -lse[o] * kLog2e;
+    dsc[o] = -sDot[h][rl] * scale;
+  }
+  float4* z = reinterpret_cast<float4*>(dq_acc + (size_t)row0 * C);
+  const int n4 = kPrepRows * C / 4;
+  for (int i = threadIdx.x; i < n4; i += blockDim.x) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+// dq_acc fp32 [rows, C] -> dqkv[:, 0:C] bf16 (row stride 3C); eight columns per thread.
+__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ dq_acc, bf16* __restrict__ dqkv,
+                                                       int rows, int C) {
+  const int per_row = C / 8;
+  const int n = rows * per_row;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int row = i / per_row, c8 = i - row * per_row;
+    const float4* src = reinterpret_cast<const float4*>(dq_acc + (size_t)row * C + c8 * 8);
+    const float4 a = __ldcs(src), c = __ldcs(src + 1);
+    *reinterpret_cast<uint4*>(dqkv + (size_t)row * 3 * C + c8 * 8) =
+        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
+  }
+}
+
+__global__ void __launch_bounds__(bwd::kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ lse,
-                       const float* __restrict__ Dv, bf16* __restrict__ dqkv, int T, int H, float scale, int* err) {
+                       const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ nl2,
+                       const float* __restrict__ dsc, bf16* __restrict__ dqkv, int T, int H, float scale, int* err) {
   using namespace bwd;
   extern __shared__ __align__(1024) uint8_t smem_raw_ab[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_ab) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + T_BYTES;
-  uint8_t* sQ = sV + T_BYTES;               // [2]
-  uint8_t* sDO = sQ + 2 * T_BYTES;          // [2]
-  uint8_t* sPT = sDO + 2 * T_BYTES;
-  uint8_t* sDST = sPT + PT_BYTES;
-  uint8_t* sDQ = sDST + PT_BYTES;
-  float* sLse = reinterpret_cast<float*>(sDQ + DQS_BYTES);  // [2][128], in log2 units after load
-  float* sD = sLse + 2 * BQRY;                              // [2][128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sD + 2 * BQRY);
+  uint8_t* sQ = sV + T_BYTES;                     // [NQS]
+  uint8_t* sDO = sQ + NQS * T_BYTES;              // [NQS]
+  uint8_t* sDST = sDO + NQS * T_BYTES;
+  uint8_t* sDQW = sDST + DST_BYTES;               // [kSoftmaxWarps][DQW_BYTES]
+  float* sNL = reinterpret_cast<float*>(sDQW + kSoftmaxWarps * DQW_BYTES);  // [NQS][BQRY]
+  float* sDS = sNL + NQS * BQRY;                                            // [NQS][BQRY]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + NQS * BQRY);
   uint64_t* kv_full = bars;
-  uint64_t* qdo_full = bars + 1;    // [2]
-  uint64_t* qdo_empty = bars + 3;   // [2]
-  uint64_t* st_full = bars + 5;
-  uint64_t* st_empty = bars + 6;
-  uint64_t* ds_full = bars + 7;
-  uint64_t* ds_empty = bars + 8;
-  uint64_t* dq_full = bars + 9;     // [2]
-  uint64_t* dq_empty = bars + 11;   // [2]
-  uint64_t* dkdv_full = bars + 13;
-  uint64_t* done = bars + 14;
-  uint64_t* gbar = bars + 15;       // group barrier of the 8 softmax-backward warps
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+  uint64_t* qdo_full = bars + 1;          // [NQS]
+  uint64_t* qdo_empty = bars + 1 + NQS;   // [NQS]
+  uint64_t* st_full = bars + 1 + 2 * NQS;
+  uint64_t* st_empty = st_full + 1;
+  uint64_t* ds_full = st_full + 2;
+  uint64_t* ds_empty = st_full + 3;
+  uint64_t* dq_full = st_full + 4;
+  uint64_t* dq_empty = st_full + 5;
+  uint64_t* dkdv_full = st_full + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(st_full + 7);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nb = T / BKEY;
-  const int kb = blockIdx.x;               // key block; block 0 has the most query blocks
-  const int bh = blockIdx.y;
+  // heaviest key blocks (kb = 0: every query block) are scheduled first
+  const int BH = gridDim.y;
+  const int lin = blockIdx.y * gridDim.x + blockIdx.x;
+  const int kb = lin / BH;
+  const int bh = lin % BH;
   const int b = bh / H, h = bh % H;
   const int C = H * HD;
   const int row_base = b * T;
@@ -418,28 +518,24 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(kv_full), 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NQS; ++i) {
       mbar_init(smem_u32(&qdo_full[i]), 1);
       mbar_init(smem_u32(&qdo_empty[i]), 1);
     }
     mbar_init(smem_u32(st_full), 1);
-    mbar_init(smem_u32(st_empty), 256);
-    mbar_init(smem_u32(ds_full), 256);
+    mbar_init(smem_u32(st_empty), kSoftmaxWarps);
+    mbar_init(smem_u32(ds_full), kSoftmaxWarps);
     mbar_init(smem_u32(ds_empty), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&dq_full[i]), 1);
-      mbar_init(smem_u32(&dq_empty[i]), 256);
-    }
+    mbar_init(smem_u32(dq_full), 1);
+    mbar_init(smem_u32(dq_empty), kSoftmaxWarps);
     mbar_init(smem_u32(dkdv_full), 1);
-    mbar_init(smem_u32(done), 1);
-    mbar_init(smem_u32(gbar), 256);
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
     tma_prefetch_desc(&tm_do);
     tma_prefetch_desc(&tm_dq);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
+    tmem_alloc(smem_u32(tmem_slot), TMEM_COLS_BWD);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -453,34 +549,29 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       mbar_arrive_expect_tx(smem_u32(kv_full), 2 * T_BYTES);
       tma_load_2d(smem_u32(sK), &tm_qkv, smem_u32(kv_full), C + h * HD, row_base + kb * BKEY);
       tma_load_2d(smem_u32(sV), &tm_qkv, smem_u32(kv_full), 2 * C + h * HD, row_base + kb * BKEY);
-      const float* lse_b = lse + (size_t)bh * T;
-      const float* D_b = Dv + (size_t)bh * T;
+      const float* nl_b = nl2 + (size_t)bh * T;
+      const float* ds_b = dsc + (size_t)bh * T;
       for (int it = 0; it < nit; ++it) {
-        const int s = it & 1, qi = kb + it;
-        if (!mbar_wait(smem_u32(&qdo_empty[s]), ((it >> 1) & 1) ^ 1, err)) break;
+        const int s = it % NQS, u = it / NQS, qi = kb + it;
+        if (!mbar_wait(smem_u32(&qdo_empty[s]), (u & 1) ^ 1, err)) break;
         const uint32_t fb = smem_u32(&qdo_full[s]);
         mbar_arrive_expect_tx(fb, 2 * T_BYTES + 2 * BQRY * 4);
         tma_load_2d(smem_u32(sQ + s * T_BYTES), &tm_qkv, fb, h * HD, row_base + qi * BQRY);
         tma_load_2d(smem_u32(sDO + s * T_BYTES), &tm_do, fb, h * HD, row_base + qi * BQRY);
-        bulk_load_1d(smem_u32(sLse + s * BQRY), lse_b + qi * BQRY, BQRY * 4, fb);
-        bulk_load_1d(smem_u32(sD + s * BQRY), D_b + qi * BQRY, BQRY * 4, fb);
+        bulk_load_1d(smem_u32(sNL + s * BQRY), nl_b + qi * BQRY, BQRY * 4, fb);
+        bulk_load_1d(smem_u32(sDS + s * BQRY), ds_b + qi * BQRY, BQRY * 4, fb);
       }
     }
   } else if (warp == 1) {
     // -------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_st = idesc_bf16_f32(BKEY, BQRY, false, false);  // S^T, dP^T
-      constexpr uint32_t id_kv = idesc_bf16_f32(BKEY, HD, false, true);     // dV, dK
+      constexpr uint32_t id_kv = idesc_bf16_f32(BKEY, HD, false, true);     // dV (A in TMEM), dK
       constexpr uint32_t id_q = idesc_bf16_f32(BQRY, HD, true, true);       // dQ
-      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      const uint32_t pt_addr = smem_u32(sPT), dst_addr = smem_u32(sDST);
-      bool ok = mbar_wait(smem_u32(kv_full), 0, err);
-      for (int it = 0; it < nit && ok; ++it) {
-        const int s = it & 1;
+      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), dst_addr = smem_u32(sDST);
+      auto issue_st = [&](int it) {
+        const int s = it % NQS;
         const uint32_t q_addr = smem_u32(sQ + s * T_BYTES), do_addr = smem_u32(sDO + s * T_BYTES);
-        if (!mbar_wait(smem_u32(&qdo_full[s]), (it >> 1) & 1, err)) { ok = false; break; }
-        if (it > 0 && !mbar_wait(smem_u32(st_empty), (it - 1) & 1, err)) { ok = false; break; }
-        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           tc_mma_bf16(tmem + C_S, smem_desc_sw128(k_addr + kk * 32, 16, 1024),
@@ -489,80 +580,85 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
                       smem_desc_sw128(do_addr + kk * 32, 16, 1024), id_st, kk > 0 ? 1u : 0u);
         }
         tc_commit(smem_u32(st_full));
-        // P^T and dS^T are in shared memory
+      };
+      bool ok = mbar_wait(smem_u32(kv_full), 0, err) && mbar_wait(smem_u32(&qdo_full[0]), 0, err);
+      if (ok) {
+        tc_fence_after();
+        issue_st(0);
+      }
+      for (int it = 0; it < nit && ok; ++it) {
+        const int s = it % NQS;
+        const uint32_t q_addr = smem_u32(sQ + s * T_BYTES), do_addr = smem_u32(sDO + s * T_BYTES);
+        if (it + 1 < nit) {
+          // block it+1's scores, once its Q/dO landed and block it's scores left TMEM
+          if (!mbar_wait(smem_u32(&qdo_full[(it + 1) % NQS]), ((it + 1) / NQS) & 1, err)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(st_empty), it & 1, err)) { ok = false; break; }
+          tc_fence_after();
+          issue_st(it + 1);
+        }
+        // P^T (tensor memory) and dS^T (shared memory) of block it are written
         if (!mbar_wait(smem_u32(ds_full), it & 1, err)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BQRY / 16; ++kk) {
           const uint32_t aoff = (kk >> 2) * (BKEY * 128) + (kk & 3) * 32;
-          tc_mma_bf16(tmem + C_DV, smem_desc_sw128(pt_addr + aoff, 16, 1024),
-                      smem_desc_sw128(do_addr + kk * 2048, 8192, 1024), id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_bf16_ts(tmem + C_DV, tmem + C_P + kk * 8, smem_desc_sw128(do_addr + kk * 2048, 8192, 1024), id_kv,
+                         (it > 0 || kk > 0) ? 1u : 0u);
           tc_mma_bf16(tmem + C_DK, smem_desc_sw128(dst_addr + aoff, 16, 1024),
                       smem_desc_sw128(q_addr + kk * 2048, 8192, 1024), id_kv, (it > 0 || kk > 0) ? 1u : 0u);
         }
-        // dQ_i = dS K into buffer it % 2 once the dQ of block it-2 has left it
-        const int qb2 = it & 1;
-        if (it > 1 && !mbar_wait(smem_u32(&dq_empty[qb2]), ((it - 2) >> 1) & 1, err)) { ok = false; break; }
+        // dQ_it once dQ_{it-1} has left tensor memory
+        if (it > 0 && !mbar_wait(smem_u32(dq_empty), (it - 1) & 1, err)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BKEY / 16; ++kk)
-          tc_mma_bf16(tmem + C_DQ + 64 * qb2, smem_desc_sw128(dst_addr + kk * 2048, BKEY * 128, 1024),
+          tc_mma_bf16(tmem + C_DQ, smem_desc_sw128(dst_addr + kk * 2048, BKEY * 128, 1024),
                       smem_desc_sw128(k_addr + kk * 2048, 8192, 1024), id_q, kk > 0 ? 1u : 0u);
-        tc_commit(smem_u32(&dq_full[qb2]));
+        tc_commit(smem_u32(dq_full));
         tc_commit(smem_u32(ds_empty));
         tc_commit(smem_u32(&qdo_empty[s]));
       }
       tc_commit(smem_u32(dkdv_full));
-      tc_commit(smem_u32(done));
-      mbar_wait(smem_u32(done), 0, err);
+      // every product has completed before the block releases tensor memory
+      mbar_wait(smem_u32(dkdv_full), 0, err);
     }
   } else {
     // -------------------------------------------------------------- softmax-backward warps
-    // warps 2..9: TMEM lane quarter q4 = warp & 3, query-column half hf
-    const int q4 = warp & 3, hf = (warp - 2) >> 2;
+    // warps 2..9: TMEM lane quarter q4 = warp & 3 (key rows), query-column half hf
+    const int q4 = warp & 3, hf = (warp - 2) >> 2, wi = warp - 2;
     const int r = q4 * 32 + lane;                  // key row (and query row for dQ)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * kLog2e;
-    const int tid = threadIdx.x - 64;              // 0..255 within the group
-    // barrier among the 256 threads of this group with a bounded wait (an mbarrier,
-    // so that a thread that gave up on an earlier wait cannot hang the others)
-    uint32_t gphase = 0;
-    auto group_sync = [&]() -> bool {
-      mbar_arrive(smem_u32(gbar));
-      const bool r2 = mbar_wait(smem_u32(gbar), gphase, err);
-      gphase ^= 1;
-      return r2;
-    };
-    // dQ of query block `jt` (TMEM buffer jt % 2; query row r, columns 32 hf ..) ->
-    // staging box hf (128-byte swizzle) -> bulk reduce-add into the accumulator
+    uint8_t* stage = sDQW + wi * DQW_BYTES;
+    // dQ of query block jt: this warp's 32 query rows x 32 columns -> staging box ->
+    // bulk reduce-add into the accumulator
     auto drain_dq = [&](int jt) -> bool {
-      const int b2 = jt & 1;
-      if (!mbar_wait(smem_u32(&dq_full[b2]), (jt >> 1) & 1, err)) return false;
+      if (!mbar_wait(smem_u32(dq_full), jt & 1, err)) return false;
       tc_fence_after();
-      if (tid == 0) bulk_wait_group_read<0>();   // the previous reduce has read the staging buffer
-      if (!group_sync()) return false;
       float v[32];
-      tmem_ld32(tmem + lane_off + C_DQ + 64 * b2 + hf * 32, v);
+      tmem_ld32(tmem + lane_off + C_DQ + hf * 32, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(dq_empty));
+        bulk_wait_group_read<0>();   // this warp's previous reduce has read the box
+      }
+      __syncwarp();
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<float4*>(sDQ + hf * (BQRY * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) =
-            make_float4(v[4 * ch] * scale, v[4 * ch + 1] * scale, v[4 * ch + 2] * scale, v[4 * ch + 3] * scale);
-      tc_fence_before();
-      mbar_arrive(smem_u32(&dq_empty[b2]));
+        *reinterpret_cast<float4*>(stage + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
+            make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
       fence_async_smem();
-      if (!group_sync()) return false;
-      if (tid == 0) {
-        const int qrow0 = row_base + (kb + jt) * BQRY;
-        tma_reduce_add_2d(&tm_dq, smem_u32(sDQ), h * HD, qrow0);
-        tma_reduce_add_2d(&tm_dq, smem_u32(sDQ + BQRY * 128), h * HD + 32, qrow0);
+      __syncwarp();
+      if (lane == 0) {
+        tma_reduce_add_2d(&tm_dq, smem_u32(stage), h * HD + hf * 32, row_base + (kb + jt) * BQRY + q4 * 32);
         bulk_commit_group();
       }
       return true;
     };
     bool ok = true;
     for (int it = 0; it < nit && ok; ++it) {
-      const int s = it & 1, qi = kb + it;
-      const bool diag = (qi == kb);
+      const int s = it % NQS;
       if (!mbar_wait(smem_u32(st_full), it & 1, err)) { ok = false; break; }
       tc_fence_after();
       // this thread's 64 query columns of S^T and dP^T; tensor memory is free again at once
@@ -574,47 +670,55 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       }
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(smem_u32(st_empty));
-      // lse / D of this query block arrived with Q_i (the MMA waited on it before S^T)
-      const float* lq = sLse + s * BQRY + hf * 64;
-      const float* dq = sD + s * BQRY + hf * 64;
-      uint32_t pp[2][16], pd[2][16];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(st_empty));
+      // -lse*log2e and -D*scale of this query block came with Q_i
+      if (!mbar_wait(smem_u32(&qdo_full[s]), (it / NQS) & 1, err)) { ok = false; break; }
+      const float4* nq = reinterpret_cast<const float4*>(sNL + s * BQRY + hf * 64);
+      const float4* dq = reinterpret_cast<const float4*>(sDS + s * BQRY + hf * 64);
+      uint32_t pp[32], pd[32];
+      const bool diag = (it == 0);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int q0 = c * 32 + 2 * i;           // within this half
-          float p0 = ex2_approx(fmaf(__uint_as_float(sv[c][2 * i]), sl2, -lq[q0] * kLog2e));
-          float p1 = ex2_approx(fmaf(__uint_as_float(sv[c][2 * i + 1]), sl2, -lq[q0 + 1] * kLog2e));
-          if (diag && r > hf * 64 + q0) p0 = 0.f;
-          if (diag && r > hf * 64 + q0 + 1) p1 = 0.f;
-          pp[c][i] = pack_bf16x2(p0, p1);
-          pd[c][i] = pack_bf16x2(p0 * (__uint_as_float(dv[c][2 * i]) - dq[q0]),
-                                 p1 * (__uint_as_float(dv[c][2 * i + 1]) - dq[q0 + 1]));
+        for (int g = 0; g < 8; ++g) {
+          const float4 n4 = nq[c * 8 + g], d4 = dq[c * 8 + g];
+          const float nn[4] = {n4.x, n4.y, n4.z, n4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+          float p[4], ds[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = g * 4 + e;       // column within this 32-column chunk
+            p[e] = ex2_approx(fmaf(__uint_as_float(sv[c][j]), sl2, nn[e]));
+            if (diag && r > hf * 64 + c * 32 + j) p[e] = 0.f;   // key after query: masked
+            ds[e] = p[e] * fmaf(__uint_as_float(dv[c][j]), scale, dd[e]);
+          }
+          pp[c * 16 + g * 2] = pack_bf16x2(p[0], p[1]);
+          pp[c * 16 + g * 2 + 1] = pack_bf16x2(p[2], p[3]);
+          pd[c * 16 + g * 2] = pack_bf16x2(ds[0], ds[1]);
+          pd[c * 16 + g * 2 + 1] = pack_bf16x2(ds[2], ds[3]);
         }
       }
-      // P^T / dS^T were last read by the MMAs of the previous query block
+      // P^T (TMEM) and dS^T (smem) were last read by the products of block it-1
       if (it > 0 && !mbar_wait(smem_u32(ds_empty), (it - 1) & 1, err)) { ok = false; break; }
+      tc_fence_after();
+      tmem_st32_u(tmem + lane_off + C_P + hf * 32, pp);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-          const int ch = c * 4 + qq;
-          const int off = hf * (BKEY * 128) + r * 128 + ((ch ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(sPT + off) =
-              make_uint4(pp[c][4 * qq], pp[c][4 * qq + 1], pp[c][4 * qq + 2], pp[c][4 * qq + 3]);
-          *reinterpret_cast<uint4*>(sDST + off) =
-              make_uint4(pd[c][4 * qq], pd[c][4 * qq + 1], pd[c][4 * qq + 2], pd[c][4 * qq + 3]);
-        }
+      for (int ch = 0; ch < 8; ++ch) {
+        const int off = hf * (BKEY * 128) + r * 128 + ((ch ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(sDST + off) = make_uint4(pd[4 * ch], pd[4 * ch + 1], pd[4 * ch + 2], pd[4 * ch + 3]);
       }
+      tmem_wait_st();
       fence_async_smem();
-      mbar_arrive(smem_u32(ds_full));
-      // while the MMAs of this block run, move the dQ of the previous block out
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(ds_full));
+      // while the products of block it run, move dQ of block it-1 out
       if (it > 0 && !drain_dq(it - 1)) { ok = false; break; }
     }
     if (ok && nit > 0) ok = drain_dq(nit - 1);
-    if (tid == 0) bulk_wait_group<0>();
-    // dK (x scale), dV for key row r, columns 32 hf ..
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
+    // dK, dV for key row r, head-dim columns 32 hf ..
     if (ok && mbar_wait(smem_u32(dkdv_full), 0, err)) {
       tc_fence_after();
       bf16* krow = dqkv + ((size_t)(row_base + kb * BKEY + r)) * 3 * C + C + h * HD + hf * 32;
@@ -623,29 +727,27 @@ __global__ void __launch_bounds__(kThreadsBwd, 1)
       tmem_ld32(tmem + lane_off + C_DK + hf * 32, v);
 #pragma unroll
       for (int i = 0; i < 32; i += 8)
-        *reinterpret_cast<uint4*>(krow + i) =
-            make_uint4(pack_bf16x2(v[i] * scale, v[i + 1] * scale), pack_bf16x2(v[i + 2] * scale, v[i + 3] * scale),
-                       pack_bf16x2(v[i + 4] * scale, v[i + 5] * scale), pack_bf16x2(v[i + 6] * scale, v[i + 7] * scale));
+        *reinterpret_cast<uint4*>(krow + i) = make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
+                                                         pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
       tmem_ld32(tmem + lane_off + C_DV + hf * 32, v);
 #pragma unroll
       for (int i = 0; i < 32; i += 8)
-        *reinterpret_cast<uint4*>(vrow + i) =
-            make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]), pack_bf16x2(v[i + 4], v[i + 5]),
-                       pack_bf16x2(v[i + 6], v[i + 7]));
+        *reinterpret_cast<uint4*>(vrow + i) = make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
+                                                         pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, TMEM_COLS);
+    tmem_dealloc(tmem, TMEM_COLS_BWD);
   }
 }
 
-// dq_acc (fp32 [B*T, C]) must be zero on entry; attn::attn_dq_convert_kernel
-// moves it into dqkv and clears it again.
-static cudaError_t bwd_main(const bf16* qkv, const bf16* dout, const float* lse, const float* Dv, float* dq_acc,
-                            bf16* dqkv, int B, int T, int H, int* err, cudaStream_t s) {
+// The whole backward. nl2 / dsc fp32 [B, H, T] and dq_acc fp32 [B*T, C] are
+// scratch (contents on entry do not matter); dqkv receives dQ | dK | dV.
+static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* nl2, float* dsc,
+                       float* dq_acc, bf16* dqkv, int B, int T, int H, int* err, cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
     cudaError_t e =
@@ -653,18 +755,25 @@ static cudaError_t bwd_main(const bf16* qkv, const bf16* dout, const float* lse,
     if (e != cudaSuccess) return e;
     attr = true;
   }
+  if (H > bwd::kMaxHeads || T % bwd::kPrepRows) return cudaErrorInvalidValue;
   const int C = H * HD;
+  const float scale = 1.0f / sqrtf((float)HD);
   CUtensorMap tm_qkv, tm_do, tm_dq;
   if (!encode_map_2d(&tm_qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qkv, 3 * (uint64_t)C, (uint64_t)B * T,
                      3 * (uint64_t)C, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_map_2d(&tm_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dout, (uint64_t)C, (uint64_t)B * T, (uint64_t)C, 64,
                      128, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !encode_map_2d(&tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, (uint64_t)C, (uint64_t)B * T, (uint64_t)C,
-                     32, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+                     32, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  bwd_prep_kernel<<<B * T / bwd::kPrepRows, 256, 0, s>>>(out, dout, lse, nl2, dsc, dq_acc, T, H, scale);
   dim3 grid(T / bwd::BKEY, B * H);
-  attn_bwd_tc_kernel<<<grid, kThreadsBwd, bwd::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, lse, Dv, dqkv, T, H,
-                                                             1.0f / sqrtf((float)HD), err);
+  attn_bwd_tc_kernel<<<grid, bwd::kThreads, bwd::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, nl2, dsc, dqkv, T, H, scale,
+                                                                  err);
+  const int n = B * T * (C / 8);
+  int blocks = (n + 255) / 256;
+  if (blocks > 148 * 8) blocks = 148 * 8;
+  bwd_post_kernel<<<blocks, 256, 0, s>>>(dq_acc, dqkv, B * T, C);
   return cudaGetLastError();
 }
 
