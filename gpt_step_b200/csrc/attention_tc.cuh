@@ -376,7 +376,12 @@ constexpr int T_BYTES = 128 * HD * 2;               // 16 KB: a 128-row tile of 
 constexpr int DST_BYTES = BKEY * BQRY * 2;          // 32 KB: dS^T
 constexpr int DQW_BYTES = 32 * 32 * 4;              // 4 KB: one warp's dQ staging box
 constexpr int kSoftmaxWarps = 8;
-constexpr int kThreads = 64 + 32 * kSoftmaxWarps;   // TMA, MMA, softmax-backward warps
+// warpgroup 0: TMA (warp 0), MMA (warp 1), two idle warps; warpgroups 1-2: softmax.
+// Launched at 168 registers a thread (three warps per scheduler), warpgroup 0
+// gives registers to the softmax warpgroups: 128 x 40 + 256 x 232 = 384 x 168.
+constexpr int kThreads = 128 + 32 * kSoftmaxWarps;
+constexpr int kLaunchRegs = 168, kCtlRegs = 88, kSoftmaxRegs = 208;
+static_assert(128 * kCtlRegs + 32 * kSoftmaxWarps * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int SMEM_BYTES = 2 * T_BYTES /*K,V*/ + NQS * 2 * T_BYTES /*Q,dO*/ + DST_BYTES +
                            kSoftmaxWarps * DQW_BYTES + NQS * 2 * BQRY * 4 /*lse, D*/ + 256 /*barriers*/ +
                            1024 /*align*/;
@@ -413,6 +418,38 @@ GPT2_DEV void tmem_st32_u(uint32_t taddr, const uint32_t (&v)[32]) {
       : "memory");
 }
 GPT2_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+template <int N>
+GPT2_DEV void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+GPT2_DEV void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+
+// P^T and dS^T of one key row (this thread) for 64 query columns. DIAG: the
+// query block is the key block itself, so keys after the query are masked.
+template <bool DIAG>
+GPT2_DEV void bwd_softmax_row(const uint32_t (&sv)[2][32], const uint32_t (&dv)[2][32], const float4* nq,
+                              const float4* dq, float sl2, float scale, int r, int col0, uint32_t (&pp)[32],
+                              uint32_t (&pd)[32]) {
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      const float4 n4 = nq[c * 8 + g], d4 = dq[c * 8 + g];
+      const float nn[4] = {n4.x, n4.y, n4.z, n4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
+      float p[4], ds[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int j = g * 4 + e;   // column within this 32-column chunk
+        p[e] = ex2_approx(fmaf(__uint_as_float(sv[c][j]), sl2, nn[e]));
+        if (DIAG && r > col0 + c * 32 + j) p[e] = 0.f;   // key after query: masked
+        ds[e] = p[e] * fmaf(__uint_as_float(dv[c][j]), scale, dd[e]);
+      }
+      pp[c * 16 + g * 2] = pack_bf16x2(p[0], p[1]);
+      pp[c * 16 + g * 2 + 1] = pack_bf16x2(p[2], p[3]);
+      pd[c * 16 + g * 2] = pack_bf16x2(ds[0], ds[1]);
+      pd[c * 16 + g * 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+    }
+  }
+}
 
 // Block: 32 consecutive query rows of one sequence, all heads. Each warp takes
 // four rows; lanes hold 16-byte chunks of O and dO, eight chunks per head.
@@ -543,89 +580,99 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // -------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      mbar_arrive_expect_tx(smem_u32(kv_full), 2 * T_BYTES);
-      tma_load_2d(smem_u32(sK), &tm_qkv, smem_u32(kv_full), C + h * HD, row_base + kb * BKEY);
-      tma_load_2d(smem_u32(sV), &tm_qkv, smem_u32(kv_full), 2 * C + h * HD, row_base + kb * BKEY);
-      const float* nl_b = nl2 + (size_t)bh * T;
-      const float* ds_b = dsc + (size_t)bh * T;
-      for (int it = 0; it < nit; ++it) {
-        const int s = it % NQS, u = it / NQS, qi = kb + it;
-        if (!mbar_wait(smem_u32(&qdo_empty[s]), (u & 1) ^ 1, err)) break;
-        const uint32_t fb = smem_u32(&qdo_full[s]);
-        mbar_arrive_expect_tx(fb, 2 * T_BYTES + 2 * BQRY * 4);
-        tma_load_2d(smem_u32(sQ + s * T_BYTES), &tm_qkv, fb, h * HD, row_base + qi * BQRY);
-        tma_load_2d(smem_u32(sDO + s * T_BYTES), &tm_do, fb, h * HD, row_base + qi * BQRY);
-        bulk_load_1d(smem_u32(sNL + s * BQRY), nl_b + qi * BQRY, BQRY * 4, fb);
-        bulk_load_1d(smem_u32(sDS + s * BQRY), ds_b + qi * BQRY, BQRY * 4, fb);
-      }
-    }
-  } else if (warp == 1) {
-    // -------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_st = idesc_bf16_f32(BKEY, BQRY, false, false);  // S^T, dP^T
-      constexpr uint32_t id_kv = idesc_bf16_f32(BKEY, HD, false, true);     // dV (A in TMEM), dK
-      constexpr uint32_t id_q = idesc_bf16_f32(BQRY, HD, true, true);       // dQ
-      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV), dst_addr = smem_u32(sDST);
-      auto issue_st = [&](int it) {
-        const int s = it % NQS;
-        const uint32_t q_addr = smem_u32(sQ + s * T_BYTES), do_addr = smem_u32(sDO + s * T_BYTES);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          tc_mma_bf16(tmem + C_S, smem_desc_sw128(k_addr + kk * 32, 16, 1024),
-                      smem_desc_sw128(q_addr + kk * 32, 16, 1024), id_st, kk > 0 ? 1u : 0u);
-          tc_mma_bf16(tmem + C_DP, smem_desc_sw128(v_addr + kk * 32, 16, 1024),
-                      smem_desc_sw128(do_addr + kk * 32, 16, 1024), id_st, kk > 0 ? 1u : 0u);
+  if (warp < 4) {
+    regs_dec<kCtlRegs>();
+    if (warp == 0) {
+      // -------------------------------------------------------------- TMA producer
+      if (lane == 0) {
+        mbar_arrive_expect_tx(smem_u32(kv_full), 2 * T_BYTES);
+        tma_load_2d(smem_u32(sK), &tm_qkv, smem_u32(kv_full), C + h * HD, row_base + kb * BKEY);
+        tma_load_2d(smem_u32(sV), &tm_qkv, smem_u32(kv_full), 2 * C + h * HD, row_base + kb * BKEY);
+        const float* nl_b = nl2 + (size_t)bh * T;
+        const float* ds_b = dsc + (size_t)bh * T;
+        for (int it = 0; it < nit; ++it) {
+          const int s = it % NQS, u = it / NQS, qi = kb + it;
+          if (!mbar_wait(smem_u32(&qdo_empty[s]), (u & 1) ^ 1, err)) break;
+          const uint32_t fb = smem_u32(&qdo_full[s]);
+          mbar_arrive_expect_tx(fb, 2 * T_BYTES + 2 * BQRY * 4);
+          tma_load_2d(smem_u32(sQ + s * T_BYTES), &tm_qkv, fb, h * HD, row_base + qi * BQRY);
+          tma_load_2d(smem_u32(sDO + s * T_BYTES), &tm_do, fb, h * HD, row_base + qi * BQRY);
+          bulk_load_1d(smem_u32(sNL + s * BQRY), nl_b + qi * BQRY, BQRY * 4, fb);
+          bulk_load_1d(smem_u32(sDS + s * BQRY), ds_b + qi * BQRY, BQRY * 4, fb);
         }
-        tc_commit(smem_u32(st_full));
-      };
-      bool ok = mbar_wait(smem_u32(kv_full), 0, err) && mbar_wait(smem_u32(&qdo_full[0]), 0, err);
-      if (ok) {
-        tc_fence_after();
-        issue_st(0);
       }
-      for (int it = 0; it < nit && ok; ++it) {
-        const int s = it % NQS;
-        const uint32_t q_addr = smem_u32(sQ + s * T_BYTES), do_addr = smem_u32(sDO + s * T_BYTES);
-        if (it + 1 < nit) {
-          // block it+1's scores, once its Q/dO landed and block it's scores left TMEM
-          if (!mbar_wait(smem_u32(&qdo_full[(it + 1) % NQS]), ((it + 1) / NQS) & 1, err)) { ok = false; break; }
-          if (!mbar_wait(smem_u32(st_empty), it & 1, err)) { ok = false; break; }
+    } else if (warp == 1) {
+      // -------------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t id_st = idesc_bf16_f32(BKEY, BQRY, false, false);  // S^T, dP^T
+        constexpr uint32_t id_kv = idesc_bf16_f32(BKEY, HD, false, true);     // dV (A in TMEM), dK
+        constexpr uint32_t id_q = idesc_bf16_f32(BQRY, HD, true, true);       // dQ
+        // Descriptors are formed once; a shared-memory offset is added in 16-byte
+        // units to the start-address field (addresses stay below 2^18, no carry).
+        const uint64_t dK_k = smem_desc_sw128(smem_u32(sK), 16, 1024);        // K, K-major
+        const uint64_t dV_k = smem_desc_sw128(smem_u32(sV), 16, 1024);        // V, K-major
+        const uint64_t dK_mn = smem_desc_sw128(smem_u32(sK), 8192, 1024);     // K, MN-major
+        const uint64_t dDS_k = smem_desc_sw128(smem_u32(sDST), 16, 1024);     // dS^T, K-major
+        const uint64_t dDS_mn = smem_desc_sw128(smem_u32(sDST), BKEY * 128, 1024);  // dS, MN-major
+        const uint64_t dQ0_k = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+        const uint64_t dQ0_mn = smem_desc_sw128(smem_u32(sQ), 8192, 1024);
+        const uint64_t dO0_k = smem_desc_sw128(smem_u32(sDO), 16, 1024);
+        const uint64_t dO0_mn = smem_desc_sw128(smem_u32(sDO), 8192, 1024);
+        constexpr uint64_t kStage = T_BYTES >> 4;   // one Q/dO stage, in descriptor units
+        auto issue_st = [&](int it) {
+          const uint64_t so = (uint64_t)(it % NQS) * kStage;
+  #pragma unroll
+          for (int kk = 0; kk < HD / 16; ++kk) {
+            tc_mma_bf16(tmem + C_S, dK_k + kk * 2, dQ0_k + so + kk * 2, id_st, kk > 0 ? 1u : 0u);
+            tc_mma_bf16(tmem + C_DP, dV_k + kk * 2, dO0_k + so + kk * 2, id_st, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(smem_u32(st_full));
+        };
+        bool ok = mbar_wait(smem_u32(kv_full), 0, err) && mbar_wait(smem_u32(&qdo_full[0]), 0, err);
+        if (ok) {
           tc_fence_after();
-          issue_st(it + 1);
+          issue_st(0);
         }
-        // P^T (tensor memory) and dS^T (shared memory) of block it are written
-        if (!mbar_wait(smem_u32(ds_full), it & 1, err)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BQRY / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * (BKEY * 128) + (kk & 3) * 32;
-          tc_mma_bf16_ts(tmem + C_DV, tmem + C_P + kk * 8, smem_desc_sw128(do_addr + kk * 2048, 8192, 1024), id_kv,
-                         (it > 0 || kk > 0) ? 1u : 0u);
-          tc_mma_bf16(tmem + C_DK, smem_desc_sw128(dst_addr + aoff, 16, 1024),
-                      smem_desc_sw128(q_addr + kk * 2048, 8192, 1024), id_kv, (it > 0 || kk > 0) ? 1u : 0u);
+        for (int it = 0; it < nit && ok; ++it) {
+          const int s = it % NQS;
+          const uint64_t so = (uint64_t)s * kStage;
+          if (it + 1 < nit) {
+            // block it+1's scores, once its Q/dO landed and block it's scores left TMEM
+            if (!mbar_wait(smem_u32(&qdo_full[(it + 1) % NQS]), ((it + 1) / NQS) & 1, err)) { ok = false; break; }
+            if (!mbar_wait(smem_u32(st_empty), it & 1, err)) { ok = false; break; }
+            tc_fence_after();
+            issue_st(it + 1);
+          }
+          // P^T (tensor memory) and dS^T (shared memory) of block it are written
+          if (!mbar_wait(smem_u32(ds_full), it & 1, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t acc0 = it > 0 ? 1u : 0u;
+  #pragma unroll
+          for (int kk = 0; kk < BQRY / 16; ++kk) {
+            const uint32_t aoff = ((kk >> 2) * (BKEY * 128) + (kk & 3) * 32) >> 4;
+            tc_mma_bf16_ts(tmem + C_DV, tmem + C_P + kk * 8, dO0_mn + so + kk * 128, id_kv, kk > 0 ? 1u : acc0);
+            tc_mma_bf16(tmem + C_DK, dDS_k + aoff, dQ0_mn + so + kk * 128, id_kv, kk > 0 ? 1u : acc0);
+          }
+          // dQ_it once dQ_{it-1} has left tensor memory
+          if (it > 0 && !mbar_wait(smem_u32(dq_empty), (it - 1) & 1, err)) { ok = false; break; }
+          tc_fence_after();
+  #pragma unroll
+          for (int kk = 0; kk < BKEY / 16; ++kk)
+            tc_mma_bf16(tmem + C_DQ, dDS_mn + kk * 128, dK_mn + kk * 128, id_q, kk > 0 ? 1u : 0u);
+          tc_commit(smem_u32(dq_full));
+          tc_commit(smem_u32(ds_empty));
+          tc_commit(smem_u32(&qdo_empty[s]));
         }
-        // dQ_it once dQ_{it-1} has left tensor memory
-        if (it > 0 && !mbar_wait(smem_u32(dq_empty), (it - 1) & 1, err)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BKEY / 16; ++kk)
-          tc_mma_bf16(tmem + C_DQ, smem_desc_sw128(dst_addr + kk * 2048, BKEY * 128, 1024),
-                      smem_desc_sw128(k_addr + kk * 2048, 8192, 1024), id_q, kk > 0 ? 1u : 0u);
-        tc_commit(smem_u32(dq_full));
-        tc_commit(smem_u32(ds_empty));
-        tc_commit(smem_u32(&qdo_empty[s]));
+        tc_commit(smem_u32(dkdv_full));
+        // every product has completed before the block releases tensor memory
+        mbar_wait(smem_u32(dkdv_full), 0, err);
       }
-      tc_commit(smem_u32(dkdv_full));
-      // every product has completed before the block releases tensor memory
-      mbar_wait(smem_u32(dkdv_full), 0, err);
     }
   } else {
+    regs_inc<kSoftmaxRegs>();
     // -------------------------------------------------------------- softmax-backward warps
-    // warps 2..9: TMEM lane quarter q4 = warp & 3 (key rows), query-column half hf
-    const int q4 = warp & 3, hf = (warp - 2) >> 2, wi = warp - 2;
+    // warps 4..11: TMEM lane quarter q4 = warp & 3 (key rows), query-column half hf
+    const int q4 = warp & 3, hf = (warp - 4) >> 2, wi = warp - 4;
     const int r = q4 * 32 + lane;                  // key row (and query row for dQ)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * kLog2e;
@@ -677,27 +724,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       const float4* nq = reinterpret_cast<const float4*>(sNL + s * BQRY + hf * 64);
       const float4* dq = reinterpret_cast<const float4*>(sDS + s * BQRY + hf * 64);
       uint32_t pp[32], pd[32];
-      const bool diag = (it == 0);
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const float4 n4 = nq[c * 8 + g], d4 = dq[c * 8 + g];
-          const float nn[4] = {n4.x, n4.y, n4.z, n4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
-          float p[4], ds[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = g * 4 + e;       // column within this 32-column chunk
-            p[e] = ex2_approx(fmaf(__uint_as_float(sv[c][j]), sl2, nn[e]));
-            if (diag && r > hf * 64 + c * 32 + j) p[e] = 0.f;   // key after query: masked
-            ds[e] = p[e] * fmaf(__uint_as_float(dv[c][j]), scale, dd[e]);
-          }
-          pp[c * 16 + g * 2] = pack_bf16x2(p[0], p[1]);
-          pp[c * 16 + g * 2 + 1] = pack_bf16x2(p[2], p[3]);
-          pd[c * 16 + g * 2] = pack_bf16x2(ds[0], ds[1]);
-          pd[c * 16 + g * 2 + 1] = pack_bf16x2(ds[2], ds[3]);
-        }
-      }
+      if (it == 0) bwd_softmax_row<true>(sv, dv, nq, dq, sl2, scale, r, hf * 64, pp, pd);
+      else bwd_softmax_row<false>(sv, dv, nq, dq, sl2, scale, r, hf * 64, pp, pd);
       // P^T (TMEM) and dS^T (smem) were last read by the products of block it-1
       if (it > 0 && !mbar_wait(smem_u32(ds_empty), (it - 1) & 1, err)) { ok = false; break; }
       tc_fence_after();
@@ -750,8 +778,13 @@ static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, c
                        float* dq_acc, bf16* dqkv, int B, int T, int H, int* err, cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
-    cudaError_t e =
-        cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::SMEM_BYTES);
+    // The register hand-over inside the kernel needs the block to be launched
+    // with kLaunchRegs registers a thread; anything less would stall it.
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_bwd_tc_kernel);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != bwd::kLaunchRegs) return cudaErrorInvalidConfiguration;
+    e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr = true;
   }
