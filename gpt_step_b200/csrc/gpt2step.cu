@@ -244,9 +244,10 @@ int ln_fwd(const bf16* x, const float* w, const float* b, bf16* y, float* mean, 
 }
 
 int ln_bwd_blocks(int rows, int C) {
-  const int warps = C <= 768 ? 8 : 4;
-  return std::min(kLnBwdBlocks, (rows + warps - 1) / warps);
+  const int warps = k::ln_bwd_warps(C);
+  return std::min(148 * k::ln_bwd_minb(C), (rows + warps - 1) / warps);
 }
+static_assert(148 * 2 <= kLnBwdBlocks, "LayerNorm partial rows");
 
 // Workspace of the LayerNorm backward: one partial row of nq * C floats per CTA
 // (nq = 2: dw, db; nq = 3 adds the column sum of dx).
@@ -291,7 +292,7 @@ int ln_bwd(const bf16* dy, const bf16* x, const float* mean, const float* rstd, 
 
 void colsum_geometry(int M, int N, int* strips, int* rows_per_strip) {
   const int gx = (N / 8 + 31) / 32;
-  int st = std::max(1, 2 * 148 / gx);
+  int st = std::max(1, 4 * 148 / gx);
   st = std::min(st, std::max(1, (M + 63) / 64));
   st = std::min(st, kMaxStrips);
   *rows_per_strip = (M + st - 1) / st;

@@ -213,31 +213,64 @@ __global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restri
 
 // LayerNorm backward: dx = rstd * (dy*w - mean(dy*w) - xhat * mean(dy*w*xhat))
 // (+ dresid, the gradient flowing along the residual stream), written in bf16.
-// Each warp keeps private column sums of dy*xhat, dy and (optionally) of its
-// output dx in shared memory; the CTA writes one partial row per quantity to
-// `part` ([grid][NQ][C], NQ = 3 with the dx sum, else 2), summed in a fixed
-// order afterwards. The dx column sum is the gradient of the bias of the
-// projection that wrote the residual stream (its output gradient is dx).
+// One warp per row, rows in a grid-stride loop; a lane always owns the same
+// columns (16-byte chunk vi = lane + 32 i), so its column sums of dy*xhat, dy
+// and (optionally) of its output dx stay in registers across rows (C <= 1024;
+// wider rows keep them in warp-private shared memory). At the end the warps'
+// sums are combined in a fixed order and the CTA writes one partial row per
+// quantity to `part` ([grid][NQ][C], NQ = 3 with the dx sum, else 2), summed in
+// a fixed order afterwards. The dx column sum is the gradient of the bias of
+// the projection that wrote the residual stream (its output gradient is dx).
+// Warps per CTA and CTAs per SM by row width: enough rows in flight per SM
+// for the HBM latency, with the register column sums unspilled.
+__host__ __device__ constexpr int ln_bwd_warps(int C) { return C <= 512 ? 8 : (C == 768 ? 12 : (C == 1024 ? 8 : 4)); }
+__host__ __device__ constexpr int ln_bwd_minb(int C) { return (C <= 512 || C > 1024) ? 2 : 1; }
 template <int C>
 struct LnBwdCfg {
-  static constexpr int WARPS = C <= 768 ? 8 : 4;
+  static constexpr int WARPS = ln_bwd_warps(C);
+  static constexpr int MINB = ln_bwd_minb(C);
   static constexpr int SMEM = WARPS * 3 * C * 4;
 };
 
 template <int C>
-__global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, 2)
+__global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, LnBwdCfg<C>::MINB)
     layernorm_bwd_kernel(const bf16* __restrict__ dy, const bf16* __restrict__ x, const float* __restrict__ mean,
                          const float* __restrict__ rstd, const float* __restrict__ w, const bf16* dresid, bf16* dx,
                          float* __restrict__ part, int rows, int with_dxsum) {
   constexpr int NV = C / 8;
   constexpr int VPL = (NV + 31) / 32;
   constexpr int WARPS = LnBwdCfg<C>::WARPS;
+  constexpr bool kRegAcc = VPL <= 4;
   extern __shared__ __align__(16) float ln_acc[];  // [WARPS][3][C]
   const int warp = threadIdx.x >> 5, l = lane_id();
   float* acc = ln_acc + warp * 3 * C;
-  for (int i = l; i < 3 * C; i += 32) acc[i] = 0.f;
-  __syncwarp();
+  float ra[kRegAcc ? VPL : 1][3][8];
+#pragma unroll
+  for (int i = 0; i < (kRegAcc ? VPL : 1); ++i)
+#pragma unroll
+    for (int q = 0; q < 3; ++q)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) ra[i][q][j] = 0.f;
+  if (!kRegAcc) {
+    for (int i = l; i < 3 * C; i += 32) acc[i] = 0.f;
+    __syncwarp();
+  }
   const int nq = with_dxsum ? 3 : 2;
+  // the weights of this lane's columns, loaded once
+  float wv[VPL][8];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int vi = l + 32 * i;
+    if (vi < NV) {
+      const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + vi * 8));
+      const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + vi * 8 + 4));
+      wv[i][0] = w0.x; wv[i][1] = w0.y; wv[i][2] = w0.z; wv[i][3] = w0.w;
+      wv[i][4] = w1.x; wv[i][5] = w1.y; wv[i][6] = w1.z; wv[i][7] = w1.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) wv[i][j] = 0.f;
+    }
+  }
   for (int row = blockIdx.x * WARPS + warp; row < rows; row += gridDim.x * WARPS) {
     const float mu = mean[row], rs = rstd[row];
     uint4 ux[VPL], ud[VPL], ur[VPL];
@@ -246,9 +279,9 @@ __global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, 2)
       const int vi = l + 32 * i;
       ur[i] = make_uint4(0u, 0u, 0u, 0u);
       if (vi < NV) {
-        ux[i] = *reinterpret_cast<const uint4*>(x + (size_t)row * C + vi * 8);
-        ud[i] = *reinterpret_cast<const uint4*>(dy + (size_t)row * C + vi * 8);
-        if (dresid != nullptr) ur[i] = *reinterpret_cast<const uint4*>(dresid + (size_t)row * C + vi * 8);
+        ux[i] = __ldcs(reinterpret_cast<const uint4*>(x + (size_t)row * C + vi * 8));
+        ud[i] = __ldcs(reinterpret_cast<const uint4*>(dy + (size_t)row * C + vi * 8));
+        if (dresid != nullptr) ur[i] = __ldcs(reinterpret_cast<const uint4*>(dresid + (size_t)row * C + vi * 8));
       }
     }
     float s1 = 0.f, s2 = 0.f;
@@ -257,20 +290,24 @@ __global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, 2)
       const int vi = l + 32 * i;
       if (vi < NV) {
         const uint32_t xw[4] = {ux[i].x, ux[i].y, ux[i].z, ux[i].w}, dw4[4] = {ud[i].x, ud[i].y, ud[i].z, ud[i].w};
-        const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + vi * 8));
-        const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + vi * 8 + 4));
-        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-        float* a0 = acc + vi * 8;
-        float* a1 = acc + C + vi * 8;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 fx = unpack_bf16x2(xw[j]), fd = unpack_bf16x2(dw4[j]);
           const float xh0 = (fx.x - mu) * rs, xh1 = (fx.y - mu) * rs;
-          a0[2 * j] += fd.x * xh0;
-          a0[2 * j + 1] += fd.y * xh1;
-          a1[2 * j] += fd.x;
-          a1[2 * j + 1] += fd.y;
-          const float g0 = fd.x * wv[2 * j], g1 = fd.y * wv[2 * j + 1];
+          if (kRegAcc) {
+            ra[i][0][2 * j] += fd.x * xh0;
+            ra[i][0][2 * j + 1] += fd.y * xh1;
+            ra[i][1][2 * j] += fd.x;
+            ra[i][1][2 * j + 1] += fd.y;
+          } else {
+            float* a0 = acc + vi * 8;
+            float* a1 = acc + C + vi * 8;
+            a0[2 * j] += fd.x * xh0;
+            a0[2 * j + 1] += fd.y * xh1;
+            a1[2 * j] += fd.x;
+            a1[2 * j + 1] += fd.y;
+          }
+          const float g0 = fd.x * wv[i][2 * j], g1 = fd.y * wv[i][2 * j + 1];
           s1 += g0 + g1;
           s2 += g0 * xh0 + g1 * xh1;
         }
@@ -283,15 +320,12 @@ __global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, 2)
       if (vi < NV) {
         const uint32_t xw[4] = {ux[i].x, ux[i].y, ux[i].z, ux[i].w}, dw4[4] = {ud[i].x, ud[i].y, ud[i].z, ud[i].w};
         const uint32_t rw[4] = {ur[i].x, ur[i].y, ur[i].z, ur[i].w};
-        const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + vi * 8));
-        const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + vi * 8 + 4));
-        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         float r[8];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 fx = unpack_bf16x2(xw[j]), fd = unpack_bf16x2(dw4[j]), fr = unpack_bf16x2(rw[j]);
-          r[2 * j] = (fd.x * wv[2 * j] - m1 - (fx.x - mu) * rs * m2) * rs + fr.x;
-          r[2 * j + 1] = (fd.y * wv[2 * j + 1] - m1 - (fx.y - mu) * rs * m2) * rs + fr.y;
+          r[2 * j] = (fd.x * wv[i][2 * j] - m1 - (fx.x - mu) * rs * m2) * rs + fr.x;
+          r[2 * j + 1] = (fd.y * wv[i][2 * j + 1] - m1 - (fx.y - mu) * rs * m2) * rs + fr.y;
         }
         const uint4 o = make_uint4(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]), pack_bf16x2(r[4], r[5]),
                                    pack_bf16x2(r[6], r[7]));
@@ -299,13 +333,32 @@ __global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, 2)
         if (with_dxsum) {
           // the bias gradient sees the stored (bf16) residual gradient
           const uint32_t ow[4] = {o.x, o.y, o.z, o.w};
-          float* a2 = acc + 2 * C + vi * 8;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const float2 f = unpack_bf16x2(ow[j]);
-            a2[2 * j] += f.x;
-            a2[2 * j + 1] += f.y;
+            if (kRegAcc) {
+              ra[i][2][2 * j] += f.x;
+              ra[i][2][2 * j + 1] += f.y;
+            } else {
+              float* a2 = acc + 2 * C + vi * 8;
+              a2[2 * j] += f.x;
+              a2[2 * j + 1] += f.y;
+            }
           }
+        }
+      }
+    }
+  }
+  if (kRegAcc) {
+#pragma unroll
+    for (int i = 0; i < (kRegAcc ? VPL : 1); ++i) {
+      const int vi = l + 32 * i;
+      if (vi < NV) {
+#pragma unroll
+        for (int q = 0; q < 3; ++q) {
+          float4* dst = reinterpret_cast<float4*>(acc + q * C + vi * 8);
+          dst[0] = make_float4(ra[i][q][0], ra[i][q][1], ra[i][q][2], ra[i][q][3]);
+          dst[1] = make_float4(ra[i][q][4], ra[i][q][5], ra[i][q][6], ra[i][q][7]);
         }
       }
     }
@@ -355,13 +408,13 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const bf16* __restr
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   if (c < N) {
     int r = r0 + ty;
-    // four independent rows per iteration keep four 16-byte loads in flight
-    for (; r + 24 < r1; r += 32) {
-      uint4 u[4];
+    // eight independent rows per iteration keep eight 16-byte loads in flight
+    for (; r + 56 < r1; r += 64) {
+      uint4 u[8];
 #pragma unroll
-      for (int k2 = 0; k2 < 4; ++k2) u[k2] = *reinterpret_cast<const uint4*>(a + (size_t)(r + 8 * k2) * N + c);
+      for (int k2 = 0; k2 < 8; ++k2) u[k2] = __ldcs(reinterpret_cast<const uint4*>(a + (size_t)(r + 8 * k2) * N + c));
 #pragma unroll
-      for (int k2 = 0; k2 < 4; ++k2) {
+      for (int k2 = 0; k2 < 8; ++k2) {
         const uint32_t w[4] = {u[k2].x, u[k2].y, u[k2].z, u[k2].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {

@@ -15,7 +15,7 @@
       Times the causal attention forward or backward (head size 64) through the
       op-level C ABI and prints TFLOP/s (causal FLOPs incl. the diagonal block).
 
-  python -m gpt_step_b200.profile_step bw --kernel ln_fwd|ln_bwd|ce --shape rows,C [--iters n]
+  python -m gpt_step_b200.profile_step bw --kernel ln_fwd|ln_bwd|ce|colsum --shape rows,C [--iters n]
       Times a bandwidth-bound kernel alone and prints GB/s of algorithmic bytes
       (for ce, C is the padded vocabulary and the real one is C - 47).
 """
@@ -160,6 +160,12 @@ def run_bw(args):
             ws = torch.empty(gs.layernorm_bwd_workspace(rows, C), dtype=torch.uint8, device="cuda")
             fn = lambda: gs.layernorm_bwd(dy, x, mean, rstd, w, dres, dx, dw, db, ws)
             nbytes = rows * (8.0 * C + 8)
+    elif args.kernel == "colsum":  # bias gradient: column sums of a rows x C bf16 matrix
+        a = bf(rows, C)
+        db = torch.zeros(C, device="cuda")
+        ws = torch.empty(gs.bias_grad_workspace(rows, C), dtype=torch.uint8, device="cuda")
+        fn = lambda: gs.bias_grad(a, db, ws)
+        nbytes = rows * C * 2.0
     else:  # ce: rows x C logits (C = padded vocabulary), real vocabulary C - 47
         z0 = bf(rows, C)
         z = torch.empty_like(z0)
@@ -199,7 +205,7 @@ def main():
     a.add_argument("--shape", default="19,1024,12")
     a.add_argument("--iters", type=int, default=20)
     w = sub.add_parser("bw")
-    w.add_argument("--kernel", choices=["ln_fwd", "ln_bwd", "ce"], default="ln_fwd")
+    w.add_argument("--kernel", choices=["ln_fwd", "ln_bwd", "ce", "colsum"], default="ln_fwd")
     w.add_argument("--shape", default="19456,768")
     w.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
