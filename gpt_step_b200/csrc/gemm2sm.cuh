@@ -31,11 +31,13 @@ constexpr int kThreads2 = 320;  // TMA, MMA, 8 epilogue warps (two per TMEM lane
 
 template <int BN>
 struct Cfg {
-  static constexpr int STAGES = 5;
+  static constexpr int STAGES = 6;
+  // epilogue staging: 4 KB per epilogue warp (two 2 KB store buffers, or one per
+  // output for the two-output GELU epilogue)
+  static constexpr int EPI_BYTES = 8 * 4096;
   static constexpr int A_BYTES = 128 * BK * 2;          // own 128 rows
   static constexpr int B_BYTES = (BN / 2) * BK * 2;     // own half of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int EPI_BYTES = 8 * 4 * 2048;       // per epilogue warp: 2 buffers x 2 outputs
   static constexpr int BAR_BYTES = 1024;
   static constexpr int SMEM = STAGES * STAGE_BYTES + EPI_BYTES + BAR_BYTES + 1024;
   static constexpr int TMEM_COLS = 2 * BN;
@@ -124,7 +126,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), 2 * 8 * 32);
+      mbar_init(smem_u32(&tempty[i]), 2 * 8);   // one arrival per epilogue warp of the pair
     }
     mbar_init(smem_u32(done), 1);
     fence_mbar_init();
@@ -188,9 +190,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
+      const int mn_tiles = p.num_m * p.num_n;
       for (int t = cid; t < p.num_tiles && ok; t += ncl, ++it) {
-        const int rest = t / p.num_m;
-        const int sp = rest / p.num_n;
+        // tile bookkeeping stays off the MMA issue path: no division without a split
+        const int sp = p.splits == 1 ? 0 : t / mn_tiles;
         const int kb0 = sp * p.kb_per_split;
         const int kb1 = min(p.nkb, kb0 + p.kb_per_split);
         const int acc = it & 1;
@@ -223,7 +226,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;              // TMEM lane quarter
     const int hv = (warp - 2) >> 2;      // column half of the tile this warp drains
-    uint8_t* wbuf = epi_smem + (warp - 2) * 8192;
+    uint8_t* wbuf = epi_smem + (warp - 2) * 4096;
     uint32_t nstore = 0;
     int it = 0;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
@@ -239,11 +242,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       const int row0 = mb * BM_PAIR + 128 * rank + q * 32;
       const int row = row0 + lane;
       const bool row_ok = row < p.M;
-#pragma unroll 1
-      for (int c = hv * (BN / 2); c < (hv + 1) * (BN / 2); c += 32) {
+      const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+      // Chunk c + 32 is read from tensor memory, and its bias / aux operands
+      // from global memory, while chunk c is processed: the epilogue of a tile
+      // then runs at about the pace of the next tile's main loop.
+      constexpr bool kBias = EPI == gemm::EPI_STORE || EPI == gemm::EPI_RESID || EPI == gemm::EPI_GELU;
+      constexpr bool kAux = EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU;
+      const bool has_bias = kBias && p.bias != nullptr;
+      const int c_beg = hv * (BN / 2), c_end = (hv + 1) * (BN / 2);
+      uint32_t vr[32];
+      float4 bn4[8];
+      uint4 an4[4];
+      auto fetch = [&](int c) {
+        tmem_ld32_async(t_row + c, vr);
         const int n = nb * BN + c;
+        if (n < p.N) {
+          if (has_bias) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) bn4[i] = __ldg(reinterpret_cast<const float4*>(p.bias + n) + i);
+          }
+          if (kAux && row_ok) {
+            const uint4* src = reinterpret_cast<const uint4*>(p.aux + (size_t)row * p.ld_aux + n);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) an4[j] = __ldcs(src + j);
+          }
+        }
+      };
+      fetch(c_beg);
+#pragma unroll 1
+      for (int c = c_beg; c < c_end; c += 32) {
+        const int n = nb * BN + c;
+        tmem_wait_ld();
         float v[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN + c, v);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vr[i]);
+        // consume this chunk's bias / aux registers, then start the next chunk's loads
+        if (n < p.N && has_bias) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[4 * i] += bn4[i].x; v[4 * i + 1] += bn4[i].y; v[4 * i + 2] += bn4[i].z; v[4 * i + 3] += bn4[i].w;
+          }
+        }
+        if (kAux && n < p.N && row_ok) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t w[4] = {an4[j].x, an4[j].y, an4[j].z, an4[j].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float2 f = unpack_bf16x2(w[h]);
+              const int i = j * 8 + h * 2;
+              if (EPI == gemm::EPI_RESID) {
+                v[i] += f.x; v[i + 1] += f.y;
+              } else {
+                v[i] *= gelu_grad_f(f.x); v[i + 1] *= gelu_grad_f(f.y);
+              }
+            }
+          }
+        }
+        if (c + 32 < c_end) fetch(c + 32);
         if (n >= p.N) continue;
         if (EPI == gemm::EPI_ACC_F32) {
           if (!row_ok) continue;
@@ -261,56 +317,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           }
           continue;
         }
-        if (EPI == gemm::EPI_STORE || EPI == gemm::EPI_RESID || EPI == gemm::EPI_GELU) {
-          if (p.bias != nullptr) {
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-              const float4 b = __ldg(reinterpret_cast<const float4*>(p.bias + n + i));
-              v[i] += b.x; v[i + 1] += b.y; v[i + 2] += b.z; v[i + 3] += b.w;
-            }
-          }
-        }
-        if ((EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU) && row_ok) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.aux + (size_t)row * p.ld_aux + n);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint4 u = src[j];
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const float2 f = unpack_bf16x2(w[h]);
-              const int i = j * 8 + h * 2;
-              if (EPI == gemm::EPI_RESID) {
-                v[i] += f.x; v[i + 1] += f.y;
-              } else {
-                v[i] *= gelu_grad_f(f.x); v[i + 1] *= gelu_grad_f(f.y);
-              }
-            }
-          }
-        }
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-        const uint32_t b = nstore & 1;
-        if (lane == 0) gemm::bulk_wait_read<1>();
+        // single-output epilogues alternate two buffers; GELU has one per output
+        const uint32_t b = EPI == gemm::EPI_GELU ? 0u : (nstore & 1);
+        if (lane == 0) {
+          if (EPI == gemm::EPI_GELU) gemm::bulk_wait_read<0>();
+          else gemm::bulk_wait_read<1>();
+        }
         __syncwarp();
         gemm::stage_row(wbuf + b * 2048, lane, pk);
         if (EPI == gemm::EPI_GELU) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(gelu_f(v[2 * i]), gelu_f(v[2 * i + 1]));
-          gemm::stage_row(wbuf + 4096 + b * 2048, lane, pk);
+          gemm::stage_row(wbuf + 2048, lane, pk);
         }
         gemm::fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
           gemm::tma_store_2d(&tmO, smem_u32(wbuf + b * 2048), n, row0);
-          if (EPI == gemm::EPI_GELU) gemm::tma_store_2d(&tmO2, smem_u32(wbuf + 4096 + b * 2048), n, row0);
+          if (EPI == gemm::EPI_GELU) gemm::tma_store_2d(&tmO2, smem_u32(wbuf + 2048), n, row0);
           gemm::bulk_commit();
         }
         ++nstore;
       }
+      tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
     }
     if (EPI != gemm::EPI_ACC_F32 && lane == 0) gemm::bulk_wait_all<0>();
   }
