@@ -307,7 +307,7 @@ def main():
         g = prof["gemm"]
         ach = g["flops"] / (g["ms"] / 1000.0) / 1e12
         pk = peaks["bf16_tflops_sustained"]
-        roof = {"bound": "tensor", "kernel": "gemm_tc_kernel (all tcgen05 GEMM launches)",
+        roof = {"bound": "tensor", "kernel": "gemm_tc2_kernel / gemm_tc_kernel (every tcgen05 GEMM launch)",
                 "achieved": round(ach, 1), "peak": pk, "unit": "TFLOP/s", "frac": round(ach / pk, 4),
                 "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
                 "traffic": None, "launches": g["launches"], "share_of_step": round(g["ms"] / ms, 4),
