@@ -42,6 +42,7 @@ enum Epi : int {
 struct Params {
   int M, N, K;
   int num_m, num_n, splits, kb_per_split, nkb, num_tiles;
+  int raster_gm;  // row tiles per raster panel (pair kernel); num_m = plain row-major order
   bf16* out;
   bf16* out2;
   int ldo;
