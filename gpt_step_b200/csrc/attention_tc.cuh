@@ -10,14 +10,14 @@
 //             S_j = Q K_j^T   (M=128, N=128, K=64)  into S[j % 2] (TMEM)
 //             O  += P_j V_j   (M=128, N=64,  K=128) into O (TMEM)
 //   warps 2-5  one query row per thread: read S_j from TMEM, online softmax in
-//             log2 units, write P_j (bf16) to shared memory as the A operand of
-//             the next MMA, rescale O in TMEM when the row maximum grows by more
+//             log2 units, write P_j (bf16 pairs) to tensor memory as the A operand
+//             of the next MMA, rescale O in TMEM when the row maximum grows by more
 //             than 2^8 (otherwise the stale maximum is kept: p <= 256 is exact
 //             enough in fp32 and bf16), finally O / l and the log-sum-exp.
 //
 // Operands: Q, K are K-major (head dimension contiguous); V is used as stored
-// ([key][head dim]) as an MN-major B operand; P is K-major. All tiles use the
-// 128-byte swizzle (rows of 64 bf16). No cluster multicast.
+// ([key][head dim]) as an MN-major B operand; P is read from tensor memory.
+// Shared tiles use the 128-byte swizzle (rows of 64 bf16). No cluster multicast.
 #pragma once
 #include "common.cuh"
 
@@ -27,14 +27,13 @@ constexpr int BQ = 128, BKV = 128, HD = 64;
 constexpr int kThreads = 192;
 constexpr int Q_BYTES = BQ * HD * 2;         // 16 KB
 constexpr int KV_BYTES = BKV * HD * 2;       // 16 KB each for K and V
-constexpr int P_BYTES = BQ * BKV * 2;        // 32 KB (two 64-key K blocks)
 constexpr int STAGES = 2;
 // No alignment slack: without static shared memory the dynamic block starts on a
-// 1 KB boundary (checked at run time), and 115,712 bytes is exactly what lets two
-// CTAs (plus the driver's 1 KB each) share an SM's 233,472 bytes.
-constexpr int SMEM_BYTES = Q_BYTES + STAGES * 2 * KV_BYTES + P_BYTES + 1024 /*barriers*/;
-constexpr int TMEM_COLS = 256;               // S [0,128), O [128,192); two CTAs share an SM
-constexpr uint32_t S_COL0 = 0, O_COL = 128;
+// 1 KB boundary (checked at run time). 82,944 bytes and 256 TMEM columns a CTA:
+// two CTAs share an SM.
+constexpr int SMEM_BYTES = Q_BYTES + STAGES * 2 * KV_BYTES + 1024 /*barriers*/;
+constexpr int TMEM_COLS = 256;               // S [0,128), O [128,192), P [192,256); two CTAs share an SM
+constexpr uint32_t S_COL0 = 0, O_COL = 128, P_COL = 192;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;    // log2(256)
@@ -51,6 +50,28 @@ GPT2_DEV void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem]^T (A: M rows in TMEM lanes, K along columns as bf16 pairs).
+GPT2_DEV void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+GPT2_DEV void tmem_st32_u(uint32_t taddr, const uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
+      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
+      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+GPT2_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
                        int T, int H, float scale, int* err) {
@@ -63,8 +84,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + Q_BYTES;                  // [STAGES][KV_BYTES]
   uint8_t* sV = sK + STAGES * KV_BYTES;        // [STAGES][KV_BYTES]
-  uint8_t* sP = sV + STAGES * KV_BYTES;        // [P_BYTES]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + P_BYTES);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + STAGES * KV_BYTES);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;     // [2]  K_j landed
   uint64_t* k_empty = bars + 3;    // [2]  S_j computed: K stage free
@@ -187,14 +207,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(smem_u32(p_full), j & 1, err)) { ok = false; break; }
         if (!mbar_wait(smem_u32(&v_full[st]), (j >> 1) & 1, err)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t p_addr = smem_u32(sP);
         const uint32_t v_addr = smem_u32(sV + st * KV_BYTES);
+        const uint64_t vd = smem_desc_sw128(v_addr, 8192, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(p_addr + (kk >> 2) * (BQ * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(v_addr + kk * 2048, 8192, 1024);
-          tc_mma_bf16(tmem + O_COL, ad, bd, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BKV / 16; ++kk)   // A = P from tensor memory, 16 keys = 8 columns a step
+          tc_mma_bf16_ts(tmem + O_COL, tmem + P_COL + kk * 8, vd + kk * 128, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(smem_u32(p_empty));
         tc_commit(smem_u32(&v_empty[st]));
         tc_commit(smem_u32(o_done));
@@ -263,18 +280,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int t = 0; t < 8; ++t) sum += spart[t];
       // the P buffer was last read by the PV product of block j-1
       if (j >= 1 && !mbar_wait(smem_u32(p_empty), (j - 1) & 1, err)) { ok = false; break; }
-      uint8_t* pb = sP;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t (&pk)[16] = pkall[c];
-        const int kb = c >> 1;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int ch = (c & 1) * 4 + q;  // 16-byte chunk within the 64-key block
-          *reinterpret_cast<uint4*>(pb + kb * (BQ * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-        }
-      }
+      tc_fence_after();
+      // P_j as bf16 pairs: keys 2i, 2i+1 of this query row in column P_COL + i
+      tmem_st32_u(tmem + lane_off + P_COL, *reinterpret_cast<const uint32_t(*)[32]>(&pkall[0][0]));
+      tmem_st32_u(tmem + lane_off + P_COL + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pkall[2][0]));
       l = l * alpha + sum;
       m = m_new;
       // O rescale (rows whose maximum moved) once the PV product of block j-1 is done
@@ -290,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_st32(tmem + lane_off + O_COL + c * 32, v);
         }
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(p_full));
     }
@@ -346,14 +355,19 @@ static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int
 // Backward (head size 64). Three kernels:
 //
 //   bwd_prep_kernel   per (batch, head, query): D = rowsum(dO o O) (the softmax
-//                     Jacobian term), stored as -D * scale, and -lse * log2(e);
-//                     clears the fp32 dQ accumulator.
+//                     Jacobian term); writes -lse/scale and -D, each as a bf16
+//                     hi + lo pair, into a 16-column operand tile per query block
+//                     (see below); clears the fp32 dQ accumulator.
 //   attn_bwd_tc_kernel  per CTA one (batch, head) and a block of 128 keys; walks
 //                     the query blocks at or after it (causal). With K, V resident
 //                     and Q_i, dO_i streamed through a three-deep ring:
-//       S^T  = K Q_i^T,  dP^T = V dO_i^T          (M=128 keys, N=128 queries, K=64)
-//       P^T  = exp2(S^T * scale*log2e - lse*log2e)  (warps 2-9, one key row each)
-//       dS^T = P^T * (dP^T - D) * scale
+//       S'^T  = [K | 1 1 0..] [Q_i | X_i]^T   = S^T - lse/scale  (M=128 keys, N=128 queries,
+//       dP'^T = [V | 0 0 1 1 0..] [dO_i | X_i]^T = dP^T - D       K = 64 + one 16-wide step)
+//       P^T  = exp2(S'^T * scale*log2e)       (softmax warps, one key row each)
+//       dS^T = P^T * dP'^T * scale
+//     where X_i holds (hi, lo) of -lse/scale and of -D per query: the per-query
+//     terms enter through the tensor core, so the softmax warps read no shared
+//     memory (their loads would queue behind the tensor core's operand reads).
 //       dV  += P^T dO_i   (A = P^T from tensor memory)   (M=128 keys, N=64, K=128)
 //       dK  += dS^T Q_i   (A = dS^T from shared memory)
 //       dQ_i = dS K       (A = dS^T read MN-major)       (M=128 queries, N=64, K=128)
@@ -380,16 +394,33 @@ constexpr int kSoftmaxWarps = 8;
 // Launched at 168 registers a thread (three warps per scheduler), warpgroup 0
 // gives registers to the softmax warpgroups: 128 x 40 + 256 x 232 = 384 x 168.
 constexpr int kThreads = 128 + 32 * kSoftmaxWarps;
-constexpr int kLaunchRegs = 168, kCtlRegs = 88, kSoftmaxRegs = 208;
+constexpr int kLaunchRegs = 168, kCtlRegs = 152, kSoftmaxRegs = 176;
 static_assert(128 * kCtlRegs + 32 * kSoftmaxWarps * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
+constexpr int XT_BYTES = 128 * 16 * 2;              // 4 KB: a 128 x 16 extra-K operand tile
 constexpr int SMEM_BYTES = 2 * T_BYTES /*K,V*/ + NQS * 2 * T_BYTES /*Q,dO*/ + DST_BYTES +
-                           kSoftmaxWarps * DQW_BYTES + NQS * 2 * BQRY * 4 /*lse, D*/ + 256 /*barriers*/ +
-                           1024 /*align*/;
+                           kSoftmaxWarps * DQW_BYTES + NQS * XT_BYTES /*X_i*/ + 2 * XT_BYTES /*K', V' columns*/ +
+                           256 /*barriers*/ + 1024 /*align*/;
 constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 320, C_DQ = 384, C_P = 448;
 constexpr int TMEM_COLS_BWD = 512;
 constexpr int kPrepRows = 32;                       // query rows per prep block
 constexpr int kMaxHeads = 64;
 }  // namespace bwd
+
+// Extra-K operand tiles (128 rows x 16 bf16) use the tensor core's non-swizzled
+// K-major layout: 8-row x 16-byte core matrices stored as 128 contiguous bytes,
+// the two core matrices of a row group adjacent (128 bytes apart along K) and
+// row groups 256 bytes apart. Byte offset of (row, col):
+__host__ __device__ constexpr int xt_offset(int row, int col) {
+  return ((row >> 3) * 2 + (col >> 3)) * 128 + (row & 7) * 16 + (col & 7) * 2;
+}
+GPT2_DEV uint64_t smem_desc_interleave(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100; layout 0: no swizzle
+  return d;
+}
 
 GPT2_DEV void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -397,27 +428,7 @@ GPT2_DEV void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32
                : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]^T (A: M rows in TMEM lanes, K along columns as bf16 pairs).
-GPT2_DEV void tc_mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
-GPT2_DEV void tmem_st32_u(uint32_t taddr, const uint32_t (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]),
-      "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]),
-      "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
-      : "memory");
-}
-GPT2_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 template <int N>
 GPT2_DEV void regs_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
 template <int N>
@@ -426,22 +437,19 @@ GPT2_DEV void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::
 // P^T and dS^T of one key row (this thread) for 64 query columns. DIAG: the
 // query block is the key block itself, so keys after the query are masked.
 template <bool DIAG>
-GPT2_DEV void bwd_softmax_row(const uint32_t (&sv)[2][32], const uint32_t (&dv)[2][32], const float4* nq,
-                              const float4* dq, float sl2, float scale, int r, int col0, uint32_t (&pp)[32],
-                              uint32_t (&pd)[32]) {
+GPT2_DEV void bwd_softmax_row(const uint32_t (&sv)[2][32], const uint32_t (&dv)[2][32], float sl2, float scale,
+                              int r, int col0, uint32_t (&pp)[32], uint32_t (&pd)[32]) {
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
-      const float4 n4 = nq[c * 8 + g], d4 = dq[c * 8 + g];
-      const float nn[4] = {n4.x, n4.y, n4.z, n4.w}, dd[4] = {d4.x, d4.y, d4.z, d4.w};
       float p[4], ds[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int j = g * 4 + e;   // column within this 32-column chunk
-        p[e] = ex2_approx(fmaf(__uint_as_float(sv[c][j]), sl2, nn[e]));
+        p[e] = ex2_approx(__uint_as_float(sv[c][j]) * sl2);          // S' already holds -lse/scale
         if (DIAG && r > col0 + c * 32 + j) p[e] = 0.f;   // key after query: masked
-        ds[e] = p[e] * fmaf(__uint_as_float(dv[c][j]), scale, dd[e]);
+        ds[e] = p[e] * (__uint_as_float(dv[c][j]) * scale);          // dP' already holds -D
       }
       pp[c * 16 + g * 2] = pack_bf16x2(p[0], p[1]);
       pp[c * 16 + g * 2 + 1] = pack_bf16x2(p[2], p[3]);
@@ -454,9 +462,8 @@ GPT2_DEV void bwd_softmax_row(const uint32_t (&sv)[2][32], const uint32_t (&dv)[
 // Block: 32 consecutive query rows of one sequence, all heads. Each warp takes
 // four rows; lanes hold 16-byte chunks of O and dO, eight chunks per head.
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
-                                                       const float* __restrict__ lse, float* __restrict__ nl2,
-                                                       float* __restrict__ dsc, float* __restrict__ dq_acc, int T,
-                                                       int H, float scale) {
+                                                       const float* __restrict__ lse, uint8_t* __restrict__ xtiles,
+                                                       float* __restrict__ dq_acc, int T, int H, float scale) {
   using namespace bwd;
   __shared__ float sDot[kMaxHeads][kPrepRows];
   const int C = H * HD;
@@ -487,11 +494,19 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ 
     }
   }
   __syncthreads();
+  // X tile of query block (b, h, t / 128), row t % 128: columns 0,1 = (hi, lo) of
+  // -lse/scale, columns 2,3 = (hi, lo) of -D, the rest 0
   for (int i = threadIdx.x; i < H * kPrepRows; i += blockDim.x) {
     const int h = i / kPrepRows, rl = i % kPrepRows;
-    const size_t o = ((size_t)b * H + h) * T + t0 + rl;
-    nl2[o] = -lse[o] * kLog2e;
-    dsc[o] = -sDot[h][rl] * scale;
+    const int t = t0 + rl;
+    const size_t o = ((size_t)b * H + h) * T + t;
+    const float x1 = -lse[o] / scale, x2 = -sDot[h][rl];
+    const float h1 = __bfloat162float(__float2bfloat16_rn(x1)), h2 = __bfloat162float(__float2bfloat16_rn(x2));
+    uint8_t* tile = xtiles + (((size_t)b * H + h) * (T / BQRY) + t / BQRY) * XT_BYTES;
+    const int qr = t % BQRY;
+    *reinterpret_cast<uint4*>(tile + xt_offset(qr, 0)) =
+        make_uint4(pack_bf16x2(h1, x1 - h1), pack_bf16x2(h2, x2 - h2), 0u, 0u);
+    *reinterpret_cast<uint4*>(tile + xt_offset(qr, 8)) = make_uint4(0u, 0u, 0u, 0u);
   }
   float4* z = reinterpret_cast<float4*>(dq_acc + (size_t)row0 * C);
   const int n4 = kPrepRows * C / 4;
@@ -514,8 +529,8 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
 
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_dq, const float* __restrict__ nl2,
-                       const float* __restrict__ dsc, bf16* __restrict__ dqkv, int T, int H, float scale, int* err) {
+                       const __grid_constant__ CUtensorMap tm_dq, const uint8_t* __restrict__ xtiles,
+                       bf16* __restrict__ dqkv, int T, int H, float scale, int* err) {
   using namespace bwd;
   extern __shared__ __align__(1024) uint8_t smem_raw_ab[];
   uint8_t* smem =
@@ -526,9 +541,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   uint8_t* sDO = sQ + NQS * T_BYTES;              // [NQS]
   uint8_t* sDST = sDO + NQS * T_BYTES;
   uint8_t* sDQW = sDST + DST_BYTES;               // [kSoftmaxWarps][DQW_BYTES]
-  float* sNL = reinterpret_cast<float*>(sDQW + kSoftmaxWarps * DQW_BYTES);  // [NQS][BQRY]
-  float* sDS = sNL + NQS * BQRY;                                            // [NQS][BQRY]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sDS + NQS * BQRY);
+  uint8_t* sXQ = sDQW + kSoftmaxWarps * DQW_BYTES;  // [NQS] X_i tiles
+  uint8_t* sXK = sXQ + NQS * XT_BYTES;              // K' extra columns: 1 1 0 ..
+  uint8_t* sXV = sXK + XT_BYTES;                    // V' extra columns: 0 0 1 1 0 ..
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sXV + XT_BYTES);
   uint64_t* kv_full = bars;
   uint64_t* qdo_full = bars + 1;          // [NQS]
   uint64_t* qdo_empty = bars + 1 + NQS;   // [NQS]
@@ -571,6 +587,14 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     tma_prefetch_desc(&tm_do);
     tma_prefetch_desc(&tm_dq);
   }
+  // constant extra-K columns of K' and V' (1.0 in bf16 is 0x3F80)
+  for (int i = threadIdx.x; i < BKEY * 2; i += blockDim.x) {
+    const int row = i >> 1, half = i & 1;
+    const uint32_t one2 = 0x3F803F80u;
+    *reinterpret_cast<uint4*>(sXK + xt_offset(row, 8 * half)) = make_uint4(half ? 0u : one2, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(sXV + xt_offset(row, 8 * half)) = make_uint4(0u, half ? 0u : one2, 0u, 0u);
+  }
+  fence_async_smem();
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), TMEM_COLS_BWD);
     tmem_relinquish();
@@ -588,17 +612,15 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         mbar_arrive_expect_tx(smem_u32(kv_full), 2 * T_BYTES);
         tma_load_2d(smem_u32(sK), &tm_qkv, smem_u32(kv_full), C + h * HD, row_base + kb * BKEY);
         tma_load_2d(smem_u32(sV), &tm_qkv, smem_u32(kv_full), 2 * C + h * HD, row_base + kb * BKEY);
-        const float* nl_b = nl2 + (size_t)bh * T;
-        const float* ds_b = dsc + (size_t)bh * T;
+        const uint8_t* x_b = xtiles + (size_t)bh * (T / BQRY) * XT_BYTES;
         for (int it = 0; it < nit; ++it) {
           const int s = it % NQS, u = it / NQS, qi = kb + it;
           if (!mbar_wait(smem_u32(&qdo_empty[s]), (u & 1) ^ 1, err)) break;
           const uint32_t fb = smem_u32(&qdo_full[s]);
-          mbar_arrive_expect_tx(fb, 2 * T_BYTES + 2 * BQRY * 4);
+          mbar_arrive_expect_tx(fb, 2 * T_BYTES + XT_BYTES);
           tma_load_2d(smem_u32(sQ + s * T_BYTES), &tm_qkv, fb, h * HD, row_base + qi * BQRY);
           tma_load_2d(smem_u32(sDO + s * T_BYTES), &tm_do, fb, h * HD, row_base + qi * BQRY);
-          bulk_load_1d(smem_u32(sNL + s * BQRY), nl_b + qi * BQRY, BQRY * 4, fb);
-          bulk_load_1d(smem_u32(sDS + s * BQRY), ds_b + qi * BQRY, BQRY * 4, fb);
+          bulk_load_1d(smem_u32(sXQ + s * XT_BYTES), x_b + (size_t)qi * XT_BYTES, XT_BYTES, fb);
         }
       }
     } else if (warp == 1) {
@@ -618,14 +640,22 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         const uint64_t dQ0_mn = smem_desc_sw128(smem_u32(sQ), 8192, 1024);
         const uint64_t dO0_k = smem_desc_sw128(smem_u32(sDO), 16, 1024);
         const uint64_t dO0_mn = smem_desc_sw128(smem_u32(sDO), 8192, 1024);
+      const uint64_t dXK = smem_desc_interleave(smem_u32(sXK), 128, 256);
+      const uint64_t dXV = smem_desc_interleave(smem_u32(sXV), 128, 256);
+      const uint64_t dXQ0 = smem_desc_interleave(smem_u32(sXQ), 128, 256);
+      constexpr uint64_t kXStage = XT_BYTES >> 4;
         constexpr uint64_t kStage = T_BYTES >> 4;   // one Q/dO stage, in descriptor units
         auto issue_st = [&](int it) {
           const uint64_t so = (uint64_t)(it % NQS) * kStage;
-  #pragma unroll
+          const uint64_t sx = (uint64_t)(it % NQS) * kXStage;
+#pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             tc_mma_bf16(tmem + C_S, dK_k + kk * 2, dQ0_k + so + kk * 2, id_st, kk > 0 ? 1u : 0u);
             tc_mma_bf16(tmem + C_DP, dV_k + kk * 2, dO0_k + so + kk * 2, id_st, kk > 0 ? 1u : 0u);
           }
+          // the per-query terms: S^T - lse/scale, dP^T - D
+          tc_mma_bf16(tmem + C_S, dXK, dXQ0 + sx, id_st, 1u);
+          tc_mma_bf16(tmem + C_DP, dXV, dXQ0 + sx, id_st, 1u);
           tc_commit(smem_u32(st_full));
         };
         bool ok = mbar_wait(smem_u32(kv_full), 0, err) && mbar_wait(smem_u32(&qdo_full[0]), 0, err);
@@ -647,7 +677,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           if (!mbar_wait(smem_u32(ds_full), it & 1, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t acc0 = it > 0 ? 1u : 0u;
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < BQRY / 16; ++kk) {
             const uint32_t aoff = ((kk >> 2) * (BKEY * 128) + (kk & 3) * 32) >> 4;
             tc_mma_bf16_ts(tmem + C_DV, tmem + C_P + kk * 8, dO0_mn + so + kk * 128, id_kv, kk > 0 ? 1u : acc0);
@@ -656,7 +686,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           // dQ_it once dQ_{it-1} has left tensor memory
           if (it > 0 && !mbar_wait(smem_u32(dq_empty), (it - 1) & 1, err)) { ok = false; break; }
           tc_fence_after();
-  #pragma unroll
+#pragma unroll
           for (int kk = 0; kk < BKEY / 16; ++kk)
             tc_mma_bf16(tmem + C_DQ, dDS_mn + kk * 128, dK_mn + kk * 128, id_q, kk > 0 ? 1u : 0u);
           tc_commit(smem_u32(dq_full));
@@ -705,7 +735,6 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     };
     bool ok = true;
     for (int it = 0; it < nit && ok; ++it) {
-      const int s = it % NQS;
       if (!mbar_wait(smem_u32(st_full), it & 1, err)) { ok = false; break; }
       tc_fence_after();
       // this thread's 64 query columns of S^T and dP^T; tensor memory is free again at once
@@ -719,13 +748,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(st_empty));
-      // -lse*log2e and -D*scale of this query block came with Q_i
-      if (!mbar_wait(smem_u32(&qdo_full[s]), (it / NQS) & 1, err)) { ok = false; break; }
-      const float4* nq = reinterpret_cast<const float4*>(sNL + s * BQRY + hf * 64);
-      const float4* dq = reinterpret_cast<const float4*>(sDS + s * BQRY + hf * 64);
       uint32_t pp[32], pd[32];
-      if (it == 0) bwd_softmax_row<true>(sv, dv, nq, dq, sl2, scale, r, hf * 64, pp, pd);
-      else bwd_softmax_row<false>(sv, dv, nq, dq, sl2, scale, r, hf * 64, pp, pd);
+      if (it == 0) bwd_softmax_row<true>(sv, dv, sl2, scale, r, hf * 64, pp, pd);
+      else bwd_softmax_row<false>(sv, dv, sl2, scale, r, hf * 64, pp, pd);
       // P^T (TMEM) and dS^T (smem) were last read by the products of block it-1
       if (it > 0 && !mbar_wait(smem_u32(ds_empty), (it - 1) & 1, err)) { ok = false; break; }
       tc_fence_after();
@@ -772,9 +797,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   }
 }
 
-// The whole backward. nl2 / dsc fp32 [B, H, T] and dq_acc fp32 [B*T, C] are
+// The whole backward. xtiles (B*H*T*32 bytes) and dq_acc fp32 [B*T, C] are
 // scratch (contents on entry do not matter); dqkv receives dQ | dK | dV.
-static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* nl2, float* dsc,
+static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, uint8_t* xtiles,
                        float* dq_acc, bf16* dqkv, int B, int T, int H, int* err, cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
@@ -799,9 +824,9 @@ static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, c
       !encode_map_2d(&tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, (uint64_t)C, (uint64_t)B * T, (uint64_t)C,
                      32, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  bwd_prep_kernel<<<B * T / bwd::kPrepRows, 256, 0, s>>>(out, dout, lse, nl2, dsc, dq_acc, T, H, scale);
+  bwd_prep_kernel<<<B * T / bwd::kPrepRows, 256, 0, s>>>(out, dout, lse, xtiles, dq_acc, T, H, scale);
   dim3 grid(T / bwd::BKEY, B * H);
-  attn_bwd_tc_kernel<<<grid, bwd::kThreads, bwd::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, nl2, dsc, dqkv, T, H, scale,
+  attn_bwd_tc_kernel<<<grid, bwd::kThreads, bwd::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, xtiles, dqkv, T, H, scale,
                                                                   err);
   const int n = B * T * (C / 8);
   int blocks = (n + 255) / 256;

@@ -132,7 +132,7 @@ void make_layout(const Dims& d, Layout* lay) {
   lay->dqkv = take(N * 3 * C * 2);
   lay->datty = take(N * C * 2);
   lay->dq_acc = take(N * C * 4);
-  lay->attD = take(2 * N * d.H * 4);
+  lay->attD = take(N * d.H * 32);
   lay->ln_part = take((size_t)kLnBwdBlocks * 3 * C * 4);
   lay->col_part = take((size_t)kMaxStrips * 4 * C * 4);
   lay->norm_part = take(kNormBlocks * 8);
@@ -341,8 +341,8 @@ int attention_bwd(const bf16* qkv, const bf16* out, const bf16* dout, const floa
   if (T % 64) return GPT2_ERR_ARG;
   cudaError_t e;
   if (hd == 64 && T % attn_tc::bwd::BKEY == 0 && H <= attn_tc::bwd::kMaxHeads && err != nullptr) {
-    // Dv holds two [B, H, T] arrays here: -lse*log2(e) and -D*scale
-    e = attn_tc::bwd_run(qkv, out, dout, lse, Dv, Dv + (size_t)B * H * T, dq_acc, dqkv, B, T, H, err, s);
+    // Dv holds the 16-column per-query operand tiles here (32 bytes per query and head)
+    e = attn_tc::bwd_run(qkv, out, dout, lse, reinterpret_cast<uint8_t*>(Dv), dq_acc, dqkv, B, T, H, err, s);
   } else if (hd == 64) e = attn::bwd<64>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
   else if (hd == 32) e = attn::bwd<32>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
   else return GPT2_ERR_ARG;
@@ -1063,7 +1063,7 @@ int gpt2op_attention_fwd(const void* qkv, void* out, float* lse, int B, int T, i
 }
 
 size_t gpt2op_attention_bwd_workspace(int B, int T, int H, int hd) {
-  return (size_t)B * T * H * hd * 4 + 2 * (size_t)B * H * T * 4;
+  return (size_t)B * T * H * hd * 4 + (size_t)B * H * T * 32;
 }
 
 int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv, int B,

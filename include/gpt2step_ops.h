@@ -100,9 +100,9 @@ int gpt2op_attention_fwd(const void* qkv, void* out, float* lse, int B, int T, i
 
 /* Attention backward from the saved output and lse: dqkv bf16 [B,T,3C]. Head
  * size 64 with T % 128 == 0 (and H <= 64) runs on tcgen05, other shapes on
- * mma.sync. The workspace (fp32 dQ accumulator [B*T, C] followed by two fp32
- * [B, H, T] per-query arrays) must be 16-byte aligned; its contents on entry do
- * not matter. Concurrent calls must not share a workspace. */
+ * mma.sync. The workspace (fp32 dQ accumulator [B*T, C] followed by 32 bytes
+ * per query and head of per-query terms) must be 16-byte aligned; its contents
+ * on entry do not matter. Concurrent calls must not share a workspace. */
 size_t gpt2op_attention_bwd_workspace(int B, int T, int H, int hd);
 int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv, int B,
                          int T, int H, int hd, void* workspace, size_t ws_bytes, int* dev_err, void* stream);
