@@ -224,7 +224,8 @@ namespace launch {
 template <int C>
 void ln_fwd_c(const bf16* x, const float* w, const float* b, bf16* y, float* mean, float* rstd, int rows,
               cudaStream_t s) {
-  k::layernorm_fwd_kernel<C><<<(rows + 7) / 8, 256, 0, s>>>(x, w, b, y, mean, rstd, rows);
+  constexpr int rows_per_cta = 8 * k::kLnFwdRows;
+  k::layernorm_fwd_kernel<C><<<(rows + rows_per_cta - 1) / rows_per_cta, 256, 0, s>>>(x, w, b, y, mean, rstd, rows);
 }
 
 int ln_fwd(const bf16* x, const float* w, const float* b, bf16* y, float* mean, float* rstd, int rows, int C,

@@ -139,9 +139,11 @@ __global__ void embed_bwd_wte_kernel(const int32_t* __restrict__ tok, const bf16
 }
 
 // ---------------------------------------------------------------------------
-// a2/a6/a9  LayerNorm forward: one warp per row, fp32 statistics (eps 1e-5,
-// biased variance), y = (x - mean) * rstd * w + b in bf16.
+// a2/a6/a9  LayerNorm forward: one warp per LN_ROWS rows (all their loads in
+// flight before any arithmetic), fp32 statistics (eps 1e-5, biased variance),
+// y = (x - mean) * rstd * w + b in bf16.
 // ---------------------------------------------------------------------------
+constexpr int kLnFwdRows = 2;   // rows per warp
 template <int C>
 __global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restrict__ x, const float* __restrict__ w,
                                                             const float* __restrict__ b, bf16* __restrict__ y,
@@ -149,18 +151,28 @@ __global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restri
                                                             int rows) {
   constexpr int NV = C / 8;                 // 16-byte vectors per row
   constexpr int VPL = (NV + 31) / 32;       // vectors per lane
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  constexpr int R = kLnFwdRows;
+  const int row0 = (blockIdx.x * 8 + (threadIdx.x >> 5)) * R;
   const int l = lane_id();
-  if (row >= rows) return;
-  const bf16* xr = x + (size_t)row * C;
-  float v[VPL][8];
-  float s = 0.f;
+  if (row0 >= rows) return;
+  uint4 u[R][VPL];
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int vi = l + 32 * i;
-    if (vi < NV) {
-      const uint4 u = *reinterpret_cast<const uint4*>(xr + vi * 8);
-      const uint32_t wv[4] = {u.x, u.y, u.z, u.w};
+  for (int k = 0; k < R; ++k)
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = l + 32 * i;
+      u[k][i] = (vi < NV && row0 + k < rows) ? __ldcs(reinterpret_cast<const uint4*>(x + (size_t)(row0 + k) * C) + vi)
+                                              : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+  for (int k = 0; k < R; ++k) {
+    const int row = row0 + k;
+    if (row >= rows) break;
+    float v[VPL][8];
+    float s = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const uint32_t wv[4] = {u[k][i].x, u[k][i].y, u[k][i].z, u[k][i].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 f = unpack_bf16x2(wv[j]);
@@ -168,46 +180,43 @@ __global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restri
         v[i][2 * j + 1] = f.y;
         s += f.x + f.y;
       }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) v[i][j] = 0.f;
     }
-  }
-  const float mu = warp_sum(s) * (1.0f / C);
-  float ss = 0.f;
+    const float mu = warp_sum(s) * (1.0f / C);
+    float ss = 0.f;
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    if (l + 32 * i < NV) {
+    for (int i = 0; i < VPL; ++i) {
+      if (l + 32 * i < NV) {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float d = v[i][j] - mu;
-        ss += d * d;
+        for (int j = 0; j < 8; ++j) {
+          const float d = v[i][j] - mu;
+          ss += d * d;
+        }
       }
     }
-  }
-  const float rs = rsqrtf(warp_sum(ss) * (1.0f / C) + 1e-5f);
-  bf16* yr = y + (size_t)row * C;
+    const float rs = rsqrtf(warp_sum(ss) * (1.0f / C) + 1e-5f);
+    bf16* yr = y + (size_t)row * C;
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int vi = l + 32 * i;
-    if (vi < NV) {
-      const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + vi * 8));
-      const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + vi * 8 + 4));
-      const float4 b0 = __ldg(reinterpret_cast<const float4*>(b + vi * 8));
-      const float4 b1 = __ldg(reinterpret_cast<const float4*>(b + vi * 8 + 4));
-      const float ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-      const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-      uint32_t o[4];
+    for (int i = 0; i < VPL; ++i) {
+      const int vi = l + 32 * i;
+      if (vi < NV) {
+        const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + vi * 8));
+        const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + vi * 8 + 4));
+        const float4 b0 = __ldg(reinterpret_cast<const float4*>(b + vi * 8));
+        const float4 b1 = __ldg(reinterpret_cast<const float4*>(b + vi * 8 + 4));
+        const float ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+        const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        uint32_t o[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j)
-        o[j] = pack_bf16x2((v[i][2 * j] - mu) * rs * ww[2 * j] + bb[2 * j],
-                           (v[i][2 * j + 1] - mu) * rs * ww[2 * j + 1] + bb[2 * j + 1]);
-      *reinterpret_cast<uint4*>(yr + vi * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int j = 0; j < 4; ++j)
+          o[j] = pack_bf16x2((v[i][2 * j] - mu) * rs * ww[2 * j] + bb[2 * j],
+                             (v[i][2 * j + 1] - mu) * rs * ww[2 * j + 1] + bb[2 * j + 1]);
+        *reinterpret_cast<uint4*>(yr + vi * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
     }
-  }
-  if (l == 0) {
-    mean[row] = mu;
-    rstd[row] = rs;
+    if (l == 0) {
+      mean[row] = mu;
+      rstd[row] = rs;
+    }
   }
 }
 
@@ -467,36 +476,48 @@ __global__ void colsum_final_kernel(const float* __restrict__ part, float* __res
 // j < V and exactly 0 for the padded columns j >= V ("Pretraining and adapting
 // a language model on a dependency-free stack", §4.1). loss = lse - z[target].
 // ---------------------------------------------------------------------------
+constexpr float kLog2eF = 1.4426950408889634f, kLn2F = 0.6931471805599453f;
 constexpr int kCeThreads = 256;
 constexpr int kCeUnroll = 4;
 
-// Online (max, sum of exp) update with the real columns of one 8-wide vector.
-GPT2_DEV void ce_accumulate(uint4 u, int col0, int V, float& m, float& s) {
+// Base-2 online softmax: logits are scaled by log2(e) once (y = z * log2e), so
+// every exponential is one ex2 of an FFMA. Only the row's last 8-wide chunks can
+// hold padded ids (>= V); full chunks skip the per-element column test.
+GPT2_DEV void bf16x8_to_f32(uint4 u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-  float f[8];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    const float2 t = unpack_bf16x2(w[j]);
-    f[2 * j] = t.x;
-    f[2 * j + 1] = t.y;
+    f[2 * j] = __uint_as_float(w[j] << 16);
+    f[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
   }
+}
+
+// Online (max, sum of 2^(y - max)) over the real columns of one chunk, in log2 units.
+GPT2_DEV void ce_accumulate(uint4 u, int col0, int V, float& m, float& s) {
+  float f[8];
+  bf16x8_to_f32(u, f);
+  const bool full = col0 + 8 <= V;
   float lm = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < 8; ++j)
-    if (col0 + j < V) lm = fmaxf(lm, f[j]);
+  for (int j = 0; j < 8; ++j) {
+    f[j] *= kLog2eF;
+    if (full || col0 + j < V) lm = fmaxf(lm, f[j]);
+  }
   if (lm == -INFINITY) return;
-  const float nm = fmaxf(m, lm);
+  if (lm > m) {
+    s *= ex2_approx(m - lm);
+    m = lm;
+  }
   float acc = 0.f;
 #pragma unroll
   for (int j = 0; j < 8; ++j)
-    if (col0 + j < V) acc += __expf(f[j] - nm);
-  s = s * __expf(m - nm) + acc;
-  m = nm;
+    if (full || col0 + j < V) acc += ex2_approx(f[j] - m);
+  s += acc;
 }
 
 GPT2_DEV void ce_combine(float& m, float& s, float om, float os) {
   const float nm = fmaxf(m, om);
-  s = (nm == -INFINITY) ? 0.f : s * __expf(m - nm) + os * __expf(om - nm);
+  s = (nm == -INFINITY) ? 0.f : s * ex2_approx(m - nm) + os * ex2_approx(om - nm);
   m = nm;
 }
 
@@ -542,7 +563,8 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
     if (l == 0) { bc[0] = m; bc[1] = s; }
   }
   __syncthreads();
-  const float M = bc[0], inv = 1.0f / bc[1];
+  const float M2 = bc[0];                      // row max in log2 units
+  const float S2 = bc[1];                      // sum of 2^(y - M2)
   int t = targets[row];
   const bool tok_ok = (t >= 0 && t < V);
   if (!tok_ok) {
@@ -550,11 +572,13 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
     t = -1;
   }
   if (threadIdx.x == 0) {
+    // loss = lse - z[t] = (M2 + log2 S2) * ln2 - z[t]
     const float zt = tok_ok ? __bfloat162float(logits[(size_t)row * Vp + t]) : 0.f;
-    losses[row] = tok_ok ? (M + logf(bc[1]) - zt) : 0.f;
+    losses[row] = tok_ok ? ((M2 + log2f(S2)) * kLn2F - zt) : 0.f;
   }
   if (!write_grad) return;
   __syncthreads();  // the target logit is read before the row is overwritten
+  const float g = dscale / S2;                 // dz = (2^(y - M2) / S2 - [col == t]) * dscale
   for (int i0 = threadIdx.x; i0 < nv; i0 += kCeThreads * kCeUnroll) {
     uint4 u[kCeUnroll];
 #pragma unroll
@@ -566,18 +590,20 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
     for (int k2 = 0; k2 < kCeUnroll; ++k2) {
       const int i = i0 + k2 * kCeThreads;
       if (i >= nv) continue;
-      const uint32_t w[4] = {u[k2].x, u[k2].y, u[k2].z, u[k2].w};
-      uint32_t o[4];
+      const int c0 = i * 8;
+      float f[8];
+      bf16x8_to_f32(u[k2], f);
+      float gv[8];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = unpack_bf16x2(w[j]);
-        const int c0 = i * 8 + 2 * j;
-        float g0 = 0.f, g1 = 0.f;
-        if (c0 < V) g0 = (__expf(f.x - M) * inv - (c0 == t ? 1.f : 0.f)) * dscale;
-        if (c0 + 1 < V) g1 = (__expf(f.y - M) * inv - (c0 + 1 == t ? 1.f : 0.f)) * dscale;
-        o[j] = pack_bf16x2(g0, g1);
+      for (int j = 0; j < 8; ++j) gv[j] = ex2_approx(fmaf(f[j], kLog2eF, -M2)) * g;
+      if (c0 + 8 > V) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (c0 + j >= V) gv[j] = 0.f;       // padded ids: exactly zero gradient
       }
-      __stcs(zr + i, make_uint4(o[0], o[1], o[2], o[3]));
+      if ((unsigned)(t - c0) < 8u) gv[t - c0] -= dscale;
+      __stcs(zr + i, make_uint4(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]), pack_bf16x2(gv[4], gv[5]),
+                                pack_bf16x2(gv[6], gv[7])));
     }
   }
 }
