@@ -358,9 +358,12 @@ static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int
 //                     Jacobian term); writes -lse/scale and -D, each as a bf16
 //                     hi + lo pair, into a 16-column operand tile per query block
 //                     (see below); clears the fp32 dQ accumulator.
-//   attn_bwd_tc_kernel  per CTA one (batch, head) and a block of 128 keys; walks
-//                     the query blocks at or after it (causal). With K, V resident
-//                     and Q_i, dO_i streamed through a three-deep ring:
+//   attn_bwd_tc_kernel  persistent, one CTA per SM; a work item is one (batch,
+//                     head) and a block of 128 keys, which walks the query blocks
+//                     at or after it (causal). The next item's K, V load as soon as
+//                     the last product of the current one has read them, so one
+//                     item's epilogue overlaps the next one's first loads. With
+//                     K, V resident and Q_i, dO_i streamed through a three-deep ring:
 //       S'^T  = [K | 1 1 0..] [Q_i | X_i]^T   = S^T - lse/scale  (M=128 keys, N=128 queries,
 //       dP'^T = [V | 0 0 1 1 0..] [dO_i | X_i]^T = dP^T - D       K = 64 + one 16-wide step)
 //       P^T  = exp2(S'^T * scale*log2e)       (softmax warps, one key row each)
@@ -530,7 +533,7 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
                        const __grid_constant__ CUtensorMap tm_dq, const uint8_t* __restrict__ xtiles,
-                       bf16* __restrict__ dqkv, int T, int H, float scale, int* err) {
+                       bf16* __restrict__ dqkv, int T, int H, int BH, float scale, int* err) {
   using namespace bwd;
   extern __shared__ __align__(1024) uint8_t smem_raw_ab[];
   uint8_t* smem =
@@ -546,31 +549,32 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   uint8_t* sXV = sXK + XT_BYTES;                    // V' extra columns: 0 0 1 1 0 ..
   uint64_t* bars = reinterpret_cast<uint64_t*>(sXV + XT_BYTES);
   uint64_t* kv_full = bars;
-  uint64_t* qdo_full = bars + 1;          // [NQS]
-  uint64_t* qdo_empty = bars + 1 + NQS;   // [NQS]
-  uint64_t* st_full = bars + 1 + 2 * NQS;
+  uint64_t* kv_empty = bars + 1;
+  uint64_t* qdo_full = bars + 2;          // [NQS]
+  uint64_t* qdo_empty = bars + 2 + NQS;   // [NQS]
+  uint64_t* st_full = bars + 2 + 2 * NQS;
   uint64_t* st_empty = st_full + 1;
   uint64_t* ds_full = st_full + 2;
   uint64_t* ds_empty = st_full + 3;
   uint64_t* dq_full = st_full + 4;
   uint64_t* dq_empty = st_full + 5;
   uint64_t* dkdv_full = st_full + 6;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(st_full + 7);
+  uint64_t* dkdv_empty = st_full + 7;
+  uint64_t* done = st_full + 8;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(st_full + 9);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nb = T / BKEY;
-  // heaviest key blocks (kb = 0: every query block) are scheduled first
-  const int BH = gridDim.y;
-  const int lin = blockIdx.y * gridDim.x + blockIdx.x;
-  const int kb = lin / BH;
-  const int bh = lin % BH;
-  const int b = bh / H, h = bh % H;
   const int C = H * HD;
-  const int row_base = b * T;
-  const int nit = nb - kb;                 // query blocks kb .. nb-1
+  // Persistent: this CTA takes work items blockIdx.x, blockIdx.x + gridDim.x, ..
+  // of the nb * BH (key block, batch-head) items; heaviest key blocks (kb = 0:
+  // every query block) come first. Barrier phases run over g, the CTA's count of
+  // query blocks processed, and over j, its count of items.
+  const int n_items = nb * BH;
 
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(kv_full), 1);
+    mbar_init(smem_u32(kv_empty), 1);
     for (int i = 0; i < NQS; ++i) {
       mbar_init(smem_u32(&qdo_full[i]), 1);
       mbar_init(smem_u32(&qdo_empty[i]), 1);
@@ -582,6 +586,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     mbar_init(smem_u32(dq_full), 1);
     mbar_init(smem_u32(dq_empty), kSoftmaxWarps);
     mbar_init(smem_u32(dkdv_full), 1);
+    mbar_init(smem_u32(dkdv_empty), kSoftmaxWarps);
+    mbar_init(smem_u32(done), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tm_qkv);
     tma_prefetch_desc(&tm_do);
@@ -609,18 +615,31 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     if (warp == 0) {
       // -------------------------------------------------------------- TMA producer
       if (lane == 0) {
-        mbar_arrive_expect_tx(smem_u32(kv_full), 2 * T_BYTES);
-        tma_load_2d(smem_u32(sK), &tm_qkv, smem_u32(kv_full), C + h * HD, row_base + kb * BKEY);
-        tma_load_2d(smem_u32(sV), &tm_qkv, smem_u32(kv_full), 2 * C + h * HD, row_base + kb * BKEY);
-        const uint8_t* x_b = xtiles + (size_t)bh * (T / BQRY) * XT_BYTES;
-        for (int it = 0; it < nit; ++it) {
-          const int s = it % NQS, u = it / NQS, qi = kb + it;
-          if (!mbar_wait(smem_u32(&qdo_empty[s]), (u & 1) ^ 1, err)) break;
+        bool ok = true;
+        int g = 0;
+        auto load_qdo = [&](int gq, int bh, int row_base, int h, int qi) -> bool {
+          const int s = gq % NQS, u = gq / NQS;
+          if (!mbar_wait(smem_u32(&qdo_empty[s]), (u & 1) ^ 1, err)) return false;
           const uint32_t fb = smem_u32(&qdo_full[s]);
           mbar_arrive_expect_tx(fb, 2 * T_BYTES + XT_BYTES);
           tma_load_2d(smem_u32(sQ + s * T_BYTES), &tm_qkv, fb, h * HD, row_base + qi * BQRY);
           tma_load_2d(smem_u32(sDO + s * T_BYTES), &tm_do, fb, h * HD, row_base + qi * BQRY);
-          bulk_load_1d(smem_u32(sXQ + s * XT_BYTES), x_b + (size_t)qi * XT_BYTES, XT_BYTES, fb);
+          bulk_load_1d(smem_u32(sXQ + s * XT_BYTES), xtiles + ((size_t)bh * nb + qi) * XT_BYTES, XT_BYTES, fb);
+          return true;
+        };
+        for (int i = blockIdx.x, j = 0; i < n_items && ok; i += gridDim.x, ++j) {
+          const int kb = i / BH, bh = i % BH, b = bh / H, h = bh % H;
+          const int row_base = b * T, nit = nb - kb;
+          // the first query block of this item may land before its keys
+          ok = load_qdo(g, bh, row_base, h, kb);
+          // K, V once the previous item's products no longer read them
+          if (ok && j > 0 && !mbar_wait(smem_u32(kv_empty), (j - 1) & 1, err)) ok = false;
+          if (!ok) break;
+          mbar_arrive_expect_tx(smem_u32(kv_full), 2 * T_BYTES);
+          tma_load_2d(smem_u32(sK), &tm_qkv, smem_u32(kv_full), C + h * HD, row_base + kb * BKEY);
+          tma_load_2d(smem_u32(sV), &tm_qkv, smem_u32(kv_full), 2 * C + h * HD, row_base + kb * BKEY);
+          for (int it = 1; it < nit && ok; ++it) ok = load_qdo(g + it, bh, row_base, h, kb + it);
+          g += nit;
         }
       }
     } else if (warp == 1) {
@@ -640,14 +659,14 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         const uint64_t dQ0_mn = smem_desc_sw128(smem_u32(sQ), 8192, 1024);
         const uint64_t dO0_k = smem_desc_sw128(smem_u32(sDO), 16, 1024);
         const uint64_t dO0_mn = smem_desc_sw128(smem_u32(sDO), 8192, 1024);
-      const uint64_t dXK = smem_desc_interleave(smem_u32(sXK), 128, 256);
-      const uint64_t dXV = smem_desc_interleave(smem_u32(sXV), 128, 256);
-      const uint64_t dXQ0 = smem_desc_interleave(smem_u32(sXQ), 128, 256);
-      constexpr uint64_t kXStage = XT_BYTES >> 4;
+        const uint64_t dXK = smem_desc_interleave(smem_u32(sXK), 128, 256);
+        const uint64_t dXV = smem_desc_interleave(smem_u32(sXV), 128, 256);
+        const uint64_t dXQ0 = smem_desc_interleave(smem_u32(sXQ), 128, 256);
+        constexpr uint64_t kXStage = XT_BYTES >> 4;
         constexpr uint64_t kStage = T_BYTES >> 4;   // one Q/dO stage, in descriptor units
-        auto issue_st = [&](int it) {
-          const uint64_t so = (uint64_t)(it % NQS) * kStage;
-          const uint64_t sx = (uint64_t)(it % NQS) * kXStage;
+        auto issue_st = [&](int gq) {
+          const uint64_t so = (uint64_t)(gq % NQS) * kStage;
+          const uint64_t sx = (uint64_t)(gq % NQS) * kXStage;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
             tc_mma_bf16(tmem + C_S, dK_k + kk * 2, dQ0_k + so + kk * 2, id_st, kk > 0 ? 1u : 0u);
@@ -658,44 +677,55 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           tc_mma_bf16(tmem + C_DP, dXV, dXQ0 + sx, id_st, 1u);
           tc_commit(smem_u32(st_full));
         };
-        bool ok = mbar_wait(smem_u32(kv_full), 0, err) && mbar_wait(smem_u32(&qdo_full[0]), 0, err);
-        if (ok) {
+        bool ok = true;
+        int g = 0;
+        for (int i = blockIdx.x, j = 0; i < n_items && ok; i += gridDim.x, ++j) {
+          const int nit = nb - i / BH;
+          // this item's keys, its first query block, and the previous scores out of TMEM
+          if (!mbar_wait(smem_u32(kv_full), j & 1, err)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&qdo_full[g % NQS]), (g / NQS) & 1, err)) { ok = false; break; }
+          if (g > 0 && !mbar_wait(smem_u32(st_empty), (g - 1) & 1, err)) { ok = false; break; }
           tc_fence_after();
-          issue_st(0);
-        }
-        for (int it = 0; it < nit && ok; ++it) {
-          const int s = it % NQS;
-          const uint64_t so = (uint64_t)s * kStage;
-          if (it + 1 < nit) {
-            // block it+1's scores, once its Q/dO landed and block it's scores left TMEM
-            if (!mbar_wait(smem_u32(&qdo_full[(it + 1) % NQS]), ((it + 1) / NQS) & 1, err)) { ok = false; break; }
-            if (!mbar_wait(smem_u32(st_empty), it & 1, err)) { ok = false; break; }
+          issue_st(g);
+          for (int it = 0; it < nit && ok; ++it) {
+            const int gc = g + it;
+            const uint64_t so = (uint64_t)(gc % NQS) * kStage;
+            if (it + 1 < nit) {
+              // block it+1's scores, once its Q/dO landed and block it's scores left TMEM
+              if (!mbar_wait(smem_u32(&qdo_full[(gc + 1) % NQS]), ((gc + 1) / NQS) & 1, err)) { ok = false; break; }
+              if (!mbar_wait(smem_u32(st_empty), gc & 1, err)) { ok = false; break; }
+              tc_fence_after();
+              issue_st(gc + 1);
+            }
+            // P^T (tensor memory) and dS^T (shared memory) of block it are written
+            if (!mbar_wait(smem_u32(ds_full), gc & 1, err)) { ok = false; break; }
+            // the previous item's dK, dV have left tensor memory
+            if (it == 0 && j > 0 && !mbar_wait(smem_u32(dkdv_empty), (j - 1) & 1, err)) { ok = false; break; }
             tc_fence_after();
-            issue_st(it + 1);
-          }
-          // P^T (tensor memory) and dS^T (shared memory) of block it are written
-          if (!mbar_wait(smem_u32(ds_full), it & 1, err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t acc0 = it > 0 ? 1u : 0u;
+            const uint32_t acc0 = it > 0 ? 1u : 0u;
 #pragma unroll
-          for (int kk = 0; kk < BQRY / 16; ++kk) {
-            const uint32_t aoff = ((kk >> 2) * (BKEY * 128) + (kk & 3) * 32) >> 4;
-            tc_mma_bf16_ts(tmem + C_DV, tmem + C_P + kk * 8, dO0_mn + so + kk * 128, id_kv, kk > 0 ? 1u : acc0);
-            tc_mma_bf16(tmem + C_DK, dDS_k + aoff, dQ0_mn + so + kk * 128, id_kv, kk > 0 ? 1u : acc0);
-          }
-          // dQ_it once dQ_{it-1} has left tensor memory
-          if (it > 0 && !mbar_wait(smem_u32(dq_empty), (it - 1) & 1, err)) { ok = false; break; }
-          tc_fence_after();
+            for (int kk = 0; kk < BQRY / 16; ++kk) {
+              const uint32_t aoff = ((kk >> 2) * (BKEY * 128) + (kk & 3) * 32) >> 4;
+              tc_mma_bf16_ts(tmem + C_DV, tmem + C_P + kk * 8, dO0_mn + so + kk * 128, id_kv, kk > 0 ? 1u : acc0);
+              tc_mma_bf16(tmem + C_DK, dDS_k + aoff, dQ0_mn + so + kk * 128, id_kv, kk > 0 ? 1u : acc0);
+            }
+            // dQ of this block once the previous block's dQ has left tensor memory
+            if (gc > 0 && !mbar_wait(smem_u32(dq_empty), (gc - 1) & 1, err)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < BKEY / 16; ++kk)
-            tc_mma_bf16(tmem + C_DQ, dDS_mn + kk * 128, dK_mn + kk * 128, id_q, kk > 0 ? 1u : 0u);
-          tc_commit(smem_u32(dq_full));
-          tc_commit(smem_u32(ds_empty));
-          tc_commit(smem_u32(&qdo_empty[s]));
+            for (int kk = 0; kk < BKEY / 16; ++kk)
+              tc_mma_bf16(tmem + C_DQ, dDS_mn + kk * 128, dK_mn + kk * 128, id_q, kk > 0 ? 1u : 0u);
+            tc_commit(smem_u32(dq_full));
+            tc_commit(smem_u32(ds_empty));
+            tc_commit(smem_u32(&qdo_empty[gc % NQS]));
+          }
+          tc_commit(smem_u32(dkdv_full));   // this item's dK, dV are complete
+          tc_commit(smem_u32(kv_empty));    // and its K, V are no longer read
+          g += nit;
         }
-        tc_commit(smem_u32(dkdv_full));
         // every product has completed before the block releases tensor memory
-        mbar_wait(smem_u32(dkdv_full), 0, err);
+        tc_commit(smem_u32(done));
+        mbar_wait(smem_u32(done), 0, err);
       }
     }
   } else {
@@ -707,10 +737,10 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * kLog2e;
     uint8_t* stage = sDQW + wi * DQW_BYTES;
-    // dQ of query block jt: this warp's 32 query rows x 32 columns -> staging box ->
-    // bulk reduce-add into the accumulator
-    auto drain_dq = [&](int jt) -> bool {
-      if (!mbar_wait(smem_u32(dq_full), jt & 1, err)) return false;
+    // dQ of query block gq (rows qrow0.., columns hc..): this warp's 32 query rows
+    // x 32 columns -> staging box -> bulk reduce-add into the accumulator
+    auto drain_dq = [&](int gq, int hc, int qrow0) -> bool {
+      if (!mbar_wait(smem_u32(dq_full), gq & 1, err)) return false;
       tc_fence_after();
       float v[32];
       tmem_ld32(tmem + lane_off + C_DQ + hf * 32, v);
@@ -728,66 +758,81 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_reduce_add_2d(&tm_dq, smem_u32(stage), h * HD + hf * 32, row_base + (kb + jt) * BQRY + q4 * 32);
+        tma_reduce_add_2d(&tm_dq, smem_u32(stage), hc + hf * 32, qrow0 + q4 * 32);
         bulk_commit_group();
       }
       return true;
     };
     bool ok = true;
-    for (int it = 0; it < nit && ok; ++it) {
-      if (!mbar_wait(smem_u32(st_full), it & 1, err)) { ok = false; break; }
-      tc_fence_after();
-      // this thread's 64 query columns of S^T and dP^T; tensor memory is free again at once
-      uint32_t sv[2][32], dv[2][32];
+    int g = 0;
+    int prev_hc = 0, prev_qrow0 = 0;   // where the previous block's dQ goes
+    for (int i = blockIdx.x, j = 0; i < n_items && ok; i += gridDim.x, ++j) {
+      const int kb = i / BH, bh = i % BH, b = bh / H, h = bh % H;
+      const int row_base = b * T, nit = nb - kb;
+      for (int it = 0; it < nit && ok; ++it) {
+        const int gc = g + it;
+        if (!mbar_wait(smem_u32(st_full), gc & 1, err)) { ok = false; break; }
+        tc_fence_after();
+        // this thread's 64 query columns of S'^T and dP'^T; tensor memory is free again at once
+        uint32_t sv[2][32], dv[2][32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        tmem_ld32_async(tmem + lane_off + C_S + hf * 64 + c * 32, sv[c]);
-        tmem_ld32_async(tmem + lane_off + C_DP + hf * 64 + c * 32, dv[c]);
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(st_empty));
-      uint32_t pp[32], pd[32];
-      if (it == 0) bwd_softmax_row<true>(sv, dv, sl2, scale, r, hf * 64, pp, pd);
-      else bwd_softmax_row<false>(sv, dv, sl2, scale, r, hf * 64, pp, pd);
-      // P^T (TMEM) and dS^T (smem) were last read by the products of block it-1
-      if (it > 0 && !mbar_wait(smem_u32(ds_empty), (it - 1) & 1, err)) { ok = false; break; }
-      tc_fence_after();
-      tmem_st32_u(tmem + lane_off + C_P + hf * 32, pp);
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32_async(tmem + lane_off + C_S + hf * 64 + c * 32, sv[c]);
+          tmem_ld32_async(tmem + lane_off + C_DP + hf * 64 + c * 32, dv[c]);
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(st_empty));
+        uint32_t pp[32], pd[32];
+        if (it == 0) bwd_softmax_row<true>(sv, dv, sl2, scale, r, hf * 64, pp, pd);
+        else bwd_softmax_row<false>(sv, dv, sl2, scale, r, hf * 64, pp, pd);
+        // P^T (TMEM) and dS^T (smem) were last read by the products of the previous block
+        if (gc > 0 && !mbar_wait(smem_u32(ds_empty), (gc - 1) & 1, err)) { ok = false; break; }
+        tc_fence_after();
+        tmem_st32_u(tmem + lane_off + C_P + hf * 32, pp);
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        const int off = hf * (BKEY * 128) + r * 128 + ((ch ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(sDST + off) = make_uint4(pd[4 * ch], pd[4 * ch + 1], pd[4 * ch + 2], pd[4 * ch + 3]);
+        for (int ch = 0; ch < 8; ++ch) {
+          const int off = hf * (BKEY * 128) + r * 128 + ((ch ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(sDST + off) = make_uint4(pd[4 * ch], pd[4 * ch + 1], pd[4 * ch + 2], pd[4 * ch + 3]);
+        }
+        tmem_wait_st();
+        fence_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(ds_full));
+        // while the products of this block run, move the previous block's dQ out
+        if (gc > 0 && !drain_dq(gc - 1, prev_hc, prev_qrow0)) { ok = false; break; }
+        prev_hc = h * HD;
+        prev_qrow0 = row_base + (kb + it) * BQRY;
       }
-      tmem_wait_st();
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(ds_full));
-      // while the products of block it run, move dQ of block it-1 out
-      if (it > 0 && !drain_dq(it - 1)) { ok = false; break; }
-    }
-    if (ok && nit > 0) ok = drain_dq(nit - 1);
-    if (lane == 0) bulk_wait_group<0>();
-    __syncwarp();
-    // dK, dV for key row r, head-dim columns 32 hf ..
-    if (ok && mbar_wait(smem_u32(dkdv_full), 0, err)) {
+      if (!ok) break;
+      g += nit;
+      // dK, dV of this item for key row r, head-dim columns 32 hf ..
+      if (!mbar_wait(smem_u32(dkdv_full), j & 1, err)) { ok = false; break; }
       tc_fence_after();
       bf16* krow = dqkv + ((size_t)(row_base + kb * BKEY + r)) * 3 * C + C + h * HD + hf * 32;
       bf16* vrow = krow + C;
       float v[32];
       tmem_ld32(tmem + lane_off + C_DK + hf * 32, v);
 #pragma unroll
-      for (int i = 0; i < 32; i += 8)
-        *reinterpret_cast<uint4*>(krow + i) = make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
-                                                         pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
+      for (int i2 = 0; i2 < 32; i2 += 8)
+        *reinterpret_cast<uint4*>(krow + i2) =
+            make_uint4(pack_bf16x2(v[i2], v[i2 + 1]), pack_bf16x2(v[i2 + 2], v[i2 + 3]),
+                       pack_bf16x2(v[i2 + 4], v[i2 + 5]), pack_bf16x2(v[i2 + 6], v[i2 + 7]));
       tmem_ld32(tmem + lane_off + C_DV + hf * 32, v);
 #pragma unroll
-      for (int i = 0; i < 32; i += 8)
-        *reinterpret_cast<uint4*>(vrow + i) = make_uint4(pack_bf16x2(v[i], v[i + 1]), pack_bf16x2(v[i + 2], v[i + 3]),
-                                                         pack_bf16x2(v[i + 4], v[i + 5]), pack_bf16x2(v[i + 6], v[i + 7]));
+      for (int i2 = 0; i2 < 32; i2 += 8)
+        *reinterpret_cast<uint4*>(vrow + i2) =
+            make_uint4(pack_bf16x2(v[i2], v[i2 + 1]), pack_bf16x2(v[i2 + 2], v[i2 + 3]),
+                       pack_bf16x2(v[i2 + 4], v[i2 + 5]), pack_bf16x2(v[i2 + 6], v[i2 + 7]));
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(dkdv_empty));
     }
+    if (ok && g > 0) ok = drain_dq(g - 1, prev_hc, prev_qrow0);
+    if (lane == 0) bulk_wait_group<0>();
+    __syncwarp();
   }
   tc_fence_before();
   __syncthreads();
@@ -825,8 +870,16 @@ static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, c
                      32, 32, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   bwd_prep_kernel<<<B * T / bwd::kPrepRows, 256, 0, s>>>(out, dout, lse, xtiles, dq_acc, T, H, scale);
-  dim3 grid(T / bwd::BKEY, B * H);
-  attn_bwd_tc_kernel<<<grid, bwd::kThreads, bwd::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, xtiles, dqkv, T, H, scale,
+  const int n_items = (T / bwd::BKEY) * B * H;
+  static int sms = 0;   // one persistent CTA per SM
+  if (sms == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return cudaErrorInvalidValue;
+    sms = v;
+  }
+  const int grid = n_items < sms ? n_items : sms;
+  attn_bwd_tc_kernel<<<grid, bwd::kThreads, bwd::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, xtiles, dqkv, T, H, B * H, scale,
                                                                   err);
   const int n = B * T * (C / 8);
   int blocks = (n + 255) / 256;
