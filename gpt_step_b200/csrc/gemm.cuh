@@ -43,6 +43,7 @@ struct Params {
   int M, N, K;
   int num_m, num_n, splits, kb_per_split, nkb, num_tiles;
   int raster_gm;  // row tiles per raster panel (pair kernel); num_m = plain row-major order
+  float* colsum;  // pair kernel, EPI_DGELU: column sums of the (bf16) output added here, or null
   bf16* out;
   bf16* out2;
   int ldo;
@@ -389,6 +390,7 @@ struct Call {
   int* err;
   int force_bn;      // 0: automatic
   int force_splits;  // 0: automatic
+  float* colsum;     // EPI_DGELU with >= 256 rows: add the output's column sums here (else null)
 };
 
 // Tile width: whole waves of 148 SMs, with 128-wide tiles charged 1.3x because a

@@ -335,6 +335,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+        if (EPI == gemm::EPI_DGELU && p.colsum != nullptr) {
+          // column sums of the stored (bf16) values over this warp's 32 rows: a
+          // transpose-reduce leaves column `lane` of the chunk in cs[0]
+          float cs[32];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 f = unpack_bf16x2(pk[i]);
+            cs[2 * i] = row_ok ? f.x : 0.f;
+            cs[2 * i + 1] = row_ok ? f.y : 0.f;
+          }
+#pragma unroll
+          for (int k = 16; k >= 1; k >>= 1) {
+            const bool upper = (lane & k) != 0;
+#pragma unroll
+            for (int i = 0; i < k; ++i) {
+              const float send = upper ? cs[i] : cs[i + k];
+              const float keep = upper ? cs[i + k] : cs[i];
+              cs[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+            }
+          }
+          atomicAdd(p.colsum + n + lane, cs[0]);
+        }
         // single-output epilogues alternate two buffers; GELU has one per output
         const uint32_t b = EPI == gemm::EPI_GELU ? 0u : (nstore & 1);
         if (lane == 0) {
@@ -402,12 +424,21 @@ namespace gemm2 {
 // on outputs 768 wide).
 constexpr int kRasterRows = 16, kRasterRowsWgrad = 8;
 
+// Whether run() takes the pair kernel for this call (the only one with fused
+// column sums).
+static bool uses_pair(const gemm::Call& c) {
+  using namespace gemm;
+  const int BN = (c.kind == WGRAD && !c.force_bn && c.N % 256 == 0) ? 256 : choose_bn(c);
+  return BN == 256 && c.M >= BM_PAIR && c.force_bn != 128;
+}
+
 static int run(const gemm::Call& c, cudaStream_t s) {
   using namespace gemm;
   if (c.M <= 0 || c.N <= 0 || c.K <= 0) return GPT2_ERR_ARG;
   if (c.N % 32 || c.K % BK) return GPT2_ERR_ARG;
   const int BN = (c.kind == WGRAD && !c.force_bn && c.N % 256 == 0) ? 256 : choose_bn(c);
   const bool pair = (BN == 256) && c.M >= BM_PAIR && c.force_bn != 128;
+  if (!pair && c.colsum) return GPT2_ERR_ARG;   // fused column sums need the pair kernel
   if (!pair) return gemm::run(c, s);
   Params p{};
   p.M = c.M; p.N = c.N; p.K = c.K;
@@ -435,6 +466,7 @@ static int run(const gemm::Call& c, cudaStream_t s) {
   p.splits = (p.nkb + p.kb_per_split - 1) / p.kb_per_split;
   p.num_tiles = p.num_m * p.num_n * p.splits;
   p.raster_gm = std::min(p.num_m, c.kind == WGRAD ? kRasterRowsWgrad : kRasterRows);
+  p.colsum = c.epi == EPI_DGELU ? c.colsum : nullptr;
   p.out = c.out; p.out2 = c.out2; p.ldo = c.ldo;
   p.aux = c.aux; p.ld_aux = c.ld_aux; p.bias = c.bias;
   p.outf = c.outf; p.ldf = c.ldf; p.err = c.err;

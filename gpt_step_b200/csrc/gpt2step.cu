@@ -555,6 +555,7 @@ int backward(gpt2_model* m, const int32_t* tok) {
     bf16* fchg = m->at<bf16>(y.fchg) + l * NC * 4;
     float* lse = m->at<float>(y.lse) + (size_t)l * d.N * d.H;
 
+    bool fused_fcb = false;   // fc bias gradient summed in the d4c epilogue
     // MLP projection
     {
       gemm::Call c = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, C, 4 * C, N, err);
@@ -565,6 +566,10 @@ int backward(gpt2_model* m, const int32_t* tok) {
       gemm::Call c = gemm_call(gemm::DGRAD, gemm::EPI_DGELU, N, 4 * C, C, err);
       c.a = dresid; c.lda = C; c.b = m->W(K_FCPROJW, l); c.ldb = 4 * C; c.out = d4c; c.ldo = 4 * C;
       c.aux = fch; c.ld_aux = 4 * C;
+      // the MLP fc bias gradient is the column sum of d4c, added in the epilogue
+      c.colsum = m->G(K_FCB, l);
+      fused_fcb = gemm2::uses_pair(c);
+      if (!fused_fcb) c.colsum = nullptr;
       GPT2_TRY(run_gemm(m, c));
     }
     // MLP fc
@@ -573,7 +578,7 @@ int backward(gpt2_model* m, const int32_t* tok) {
       c.a = d4c; c.lda = 4 * C; c.b = ln2; c.ldb = C; c.outf = m->G(K_FCW, l); c.ldf = C;
       GPT2_TRY(run_gemm(m, c));
     }
-    GPT2_TRY(bias_grad_m(m, d4c, m->G(K_FCB, l), N, 4 * C));
+    if (!fused_fcb) GPT2_TRY(bias_grad_m(m, d4c, m->G(K_FCB, l), N, 4 * C));
     {
       gemm::Call c = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, 4 * C, err);
       c.a = d4c; c.lda = 4 * C; c.b = m->W(K_FCW, l); c.ldb = C; c.out = dln; c.ldo = C;
