@@ -215,6 +215,21 @@ GPT2_DEV float2 unpack_bf16x2(uint32_t u) {
   return __bfloat1622float2(h);
 }
 
+// Column sums over a warp's 32 rows: lane l holds row l's 32 values in cs[];
+// after a transpose-reduce (31 shuffles) cs[0] of lane l is the sum of column l.
+GPT2_DEV void warp_colsum32(float (&cs)[32], int lane) {
+#pragma unroll
+  for (int k = 16; k >= 1; k >>= 1) {
+    const bool upper = (lane & k) != 0;
+#pragma unroll
+    for (int i = 0; i < k; ++i) {
+      const float send = upper ? cs[i] : cs[i + k];
+      const float keep = upper ? cs[i + k] : cs[i];
+      cs[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
+    }
+  }
+}
+
 GPT2_DEV float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -345,16 +345,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             cs[2 * i] = row_ok ? f.x : 0.f;
             cs[2 * i + 1] = row_ok ? f.y : 0.f;
           }
-#pragma unroll
-          for (int k = 16; k >= 1; k >>= 1) {
-            const bool upper = (lane & k) != 0;
-#pragma unroll
-            for (int i = 0; i < k; ++i) {
-              const float send = upper ? cs[i] : cs[i + k];
-              const float keep = upper ? cs[i + k] : cs[i];
-              cs[i] = keep + __shfl_xor_sync(0xffffffffu, send, k);
-            }
-          }
+          warp_colsum32(cs, lane);
           atomicAdd(p.colsum + n + lane, cs[0]);
         }
         // single-output epilogues alternate two buffers; GELU has one per output

@@ -226,6 +226,28 @@ def test_host_train_step_matches_device_calls():
     assert l1 == pytest.approx(l2, abs=1e-6) and n1 == pytest.approx(n2, rel=1e-3)
 
 
+# --- head size 64: the tcgen05 attention path with fused bias gradients ----------------------
+
+def test_head64_accumulated_gradients_match_oracle():
+    """Head size 64 and T a multiple of 128 take the tcgen05 attention (the tiny and
+    small configurations use head size 32), and the GELU-backward GEMM epilogue
+    adds the MLP fc bias gradient by atomics. Two micro-steps check that the
+    gradients accumulate."""
+    m, ocfg = pair("tiny", n_head=2, seq_len=256, micro_batch=2)
+    batches = batch_for("tiny", ocfg, n=2)
+    p = G.init_params(ocfg, 1337)
+    og = None
+    for x, y in batches:
+        loss = m.fwd_bwd(i32(x), i32(y), want_loss=True)
+        oloss, g = G.fwd_bwd(ocfg, p, x, y)
+        assert abs(loss - oloss) <= LOSS_TOL
+        og = g if og is None else {k: og[k] + g[k] for k in og}
+    grads = m.read_all(gs.GPT2_GRADS)
+    ogn = oracle_named(ocfg, og)
+    for name, a in grads.items():
+        assert rel_l2(a, ogn[name]) <= GRAD_TOL, (name, rel_l2(a, ogn[name]))
+
+
 # --- the small configuration: full context length, many tiles --------------------------------
 
 def test_small_config_step_parity():
