@@ -16,6 +16,9 @@
 //             all 256 epilogue threads of the pair arrive (the odd CTA remotely)
 // No TMA multicast is used: every load reads global memory into its own CTA.
 #pragma once
+#include <algorithm>
+#include <vector>
+
 #include "gemm.cuh"
 
 namespace gemm2 {
@@ -112,11 +115,16 @@ GPT2_DEV void tile_coords(const gemm::Params& p, int t, int& mb, int& nb, int& s
   nb = within / rows;
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
+// With GROUP, a second product (a weight gradient: MN-major A and B, fp32
+// accumulate; maps tmA1/tmB1, parameters p1) follows the first one's tiles in
+// the same persistent tile list, so its tiles fill the first one's last wave
+// and both share one pipeline fill and drain.
+template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
-                    const Params p) {
+                    const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA1,
+                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ Params p1) {
   using C = Cfg<BN>;
   constexpr int S = C::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw2[];
@@ -135,6 +143,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   const uint32_t rank = cluster_rank();
   const bool leader = (rank == 0);
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const int total_tiles = p.num_tiles + (GROUP ? p1.num_tiles : 0);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -149,6 +158,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (GROUP) {
+      tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmB1);
+    }
     if (EPI != gemm::EPI_ACC_F32) tma_prefetch_desc(&tmO);
     if (EPI == gemm::EPI_GELU) tma_prefetch_desc(&tmO2);
   }
@@ -167,11 +180,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = cid; t < p.num_tiles && ok; t += ncl) {
+      for (int t = cid; t < total_tiles && ok; t += ncl) {
+        const bool second = GROUP && t >= p.num_tiles;
+        const Params& q = second ? p1 : p;
         int mb, nb, sp;
-        tile_coords(p, t, mb, nb, sp);
-        const int kb0 = sp * p.kb_per_split;
-        const int kb1 = min(p.nkb, kb0 + p.kb_per_split);
+        tile_coords(q, second ? t - p.num_tiles : t, mb, nb, sp);
+        const int kb0 = sp * q.kb_per_split;
+        const int kb1 = min(q.nkb, kb0 + q.kb_per_split);
         const int m0 = mb * BM_PAIR + 128 * rank;
         const int n0 = nb * BN + (BN / 2) * rank;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -181,17 +196,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t sb = sa + C::A_BYTES;
           const int k0 = kb * BK;
-          if (A_MN) {
+          if (second) {
 #pragma unroll
-            for (int j = 0; j < 2; ++j) tma_load_2d_pair(sa + j * 8192, &tmA, fb, m0 + 64 * j, k0);
-          } else {
-            tma_load_2d_pair(sa, &tmA, fb, k0, m0);
-          }
-          if (B_MN) {
+            for (int j = 0; j < 2; ++j) tma_load_2d_pair(sa + j * 8192, &tmA1, fb, m0 + 64 * j, k0);
 #pragma unroll
-            for (int j = 0; j < BN / 128; ++j) tma_load_2d_pair(sb + j * 8192, &tmB, fb, n0 + 64 * j, k0);
+            for (int j = 0; j < BN / 128; ++j) tma_load_2d_pair(sb + j * 8192, &tmB1, fb, n0 + 64 * j, k0);
           } else {
-            tma_load_2d_pair(sb, &tmB, fb, k0, n0);
+            if (A_MN) {
+#pragma unroll
+              for (int j = 0; j < 2; ++j) tma_load_2d_pair(sa + j * 8192, &tmA, fb, m0 + 64 * j, k0);
+            } else {
+              tma_load_2d_pair(sa, &tmA, fb, k0, m0);
+            }
+            if (B_MN) {
+#pragma unroll
+              for (int j = 0; j < BN / 128; ++j) tma_load_2d_pair(sb + j * 8192, &tmB, fb, n0 + 64 * j, k0);
+            } else {
+              tma_load_2d_pair(sb, &tmB, fb, k0, n0);
+            }
           }
           if (++stage == S) { stage = 0; phase ^= 1; }
         }
@@ -200,17 +222,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = idesc_bf16_f32(BM_PAIR, BN, A_MN, B_MN);
+      constexpr uint32_t idesc0 = idesc_bf16_f32(BM_PAIR, BN, A_MN, B_MN);
+      constexpr uint32_t idesc1 = idesc_bf16_f32(BM_PAIR, BN, true, true);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      const int mn_tiles = p.num_m * p.num_n;
-      for (int t = cid; t < p.num_tiles && ok; t += ncl, ++it) {
+      for (int t = cid; t < total_tiles && ok; t += ncl, ++it) {
+        const bool second = GROUP && t >= p.num_tiles;
+        const Params& q = second ? p1 : p;
+        const int tt = second ? t - p.num_tiles : t;
         // tile bookkeeping stays off the MMA issue path: no division without a split
-        const int sp = p.splits == 1 ? 0 : t / mn_tiles;
-        const int kb0 = sp * p.kb_per_split;
-        const int kb1 = min(p.nkb, kb0 + p.kb_per_split);
+        const int sp = q.splits == 1 ? 0 : tt / (q.num_m * q.num_n);
+        const int kb0 = sp * q.kb_per_split;
+        const int kb1 = min(q.nkb, kb0 + q.kb_per_split);
+        const bool a_mn = second || A_MN, b_mn = second || B_MN;
+        const uint32_t idesc = second ? idesc1 : idesc0;
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, p.err)) { ok = false; break; }
@@ -223,9 +250,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           const uint32_t sb = sa + C::A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-            const uint64_t ad = A_MN ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
+            const uint64_t ad = a_mn ? smem_desc_sw128(sa + kk * 2048, 8192, 1024)
                                      : smem_desc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = B_MN ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
+            const uint64_t bd = b_mn ? smem_desc_sw128(sb + kk * 2048, 8192, 1024)
                                      : smem_desc_sw128(sb + kk * 32, 16, 1024);
             tc_mma2_bf16(d_tmem, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
           }
@@ -246,9 +273,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     int it = 0;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
-    for (int t = cid; t < p.num_tiles; t += ncl, ++it) {
+    for (int t = cid; t < total_tiles; t += ncl, ++it) {
+      const bool second = GROUP && t >= p.num_tiles;
       int mb, nb, sp;
-      tile_coords(p, t, mb, nb, sp);
+      tile_coords(second ? p1 : p, second ? t - p.num_tiles : t, mb, nb, sp);
       (void)sp;
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
@@ -256,70 +284,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       tc_fence_after();
       const int row0 = mb * BM_PAIR + 128 * rank + q * 32;
       const int row = row0 + lane;
-      const bool row_ok = row < p.M;
+      const bool row_ok = row < (second ? p1.M : p.M);
       const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
-      // Chunk c + 32 is read from tensor memory, and its bias / aux operands
-      // from global memory, while chunk c is processed: the epilogue of a tile
-      // then runs at about the pace of the next tile's main loop.
-      constexpr bool kBias = EPI == gemm::EPI_STORE || EPI == gemm::EPI_RESID || EPI == gemm::EPI_GELU;
-      constexpr bool kAux = EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU;
-      const bool has_bias = kBias && p.bias != nullptr;
-      const int c_beg = hv * (BN / 2), c_end = (hv + 1) * (BN / 2);
-      uint32_t vr[32];
-      float4 bn4[8];
-      uint4 an4[4];
-      auto fetch = [&](int c) {
-        tmem_ld32_async(t_row + c, vr);
-        const int n = nb * BN + c;
-        if (n < p.N) {
-          if (has_bias) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) bn4[i] = __ldg(reinterpret_cast<const float4*>(p.bias + n) + i);
-          }
-          if (kAux && row_ok) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.aux + (size_t)row * p.ld_aux + n);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) an4[j] = __ldcs(src + j);
-          }
-        }
-      };
-      fetch(c_beg);
+      if (second) {
+        // weight-gradient tile: fp32 accumulate (vector atomics when K is split)
 #pragma unroll 1
-      for (int c = c_beg; c < c_end; c += 32) {
-        const int n = nb * BN + c;
-        tmem_wait_ld();
-        float v[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vr[i]);
-        // consume this chunk's bias / aux registers, then start the next chunk's loads
-        if (n < p.N && has_bias) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[4 * i] += bn4[i].x; v[4 * i + 1] += bn4[i].y; v[4 * i + 2] += bn4[i].z; v[4 * i + 3] += bn4[i].w;
-          }
-        }
-        if (kAux && n < p.N && row_ok) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t w[4] = {an4[j].x, an4[j].y, an4[j].z, an4[j].w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const float2 f = unpack_bf16x2(w[h]);
-              const int i = j * 8 + h * 2;
-              if (EPI == gemm::EPI_RESID) {
-                v[i] += f.x; v[i + 1] += f.y;
-              } else {
-                v[i] *= gelu_grad_f(f.x); v[i + 1] *= gelu_grad_f(f.y);
-              }
-            }
-          }
-        }
-        if (c + 32 < c_end) fetch(c + 32);
-        if (n >= p.N) continue;
-        if (EPI == gemm::EPI_ACC_F32) {
-          if (!row_ok) continue;
-          float* dst = p.outf + (size_t)row * p.ldf + n;
-          if (p.splits > 1) {
+        for (int c = hv * (BN / 2); c < (hv + 1) * (BN / 2); c += 32) {
+          float v[32];
+          tmem_ld32(t_row + c, v);
+          const int n = nb * BN + c;
+          if (n >= p1.N || !row_ok) continue;
+          float* dst = p1.outf + (size_t)row * p1.ldf + n;
+          if (p1.splits > 1) {
 #pragma unroll
             for (int i = 0; i < 32; i += 4) gemm::red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
           } else {
@@ -330,45 +306,120 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
               *reinterpret_cast<float4*>(dst + i) = o;
             }
           }
-          continue;
         }
-        uint32_t pk[16];
+      } else {
+        // Chunk c + 32 is read from tensor memory, and its bias / aux operands
+        // from global memory, while chunk c is processed: the epilogue of a tile
+        // then runs at about the pace of the next tile's main loop.
+        constexpr bool kBias = EPI == gemm::EPI_STORE || EPI == gemm::EPI_RESID || EPI == gemm::EPI_GELU;
+        constexpr bool kAux = EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU;
+        const bool has_bias = kBias && p.bias != nullptr;
+        const int c_beg = hv * (BN / 2), c_end = (hv + 1) * (BN / 2);
+        uint32_t vr[32];
+        float4 bn4[8];
+        uint4 an4[4];
+        auto fetch = [&](int c) {
+          tmem_ld32_async(t_row + c, vr);
+          const int n = nb * BN + c;
+          if (n < p.N) {
+            if (has_bias) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
-        if (EPI == gemm::EPI_DGELU && p.colsum != nullptr) {
-          // column sums of the stored (bf16) values over this warp's 32 rows: a
-          // transpose-reduce leaves column `lane` of the chunk in cs[0]
-          float cs[32];
+              for (int i = 0; i < 8; ++i) bn4[i] = __ldg(reinterpret_cast<const float4*>(p.bias + n) + i);
+            }
+            if (kAux && row_ok) {
+              const uint4* src = reinterpret_cast<const uint4*>(p.aux + (size_t)row * p.ld_aux + n);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 f = unpack_bf16x2(pk[i]);
-            cs[2 * i] = row_ok ? f.x : 0.f;
-            cs[2 * i + 1] = row_ok ? f.y : 0.f;
+              for (int j = 0; j < 4; ++j) an4[j] = __ldcs(src + j);
+            }
           }
-          warp_colsum32(cs, lane);
-          atomicAdd(p.colsum + n + lane, cs[0]);
-        }
-        // single-output epilogues alternate two buffers; GELU has one per output
-        const uint32_t b = EPI == gemm::EPI_GELU ? 0u : (nstore & 1);
-        if (lane == 0) {
-          if (EPI == gemm::EPI_GELU) gemm::bulk_wait_read<0>();
-          else gemm::bulk_wait_read<1>();
-        }
-        __syncwarp();
-        gemm::stage_row(wbuf + b * 2048, lane, pk);
-        if (EPI == gemm::EPI_GELU) {
+        };
+        fetch(c_beg);
+#pragma unroll 1
+        for (int c = c_beg; c < c_end; c += 32) {
+          const int n = nb * BN + c;
+          tmem_wait_ld();
+          float v[32];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(gelu_f(v[2 * i]), gelu_f(v[2 * i + 1]));
-          gemm::stage_row(wbuf + 2048, lane, pk);
+          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vr[i]);
+          // consume this chunk's bias / aux registers, then start the next chunk's loads
+          if (n < p.N && has_bias) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              v[4 * i] += bn4[i].x; v[4 * i + 1] += bn4[i].y; v[4 * i + 2] += bn4[i].z; v[4 * i + 3] += bn4[i].w;
+            }
+          }
+          if (kAux && n < p.N && row_ok) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t w[4] = {an4[j].x, an4[j].y, an4[j].z, an4[j].w};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const float2 f = unpack_bf16x2(w[h]);
+                const int i = j * 8 + h * 2;
+                if (EPI == gemm::EPI_RESID) {
+                  v[i] += f.x; v[i + 1] += f.y;
+                } else {
+                  v[i] *= gelu_grad_f(f.x); v[i + 1] *= gelu_grad_f(f.y);
+                }
+              }
+            }
+          }
+          if (c + 32 < c_end) fetch(c + 32);
+          if (n >= p.N) continue;
+          if (EPI == gemm::EPI_ACC_F32) {
+            if (!row_ok) continue;
+            float* dst = p.outf + (size_t)row * p.ldf + n;
+            if (p.splits > 1) {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) gemm::red_add_v4(dst + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; i += 4) {
+                float4 o = *reinterpret_cast<float4*>(dst + i);
+                o.x += v[i]; o.y += v[i + 1]; o.z += v[i + 2]; o.w += v[i + 3];
+                *reinterpret_cast<float4*>(dst + i) = o;
+              }
+            }
+            continue;
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          if (EPI == gemm::EPI_DGELU && p.colsum != nullptr) {
+            // column sums of the stored (bf16) values over this warp's 32 rows: a
+            // transpose-reduce leaves column `lane` of the chunk in cs[0]
+            float cs[32];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 f = unpack_bf16x2(pk[i]);
+              cs[2 * i] = row_ok ? f.x : 0.f;
+              cs[2 * i + 1] = row_ok ? f.y : 0.f;
+            }
+            warp_colsum32(cs, lane);
+            atomicAdd(p.colsum + n + lane, cs[0]);
+          }
+          // single-output epilogues alternate two buffers; GELU has one per output
+          const uint32_t b = EPI == gemm::EPI_GELU ? 0u : (nstore & 1);
+          if (lane == 0) {
+            if (EPI == gemm::EPI_GELU) gemm::bulk_wait_read<0>();
+            else gemm::bulk_wait_read<1>();
+          }
+          __syncwarp();
+          gemm::stage_row(wbuf + b * 2048, lane, pk);
+          if (EPI == gemm::EPI_GELU) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(gelu_f(v[2 * i]), gelu_f(v[2 * i + 1]));
+            gemm::stage_row(wbuf + 2048, lane, pk);
+          }
+          gemm::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            gemm::tma_store_2d(&tmO, smem_u32(wbuf + b * 2048), n, row0);
+            if (EPI == gemm::EPI_GELU) gemm::tma_store_2d(&tmO2, smem_u32(wbuf + 2048), n, row0);
+            gemm::bulk_commit();
+          }
+          ++nstore;
         }
-        gemm::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          gemm::tma_store_2d(&tmO, smem_u32(wbuf + b * 2048), n, row0);
-          if (EPI == gemm::EPI_GELU) gemm::tma_store_2d(&tmO2, smem_u32(wbuf + 2048), n, row0);
-          gemm::bulk_commit();
-        }
-        ++nstore;
       }
       tmem_wait_ld();
       tc_fence_before();
@@ -386,20 +437,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   }
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool GROUP = false>
 static cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                              const CUtensorMap& to2, Params p, cudaStream_t s) {
+                              const CUtensorMap& to2, const Params& p, cudaStream_t s,
+                              const CUtensorMap* ta1 = nullptr, const CUtensorMap* tb1 = nullptr,
+                              const Params* p1 = nullptr) {
   using C = Cfg<BN>;
-  auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EPI>;
+  auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EPI, GROUP>;
   static bool attr_set = false;
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
+  Params q1{};
+  if (GROUP) q1 = *p1;
+  const int total = p.num_tiles + q1.num_tiles;
   const int pairs = gemm::num_sms() / 2;
-  const int grid = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
-  kern<<<grid, kThreads2, C::SMEM, s>>>(ta, tb, to, to2, p);
+  const int grid = 2 * (total < pairs ? total : pairs);
+  kern<<<grid, kThreads2, C::SMEM, s>>>(ta, tb, to, to2, p, GROUP ? *ta1 : ta, GROUP ? *tb1 : tb, q1);
   return cudaGetLastError();
 }
 
@@ -423,15 +479,13 @@ static bool uses_pair(const gemm::Call& c) {
   return BN == 256 && c.M >= BM_PAIR && c.force_bn != 128;
 }
 
-static int run(const gemm::Call& c, cudaStream_t s) {
+// Tile parameters and tensor maps of one pair-kernel product. splits > 0 forces
+// the reduction split of a weight gradient.
+static int prepare(const gemm::Call& c, int splits_forced, Params& p, CUtensorMap& ta, CUtensorMap& tb,
+                   CUtensorMap& to, CUtensorMap& to2) {
   using namespace gemm;
-  if (c.M <= 0 || c.N <= 0 || c.K <= 0) return GPT2_ERR_ARG;
-  if (c.N % 32 || c.K % BK) return GPT2_ERR_ARG;
-  const int BN = (c.kind == WGRAD && !c.force_bn && c.N % 256 == 0) ? 256 : choose_bn(c);
-  const bool pair = (BN == 256) && c.M >= BM_PAIR && c.force_bn != 128;
-  if (!pair && c.colsum) return GPT2_ERR_ARG;   // fused column sums need the pair kernel
-  if (!pair) return gemm::run(c, s);
-  Params p{};
+  const int BN = 256;
+  p = Params{};
   p.M = c.M; p.N = c.N; p.K = c.K;
   p.num_m = (c.M + BM_PAIR - 1) / BM_PAIR;
   p.num_n = (c.N + BN - 1) / BN;
@@ -439,7 +493,9 @@ static int run(const gemm::Call& c, cudaStream_t s) {
   int splits = 1;
   if (c.kind == WGRAD) {
     // waves of SM pairs: the split search sees pair tiles against 74 pairs
-    if (c.force_splits) {
+    if (splits_forced > 0) {
+      splits = splits_forced;
+    } else if (c.force_splits) {
       splits = c.force_splits;
     } else {
       const long pairs = num_sms() / 2;
@@ -462,7 +518,6 @@ static int run(const gemm::Call& c, cudaStream_t s) {
   p.aux = c.aux; p.ld_aux = c.ld_aux; p.bias = c.bias;
   p.outf = c.outf; p.ldf = c.ldf; p.err = c.err;
 
-  CUtensorMap ta, tb, to, to2;
   memset(&to, 0, sizeof(to));
   memset(&to2, 0, sizeof(to2));
   bool ok;
@@ -481,6 +536,20 @@ static int run(const gemm::Call& c, cudaStream_t s) {
     if (c.epi == EPI_GELU && !make_map(&to2, c.out2, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
       return GPT2_ERR_ARG;
   }
+  return GPT2_OK;
+}
+
+static int run(const gemm::Call& c, cudaStream_t s) {
+  using namespace gemm;
+  if (c.M <= 0 || c.N <= 0 || c.K <= 0) return GPT2_ERR_ARG;
+  if (c.N % 32 || c.K % BK) return GPT2_ERR_ARG;
+  const bool pair = uses_pair(c);
+  if (!pair && c.colsum) return GPT2_ERR_ARG;   // fused column sums need the pair kernel
+  if (!pair) return gemm::run(c, s);
+  Params p;
+  CUtensorMap ta, tb, to, to2;
+  const int st = prepare(c, 0, p, ta, tb, to, to2);
+  if (st != GPT2_OK) return st;
   cudaError_t e = cudaErrorInvalidValue;
   if (c.kind == FWD) {
     switch (c.epi) {
@@ -498,6 +567,55 @@ static int run(const gemm::Call& c, cudaStream_t s) {
   } else {
     if (c.epi != EPI_ACC_F32) return GPT2_ERR_ARG;
     e = launch_tc2<256, true, true, EPI_ACC_F32>(ta, tb, to, to2, p, s);
+  }
+  return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
+}
+
+// A layer's input gradient (dgrad, c0) and weight gradient (wgrad, c1) in one
+// launch: c1's tiles follow c0's in the persistent tile list, its reduction
+// split chosen so that its tiles carry about as many k-blocks as c0's. Falls
+// back to two launches when either product does not take the pair kernel.
+static int run_group(const gemm::Call& c0, const gemm::Call& c1, cudaStream_t s, int* launches) {
+  using namespace gemm;
+  const bool ok_shapes = c0.kind == DGRAD && c1.kind == WGRAD && c1.epi == EPI_ACC_F32 && c0.M > 0 &&
+                         c0.N % 32 == 0 && c0.K % BK == 0 && c1.K % BK == 0 && c1.K > 0 && uses_pair(c0) &&
+                         uses_pair(c1) && c1.N % 256 == 0;
+  *launches = ok_shapes ? 1 : 2;
+  if (!ok_shapes) {
+    const int st = gemm2::run(c0, s);
+    return st != GPT2_OK ? st : gemm2::run(c1, s);
+  }
+  Params p0, p1;
+  CUtensorMap ta0, tb0, to0, to20, ta1, tb1, to1, to21;
+  int st = prepare(c0, 0, p0, ta0, tb0, to0, to20);
+  if (st != GPT2_OK) return st;
+  // The wgrad split that minimises the estimated finish time of the busiest SM
+  // pair under the round-robin tile order: a tile costs its k-blocks plus an
+  // epilogue allowance, a split tile a further allowance for its fp32 atomic pass.
+  const int nkb1 = c1.K / BK;
+  const long tiles1 = (long)((c1.M + BM_PAIR - 1) / BM_PAIR) * (c1.N / 256);
+  const int pairs = num_sms() / 2;
+  constexpr int kEpi = 2, kAtomic = 8;
+  int splits1 = 1;
+  long best = -1;
+  std::vector<long> load(pairs);
+  for (int sp = 1; sp <= 32 && nkb1 >= 8 * sp; ++sp) {
+    const int kbps = (nkb1 + sp - 1) / sp;
+    const int nsp = (nkb1 + kbps - 1) / kbps;
+    std::fill(load.begin(), load.end(), 0L);
+    long t = 0;
+    for (long i = 0; i < p0.num_tiles; ++i, ++t) load[t % pairs] += p0.nkb + kEpi;
+    for (long i = 0; i < tiles1 * nsp; ++i, ++t) load[t % pairs] += kbps + kEpi + (nsp > 1 ? kAtomic : 0);
+    const long mk = *std::max_element(load.begin(), load.end());
+    if (best < 0 || mk < best) { best = mk; splits1 = nsp; }
+  }
+  st = prepare(c1, splits1, p1, ta1, tb1, to1, to21);
+  if (st != GPT2_OK) return st;
+  cudaError_t e = cudaErrorInvalidValue;
+  switch (c0.epi) {
+    case EPI_STORE: e = launch_tc2<256, false, true, EPI_STORE, true>(ta0, tb0, to0, to20, p0, s, &ta1, &tb1, &p1); break;
+    case EPI_DGELU: e = launch_tc2<256, false, true, EPI_DGELU, true>(ta0, tb0, to0, to20, p0, s, &ta1, &tb1, &p1); break;
+    default: return GPT2_ERR_ARG;
   }
   return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }

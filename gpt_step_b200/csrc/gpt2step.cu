@@ -405,6 +405,15 @@ int run_gemm(gpt2_model* m, const gemm::Call& c) {
   return st;
 }
 
+// A layer's dgrad (c0) and wgrad (c1) as one grouped launch where possible.
+int run_gemm_group(gpt2_model* m, const gemm::Call& c0, const gemm::Call& c1) {
+  const size_t p = prof_begin(m);
+  int nl = 2;
+  const int st = gemm2::run_group(c0, c1, m->stream, &nl);
+  prof_end(m, p, PC_GEMM, 2.0 * c0.M * c0.N * c0.K + 2.0 * c1.M * c1.N * c1.K, nl);
+  return st;
+}
+
 int ln_fwd_m(gpt2_model* m, const bf16* x, int kw, int kb, int l, bf16* y, float* mean, float* rstd, int rows) {
   const int C = m->lay.d.C;
   const size_t p = prof_begin(m);
@@ -556,46 +565,38 @@ int backward(gpt2_model* m, const int32_t* tok) {
     float* lse = m->at<float>(y.lse) + (size_t)l * d.N * d.H;
 
     bool fused_fcb = false;   // fc bias gradient summed in the d4c epilogue
-    // MLP projection
+    // Each linear layer's input gradient (dgrad) and weight gradient (wgrad) run as
+    // one grouped launch: the wgrad tiles fill the dgrad's last wave.
+    // MLP projection (the GELU' epilogue also sums the fc bias gradient)
     {
-      gemm::Call c = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, C, 4 * C, N, err);
-      c.a = dresid; c.lda = C; c.b = fchg; c.ldb = 4 * C; c.outf = m->G(K_FCPROJW, l); c.ldf = 4 * C;
-      GPT2_TRY(run_gemm(m, c));
-    }
-    {
-      gemm::Call c = gemm_call(gemm::DGRAD, gemm::EPI_DGELU, N, 4 * C, C, err);
-      c.a = dresid; c.lda = C; c.b = m->W(K_FCPROJW, l); c.ldb = 4 * C; c.out = d4c; c.ldo = 4 * C;
-      c.aux = fch; c.ld_aux = 4 * C;
-      // the MLP fc bias gradient is the column sum of d4c, added in the epilogue
-      c.colsum = m->G(K_FCB, l);
-      fused_fcb = gemm2::uses_pair(c);
-      if (!fused_fcb) c.colsum = nullptr;
-      GPT2_TRY(run_gemm(m, c));
+      gemm::Call cw = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, C, 4 * C, N, err);
+      cw.a = dresid; cw.lda = C; cw.b = fchg; cw.ldb = 4 * C; cw.outf = m->G(K_FCPROJW, l); cw.ldf = 4 * C;
+      gemm::Call cd = gemm_call(gemm::DGRAD, gemm::EPI_DGELU, N, 4 * C, C, err);
+      cd.a = dresid; cd.lda = C; cd.b = m->W(K_FCPROJW, l); cd.ldb = 4 * C; cd.out = d4c; cd.ldo = 4 * C;
+      cd.aux = fch; cd.ld_aux = 4 * C;
+      cd.colsum = m->G(K_FCB, l);
+      fused_fcb = gemm2::uses_pair(cd);
+      if (!fused_fcb) cd.colsum = nullptr;
+      GPT2_TRY(run_gemm_group(m, cd, cw));
     }
     // MLP fc
     {
-      gemm::Call c = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, 4 * C, C, N, err);
-      c.a = d4c; c.lda = 4 * C; c.b = ln2; c.ldb = C; c.outf = m->G(K_FCW, l); c.ldf = C;
-      GPT2_TRY(run_gemm(m, c));
+      gemm::Call cw = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, 4 * C, C, N, err);
+      cw.a = d4c; cw.lda = 4 * C; cw.b = ln2; cw.ldb = C; cw.outf = m->G(K_FCW, l); cw.ldf = C;
+      gemm::Call cd = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, 4 * C, err);
+      cd.a = d4c; cd.lda = 4 * C; cd.b = m->W(K_FCW, l); cd.ldb = C; cd.out = dln; cd.ldo = C;
+      GPT2_TRY(run_gemm_group(m, cd, cw));
     }
     if (!fused_fcb) GPT2_TRY(bias_grad_m(m, d4c, m->G(K_FCB, l), N, 4 * C));
-    {
-      gemm::Call c = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, 4 * C, err);
-      c.a = d4c; c.lda = 4 * C; c.b = m->W(K_FCW, l); c.ldb = C; c.out = dln; c.ldo = C;
-      GPT2_TRY(run_gemm(m, c));
-    }
     GPT2_TRY(ln_bwd_m(m, dln, xmid, m->at<float>(y.ln2_mean) + l * d.N, m->at<float>(y.ln2_rstd) + l * d.N, K_LN2W,
                       K_LN2B, l, dresid, dresid, m->G(K_ATTPROJB, l)));
     // attention projection
     {
-      gemm::Call c = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, C, C, N, err);
-      c.a = dresid; c.lda = C; c.b = atty; c.ldb = C; c.outf = m->G(K_ATTPROJW, l); c.ldf = C;
-      GPT2_TRY(run_gemm(m, c));
-    }
-    {
-      gemm::Call c = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, C, err);
-      c.a = dresid; c.lda = C; c.b = m->W(K_ATTPROJW, l); c.ldb = C; c.out = datty; c.ldo = C;
-      GPT2_TRY(run_gemm(m, c));
+      gemm::Call cw = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, C, C, N, err);
+      cw.a = dresid; cw.lda = C; cw.b = atty; cw.ldb = C; cw.outf = m->G(K_ATTPROJW, l); cw.ldf = C;
+      gemm::Call cd = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, C, err);
+      cd.a = dresid; cd.lda = C; cd.b = m->W(K_ATTPROJW, l); cd.ldb = C; cd.out = datty; cd.ldo = C;
+      GPT2_TRY(run_gemm_group(m, cd, cw));
     }
     {
       const size_t p = prof_begin(m);
@@ -605,16 +606,13 @@ int backward(gpt2_model* m, const int32_t* tok) {
     }
     // QKV projection
     {
-      gemm::Call c = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, 3 * C, C, N, err);
-      c.a = dqkv; c.lda = 3 * C; c.b = ln1; c.ldb = C; c.outf = m->G(K_QKVW, l); c.ldf = C;
-      GPT2_TRY(run_gemm(m, c));
+      gemm::Call cw = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, 3 * C, C, N, err);
+      cw.a = dqkv; cw.lda = 3 * C; cw.b = ln1; cw.ldb = C; cw.outf = m->G(K_QKVW, l); cw.ldf = C;
+      gemm::Call cd = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, 3 * C, err);
+      cd.a = dqkv; cd.lda = 3 * C; cd.b = m->W(K_QKVW, l); cd.ldb = C; cd.out = dln; cd.ldo = C;
+      GPT2_TRY(run_gemm_group(m, cd, cw));
     }
     GPT2_TRY(bias_grad_m(m, dqkv, m->G(K_QKVB, l), N, 3 * C));
-    {
-      gemm::Call c = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, 3 * C, err);
-      c.a = dqkv; c.lda = 3 * C; c.b = m->W(K_QKVW, l); c.ldb = C; c.out = dln; c.ldo = C;
-      GPT2_TRY(run_gemm(m, c));
-    }
     GPT2_TRY(ln_bwd_m(m, dln, x_in, m->at<float>(y.ln1_mean) + l * d.N, m->at<float>(y.ln1_rstd) + l * d.N, K_LN1W,
                       K_LN1B, l, dresid, dresid, l > 0 ? m->G(K_FCPROJB, l - 1) : nullptr));
   }
