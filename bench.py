@@ -191,9 +191,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from gpt_step_b200.replicas import job_throughput, max_over_ranks, rank_env, replica_seed
+    rank, world, local_rank = rank_env()
 
     if args.impl == "reference":
         run_reference(args, rank, world)
@@ -216,10 +215,10 @@ def main():
     w = workloads.WORKLOADS[WORKLOAD]
     B, T, A = w["micro_batch"], w["seq_len"], w["grad_accum"]
     cfg = gs.Config.make(**workloads.model_args(WORKLOAD))
-    model = gs.GPT2(cfg, 1337 + rank)
+    model = gs.GPT2(cfg, replica_seed(1337, rank))
     n_steps = args.warmup + args.steps
     n_win = n_steps * A * B
-    src = synth.TokenSource(B, T, cfg.vocab_real, 1337 + rank, w["mean_doc_len"], n_win)
+    src = synth.TokenSource(B, T, cfg.vocab_real, replica_seed(1337, rank), w["mean_doc_len"], n_win)
     xs, ys = [], []
     for _ in range(n_steps * A):
         x, y = src.get()
@@ -268,13 +267,9 @@ def main():
     prof = model.profile_read()
     model.profile(False)
     barrier()
-    t_max = ms
-    if world > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_max = float(t.item())
+    t_max = max_over_ranks(ms, device="cuda")
     tokens = args.steps * A * B * T * world
-    value = tokens / (t_max / 1000.0)
+    value = job_throughput(args.steps * A * B * T, world, t_max)
 
     # end to end through the host-buffer C-ABI call
     e2e = None
@@ -292,12 +287,8 @@ def main():
             model.train_step_host_ptr(htok.data_ptr(), htgt.data_ptr(), A, 2 * n_steps + k)
         e1.record(stream)
         barrier()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ems], device="cuda")
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": tokens / (ems / 1000.0), "unit": "tokens/s",
+        ems = max_over_ranks(e0.elapsed_time(e1), device="cuda")
+        e2e = {"value": job_throughput(args.steps * A * B * T, world, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": 2 * A * B * T * 4, "d2h_bytes_per_step": 8,
                "api": "gpt2_train_step_host (pinned host tokens/targets)"}
 
