@@ -284,6 +284,28 @@ def softmax_ce(z, targets, V):
     return losses, dz
 
 
+def softmax_ce_masked(z, targets, V, ignore_index=-1):
+    """Cross-entropy with an ignore index per target: the loss is taken only on
+    chosen positions ("Pretraining and adapting a language model on a
+    dependency-free stack" takes the adapter's loss on answers rather than
+    questions). Rows whose target equals `ignore_index` contribute loss 0 and a
+    gradient of exactly zero; the others are softmax_ce's rows, and the mean is
+    over the kept rows only.
+
+    z [N, Vp], targets [N]. Returns (per-row losses [N], dz of the mean loss over
+    kept rows, number of kept rows).
+    """
+    keep = targets != ignore_index
+    n_keep = int(keep.sum())
+    losses = np.zeros(z.shape[0])
+    dz = np.zeros_like(z)
+    if n_keep:
+        lk, dk = softmax_ce(z[keep], targets[keep], V)
+        losses[keep] = lk
+        dz[keep] = dk           # softmax_ce of the kept rows already divides by n_keep
+    return losses, dz, n_keep
+
+
 # ----------------------------------------------------------------------------
 # forward / backward of the whole model
 # ----------------------------------------------------------------------------

@@ -231,3 +231,51 @@ def test_zipf_stream_statistics():
     assert abs(np.mean(doc == 1) - 2 ** -1.1 / H) < 3e-3
     x, y = synth.windows(s, 4, 1024)
     assert np.array_equal(x[:, 1:], y[:, :-1])
+
+
+# --- masked-target cross-entropy (an ignore index per target) -------------------------------
+
+def test_masked_ce_without_ignored_rows_is_plain_ce():
+    rng = np.random.default_rng(7)
+    z = rng.standard_normal((5, 24))
+    t = rng.integers(0, 20, 5)
+    l0, d0 = G.softmax_ce(z, t, 20)
+    l1, d1, n = G.softmax_ce_masked(z, t, 20)
+    assert n == 5
+    np.testing.assert_allclose(l1, l0, rtol=0, atol=0)
+    np.testing.assert_allclose(d1, d0, rtol=0, atol=0)
+
+
+def test_masked_ce_all_ignored_is_zero():
+    z = np.random.default_rng(8).standard_normal((3, 8))
+    l, d, n = G.softmax_ce_masked(z, np.full(3, -1), 6)
+    assert n == 0 and not l.any() and not d.any()
+
+
+def test_masked_ce_gradient_by_finite_differences():
+    """The gradient is that of the mean loss over the kept rows (central
+    differences in fp64); ignored rows and padded columns get exactly zero."""
+    rng = np.random.default_rng(9)
+    N, V, Vp = 6, 10, 16
+    z = rng.standard_normal((N, Vp))
+    t = np.array([2, -1, 7, -1, 0, 9])
+    _, dz, n = G.softmax_ce_masked(z, t, V)
+    assert n == 4
+    keep = t != -1
+
+    def mean_loss(zz):
+        zr = zz[:, :V]
+        m = zr.max(axis=1)
+        lse = m + np.log(np.exp(zr - m[:, None]).sum(axis=1))
+        return np.mean((lse - zz[np.arange(N), np.where(keep, t, 0)])[keep])
+
+    h = 1e-6
+    num = np.zeros_like(z)
+    for i in range(N):
+        for j in range(Vp):
+            zp, zm = z.copy(), z.copy()
+            zp[i, j] += h
+            zm[i, j] -= h
+            num[i, j] = (mean_loss(zp) - mean_loss(zm)) / (2 * h)
+    np.testing.assert_allclose(dz, num, atol=1e-8)
+    assert not dz[~keep].any() and not dz[:, V:].any()
