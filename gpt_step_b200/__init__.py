@@ -95,6 +95,7 @@ _SIGNATURES = {
     "gpt2op_attention_bwd_workspace": (_SZ, [_I, _I, _I, _I]),
     "gpt2op_attention_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P]),
     "gpt2op_softmax_ce": (_I, [_P, _P, _P, _I, _I, _I, _F, _P, _P]),
+    "gpt2op_softmax_ce_masked": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P]),
     "gpt2op_embedding_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "gpt2op_embedding_bwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
 }
@@ -382,6 +383,13 @@ def softmax_ce(logits, targets, losses, V, dscale, err, stream=None):
     N, Vp = logits.shape
     check(lib().gpt2op_softmax_ce(_ptr(logits), _ptr(targets), _ptr(losses), N, V, Vp, dscale,
                                   _ptr(err), _s(stream)), "gpt2op_softmax_ce")
+
+
+def softmax_ce_masked(logits, targets, losses, V, ignore_index, dscale, err, stream=None):
+    """Softmax-CE where rows with target == ignore_index get loss 0 and zero gradient."""
+    N, Vp = logits.shape
+    check(lib().gpt2op_softmax_ce_masked(_ptr(logits), _ptr(targets), _ptr(losses), N, V, Vp, ignore_index,
+                                         dscale, _ptr(err), _s(stream)), "gpt2op_softmax_ce_masked")
 
 
 def embedding_fwd(tokens, wte, wpe, out, V, err, stream=None):

@@ -13,6 +13,7 @@
 //             -> LN2 -> fc + GELU -> proj (+res)] -> LN_f -> tied head -> CE
 //   backward  the same in reverse, weight gradients accumulated in fp32
 //   update    global norm over all gradients / micro-steps, clip, AdamW
+#include <limits.h>
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
@@ -317,11 +318,13 @@ int bias_grad(const bf16* dout, float* db, int M, int N, float* part, size_t par
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
+// ignore_index: targets equal to it are skipped (INT_MIN: none are)
 int softmax_ce(bf16* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,
-               int write_grad, int* err, cudaStream_t s) {
+               int write_grad, int* err, cudaStream_t s, int ignore_index = INT_MIN) {
   if (Vp % 8 || V > Vp || V <= 0) return GPT2_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(logits) & 15) != 0) return GPT2_ERR_ARG;
-  k::softmax_ce_kernel<<<N, k::kCeThreads, 0, s>>>(logits, targets, losses, V, Vp, dscale, write_grad, err);
+  k::softmax_ce_kernel<<<N, k::kCeThreads, 0, s>>>(logits, targets, losses, V, Vp, dscale, write_grad, err,
+                                                    ignore_index);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -1088,6 +1091,13 @@ int gpt2op_softmax_ce(void* logits, const int32_t* targets, float* losses, int N
   if (!logits || !targets || !losses || !dev_err || N <= 0) return GPT2_ERR_ARG;
   return launch::softmax_ce(static_cast<bf16*>(logits), targets, losses, N, V, Vp, dscale, 1, dev_err,
                             static_cast<cudaStream_t>(stream));
+}
+
+int gpt2op_softmax_ce_masked(void* logits, const int32_t* targets, float* losses, int N, int V, int Vp,
+                             int ignore_index, float dscale, int* dev_err, void* stream) {
+  if (!logits || !targets || !losses || !dev_err || N <= 0 || ignore_index == INT_MIN) return GPT2_ERR_ARG;
+  return launch::softmax_ce(static_cast<bf16*>(logits), targets, losses, N, V, Vp, dscale, 1, dev_err,
+                            static_cast<cudaStream_t>(stream), ignore_index);
 }
 
 int gpt2op_embedding_fwd(const int32_t* tokens, const void* wte, const void* wpe, void* out, int B, int T, int C, int V,

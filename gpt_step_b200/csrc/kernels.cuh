@@ -521,19 +521,28 @@ GPT2_DEV void ce_combine(float& m, float& s, float om, float os) {
   m = nm;
 }
 
-// One CTA per row, no shared-memory staging: pass 1 streams the bf16 row
+// One CTA per row, no shared-memory staging (rows whose target equals
+// ignore_index, when one is given, get loss 0 and a zero gradient): pass 1 streams the bf16 row
 // (kCeUnroll 16-byte loads in flight per thread) for the running (max, sum of
 // exp) over the real columns; pass 2 reads the row again (from L2) and
 // overwrites it with dz.
 __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict__ logits,
                                                                 const int32_t* __restrict__ targets,
                                                                 float* __restrict__ losses, int V, int Vp,
-                                                                float dscale, int write_grad, int* err) {
+                                                                float dscale, int write_grad, int* err,
+                                                                int ignore_index) {
   __shared__ float red_m[kCeThreads / 32], red_s[kCeThreads / 32];
   __shared__ float bc[2];
   const int row = blockIdx.x;
   uint4* zr = reinterpret_cast<uint4*>(logits + (size_t)row * Vp);
   const int nv = Vp / 8;
+  if (targets[row] == ignore_index) {
+    // an ignored position: loss 0, gradient exactly 0, not an error
+    if (threadIdx.x == 0) losses[row] = 0.f;
+    if (write_grad)
+      for (int i = threadIdx.x; i < nv; i += kCeThreads) __stcs(zr + i, make_uint4(0u, 0u, 0u, 0u));
+    return;
+  }
   float m = -INFINITY, s = 0.f;
   for (int i0 = threadIdx.x; i0 < nv; i0 += kCeThreads * kCeUnroll) {
     uint4 u[kCeUnroll];

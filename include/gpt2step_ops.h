@@ -115,6 +115,16 @@ int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, con
 int gpt2op_softmax_ce(void* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,
                       int* dev_err, void* stream);
 
+/* Cross-entropy with an ignore index per target (the loss taken only on chosen
+ * positions, e.g. the answers of question/answer text; "Pretraining and
+ * adapting a language model on a dependency-free stack" trains its adapter that
+ * way). The pages have no kernel for it: this is the vocabulary-masked
+ * softmax-CE above where rows whose target equals ignore_index (any value but
+ * INT_MIN) get loss 0 and a gradient of exactly 0 and raise no error. dscale is
+ * the caller's, normally 1 / (number of kept rows) for the mean over kept rows. */
+int gpt2op_softmax_ce_masked(void* logits, const int32_t* targets, float* losses, int N, int V, int Vp,
+                             int ignore_index, float dscale, int* dev_err, void* stream);
+
 /* Token + position embedding: out[b,t,:] = wte[tok[b,t],:] + wpe[t,:] (bf16).
  * Ids outside [0, V) read row 0 and set flag 1 in dev_err. */
 int gpt2op_embedding_fwd(const int32_t* tokens, const void* wte, const void* wpe, void* out, int B, int T, int C,

@@ -172,6 +172,27 @@ def test_softmax_ce(N, V, Vp):
     assert int(err[0]) & 1
 
 
+@pytest.mark.parametrize("N,V,Vp,ignore", [(64, 1000, 1024, -100), (37, 4353, 4480, -1), (16, 50257, 50304, -1)])
+def test_softmax_ce_masked(N, V, Vp, ignore):
+    """Ignore index per target: ignored rows give loss 0 and an exactly zero
+    gradient row and raise no error; kept rows match the oracle's mean over kept rows."""
+    z = rnd((N, Vp), 27, 2.0)
+    t = np.random.default_rng(28).integers(0, V, N)
+    t[::3] = ignore
+    zd = bf16(z)
+    losses = torch.empty(N, device="cuda")
+    err = err_word()
+    n_keep = int((t != ignore).sum())
+    gs.softmax_ce_masked(zd, i32(t), losses, V, ignore, 1.0 / n_keep, err)
+    lr, dzr, n = G.softmax_ce_masked(rounded(z), t, V, ignore)
+    assert n == n_keep
+    assert np.max(np.abs(host(losses) - lr)) < 1e-4
+    dz = host(zd)
+    assert np.all(dz[t == ignore] == 0.0) and np.all(dz[:, V:] == 0.0)
+    assert rel_l2(dz, dzr) < BF16_TOL
+    assert int(err.sum()) == 0
+
+
 # --- a1: embeddings -----------------------------------------------------------------------
 
 def test_embedding_fwd_bwd():
