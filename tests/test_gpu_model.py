@@ -305,3 +305,45 @@ def test_gpt2_124m_bench_configuration_sampled():
     norm = m.clip_adamw(0, want_norm=True)
     assert np.isfinite(norm) and norm > 0
     assert np.all(m.read(gs.GPT2_PARAMS, 0)[ocfg.V:] == 0.0)
+
+
+def test_checkpoint_resume_continues_the_run(tmp_path):
+    """A run stopped at a checkpoint and restored into a model of another seed
+    continues the uninterrupted run: the restored fp32 weights and moments are
+    bitwise the saved ones, the held-out loss (forward only, no atomics) is bitwise
+    equal, and the following steps track the uninterrupted ones to fp32 summation
+    order (the split-K weight gradients add in an unspecified order)."""
+    from gpt_step_b200 import checkpoint as ck
+    over = dict(total_steps=10, warmup_steps=2, grad_accum=2)
+    args = workloads.model_args("tiny", **over)
+    w = workloads.WORKLOADS["tiny"]
+    B, T, V = args["micro_batch"], args["seq_len"], args["vocab_real"]
+    hx, hy = synth.uniform_next_token_batch(B, T, V, 4242)
+    hx, hy = i32(hx), i32(hy)
+    ev = lambda m: m.eval_loss(hx, hy)
+    cad = ck.Cadence(eval_every=2, ckpt_every=2)
+    src = lambda: synth.TokenSource(B, T, V, 1337, w["mean_doc_len"], 64)
+
+    a = gs.GPT2(gs.Config.make(**args), 1337)
+    ra = ck.run(a, src(), 0, 4, i32, cad, str(tmp_path / "a"), ev)
+    path = ck.ckpt_path(str(tmp_path / "a"), 2)
+    saved = np.load(path)
+
+    b = gs.GPT2(gs.Config.make(**args), 999)
+    h = ck.load(b, path)
+    assert h["step"] == 2
+    for i, t in enumerate(b.tensors()):
+        for key, what in (("param", gs.GPT2_PARAMS), ("m", gs.GPT2_ADAM_M), ("v", gs.GPT2_ADAM_V)):
+            assert np.array_equal(b.read(what, i), saved[f"{key}/{t.name}"]), (key, t.name)
+    assert ev(b) == ra[1]["eval_loss"]
+    s = src()
+    s.next = h["data_cursor"]
+    rb = ck.run(b, s, h["step"], 4, i32, cad, None, ev)
+    for x, y in zip(ra[2:], rb):
+        assert x["step"] == y["step"]
+        assert y["loss"] == pytest.approx(x["loss"], rel=1e-5)
+        assert y["grad_norm"] == pytest.approx(x["grad_norm"], rel=1e-4)
+    for i, t in enumerate(a.tensors()):
+        assert np.max(np.abs(a.read(gs.GPT2_PARAMS, i) - b.read(gs.GPT2_PARAMS, i))) <= 2e-6, t.name
+    a.close()
+    b.close()
