@@ -96,6 +96,8 @@ _SIGNATURES = {
     "gpt2op_attention_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P]),
     "gpt2op_softmax_ce": (_I, [_P, _P, _P, _I, _I, _I, _F, _P, _P]),
     "gpt2op_softmax_ce_masked": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P]),
+    "gpt2op_lm_head_ce_workspace": (_SZ, [_I, _I]),
+    "gpt2op_lm_head_ce": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P]),
     "gpt2op_embedding_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "gpt2op_embedding_bwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
 }
@@ -390,6 +392,20 @@ def softmax_ce_masked(logits, targets, losses, V, ignore_index, dscale, err, str
     N, Vp = logits.shape
     check(lib().gpt2op_softmax_ce_masked(_ptr(logits), _ptr(targets), _ptr(losses), N, V, Vp, ignore_index,
                                          dscale, _ptr(err), _s(stream)), "gpt2op_softmax_ce_masked")
+
+
+def lm_head_ce_workspace(N, Vp):
+    return lib().gpt2op_lm_head_ce_workspace(N, Vp)
+
+
+def lm_head_ce(h, wte, targets, logits, losses, V, dscale, write_grad, ws, err, stream=None):
+    """Tied lm_head GEMM + softmax-CE: logits = h . wte^T, then losses (and dz in place)."""
+    N, C = h.shape
+    Vp = wte.shape[0]
+    check(lib().gpt2op_lm_head_ce(_ptr(h), _ptr(wte), _ptr(targets), _ptr(logits), _ptr(losses), N, C, V, Vp,
+                                  dscale, 1 if write_grad else 0, _ptr(ws),
+                                  0 if ws is None else ws.numel() * ws.element_size(), _ptr(err), _s(stream)),
+          "gpt2op_lm_head_ce")
 
 
 def embedding_fwd(tokens, wte, wpe, out, V, err, stream=None):

@@ -37,6 +37,8 @@ enum Epi : int {
   EPI_GELU = 2,     // out = bf16(acc + bias); out2 = bf16(GELU(acc + bias))
   EPI_DGELU = 3,    // out = bf16(acc * GELU'(aux))
   EPI_ACC_F32 = 4,  // outf += acc (fp32; atomic when the reduction is split)
+  EPI_LSE = 5,      // pair kernel only: out = bf16(acc), and per row and half tile the
+                    // running (max, sum of 2^) of log2(e) * out over columns < lse_V
 };
 
 struct Params {
@@ -44,6 +46,8 @@ struct Params {
   int num_m, num_n, splits, kb_per_split, nkb, num_tiles;
   int raster_gm;  // row tiles per raster panel (pair kernel); num_m = plain row-major order
   float* colsum;  // pair kernel, EPI_DGELU: column sums of the (bf16) output added here, or null
+  float2* lse_part;  // pair kernel, EPI_LSE: [M][lse_slots] (max, sum) partials, slot = 2 * n_tile + half
+  int lse_V, lse_slots;
   bf16* out;
   bf16* out2;
   int ldo;
@@ -391,6 +395,8 @@ struct Call {
   int force_bn;      // 0: automatic
   int force_splits;  // 0: automatic
   float* colsum;     // EPI_DGELU with >= 256 rows: add the output's column sums here (else null)
+  float2* lse_part;  // EPI_LSE: [M][2 * ceil(N / 256)] row partials (see Params)
+  int lse_V;         // EPI_LSE: columns >= lse_V are stored but left out of the partials
 };
 
 // Tile width: whole waves of 148 SMs, with 128-wide tiles charged 1.3x because a
@@ -421,7 +427,7 @@ static int choose_splits(long tiles, int nkb) {
 }
 
 static int run(const Call& c, cudaStream_t s) {
-  if (c.M <= 0 || c.N <= 0 || c.K <= 0) return GPT2_ERR_ARG;
+  if (c.M <= 0 || c.N <= 0 || c.K <= 0 || c.epi == EPI_LSE) return GPT2_ERR_ARG;
   if (c.N % 32 || c.K % BK) return GPT2_ERR_ARG;
   // weight gradients take full-width tiles; the split of the reduction fills the waves
   const int BN = (c.kind == WGRAD && !c.force_bn && c.N % 256 == 0) ? 256 : choose_bn(c);

@@ -311,7 +311,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         // Chunk c + 32 is read from tensor memory, and its bias / aux operands
         // from global memory, while chunk c is processed: the epilogue of a tile
         // then runs at about the pace of the next tile's main loop.
-        constexpr bool kBias = EPI == gemm::EPI_STORE || EPI == gemm::EPI_RESID || EPI == gemm::EPI_GELU;
+        constexpr bool kBias = EPI == gemm::EPI_STORE || EPI == gemm::EPI_RESID || EPI == gemm::EPI_GELU ||
+                               EPI == gemm::EPI_LSE;
+        constexpr bool kLse = EPI == gemm::EPI_LSE;
+        // EPI_LSE: this row's running max (log2 units) and sum of 2^(y - max) over the half tile
+        float lse_m = -INFINITY, lse_s = 0.f;
         constexpr bool kAux = EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU;
         const bool has_bias = kBias && p.bias != nullptr;
         const int c_beg = hv * (BN / 2), c_end = (hv + 1) * (BN / 2);
@@ -385,6 +389,49 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          if (kLse) {
+            // over the stored bf16 values f: chunk max by a bf16x2 tree (exact, and
+            // max(f) * log2(e) rounds to the max of the scaled values), then the sum
+            // of 2^(f log2(e) - max) in four independent accumulators
+            const float kL2e = 1.4426950408889634f;
+            float cm;
+            float f[32];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float2 u = unpack_bf16x2(pk[i]);
+              f[2 * i] = u.x;
+              f[2 * i + 1] = u.y;
+            }
+            if (n + 32 <= p.lse_V) {
+              __nv_bfloat162 h[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) h[i] = *reinterpret_cast<const __nv_bfloat162*>(&pk[i]);
+#pragma unroll
+              for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+                for (int i = 0; i < w; ++i) h[i] = __hmax2(h[i], h[i + w]);
+              const float2 hm = __bfloat1622float2(h[0]);
+              cm = fmaxf(hm.x, hm.y) * kL2e;
+            } else {
+              cm = -INFINITY;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                if (n + i >= p.lse_V) f[i] = -INFINITY;   // padded ids: 2^-inf = 0
+                cm = fmaxf(cm, f[i]);
+              }
+              cm *= kL2e;
+            }
+            if (cm > lse_m) {
+              lse_s *= ex2_approx(lse_m - cm);
+              lse_m = cm;
+            }
+            if (cm != -INFINITY) {
+              float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int i = 0; i < 32; ++i) a[i & 3] += ex2_approx(fmaf(f[i], kL2e, -lse_m));
+              lse_s += (a[0] + a[1]) + (a[2] + a[3]);
+            }
+          }
           if (EPI == gemm::EPI_DGELU && p.colsum != nullptr) {
             // column sums of the stored (bf16) values over this warp's 32 rows: a
             // transpose-reduce leaves column `lane` of the chunk in cs[0]
@@ -420,6 +467,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
           }
           ++nstore;
         }
+        if (kLse && row_ok) p.lse_part[(size_t)row * p.lse_slots + 2 * nb + hv] = make_float2(lse_m, lse_s);
       }
       tmem_wait_ld();
       tc_fence_before();
@@ -514,6 +562,12 @@ static int prepare(const gemm::Call& c, int splits_forced, Params& p, CUtensorMa
   p.num_tiles = p.num_m * p.num_n * p.splits;
   p.raster_gm = std::min(p.num_m, c.kind == WGRAD ? kRasterRowsWgrad : kRasterRows);
   p.colsum = c.epi == EPI_DGELU ? c.colsum : nullptr;
+  if (c.epi == EPI_LSE) {
+    if (c.kind != FWD || !c.lse_part || c.lse_V <= 0 || c.lse_V > c.N) return GPT2_ERR_ARG;
+    p.lse_part = c.lse_part;
+    p.lse_V = c.lse_V;
+    p.lse_slots = 2 * p.num_n;
+  }
   p.out = c.out; p.out2 = c.out2; p.ldo = c.ldo;
   p.aux = c.aux; p.ld_aux = c.ld_aux; p.bias = c.bias;
   p.outf = c.outf; p.ldf = c.ldf; p.err = c.err;
@@ -545,7 +599,7 @@ static int run(const gemm::Call& c, cudaStream_t s) {
   if (c.N % 32 || c.K % BK) return GPT2_ERR_ARG;
   const bool pair = uses_pair(c);
   if (!pair && c.colsum) return GPT2_ERR_ARG;   // fused column sums need the pair kernel
-  if (!pair) return gemm::run(c, s);
+  if (!pair) return gemm::run(c, s);   // refuses EPI_LSE
   Params p;
   CUtensorMap ta, tb, to, to2;
   const int st = prepare(c, 0, p, ta, tb, to, to2);
@@ -556,6 +610,7 @@ static int run(const gemm::Call& c, cudaStream_t s) {
       case EPI_STORE: e = launch_tc2<256, false, false, EPI_STORE>(ta, tb, to, to2, p, s); break;
       case EPI_RESID: e = launch_tc2<256, false, false, EPI_RESID>(ta, tb, to, to2, p, s); break;
       case EPI_GELU: e = launch_tc2<256, false, false, EPI_GELU>(ta, tb, to, to2, p, s); break;
+      case EPI_LSE: e = launch_tc2<256, false, false, EPI_LSE>(ta, tb, to, to2, p, s); break;
       default: return GPT2_ERR_ARG;
     }
   } else if (c.kind == DGRAD) {

@@ -79,11 +79,14 @@ struct Layout {
   long P;  // flat length (padded, multiple of 64)
   size_t params, grads, adam_m, adam_v, pbf;
   size_t resid, ln1, ln1_mean, ln1_rstd, qkv, atty, lse, resid_mid, ln2, ln2_mean, ln2_rstd, fch, fchg;
-  size_t lnf, lnf_mean, lnf_rstd, logits;
+  size_t lnf, lnf_mean, lnf_rstd, logits, lse_part;
   size_t dresid, dln, d4c, dqkv, datty, dq_acc, attD;
   size_t ln_part, col_part, norm_part, losses, scalars, eval_acc, err, tok, tgt;
   size_t total;
 };
+
+// (max, sum) partials per logits row that the lm_head GEMM leaves: two per 256-wide tile
+inline int lse_slots(int Vp) { return 2 * ((Vp + 255) / 256); }
 
 void make_layout(const Dims& d, Layout* lay) {
   lay->d = d;
@@ -127,6 +130,7 @@ void make_layout(const Dims& d, Layout* lay) {
   lay->lnf_mean = take(N * 4);
   lay->lnf_rstd = take(N * 4);
   lay->logits = take(N * (size_t)d.Vp * 2);
+  lay->lse_part = take(N * (size_t)lse_slots(d.Vp) * 8);
   lay->dresid = take(N * C * 2);
   lay->dln = take(N * C * 2);
   lay->d4c = take(N * 4 * C * 2);
@@ -318,13 +322,16 @@ int bias_grad(const bf16* dout, float* db, int M, int N, float* part, size_t par
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
-// ignore_index: targets equal to it are skipped (INT_MIN: none are)
+// ignore_index: targets equal to it are skipped (INT_MIN: none are). part: the
+// logits GEMM's EPI_LSE row partials ([N][slots]), or null to scan the row.
 int softmax_ce(bf16* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,
-               int write_grad, int* err, cudaStream_t s, int ignore_index = INT_MIN) {
+               int write_grad, int* err, cudaStream_t s, int ignore_index = INT_MIN,
+               const float2* part = nullptr, int slots = 0) {
   if (Vp % 8 || V > Vp || V <= 0) return GPT2_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(logits) & 15) != 0) return GPT2_ERR_ARG;
+  if (part && slots <= 0) return GPT2_ERR_ARG;
   k::softmax_ce_kernel<<<N, k::kCeThreads, 0, s>>>(logits, targets, losses, V, Vp, dscale, write_grad, err,
-                                                    ignore_index);
+                                                    ignore_index, part, slots);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -490,17 +497,29 @@ int forward(gpt2_model* m, const int32_t* tok, const int32_t* tgt, int b, bool t
   GPT2_TRY(ln_fwd_m(m, resid + L * NC, K_LNFW, K_LNFB, 0, lnf, m->at<float>(y.lnf_mean), m->at<float>(y.lnf_rstd),
                     (int)N));
   bf16* logits = m->at<bf16>(y.logits);
+  // the pair kernel's epilogue also leaves each row's (max, sum) partials, so the
+  // cross-entropy reads the logits once
+  float2* lse_part = nullptr;
   {
     gemm::Call c = gemm_call(gemm::FWD, gemm::EPI_STORE, (int)N, d.Vp, C, err);
     c.a = lnf; c.lda = C; c.b = m->W(K_WTE); c.ldb = C; c.out = logits; c.ldo = d.Vp;
+    if (gemm2::uses_pair(c)) {
+      lse_part = m->at<float2>(y.lse_part);
+      c.epi = gemm::EPI_LSE; c.lse_part = lse_part; c.lse_V = d.V;
+    }
     GPT2_TRY(run_gemm(m, c));
   }
   float* losses = m->at<float>(y.losses);
   {
     const size_t p = prof_begin(m);
-    GPT2_TRY(launch::softmax_ce(logits, tgt, losses, (int)N, d.V, d.Vp, 1.0f / (float)N, train ? 1 : 0, err, s));
+    GPT2_TRY(launch::softmax_ce(logits, tgt, losses, (int)N, d.V, d.Vp, 1.0f / (float)N, train ? 1 : 0, err, s,
+                                INT_MIN, lse_part, lse_slots(d.Vp)));
     k::loss_reduce_kernel<<<1, 1024, 0, s>>>(losses, (int)N, loss_acc, &m->sc()->micro_loss);
-    prof_end(m, p, PC_CE, (double)N * d.Vp * (train ? 4.0 : 2.0), 2);
+    // algorithmic bytes: the logits read (and overwritten when training), or with
+    // the GEMM's partials those plus the partials, and no row scan for a loss alone
+    const double part_bytes = lse_part ? (double)N * lse_slots(d.Vp) * 8.0 : 0.0;
+    const double row_bytes = train ? 4.0 * d.Vp : (lse_part ? 2.0 : 2.0 * d.Vp);
+    prof_end(m, p, PC_CE, (double)N * row_bytes + part_bytes, 2);
   }
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
@@ -1091,6 +1110,33 @@ int gpt2op_softmax_ce(void* logits, const int32_t* targets, float* losses, int N
   if (!logits || !targets || !losses || !dev_err || N <= 0) return GPT2_ERR_ARG;
   return launch::softmax_ce(static_cast<bf16*>(logits), targets, losses, N, V, Vp, dscale, 1, dev_err,
                             static_cast<cudaStream_t>(stream));
+}
+
+size_t gpt2op_lm_head_ce_workspace(int N, int Vp) {
+  if (N <= 0 || Vp <= 0) return 0;
+  return (size_t)N * lse_slots(Vp) * 8;
+}
+
+int gpt2op_lm_head_ce(const void* h, const void* wte, const int32_t* targets, void* logits, float* losses, int N,
+                      int C, int V, int Vp, float dscale, int write_grad, void* workspace, size_t ws_bytes,
+                      int* dev_err, void* stream) {
+  if (!h || !wte || !targets || !logits || !losses || !dev_err || N <= 0 || C <= 0 || V <= 0 || V > Vp)
+    return GPT2_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  gemm::Call c = gemm_call(gemm::FWD, gemm::EPI_STORE, N, Vp, C, dev_err);
+  c.a = static_cast<const bf16*>(h); c.lda = C; c.b = static_cast<const bf16*>(wte); c.ldb = C;
+  c.out = static_cast<bf16*>(logits); c.ldo = Vp;
+  if (!workspace || ws_bytes < gpt2op_lm_head_ce_workspace(N, Vp) || (reinterpret_cast<uintptr_t>(workspace) & 7) != 0)
+    return GPT2_ERR_ARG;
+  float2* part = nullptr;
+  if (gemm2::uses_pair(c)) {
+    part = static_cast<float2*>(workspace);
+    c.epi = gemm::EPI_LSE; c.lse_part = part; c.lse_V = V;
+  }
+  const int st = gemm2::run(c, s);
+  if (st != GPT2_OK) return st;
+  return launch::softmax_ce(static_cast<bf16*>(logits), targets, losses, N, V, Vp, dscale, write_grad ? 1 : 0,
+                            dev_err, s, INT_MIN, part, lse_slots(Vp));
 }
 
 int gpt2op_softmax_ce_masked(void* logits, const int32_t* targets, float* losses, int N, int V, int Vp,

@@ -525,12 +525,15 @@ GPT2_DEV void ce_combine(float& m, float& s, float om, float os) {
 // ignore_index, when one is given, get loss 0 and a zero gradient): pass 1 streams the bf16 row
 // (kCeUnroll 16-byte loads in flight per thread) for the running (max, sum of
 // exp) over the real columns; pass 2 reads the row again (from L2) and
-// overwrites it with dz.
+// overwrites it with dz. With `part` given, pass 1 instead combines the row's
+// `slots` (max, sum) partials that the logits GEMM's epilogue left (the same
+// base-2 quantities over the same stored values), and the row is read once.
 __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict__ logits,
                                                                 const int32_t* __restrict__ targets,
                                                                 float* __restrict__ losses, int V, int Vp,
                                                                 float dscale, int write_grad, int* err,
-                                                                int ignore_index) {
+                                                                int ignore_index, const float2* __restrict__ part,
+                                                                int slots) {
   __shared__ float red_m[kCeThreads / 32], red_s[kCeThreads / 32];
   __shared__ float bc[2];
   const int row = blockIdx.x;
@@ -544,17 +547,25 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
     return;
   }
   float m = -INFINITY, s = 0.f;
-  for (int i0 = threadIdx.x; i0 < nv; i0 += kCeThreads * kCeUnroll) {
-    uint4 u[kCeUnroll];
-#pragma unroll
-    for (int k2 = 0; k2 < kCeUnroll; ++k2) {
-      const int i = i0 + k2 * kCeThreads;
-      u[k2] = i < nv ? __ldcg(zr + i) : make_uint4(0u, 0u, 0u, 0u);
+  if (part != nullptr) {
+    const float2* pr = part + (size_t)row * slots;
+    for (int i = threadIdx.x; i < slots; i += kCeThreads) {
+      const float2 v = __ldcs(pr + i);
+      ce_combine(m, s, v.x, v.y);
     }
+  } else {
+    for (int i0 = threadIdx.x; i0 < nv; i0 += kCeThreads * kCeUnroll) {
+      uint4 u[kCeUnroll];
 #pragma unroll
-    for (int k2 = 0; k2 < kCeUnroll; ++k2) {
-      const int i = i0 + k2 * kCeThreads;
-      if (i < nv) ce_accumulate(u[k2], i * 8, V, m, s);
+      for (int k2 = 0; k2 < kCeUnroll; ++k2) {
+        const int i = i0 + k2 * kCeThreads;
+        u[k2] = i < nv ? __ldcg(zr + i) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int k2 = 0; k2 < kCeUnroll; ++k2) {
+        const int i = i0 + k2 * kCeThreads;
+        if (i < nv) ce_accumulate(u[k2], i * 8, V, m, s);
+      }
     }
   }
 #pragma unroll

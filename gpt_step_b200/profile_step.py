@@ -15,6 +15,12 @@
       Times the causal attention forward or backward (head size 64) through the
       op-level C ABI and prints TFLOP/s (causal FLOPs incl. the diagonal block).
 
+  python -m gpt_step_b200.profile_step head --shape N,C,Vp [--iters n]
+      Times the tied lm_head + softmax-CE both ways: the plain GEMM followed by
+      the two-pass CE, and the GEMM whose epilogue leaves the row partials
+      followed by the one-pass CE (real vocabulary Vp - 47), each alone and
+      together, in milliseconds.
+
   python -m gpt_step_b200.profile_step bw --kernel ln_fwd|ln_bwd|ce|colsum --shape rows,C [--iters n]
       Times a bandwidth-bound kernel alone and prints GB/s of algorithmic bytes
       (for ce, C is the padded vocabulary and the real one is C - 47).
@@ -189,6 +195,50 @@ def run_bw(args):
                       "gbs": nbytes / (ms / 1000.0) / 1e9}))
 
 
+def _time(fn, iters):
+    import torch
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters
+
+
+def run_head(args):
+    import torch
+
+    import gpt_step_b200 as gs
+    from gpt_step_b200 import build
+    build.build()
+    N, C, Vp = (int(v) for v in args.shape.split(","))
+    V = Vp - 47
+    rng = np.random.default_rng(0)
+    bf = lambda s, sc: torch.tensor(rng.standard_normal(s).astype(np.float32) * sc).to(torch.bfloat16).cuda()
+    h, w = bf((N, C), 1.0), bf((Vp, C), 0.05)
+    t = torch.tensor(rng.integers(0, V, N), dtype=torch.int32, device="cuda")
+    logits = torch.empty(N, Vp, dtype=torch.bfloat16, device="cuda")
+    losses = torch.empty(N, device="cuda")
+    ws = torch.empty(gs.lm_head_ce_workspace(N, Vp), dtype=torch.uint8, device="cuda")
+    err = torch.zeros(4, dtype=torch.int32, device="cuda")
+    gemm = lambda: gs.linear_fwd(h, w, None, None, logits, err)
+    ce2 = lambda: gs.softmax_ce(logits, t, losses, V, 1.0 / N, err)
+    out = {"N": N, "C": C, "Vp": Vp}
+    out["gemm_store_ms"] = _time(gemm, args.iters)
+    out["gemm_lse_plus_loss_only_ms"] = _time(
+        lambda: gs.lm_head_ce(h, w, t, logits, losses, V, 1.0 / N, False, ws, err), args.iters)
+    out["ce_two_pass_ms"] = _time(lambda: (gemm(), ce2()), args.iters) - out["gemm_store_ms"]
+    out["unfused_total_ms"] = out["gemm_store_ms"] + out["ce_two_pass_ms"]
+    out["fused_total_ms"] = _time(lambda: gs.lm_head_ce(h, w, t, logits, losses, V, 1.0 / N, True, ws, err),
+                                  args.iters)
+    out["err"] = int(err.sum())
+    print(json.dumps(out))
+
+
 def main():
     ap = argparse.ArgumentParser()
     sub = ap.add_subparsers(dest="mode", required=True)
@@ -204,12 +254,15 @@ def main():
     a.add_argument("--dir", choices=["fwd", "bwd"], default="fwd")
     a.add_argument("--shape", default="19,1024,12")
     a.add_argument("--iters", type=int, default=20)
+    hp = sub.add_parser("head")
+    hp.add_argument("--shape", default="19456,768,50304")
+    hp.add_argument("--iters", type=int, default=20)
     w = sub.add_parser("bw")
     w.add_argument("--kernel", choices=["ln_fwd", "ln_bwd", "ce", "colsum"], default="ln_fwd")
     w.add_argument("--shape", default="19456,768")
     w.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()
-    {"step": run_step, "gemm": run_gemm, "attn": run_attn, "bw": run_bw}[args.mode](args)
+    {"step": run_step, "gemm": run_gemm, "attn": run_attn, "bw": run_bw, "head": run_head}[args.mode](args)
 
 
 if __name__ == "__main__":

@@ -115,6 +115,25 @@ int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, con
 int gpt2op_softmax_ce(void* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,
                       int* dev_err, void* stream);
 
+/* The tied lm_head and the softmax-CE as one op ("Pretraining and adapting a
+ * language model on a dependency-free stack" §4.1: logits = ln_f output x wte^T,
+ * softmax over the V real ids). h bf16 [N,C] and wte bf16 [Vp,C] row-major;
+ * logits bf16 [N,Vp] (caller-owned, 16-byte aligned) receive the logits, then,
+ * when write_grad is non-zero, are overwritten with dz exactly as
+ * gpt2op_softmax_ce does; losses fp32 [N]. When the GEMM runs on CTA pairs
+ * (N >= 256 rows and 256-wide tiles chosen, as for the model's logits), its
+ * epilogue also writes each row's running (max, sum of 2^) over every 128
+ * columns of the stored bf16 logits into the workspace, so the cross-entropy
+ * reads the logits once (not at all for losses alone); otherwise the two-pass
+ * kernel runs. The workspace (gpt2op_lm_head_ce_workspace bytes, 8-byte
+ * aligned, contents on entry irrelevant) is required either way. Errors as
+ * gpt2op_softmax_ce; a missing, short or misaligned workspace returns
+ * GPT2_ERR_ARG before any launch. */
+size_t gpt2op_lm_head_ce_workspace(int N, int Vp);
+int gpt2op_lm_head_ce(const void* h, const void* wte, const int32_t* targets, void* logits, float* losses, int N,
+                      int C, int V, int Vp, float dscale, int write_grad, void* workspace, size_t ws_bytes,
+                      int* dev_err, void* stream);
+
 /* Cross-entropy with an ignore index per target (the loss taken only on chosen
  * positions, e.g. the answers of question/answer text; "Pretraining and
  * adapting a language model on a dependency-free stack" trains its adapter that

@@ -172,6 +172,40 @@ def test_softmax_ce(N, V, Vp):
     assert int(err[0]) & 1
 
 
+@pytest.mark.parametrize("N,C,V,Vp", [(700, 256, 50257, 50304), (512, 768, 50257, 50304), (1024, 384, 4353, 4480),
+                                       (300, 256, 1000, 1024), (128, 128, 4353, 4480)])
+def test_lm_head_ce(N, C, V, Vp):
+    """Tied lm_head GEMM + softmax-CE. The first three shapes run the GEMM on CTA
+    pairs, whose epilogue leaves per-row (max, sum) partials so that the CE reads
+    the logits once (700 rows: a ragged last row tile); the last two take the
+    single-CTA GEMM and the two-pass CE. Losses agree with the oracle's CE of the stored bf16 logits
+    to fp32 rounding, padded columns (given large logits here) are left out, and
+    the gradient matches the oracle's."""
+    h, w = rnd((N, C), 29), rnd((Vp, C), 30, 0.05)
+    w[V:] = rnd((Vp - V, C), 31, 0.5)   # padded ids: large logits that must not count
+    t = np.random.default_rng(32).integers(0, V, N)
+    hd, wd, td = bf16(h), bf16(w), i32(t)
+    ws_bytes = gs.lm_head_ce_workspace(N, Vp)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+    logits = torch.empty(N, Vp, dtype=torch.bfloat16, device="cuda")
+    losses = torch.empty(N, device="cuda")
+    err = err_word()
+    gs.lm_head_ce(hd, wd, td, logits, losses, V, 1.0 / N, False, ws, err)
+    z = host(logits)
+    assert rel_l2(z, rounded(h) @ rounded(w).T) < BF16_TOL
+    lr, dzr = G.softmax_ce(z, t, V)
+    l0 = host(losses)
+    assert np.max(np.abs(l0 - lr)) < 1e-4
+    gs.lm_head_ce(hd, wd, td, logits, losses, V, 1.0 / N, True, ws, err)
+    assert np.array_equal(host(losses), l0)
+    dz = host(logits)
+    assert np.all(dz[:, V:] == 0.0)
+    assert rel_l2(dz[:, :V], dzr[:, :V]) < BF16_TOL
+    assert int(err.sum()) == 0
+    with pytest.raises(gs.GPT2Error):
+        gs.lm_head_ce(hd, wd, td, logits, losses, V, 1.0 / N, True, ws[: ws_bytes - 8], err)
+
+
 @pytest.mark.parametrize("N,V,Vp,ignore", [(64, 1000, 1024, -100), (37, 4353, 4480, -1), (16, 50257, 50304, -1)])
 def test_softmax_ce_masked(N, V, Vp, ignore):
     """Ignore index per target: ignored rows give loss 0 and an exactly zero
