@@ -15,8 +15,12 @@ A step is 9 x gpt2_fwd_bwd + gpt2_clip_adamw. `value` is whole-job tokens/s
 from CUDA events over exactly K steps (max over ranks). `e2e` repeats the
 measurement through gpt2_train_step_host with pinned host token buffers (the
 host->device copies and the loss/norm readback inside the timed region).
-With --gpus N each rank trains an independent replica on its own token stream
-(no gradient exchange), so scaling is weak.
+With --gpus N the ranks train one model data-parallel (the pages' multi-card
+arrangement, §4.4): each rank takes its own micro-batches from its own token
+stream, the fp32 gradients are averaged across ranks by one NCCL all-reduce
+before every clip + AdamW (gpt_step_b200.dp), and the weights stay identical
+(checked after the timed region). Per-rank work is fixed, so scaling is weak.
+--parallel replicas instead trains N independent replicas (no exchange).
 
 --impl reference times the CPU oracle (the fp64 numpy definition of the same
 step) on the host cores on a bounded sample of the same workload.
@@ -54,7 +58,7 @@ def load_peaks():
             "source": "fallback"}
 
 
-def workload_desc(w, n_gpus):
+def workload_desc(w, n_gpus, parallel="dp"):
     return {
         "workload": (f"GPT-2 124M training step: L{w['n_layer']} H{w['n_head']} C{w['n_embd']} "
                      f"T{w['seq_len']} V{w['vocab_real']}->50304, micro-batch {w['micro_batch']} x "
@@ -62,7 +66,9 @@ def workload_desc(w, n_gpus):
         "global_batch": w["micro_batch"] * w["grad_accum"] * n_gpus,
         "seq_len": w["seq_len"],
         "tokens_per_step": w["micro_batch"] * w["grad_accum"] * w["seq_len"] * n_gpus,
-        "parallelism": f"replicas x{n_gpus}" if n_gpus > 1 else "single GPU",
+        "parallelism": ("single GPU" if n_gpus == 1 else
+                        f"dp{n_gpus} (NCCL all-reduce of the fp32 gradients per optimizer step)"
+                        if parallel == "dp" else f"replicas x{n_gpus}"),
         "l2": "inputs larger than L2 (each micro-step touches ~8 GB of activations and logits)",
         "inputs": "synthetic Zipf(1.1) token stream, geometric(1000) documents, seed 1337+rank",
     }
@@ -189,6 +195,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--parallel", default="dp", choices=["dp", "replicas"])
     args = ap.parse_args()
 
     from gpt_step_b200.replicas import job_throughput, max_over_ranks, rank_env, replica_seed
@@ -215,7 +222,11 @@ def main():
     w = workloads.WORKLOADS[WORKLOAD]
     B, T, A = w["micro_batch"], w["seq_len"], w["grad_accum"]
     cfg = gs.Config.make(**workloads.model_args(WORKLOAD))
-    model = gs.GPT2(cfg, replica_seed(1337, rank))
+    dp_mode = args.parallel == "dp"
+    # data parallel: one model (the same initial weights everywhere), per-rank data
+    model = gs.GPT2(cfg, 1337 if dp_mode else replica_seed(1337, rank))
+    from gpt_step_b200.dp import DataParallel
+    par = DataParallel(model) if dp_mode else None
     n_steps = args.warmup + args.steps
     n_win = n_steps * A * B
     src = synth.TokenSource(B, T, cfg.vocab_real, replica_seed(1337, rank), w["mean_doc_len"], n_win)
@@ -233,6 +244,8 @@ def main():
         for a in range(A):
             j = i * A + a
             model.fwd_bwd(tok[j], tgt[j])
+        if par is not None:
+            par.sync_grads()           # no-op on one rank
         model.clip_adamw(i if sched is None else sched)
 
     def barrier():
@@ -267,6 +280,8 @@ def main():
     prof = model.profile_read()
     model.profile(False)
     barrier()
+    # every rank's weights must still be identical after the data-parallel steps
+    agree = par.replicas_agree() if (par is not None and world > 1) else None
     t_max = max_over_ranks(ms, device="cuda")
     tokens = args.steps * A * B * T * world
     value = job_throughput(args.steps * A * B * T, world, t_max)
@@ -278,19 +293,27 @@ def main():
         htgt = torch.empty((A, B, T), dtype=torch.int32, pin_memory=True)
         host_batches = [(np.stack(xs[i * A:(i + 1) * A]), np.stack(ys[i * A:(i + 1) * A]))
                         for i in range(args.warmup, n_steps)]
+        multi = par is not None and world > 1
+        if multi:   # the step needs the exchange between backward and update: dp's host path
+            dtok, dtgt = torch.empty((A, B, T), dtype=torch.int32, device="cuda"), torch.empty(
+                (A, B, T), dtype=torch.int32, device="cuda")
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for k, (hx, hy) in enumerate(host_batches):
             htok.numpy()[...] = hx
             htgt.numpy()[...] = hy
-            model.train_step_host_ptr(htok.data_ptr(), htgt.data_ptr(), A, 2 * n_steps + k)
+            if multi:
+                par.step_host(htok, htgt, dtok, dtgt, 2 * n_steps + k)
+            else:
+                model.train_step_host_ptr(htok.data_ptr(), htgt.data_ptr(), A, 2 * n_steps + k)
         e1.record(stream)
         barrier()
         ems = max_over_ranks(e0.elapsed_time(e1), device="cuda")
         e2e = {"value": job_throughput(args.steps * A * B * T, world, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": 2 * A * B * T * 4, "d2h_bytes_per_step": 8,
-               "api": "gpt2_train_step_host (pinned host tokens/targets)"}
+               "api": ("DataParallel.step_host (pinned host tokens/targets, NCCL gradient average)" if multi
+                       else "gpt2_train_step_host (pinned host tokens/targets)")}
 
     peaks = load_peaks()
     roof = None
@@ -312,12 +335,14 @@ def main():
             "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 3),
             "higher_is_better": True, "scaling": "weak",
             "vs_baseline": round(value / PAGES_TOKENS_PER_S, 3),
-            "dtype": "bf16", "data": "synthetic", "config": workload_desc(w, world),
+            "dtype": "bf16", "data": "synthetic", "config": workload_desc(w, world, args.parallel),
             "mfu": round(mfu, 4), "mfu_peak": f"{peaks['bf16_tflops']} TFLOP/s bf16 dense ({peaks['source']})",
             "loss": round(loss, 4), "grad_norm": round(norm, 4),
             "gpu_launches": int(launches), "clocks": clk, "roofline": roof, "e2e": e2e,
             "kernels": prof,
         }
+        if agree is not None:
+            line["replicas_agree"] = agree
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line), flush=True)

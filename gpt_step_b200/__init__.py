@@ -80,6 +80,7 @@ _SIGNATURES = {
                               ctypes.POINTER(_I)]),
     "gpt2_read": (_I, [_P, _I, _I, _FP]),
     "gpt2_write": (_I, [_P, _I, _I, _FP]),
+    "gpt2_state_device_ptr": (_I, [_P, _I, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(_I64)]),
     "gpt2op_linear_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "gpt2op_linear_fwd_gelu": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "gpt2op_linear_dgrad": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
@@ -284,6 +285,14 @@ class GPT2:
         if a.shape != info.shape:
             raise ValueError(f"{info.name}: shape {a.shape} != {info.shape}")
         check(lib().gpt2_write(self.h, what, idx, a.ctypes.data_as(_FP)), "gpt2_write")
+
+    def state_tensor(self, what: int):
+        """The flat fp32 state array `what` as a torch view of the arena (no copy)."""
+        ptr, n = ctypes.c_void_p(), ctypes.c_int64()
+        check(lib().gpt2_state_device_ptr(self.h, what, ctypes.byref(ptr), ctypes.byref(n)),
+              "gpt2_state_device_ptr")
+        off = ptr.value - self.arena.data_ptr()
+        return self.arena[off: off + 4 * n.value].view(self.torch.float32)
 
     def read_all(self, what: int) -> dict:
         return {t.name: self.read(what, i) for i, t in enumerate(self.tensors())}

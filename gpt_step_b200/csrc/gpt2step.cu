@@ -940,6 +940,15 @@ static float* state_array(gpt2_model* m, int what) {
   }
 }
 
+int gpt2_state_device_ptr(gpt2_model* m, int what, void** dev_ptr, int64_t* count) {
+  if (!m || !dev_ptr || !count) return GPT2_ERR_ARG;
+  float* base = state_array(m, what);
+  if (!base) return GPT2_ERR_ARG;
+  *dev_ptr = base;
+  *count = (int64_t)m->lay.P;
+  return GPT2_OK;
+}
+
 int gpt2_read(gpt2_model* m, int what, int idx, float* host_dst) {
   if (!m || !host_dst || idx < 0 || idx >= (int)m->tensors.size()) return GPT2_ERR_ARG;
   float* base = state_array(m, what);

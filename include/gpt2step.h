@@ -156,6 +156,16 @@ int gpt2_tensor_info(const gpt2_model* model, int idx, const char** name, int64_
 int gpt2_read(gpt2_model* model, int what, int idx, float* host_dst);
 int gpt2_write(gpt2_model* model, int what, int idx, const float* host_src);
 
+/* Device address and length (fp32 elements, padded flat layout: every tensor
+ * at a 64-element aligned offset, gaps zero) of the whole state array `what`
+ * inside the caller's arena, for collectives over it: data-parallel ranks
+ * ("Pretraining and adapting a language model on a dependency-free stack",
+ * §4.4, three cards) average GPT2_GRADS across ranks between their last
+ * gpt2_fwd_bwd and gpt2_clip_adamw, on the model's stream. Valid while the
+ * model lives; no copy, no synchronisation. Writing GPT2_PARAMS through it
+ * does not refresh the bf16 copy (use gpt2_write). */
+int gpt2_state_device_ptr(gpt2_model* model, int what, void** dev_ptr, int64_t* count);
+
 /* Total parameter count: real vocabulary rows only (124,439,808 for GPT-2
  * 124M, §4.1) when padded == 0, all stored rows when padded != 0. */
 int64_t gpt2_num_params(const gpt2_config* cfg, int padded);

@@ -347,3 +347,43 @@ def test_checkpoint_resume_continues_the_run(tmp_path):
         assert np.max(np.abs(a.read(gs.GPT2_PARAMS, i) - b.read(gs.GPT2_PARAMS, i))) <= 2e-6, t.name
     a.close()
     b.close()
+
+
+def test_data_parallel_plumbing_on_one_rank():
+    """The flat gradient array that data-parallel ranks average (gpt2_state_device_ptr)
+    is the one gpt2_read reports, padded gaps zero; an NCCL average over a one-rank
+    group leaves it bit-identical; and DataParallel's step on one rank runs the
+    plain step and keeps the weights finite."""
+    import socket
+
+    import torch.distributed as dist
+    from gpt_step_b200 import dp
+    args = workloads.model_args("tiny")
+    m = gs.GPT2(gs.Config.make(**args), 1337)
+    x, y = synth.uniform_next_token_batch(args["micro_batch"], args["seq_len"], args["vocab_real"], 77)
+    m.fwd_bwd(i32(x), i32(y))
+    torch.cuda.synchronize()
+    g = m.state_tensor(gs.GPT2_GRADS)
+    per = sum(float(np.abs(m.read(gs.GPT2_GRADS, i).astype(np.float64)).sum()) for i in range(len(m.tensors())))
+    assert per > 0 and float(g.double().abs().sum()) == pytest.approx(per, rel=1e-12)
+    before = g.clone()
+    own = not dist.is_initialized()
+    if own:
+        with socket.socket() as s:
+            s.bind(("127.0.0.1", 0))
+            port = s.getsockname()[1]
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        dist.all_reduce(g, op=dist.ReduceOp.AVG)
+        torch.cuda.synchronize()
+        assert torch.equal(g, before)
+        d = dp.DataParallel(m)
+        assert d.world == 1
+        m.clip_adamw(0)
+        d.step([i32(x)], [i32(y)], 1)
+        loss, norm = m.last_step_stats()
+        assert math.isfinite(loss) and math.isfinite(norm) and d.replicas_agree()
+    finally:
+        if own:
+            dist.destroy_process_group()
+    m.close()
