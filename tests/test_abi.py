@@ -72,3 +72,21 @@ def test_noalloc_layernorm_bwd_rejects_oversized_calls_before_touching_the_gpu(l
     st = lib.gpt2op_layernorm_bwd_noalloc(dummy, dummy, dummy, dummy, dummy, None, dummy, dummy, dummy,
                                           100000, 1536, None)
     assert st == 1                # GPT2_ERR_ARG
+
+
+def test_head_and_masked_ce_reject_bad_arguments_before_touching_the_gpu(lib):
+    """Argument errors of the newer entry points come back as GPT2_ERR_ARG from
+    host-side checks alone (dummy pointers are never dereferenced)."""
+    assert lib.gpt2op_lm_head_ce_workspace(19456, 50304) == 19456 * 2 * 197 * 8
+    assert lib.gpt2op_lm_head_ce_workspace(0, 50304) == 0
+    d = ctypes.c_void_p(16)
+    f = ctypes.c_float(1.0)
+    # null input, V > Vp, missing workspace, short workspace
+    assert lib.gpt2op_lm_head_ce(None, d, d, d, d, 256, 64, 100, 128, f, 1, d, 1 << 20, d, None) == 1
+    assert lib.gpt2op_lm_head_ce(d, d, d, d, d, 256, 64, 129, 128, f, 1, d, 1 << 20, d, None) == 1
+    assert lib.gpt2op_lm_head_ce(d, d, d, d, d, 256, 64, 100, 128, f, 1, None, 1 << 20, d, None) == 1
+    assert lib.gpt2op_lm_head_ce(d, d, d, d, d, 256, 64, 100, 128, f, 1, d, 256 * 8 - 8, d, None) == 1
+    # the masked CE needs an ignore index (INT_MIN means none)
+    assert lib.gpt2op_softmax_ce_masked(d, d, d, 4, 100, 128, -2 ** 31, f, d, None) == 1
+    ptr, n = ctypes.c_void_p(), ctypes.c_int64()
+    assert lib.gpt2_state_device_ptr(None, 1, ctypes.byref(ptr), ctypes.byref(n)) == 1
