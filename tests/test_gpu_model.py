@@ -307,6 +307,49 @@ def test_gpt2_124m_bench_configuration_sampled():
     assert np.all(m.read(gs.GPT2_PARAMS, 0)[ocfg.V:] == 0.0)
 
 
+def test_gpt2_124m_micro_batch_64_with_held_out_pass_sampled():
+    """The large-micro-batch 124M configuration (64 x 1024 per micro-step) and its
+    held-out pass (batches of 64 x 1024 from a separately seeded stream): the
+    micro-step's per-token losses on a sampled sequence against the oracle, and the
+    held-out loss equal to the forward's mean loss on the same batch."""
+    m, ocfg = pair("gpt2_124m_b64")
+    w = workloads.WORKLOADS["gpt2_124m_b64"]
+    (x, y), = batch_for("gpt2_124m_b64", ocfg)
+    loss = m.fwd_bwd(i32(x), i32(y), want_loss=True)
+    tl = m.token_losses()
+    assert tl.shape == (64, 1024) and float(tl.mean()) == pytest.approx(loss, abs=1e-4)
+    p = G.init_params(ocfg, 1337)
+    ref = G.token_losses(ocfg, p, x[63:64], y[63:64])[0]
+    assert abs(float(tl[63].mean()) - float(ref.mean())) <= LOSS_TOL
+    assert np.max(np.abs(tl[63] - ref)) < 0.15
+    assert np.isfinite(m.clip_adamw(0, want_norm=True))
+    src = synth.TokenSource(w["eval_batch"], ocfg.T, ocfg.V, w["eval_seed"], w["mean_doc_len"], w["eval_batch"])
+    ex, ey = src.get()
+    ev = m.eval_loss(i32(ex), i32(ey))
+    assert ev == pytest.approx(m.fwd_bwd(i32(ex), i32(ey), want_loss=True), abs=1e-5)
+    m.close()
+
+
+def test_wide_configuration_sampled():
+    """The wide configuration (16 blocks, 24 heads, 1536 channels, vocabulary 8449
+    padded to 8576, micro-batch 8): per-token losses of a sampled sequence against
+    the oracle, finite gradients with zero padded rows, a finite clipped step."""
+    m, ocfg = pair("wide")
+    (x, y), = batch_for("wide", ocfg)
+    loss = m.fwd_bwd(i32(x), i32(y), want_loss=True)
+    tl = m.token_losses()
+    assert float(tl.mean()) == pytest.approx(loss, abs=1e-4)
+    p = G.init_params(ocfg, 1337)
+    ref = G.token_losses(ocfg, p, x[0:1], y[0:1])[0]
+    assert abs(float(tl[0].mean()) - float(ref.mean())) <= LOSS_TOL
+    assert np.max(np.abs(tl[0] - ref)) < 0.15
+    g = m.read_all(gs.GPT2_GRADS)
+    assert np.all(g["wte.weight"][ocfg.V:] == 0.0)
+    assert all(np.all(np.isfinite(a)) for a in g.values())
+    assert np.isfinite(m.clip_adamw(0, want_norm=True))
+    m.close()
+
+
 def test_checkpoint_resume_continues_the_run(tmp_path):
     """A run stopped at a checkpoint and restored into a model of another seed
     continues the uninterrupted run: the restored fp32 weights and moments are
