@@ -135,7 +135,7 @@ def ckpt_path(directory: str, step: int, prefix: str = "step_") -> str:
 
 
 def run(model, source, first_step: int, last_step: int, put, cadence: Cadence,
-        ckpt_dir: str | None = None, evaluate=None, log=None) -> list:
+        ckpt_dir: str | None = None, evaluate=None, log=None, par=None) -> list:
     """Optimizer steps ``first_step .. last_step-1`` with the eval and checkpoint cadence.
 
     ``source.get()`` yields host (tokens, targets) micro-batches and carries the
@@ -144,20 +144,30 @@ def run(model, source, first_step: int, last_step: int, put, cadence: Cadence,
     ``grad_accum`` micro-steps, then the clip + AdamW step. Returns the log
     records (one per step: step, the mean loss over its micro-steps, the
     pre-clip gradient norm, and the eval loss where one was due).
+
+    With ``par`` (a ``dp.DataParallel``) the run is one rank of a data-parallel
+    job: gradients are averaged across ranks before each update, the logged
+    and held-out losses are averaged across ranks, and rank 0 alone writes the
+    checkpoints. Every rank's data cursor advances alike (same micro-batch
+    count per step), so rank 0's cursor is every rank's.
     """
     records = []
     accum = model.cfg.grad_accum
+    mean = (lambda v: par.mean_over_ranks(v)) if par is not None else (lambda v: v)
+    writer = par is None or par.rank == 0
     for step in range(first_step, last_step):
         for _ in range(accum):
             x, y = source.get()
             model.fwd_bwd(put(x), put(y))
+        if par is not None:
+            par.sync_grads()
         model.clip_adamw(step)
         loss, norm = model.last_step_stats()
-        rec = {"step": step, "loss": loss, "grad_norm": norm}
+        rec = {"step": step, "loss": mean(loss), "grad_norm": norm}
         done = step + 1
         if evaluate is not None and cadence.eval_due(done):
-            rec["eval_loss"] = evaluate(model)
-        if ckpt_dir is not None and cadence.ckpt_due(done):
+            rec["eval_loss"] = mean(evaluate(model))
+        if ckpt_dir is not None and cadence.ckpt_due(done) and writer:
             os.makedirs(ckpt_dir, exist_ok=True)
             rec["checkpoint"] = save(model, ckpt_path(ckpt_dir, done), done, getattr(source, "next", None))
         records.append(rec)

@@ -147,3 +147,102 @@ def test_single_process_is_the_plain_step():
     ref.clip_adamw(0)
     assert torch.equal(m.p, ref.p)
     assert d.mean_over_ranks(2.5) == 2.5 and d.replicas_agree()
+
+
+# --- data parallel with the checkpoint / eval cadence ----------------------------------------
+
+class CkptFake(FakeModel):
+    """FakeModel in fp32 with the state interface a checkpoint needs."""
+
+    class Cfg(dict):
+        grad_accum = 2
+
+    def __init__(self, seed=0):
+        super().__init__(seed)
+        self.p = self.p.float()
+        self.g = self.g.float()
+        self.mom = {2: torch.zeros(N), 3: torch.zeros(N)}
+        self.cfg = CkptFake.Cfg(n_embd=N, grad_accum=2)
+
+    def fwd_bwd(self, x, y):
+        f = _feat(x, y).float()
+        self.g += 0.3 * self.p - f
+        self.losses.append(float(f.sum()))
+        self.k += 1
+
+    def eval_loss(self, x, y):
+        return float(_feat(x, y).float() @ self.p)
+
+    def tensors(self):
+        from types import SimpleNamespace
+        return [SimpleNamespace(name="w", shape=(N,))]
+
+    def read(self, what, i):
+        return (self.p if what == dp.PARAMS else self.mom[what]).numpy().copy()
+
+    def write(self, what, i, a):
+        t = torch.tensor(a)
+        if what == dp.PARAMS:
+            self.p = t
+        else:
+            self.mom[what] = t
+
+
+class RankSource:
+    def __init__(self, rank):
+        self.rank, self.next = rank, 0
+
+    def get(self):
+        rng = np.random.default_rng(7919 * self.rank + self.next)
+        self.next += 1
+        return rng.integers(0, 50, (2, 8)), rng.integers(0, 50, (2, 8))
+
+
+def _ckpt_rank_main(rank, world, port, q, root):
+    import os
+
+    import torch.distributed as dist
+
+    from gpt_step_b200 import checkpoint as ck
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        cad = ck.Cadence(eval_every=2, ckpt_every=2)
+        ex, ey = _batches(5, 0, rank, world)
+        ev = lambda m: m.eval_loss(ex, ey)
+        ident = lambda a: a
+        a = CkptFake()
+        ra = ck.run(a, RankSource(rank), 0, 4, ident, cad, os.path.join(root, "a"), ev, par=dp.DataParallel(a))
+        b = CkptFake()
+        ck.run(b, RankSource(rank), 0, 2, ident, cad, os.path.join(root, "b"), ev, par=dp.DataParallel(b))
+        dist.barrier()                           # rank 0 has written step 2
+        c = CkptFake(seed=5)
+        h = ck.load(c, ck.latest(os.path.join(root, "b")))
+        s = RankSource(rank)
+        s.next = h["data_cursor"]
+        rc = ck.run(c, s, h["step"], 4, ident, cad, None, ev, par=dp.DataParallel(c))
+        strip = lambda recs: [{k: v for k, v in r.items() if k != "checkpoint"} for r in recs]
+        q.put((rank, a.p.tolist(), c.p.tolist(), strip(ra), strip(ra[:2]) + strip(rc),
+               sorted(os.listdir(os.path.join(root, "b")))))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_data_parallel_run_checkpoints_on_rank_0_and_resumes(tmp_path):
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ckpt_rank_main, args=(r, world, port, q, str(tmp_path))) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, pa, pc, ra, rresumed, files in out:
+        assert pa == pc                          # stop, restore, continue = straight run, bitwise
+        assert ra == rresumed                    # same logged (rank-averaged) losses and evals
+        assert files == ["step_0000002.npz"]     # rank 0 alone wrote, once
+    assert out[0][1] == out[1][1]                # ranks hold the same weights
+    assert out[0][3] == out[1][3]                # and log the same averaged values
+    assert [r["step"] for r in out[0][3] if "eval_loss" in r] == [1, 3]
