@@ -58,11 +58,17 @@ def save(model, path: str, step: int, data_cursor: int | None = None) -> str:
               "config": _config_dict(model.cfg), "tensors": names}
     arrays["header"] = np.frombuffer(json.dumps(header).encode(), dtype=np.uint8)
     tmp = f"{path}.tmp-{os.getpid()}"
-    with open(tmp, "wb") as f:
-        np.savez(f, **arrays)
-        f.flush()
-        os.fsync(f.fileno())
-    os.replace(tmp, path)
+    try:
+        with open(tmp, "wb") as f:
+            np.savez(f, **arrays)
+            f.flush()
+            os.fsync(f.fileno())
+        os.replace(tmp, path)
+    except BaseException:
+        # a failed save leaves any earlier checkpoint at `path` as it was
+        if os.path.exists(tmp):
+            os.remove(tmp)
+        raise
     return path
 
 

@@ -160,3 +160,21 @@ def test_resume_continues_instead_of_repeating(tmp_path):
     for w in a.state:
         for x, y in zip(a.state[w], c.state[w]):
             assert np.array_equal(x, y)
+
+
+def test_failed_save_keeps_the_previous_checkpoint(tmp_path, monkeypatch):
+    a = FakeModel(1)
+    p = ck.save(a, str(tmp_path / "c.npz"), 5, data_cursor=10)
+    b = FakeModel(2)
+
+    def boom(*args, **kw):
+        raise OSError("disk full")
+    monkeypatch.setattr(ck.np, "savez", boom)
+    with pytest.raises(OSError):
+        ck.save(b, p, 6, data_cursor=12)
+    monkeypatch.undo()
+    assert os.listdir(tmp_path) == ["c.npz"]          # no temporary left behind
+    c = FakeModel(3)
+    h = ck.load(c, p)
+    assert h["step"] == 5 and h["data_cursor"] == 10
+    assert all(np.array_equal(x, y) for x, y in zip(a.state[ck.PARAMS], c.state[ck.PARAMS]))
