@@ -267,3 +267,28 @@ def test_zero_layer_model_is_logistic_regression():
     head = (probs - Y).T @ F / F.shape[0]
     untouched = np.setdiff1d(np.arange(cfg.V), x.reshape(-1))
     np.testing.assert_allclose(g["wte"][untouched], head[untouched], rtol=1e-11, atol=1e-15)
+
+
+def test_equal_shards_average_to_the_whole_batch():
+    """The mean loss over a batch is the mean of its equal-sized shards' mean
+    losses, so its gradient is the mean of theirs. Gradient accumulation
+    ("Pretraining and adapting a language model on a dependency-free stack"
+    §4.3, 9 micro-steps per optimizer step) and the average across cards (§4.4)
+    both rely on this. So one optimizer step over 4 sequences must equal one
+    step accumulated over two shards of 2, with the same pre-clip norm."""
+    cfg = G.Config(**dict(MICRO, micro_batch=4))
+    p = perturbed_params(cfg, 23)
+    x, y = micro_batch(cfg, 24)
+    loss, g = G.fwd_bwd(cfg, p, x, y)
+    l0, g0 = G.fwd_bwd(cfg, p, x[:2], y[:2])
+    l1, g1 = G.fwd_bwd(cfg, p, x[2:], y[2:])
+    assert loss == pytest.approx(0.5 * (l0 + l1), rel=1e-13)
+    for k in g:
+        np.testing.assert_allclose(g[k], 0.5 * (g0[k] + g1[k]), rtol=1e-10, atol=1e-15)
+    pa, pb = {k: v.copy() for k, v in p.items()}, {k: v.copy() for k, v in p.items()}
+    ma, va, mb, vb = (G.zeros_like_params(cfg) for _ in range(4))
+    la, na = G.train_step(cfg, pa, ma, va, 3, [(x, y)])
+    lb, nb = G.train_step(cfg, pb, mb, vb, 3, [(x[:2], y[:2]), (x[2:], y[2:])])
+    assert la == pytest.approx(lb, rel=1e-13) and na == pytest.approx(nb, rel=1e-10)
+    for k in pa:
+        np.testing.assert_allclose(pa[k], pb[k], rtol=0, atol=1e-12)
