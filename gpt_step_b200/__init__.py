@@ -68,6 +68,7 @@ _SIGNATURES = {
     "gpt2_train_step_host": (_I, [_P, _P, _P, _I32, _I32, _FP, _FP]),
     "gpt2_token_losses": (_I, [_P, _FP, _I64]),
     "gpt2_lr": (_F, [_P, _I32]),
+    "gpt2_schedule_lr": (ctypes.c_double, [ctypes.POINTER(Config), _I32]),
     "gpt2_kernel_launches": (_I64, [_P]),
     "gpt2_profile_enable": (_I, [_P, _I]),
     "gpt2_profile_num_classes": (_I, []),
@@ -85,6 +86,7 @@ _SIGNATURES = {
     "gpt2op_linear_fwd_gelu": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "gpt2op_linear_dgrad": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "gpt2op_linear_wgrad": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
+    "gpt2op_linear_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, ctypes.POINTER(_I), _P, _P]),
     "gpt2op_bias_grad_workspace": (_SZ, [_I, _I]),
     "gpt2op_bias_grad": (_I, [_P, _P, _I, _I, _P, _SZ, _P]),
     "gpt2op_layernorm_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _P]),
@@ -101,6 +103,7 @@ _SIGNATURES = {
     "gpt2op_lm_head_ce": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P]),
     "gpt2op_embedding_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "gpt2op_embedding_bwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "gpt2op_wait_selftest": (_I, [_I64, _P, _P]),
 }
 
 
@@ -149,6 +152,11 @@ def _stream_handle(stream=None):
 
 def arena_bytes(cfg: Config) -> int:
     return lib().gpt2_arena_bytes(ctypes.byref(cfg))
+
+
+def schedule_lr(cfg: Config, step: int) -> float:
+    """The learning-rate schedule of `cfg` at `step` (host arithmetic in the library)."""
+    return lib().gpt2_schedule_lr(ctypes.byref(cfg), step)
 
 
 def num_params(cfg: Config, padded: bool = False) -> int:
@@ -334,6 +342,22 @@ def linear_wgrad(dout, inp, dw, err, splits=0, stream=None):
     K = inp.shape[1]
     check(lib().gpt2op_linear_wgrad(_ptr(dout), _ptr(inp), _ptr(dw), M, N, K, splits, _ptr(err),
                                     _s(stream)), "gpt2op_linear_wgrad")
+
+
+def linear_bwd(dout, w, inp, gelu_pre, din, dw, colsum, err, stream=None) -> int:
+    """Grouped input + weight gradient of a linear layer; returns the dw reduction split."""
+    M, N = dout.shape
+    K = w.shape[1]
+    sp = ctypes.c_int()
+    check(lib().gpt2op_linear_bwd(_ptr(dout), _ptr(w), _ptr(inp), _ptr(gelu_pre), _ptr(din), _ptr(dw),
+                                  _ptr(colsum), M, N, K, ctypes.byref(sp), _ptr(err), _s(stream)),
+          "gpt2op_linear_bwd")
+    return sp.value
+
+
+def wait_selftest(limit_ns, err, stream=None) -> int:
+    """Run the bounded-wait self-test; returns the raw status (6 = timed out as designed)."""
+    return lib().gpt2op_wait_selftest(int(limit_ns), _ptr(err), _s(stream))
 
 
 def bias_grad_workspace(M, N):

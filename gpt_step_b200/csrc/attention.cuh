@@ -512,12 +512,9 @@ constexpr int bwd_smem() {
 
 template <int HD>
 static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, fwd_smem<HD>());
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static PerDeviceOnce once;
+  cudaError_t e = smem_optin(once, attn_fwd_kernel<HD>, fwd_smem<HD>());
+  if (e != cudaSuccess) return e;
   dim3 grid(T / BLK, B * H);
   attn_fwd_kernel<HD><<<grid, 128, fwd_smem<HD>(), s>>>(qkv, out, lse, T, H, 1.0f / sqrtf((float)HD));
   return cudaGetLastError();
@@ -527,12 +524,9 @@ static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int
 template <int HD>
 static cudaError_t bwd(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dv,
                        float* dq_acc, bf16* dqkv, int B, int T, int H, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(attn_bwd_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd_smem<HD>());
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static PerDeviceOnce once;
+  cudaError_t e = smem_optin(once, attn_bwd_kernel<HD>, bwd_smem<HD>());
+  if (e != cudaSuccess) return e;
   const int rows = B * T * H;
   attn_bwd_dot_kernel<HD><<<(rows + 255) / 256, 256, 0, s>>>(out, dout, Dv, B, T, H);
   const int C = H * HD;

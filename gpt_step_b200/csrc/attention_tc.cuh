@@ -331,15 +331,14 @@ __global__ void __launch_bounds__(kThreads, 2)
 
 // qkv bf16 [B*T, 3C] (q | k | v, heads contiguous), out bf16 [B*T, C], lse fp32 [B, H, T].
 static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, int* err, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
+  static PerDeviceOnce once;
+  cudaError_t e0 = once.run([] {
     cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // ask for the whole shared-memory carveout so that two CTAs share an SM
-    e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  });
+  if (e0 != cudaSuccess) return e0;
   const int C = H * HD;
   CUtensorMap tm;
   if (!encode_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qkv, 3 * (uint64_t)C, (uint64_t)B * T, 3 * (uint64_t)C,
@@ -846,18 +845,17 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 // scratch (contents on entry do not matter); dqkv receives dQ | dK | dV.
 static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, uint8_t* xtiles,
                        float* dq_acc, bf16* dqkv, int B, int T, int H, int* err, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
+  static PerDeviceOnce once;
+  cudaError_t e0 = once.run([] {
     // The register hand-over inside the kernel needs the block to be launched
     // with kLaunchRegs registers a thread; anything less would stall it.
     cudaFuncAttributes fa;
     cudaError_t e = cudaFuncGetAttributes(&fa, attn_bwd_tc_kernel);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != bwd::kLaunchRegs) return cudaErrorInvalidConfiguration;
-    e = cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+    return cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::SMEM_BYTES);
+  });
+  if (e0 != cudaSuccess) return e0;
   if (H > bwd::kMaxHeads || T % bwd::kPrepRows) return cudaErrorInvalidValue;
   const int C = H * HD;
   const float scale = 1.0f / sqrtf((float)HD);
@@ -871,13 +869,7 @@ static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, c
     return cudaErrorInvalidValue;
   bwd_prep_kernel<<<B * T / bwd::kPrepRows, 256, 0, s>>>(out, dout, lse, xtiles, dq_acc, T, H, scale);
   const int n_items = (T / bwd::BKEY) * B * H;
-  static int sms = 0;   // one persistent CTA per SM
-  if (sms == 0) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return cudaErrorInvalidValue;
-    sms = v;
-  }
+  const int sms = device_sm_count();   // one persistent CTA per SM
   const int grid = n_items < sms ? n_items : sms;
   attn_bwd_tc_kernel<<<grid, bwd::kThreads, bwd::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, xtiles, dqkv, T, H, B * H, scale,
                                                                   err);

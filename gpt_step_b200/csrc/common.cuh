@@ -10,6 +10,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/gpt2step.h"
 
 typedef __nv_bfloat16 bf16;
@@ -73,21 +76,25 @@ GPT2_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete. Returns false (and
-// records a timeout) if it does not within kWaitLimitNs, or immediately if
-// another thread of the grid already recorded an error.
-GPT2_DEV bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+// records a timeout) if it does not within limit_ns, or as soon as another
+// thread of the grid has recorded a timeout.
+GPT2_DEV bool mbar_wait_limit(uint32_t bar, uint32_t parity, int* err, unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*(volatile int*)err & DEVERR_TIMEOUT) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         atomicOr(err, DEVERR_TIMEOUT);
         return false;
       }
     }
   }
+}
+
+GPT2_DEV bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
+  return mbar_wait_limit(bar, parity, err, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------------------
@@ -266,17 +273,64 @@ GPT2_DEV float gelu_grad_f(float u) {
 }
 
 // ---------------------------------------------------------------------------
+// host: one-time set-up per device (function attributes are per context)
+// ---------------------------------------------------------------------------
+// Runs `fn` (returning cudaError_t) once on each device that calls it, with
+// that device current; safe to call from several host threads. A failed
+// attempt is retried on the next call.
+struct PerDeviceOnce {
+  static constexpr int kMaxDevices = 64;
+  std::atomic<uint64_t> done{0};
+  std::mutex mu;
+  template <typename Fn>
+  cudaError_t run(Fn&& fn) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    const uint64_t bit = 1ull << dev;
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+    e = fn();
+    if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_release);
+    return e;
+  }
+};
+
+// Opt `kern` into `bytes` of dynamic shared memory on the current device (once per device).
+template <typename K>
+inline cudaError_t smem_optin(PerDeviceOnce& once, K* kern, int bytes) {
+  return once.run([&] {
+    return cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                bytes);
+  });
+}
+
+// Number of SMs of the current device.
+inline int device_sm_count() {
+  static std::atomic<int> cached[PerDeviceOnce::kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= PerDeviceOnce::kMaxDevices) return 148;
+  int v = cached[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+  cached[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
+
+// ---------------------------------------------------------------------------
 // host: tensor-map encoding through the driver entry point (no libcuda link)
 // ---------------------------------------------------------------------------
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+  }();
   return fn;
 }
 

@@ -339,29 +339,16 @@ static bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t 
   return encode_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, inner, outer, ld, box_inner, box_outer, swz);
 }
 
-static int g_num_sms = 0;
-
-static int num_sms() {
-  if (g_num_sms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_num_sms <= 0) g_num_sms = 148;
-  }
-  return g_num_sms;
-}
+static int num_sms() { return device_sm_count(); }
 
 template <int BN, bool A_MN, bool B_MN, int EPI>
 static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
                              const CUtensorMap& to2, Params p, cudaStream_t s) {
   using C = Cfg<BN>;
   auto kern = gemm_tc_kernel<BN, A_MN, B_MN, EPI>;
-  static bool attr_set = false;  // per template instance
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce once;  // per template instance
+  const cudaError_t e = smem_optin(once, kern, C::SMEM);
+  if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
   kern<<<grid, kThreads, C::SMEM, s>>>(ta, tb, to, to2, p);
   return cudaGetLastError();

@@ -492,12 +492,9 @@ static cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& tb, cons
                               const Params* p1 = nullptr) {
   using C = Cfg<BN>;
   auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EPI, GROUP>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  static PerDeviceOnce once;  // per template instance
+  const cudaError_t e = smem_optin(once, kern, C::SMEM);
+  if (e != cudaSuccess) return e;
   Params q1{};
   if (GROUP) q1 = *p1;
   const int total = p.num_tiles + q1.num_tiles;
@@ -630,12 +627,14 @@ static int run(const gemm::Call& c, cudaStream_t s) {
 // launch: c1's tiles follow c0's in the persistent tile list, its reduction
 // split chosen so that its tiles carry about as many k-blocks as c0's. Falls
 // back to two launches when either product does not take the pair kernel.
-static int run_group(const gemm::Call& c0, const gemm::Call& c1, cudaStream_t s, int* launches) {
+static int run_group(const gemm::Call& c0, const gemm::Call& c1, cudaStream_t s, int* launches,
+                     int* splits_out = nullptr) {
   using namespace gemm;
   const bool ok_shapes = c0.kind == DGRAD && c1.kind == WGRAD && c1.epi == EPI_ACC_F32 && c0.M > 0 &&
                          c0.N % 32 == 0 && c0.K % BK == 0 && c1.K % BK == 0 && c1.K > 0 && uses_pair(c0) &&
                          uses_pair(c1) && c1.N % 256 == 0;
   *launches = ok_shapes ? 1 : 2;
+  if (splits_out) *splits_out = 0;
   if (!ok_shapes) {
     const int st = gemm2::run(c0, s);
     return st != GPT2_OK ? st : gemm2::run(c1, s);
@@ -666,6 +665,7 @@ static int run_group(const gemm::Call& c0, const gemm::Call& c1, cudaStream_t s,
   }
   st = prepare(c1, splits1, p1, ta1, tb1, to1, to21);
   if (st != GPT2_OK) return st;
+  if (splits_out) *splits_out = p1.splits;
   cudaError_t e = cudaErrorInvalidValue;
   switch (c0.epi) {
     case EPI_STORE: e = launch_tc2<256, false, true, EPI_STORE, true>(ta0, tb0, to0, to20, p0, s, &ta1, &tb1, &p1); break;

@@ -260,16 +260,15 @@ static_assert(148 * 2 <= kLnBwdBlocks, "LayerNorm partial rows");
 size_t ln_bwd_workspace(int rows, int C, int nq = 2) { return (size_t)ln_bwd_blocks(rows, C) * nq * C * 4; }
 
 template <int C>
-void ln_bwd_c(const bf16* dy, const bf16* x, const float* mean, const float* rstd, const float* w,
-              const bf16* dresid, bf16* dx, float* part, int rows, int blocks, int with_dxsum, cudaStream_t s) {
+cudaError_t ln_bwd_c(const bf16* dy, const bf16* x, const float* mean, const float* rstd, const float* w,
+                     const bf16* dresid, bf16* dx, float* part, int rows, int blocks, int with_dxsum, cudaStream_t s) {
   using Cfg = k::LnBwdCfg<C>;
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(k::layernorm_bwd_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::SMEM);
-    attr = true;
-  }
+  static PerDeviceOnce once;
+  const cudaError_t e = smem_optin(once, k::layernorm_bwd_kernel<C>, Cfg::SMEM);
+  if (e != cudaSuccess) return e;
   k::layernorm_bwd_kernel<C><<<blocks, Cfg::WARPS * 32, Cfg::SMEM, s>>>(dy, x, mean, rstd, w, dresid, dx, part, rows,
                                                                         with_dxsum);
+  return cudaGetLastError();
 }
 
 // dbias (may be NULL) receives the column sum of dx: the bias gradient of the
@@ -281,17 +280,19 @@ int ln_bwd(const bf16* dy, const bf16* x, const float* mean, const float* rstd, 
   const int blocks = ln_bwd_blocks(rows, C);
   if (part_bytes < (size_t)blocks * nq * C * 4) return GPT2_ERR_ARG;
   const int wd = dbias ? 1 : 0;
+  cudaError_t e;
   switch (C) {
-    case 128: ln_bwd_c<128>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 256: ln_bwd_c<256>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 384: ln_bwd_c<384>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 512: ln_bwd_c<512>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 768: ln_bwd_c<768>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 1024: ln_bwd_c<1024>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 1536: ln_bwd_c<1536>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 2048: ln_bwd_c<2048>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 128: e = ln_bwd_c<128>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 256: e = ln_bwd_c<256>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 384: e = ln_bwd_c<384>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 512: e = ln_bwd_c<512>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 768: e = ln_bwd_c<768>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 1024: e = ln_bwd_c<1024>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 1536: e = ln_bwd_c<1536>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+    case 2048: e = ln_bwd_c<2048>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
     default: return GPT2_ERR_ARG;
   }
+  if (e != cudaSuccess) return GPT2_ERR_CUDA;
   k::partial_rows_reduce_kernel<<<(nq * C + 31) / 32, 256, 0, s>>>(part, blocks, nq * C, dw, db, dbias, C);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
@@ -470,7 +471,8 @@ int forward(gpt2_model* m, const int32_t* tok, const int32_t* tgt, int b, bool t
     {
       const size_t p = prof_begin(m);
       GPT2_TRY(launch::attention_fwd(qkv, atty, lse, b, T, d.H, d.hd, err, s));
-      prof_end(m, p, PC_ATTN_FWD, 2.0 * b * d.H * (double)T * (T + 64) * d.hd, 1);
+      // causal FLOPs: QK^T and PV over the T(T+1)/2 visible (query, key) pairs
+      prof_end(m, p, PC_ATTN_FWD, 2.0 * b * d.H * (double)T * (T + 1) * d.hd, 1);
     }
     {
       gemm::Call c = gemm_call(gemm::FWD, gemm::EPI_RESID, (int)N, C, C, err);
@@ -624,7 +626,8 @@ int backward(gpt2_model* m, const int32_t* tok) {
       const size_t p = prof_begin(m);
       GPT2_TRY(launch::attention_bwd(qkv, atty, datty, lse, m->at<float>(y.attD), m->at<float>(y.dq_acc), dqkv, d.B,
                                      T, d.H, d.hd, err, s));
-      prof_end(m, p, PC_ATTN_BWD, 5.0 * d.B * d.H * (double)T * (T + 64) * d.hd, 3);
+      // causal FLOPs: QK^T, dO V^T, dV, dK and dQ over the visible pairs
+      prof_end(m, p, PC_ATTN_BWD, 5.0 * d.B * d.H * (double)T * (T + 1) * d.hd, 3);
     }
     // QKV projection
     {
@@ -649,6 +652,14 @@ int backward(gpt2_model* m, const int32_t* tok) {
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
+// The status a device error word maps to (a timeout first: it means a kernel gave up early).
+int status_of_device_word(int h) {
+  if (h & DEVERR_TIMEOUT) return GPT2_ERR_TIMEOUT;
+  if (h & DEVERR_TOKEN_RANGE) return GPT2_ERR_TOKEN_RANGE;
+  if (h & DEVERR_NONFINITE) return GPT2_ERR_NONFINITE;
+  return GPT2_OK;
+}
+
 // Read and clear the device error word; map it to a status.
 int collect_device_error(gpt2_model* m) {
   int h = 0;
@@ -659,10 +670,7 @@ int collect_device_error(gpt2_model* m) {
     if (cudaMemsetAsync(m->err(), 0, sizeof(int), m->stream) != cudaSuccess) return GPT2_ERR_CUDA;
     if (cudaStreamSynchronize(m->stream) != cudaSuccess) return GPT2_ERR_CUDA;
   }
-  if (h & DEVERR_TIMEOUT) return GPT2_ERR_TIMEOUT;
-  if (h & DEVERR_TOKEN_RANGE) return GPT2_ERR_TOKEN_RANGE;
-  if (h & DEVERR_NONFINITE) return GPT2_ERR_NONFINITE;
-  return GPT2_OK;
+  return status_of_device_word(h);
 }
 
 double lr_at(const gpt2_config& c, int step) {
@@ -881,6 +889,8 @@ int gpt2_token_losses(gpt2_model* m, float* host_dst, int64_t n) {
 
 float gpt2_lr(const gpt2_model* m, int32_t step) { return m ? (float)lr_at(m->cfg, step) : 0.f; }
 
+double gpt2_schedule_lr(const gpt2_config* cfg, int32_t step) { return cfg ? lr_at(*cfg, step) : -1.0; }
+
 int64_t gpt2_kernel_launches(const gpt2_model* m) { return m ? m->launches : -1; }
 
 int gpt2_profile_enable(gpt2_model* m, int on) {
@@ -1013,6 +1023,25 @@ int gpt2op_linear_wgrad(const void* dout, const void* inp, float* dw, int M, int
   c.a = static_cast<const bf16*>(dout); c.lda = N; c.b = static_cast<const bf16*>(inp); c.ldb = K;
   c.outf = dw; c.ldf = K; c.force_splits = splits;
   return gemm2::run(c, static_cast<cudaStream_t>(stream));
+}
+
+int gpt2op_linear_bwd(const void* dout, const void* w, const void* inp, const void* gelu_pre, void* din, float* dw,
+                      float* colsum, int M, int N, int K, int* splits_out, int* dev_err, void* stream) {
+  if (!dout || !w || !inp || !din || !dw || !dev_err) return GPT2_ERR_ARG;
+  if (M < 256 || M % 64 || N % 256 || K % 256) return GPT2_ERR_ARG;
+  if (colsum && !gelu_pre) return GPT2_ERR_ARG;
+  // din[M, K] = dout[M, N] . w[N, K]: reduction N, output width K
+  gemm::Call cd = gemm_call(gemm::DGRAD, gelu_pre ? gemm::EPI_DGELU : gemm::EPI_STORE, M, K, N, dev_err);
+  cd.a = static_cast<const bf16*>(dout); cd.lda = N; cd.b = static_cast<const bf16*>(w); cd.ldb = K;
+  cd.out = static_cast<bf16*>(din); cd.ldo = K; cd.aux = static_cast<const bf16*>(gelu_pre); cd.ld_aux = K;
+  cd.colsum = colsum;
+  // dw[N, K] += dout[M, N]^T . inp[M, K]: reduction M
+  gemm::Call cw = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, N, K, M, dev_err);
+  cw.a = static_cast<const bf16*>(dout); cw.lda = N; cw.b = static_cast<const bf16*>(inp); cw.ldb = K;
+  cw.outf = dw; cw.ldf = K;
+  if (!gemm2::uses_pair(cd) || !gemm2::uses_pair(cw)) return GPT2_ERR_ARG;
+  int nl = 0;
+  return gemm2::run_group(cd, cw, static_cast<cudaStream_t>(stream), &nl, splits_out);
 }
 
 size_t gpt2op_bias_grad_workspace(int M, int N) { return launch::bias_grad_workspace(M, N); }
@@ -1153,6 +1182,16 @@ int gpt2op_softmax_ce_masked(void* logits, const int32_t* targets, float* losses
   if (!logits || !targets || !losses || !dev_err || N <= 0 || ignore_index == INT_MIN) return GPT2_ERR_ARG;
   return launch::softmax_ce(static_cast<bf16*>(logits), targets, losses, N, V, Vp, dscale, 1, dev_err,
                             static_cast<cudaStream_t>(stream), ignore_index);
+}
+
+int gpt2op_wait_selftest(int64_t limit_ns, int* dev_err, void* stream) {
+  if (!dev_err || limit_ns < 1000000 || limit_ns > 5000000000LL) return GPT2_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  k::wait_selftest_kernel<<<1, 32, 0, s>>>(dev_err, (unsigned long long)limit_ns);
+  if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) return GPT2_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, dev_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GPT2_ERR_CUDA;
+  return status_of_device_word(h);
 }
 
 int gpt2op_embedding_fwd(const int32_t* tokens, const void* wte, const void* wpe, void* out, int B, int T, int C, int V,

@@ -775,4 +775,18 @@ __global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__
     dst[i] = __float2bfloat16_rn(src[i]);
 }
 
+// Bounded-wait self-test: lane 0 waits on a barrier whose phase nothing
+// completes (its count is 1 and nobody arrives); the wait gives up after
+// limit_ns, records DEVERR_TIMEOUT in err and the kernel returns normally.
+__global__ void wait_selftest_kernel(int* err, unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0) mbar_wait_limit(smem_u32(&bar), 0, err, limit_ns);
+  __syncwarp();
+}
+
 }  // namespace k

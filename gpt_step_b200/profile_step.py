@@ -13,7 +13,7 @@
 
   python -m gpt_step_b200.profile_step attn --dir fwd|bwd --shape B,T,H [--iters n]
       Times the causal attention forward or backward (head size 64) through the
-      op-level C ABI and prints TFLOP/s (causal FLOPs incl. the diagonal block).
+      op-level C ABI and prints TFLOP/s (causal FLOPs: the T(T+1)/2 visible pairs).
 
   python -m gpt_step_b200.profile_step head --shape N,C,Vp [--iters n]
       Times the tied lm_head + softmax-CE both ways: the plain GEMM followed by
@@ -21,9 +21,10 @@
       followed by the one-pass CE (real vocabulary Vp - 47), each alone and
       together, in milliseconds.
 
-  python -m gpt_step_b200.profile_step bw --kernel ln_fwd|ln_bwd|ce|colsum --shape rows,C [--iters n]
+  python -m gpt_step_b200.profile_step bw --kernel ln_fwd|ln_bwd|ce|colsum|embed_fwd|embed_bwd --shape rows,C [--iters n]
       Times a bandwidth-bound kernel alone and prints GB/s of algorithmic bytes
-      (for ce, C is the padded vocabulary and the real one is C - 47).
+      (for ce, C is the padded vocabulary and the real one is C - 47; for the
+      embeddings, rows is B * 1024 tokens over a 50,257-id vocabulary).
 """
 from __future__ import annotations
 
@@ -119,13 +120,13 @@ def run_attn(args):
     gs.attention_fwd(qkv, out, lse, H, err)
     if args.dir == "fwd":
         fn = lambda: gs.attention_fwd(qkv, out, lse, H, err)
-        flops = 2.0 * B * H * T * (T + 128) * hd
+        flops = 2.0 * B * H * T * (T + 1) * hd   # causal: T(T+1)/2 visible pairs
     else:
         dout = torch.tensor(rng.standard_normal((B, T, C)).astype(np.float32)).to(torch.bfloat16).cuda()
         dqkv = torch.empty_like(qkv)
         ws = torch.empty(gs.attention_bwd_workspace(B, T, H, hd), dtype=torch.uint8, device="cuda")
         fn = lambda: gs.attention_bwd(qkv, out, dout, lse, dqkv, H, ws, err)
-        flops = 5.0 * B * H * T * (T + 128) * hd
+        flops = 5.0 * B * H * T * (T + 1) * hd
     for _ in range(3):
         fn()
     torch.cuda.synchronize()
@@ -166,6 +167,20 @@ def run_bw(args):
             ws = torch.empty(gs.layernorm_bwd_workspace(rows, C), dtype=torch.uint8, device="cuda")
             fn = lambda: gs.layernorm_bwd(dy, x, mean, rstd, w, dres, dx, dw, db, ws)
             nbytes = rows * (8.0 * C + 8)
+    elif args.kernel in ("embed_fwd", "embed_bwd"):  # rows = B * T tokens (T = 1024), vocabulary 50,257
+        T, V = 1024, 50257
+        Bt = rows // T
+        tok = torch.tensor(rng.integers(0, V, (Bt, T)), dtype=torch.int32, device="cuda")
+        wte, wpe = bf(V + 47, C), bf(T, C)
+        out = torch.empty(Bt, T, C, dtype=torch.bfloat16, device="cuda")
+        if args.kernel == "embed_fwd":
+            fn = lambda: gs.embedding_fwd(tok, wte, wpe, out, V, err)
+            nbytes = rows * (6.0 * C + 4)
+        else:
+            dx = bf(Bt, T, C)
+            dwte, dwpe = torch.zeros(V + 47, C, device="cuda"), torch.zeros(T, C, device="cuda")
+            fn = lambda: gs.embedding_bwd(tok, dx, dwte, dwpe, V)
+            nbytes = rows * (2.0 * C + 4) + 2.0 * rows * C * 4 + 8.0 * T * C
     elif args.kernel == "colsum":  # bias gradient: column sums of a rows x C bf16 matrix
         a = bf(rows, C)
         db = torch.zeros(C, device="cuda")
@@ -258,7 +273,8 @@ def main():
     hp.add_argument("--shape", default="19456,768,50304")
     hp.add_argument("--iters", type=int, default=20)
     w = sub.add_parser("bw")
-    w.add_argument("--kernel", choices=["ln_fwd", "ln_bwd", "ce", "colsum"], default="ln_fwd")
+    w.add_argument("--kernel", choices=["ln_fwd", "ln_bwd", "ce", "colsum", "embed_fwd", "embed_bwd"],
+                   default="ln_fwd")
     w.add_argument("--shape", default="19456,768")
     w.add_argument("--iters", type=int, default=20)
     args = ap.parse_args()

@@ -126,6 +126,12 @@ int gpt2_token_losses(gpt2_model* model, float* host_dst, int64_t n);
 /* Learning rate the schedule gives for `step` (host arithmetic only). */
 float gpt2_lr(const gpt2_model* model, int32_t step);
 
+/* The same schedule from a configuration alone, no model or GPU needed
+ * (§4.3: linear warmup over warmup_steps to max_lr, then a cosine to min_lr at
+ * total_steps; step is 0-based, warmup gives max_lr * (step + 1) / warmup_steps,
+ * steps past total_steps stay at min_lr). Returns -1 for a NULL config. */
+double gpt2_schedule_lr(const gpt2_config* cfg, int32_t step);
+
 /* Number of CUDA kernels this model has launched so far (host-side count). */
 int64_t gpt2_kernel_launches(const gpt2_model* model);
 

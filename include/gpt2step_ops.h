@@ -52,6 +52,20 @@ int gpt2op_linear_dgrad(const void* dout, const void* w, const void* gelu_pre, v
 int gpt2op_linear_wgrad(const void* dout, const void* inp, float* dw, int M, int N, int K, int splits, int* dev_err,
                         void* stream);
 
+/* Both gradients of a linear layer in one launch (§4.1 Fig. 1 backward; the
+ * form gpt2_fwd_bwd uses for every block's four linear layers):
+ *   din[M,K] = dout[M,N] . w[N,K]  (times GELU'(gelu_pre[M,K]) if gelu_pre is
+ *              not NULL; then colsum, if not NULL, fp32 [K], += the column sums
+ *              of the stored bf16 din -- the MLP fc bias gradient)
+ *   dw[N,K] (fp32) += dout[M,N]^T . inp[M,K]
+ * The weight-gradient tiles follow the input-gradient tiles in one persistent
+ * tile list; the M reduction of dw is split across CTAs (fp32 atomics) by a
+ * host-side estimate of the busiest SM pair's finish time. Requires M >= 256,
+ * M % 64 == 0, N % 256 == 0, K % 256 == 0; other shapes return GPT2_ERR_ARG.
+ * *splits_out (may be NULL) receives the dw reduction split chosen. */
+int gpt2op_linear_bwd(const void* dout, const void* w, const void* inp, const void* gelu_pre, void* din, float* dw,
+                      float* colsum, int M, int N, int K, int* splits_out, int* dev_err, void* stream);
+
 /* Bias gradient: db[N] (fp32) += sum over rows of dout[M,N] (bf16),
  * deterministic two-pass column sum. N % 8 == 0. */
 size_t gpt2op_bias_grad_workspace(int M, int N);
@@ -80,11 +94,14 @@ int gpt2op_layernorm_bwd(const void* dy, const void* x, const float* mean, const
  * the implicit device synchronisation an allocation can cause.
  * Its scratch is one fixed array inside the library, of
  * gpt2op_layernorm_bwd_noalloc_max_bytes() = 2,424,832 bytes, that every GPU
- * which loads the library keeps until the process exits. A call needing more
- * (8 * C * min(296, ceil(rows / w)) bytes, w = 8 for C <= 768 and 4 above; any
- * row count fits for C <= 1024) returns GPT2_ERR_ARG before touching the GPU. The first call on a
- * device looks up the array's device address and should come before any stream
- * capture. All calls share the array: calls that overlap on the GPU race. */
+ * which loads the library keeps until the process exits. A call fits exactly
+ * when gpt2op_layernorm_bwd_workspace(rows, C) is at most that size (the
+ * workspace is 8 * C bytes per CTA; a CTA takes 8 / 12 / 8 / 4 rows for C <= 512 /
+ * 768 / 1024 / larger, up to 296 / 148 / 148 / 296 CTAs, so any row count fits
+ * for C <= 1024); a call needing more returns GPT2_ERR_ARG before touching the
+ * GPU. The first call on a device looks up the array's device address and
+ * should come before any stream capture. All calls share the array: calls that
+ * overlap on the GPU race. */
 size_t gpt2op_layernorm_bwd_noalloc_max_bytes(void);
 int gpt2op_layernorm_bwd_noalloc(const void* dy, const void* x, const float* mean, const float* rstd, const float* w,
                                  const void* dresid, void* dx, float* dw, float* db, int rows, int C, void* stream);
@@ -152,6 +169,16 @@ int gpt2op_embedding_fwd(const int32_t* tokens, const void* wte, const void* wpe
 /* Embedding backward: dwte[tok,:] += dx (fp32 atomics), dwpe[t,:] += sum_b dx. */
 int gpt2op_embedding_bwd(const int32_t* tokens, const void* dx, float* dwte, float* dwpe, int B, int T, int C, int V,
                          void* stream);
+
+/* Self-test of the bounded device wait that every mbarrier wait of this
+ * library uses (no counterpart on the pages: it checks the library's own
+ * failure handling). One CTA waits on a shared-memory barrier that nothing
+ * completes, gives up after limit_ns (1 ms .. 5 s) of %globaltimer time,
+ * records flag 4 in dev_err (a device int the caller zeroes) and returns, so
+ * the context stays usable. The call synchronises `stream` and returns the
+ * status the step's calls map that word to: GPT2_ERR_TIMEOUT when the wait
+ * ran out, GPT2_OK if it did not, GPT2_ERR_ARG for a limit out of range. */
+int gpt2op_wait_selftest(int64_t limit_ns, int* dev_err, void* stream);
 
 #ifdef __cplusplus
 }

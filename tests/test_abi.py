@@ -90,3 +90,33 @@ def test_head_and_masked_ce_reject_bad_arguments_before_touching_the_gpu(lib):
     assert lib.gpt2op_softmax_ce_masked(d, d, d, 4, 100, 128, -2 ** 31, f, d, None) == 1
     ptr, n = ctypes.c_void_p(), ctypes.c_int64()
     assert lib.gpt2_state_device_ptr(None, 1, ctypes.byref(ptr), ctypes.byref(n)) == 1
+
+
+def test_schedule_matches_the_oracle_on_the_cpu(lib):
+    """The library's warmup + cosine schedule (the one gpt2_clip_adamw applies)
+    against the oracle's lr_at, across warmup, the cosine branch and past its end."""
+    from oracle import gpt2 as G
+    for name in ("gpt2_124m", "small", "tiny"):
+        args = workloads.model_args(name)
+        cfg, ocfg = gs.Config.make(**args), G.Config(**args)
+        S, W = args["total_steps"], args["warmup_steps"]
+        steps = sorted({0, 1, W // 2, max(W - 1, 0), W, W + 1, (W + S) // 2, S - 1, S, S + 100, 3 * S})
+        for s in steps:
+            # the C config holds max_lr as a float (6e-4 -> 6.0000002e-4): agreement to that rounding
+            assert gs.schedule_lr(cfg, s) == pytest.approx(G.lr_at(ocfg, s), rel=1e-7, abs=1e-18), (name, s)
+    c124 = gs.Config.make(**workloads.model_args("gpt2_124m"))
+    assert gs.schedule_lr(c124, 699) == pytest.approx(6e-4, rel=1e-7)
+    assert gs.schedule_lr(c124, 9782) == pytest.approx(3e-4, rel=1e-4)
+    assert lib.gpt2_schedule_lr(None, 0) == -1.0
+
+
+def test_grouped_backward_and_wait_selftest_reject_bad_arguments(lib):
+    d = ctypes.c_void_p(16)
+    # M below one pair tile, N or K not multiples of 256, colsum without GELU'
+    assert lib.gpt2op_linear_bwd(d, d, d, None, d, d, None, 128, 768, 768, None, d, None) == 1
+    assert lib.gpt2op_linear_bwd(d, d, d, None, d, d, None, 1024, 640, 768, None, d, None) == 1
+    assert lib.gpt2op_linear_bwd(d, d, d, None, d, d, None, 1024, 768, 704, None, d, None) == 1
+    assert lib.gpt2op_linear_bwd(d, d, d, None, d, d, d, 1024, 768, 768, None, d, None) == 1
+    assert lib.gpt2op_wait_selftest(10, d, None) == 1            # limit below 1 ms
+    assert lib.gpt2op_wait_selftest(10 ** 10, d, None) == 1      # above 5 s
+    assert lib.gpt2op_wait_selftest(10 ** 7, None, None) == 1

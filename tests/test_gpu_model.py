@@ -142,8 +142,20 @@ def test_eval_loss_and_token_losses_match_forward():
     assert m.eval_loss(i32(x2), i32(y2)) == pytest.approx(loss, abs=1e-5)
 
 
-def test_adamw_on_identical_fp32_gradients():
-    m, ocfg = pair("tiny")
+# steps of the 124M schedule (warmup 700 to 6e-4, cosine to 0 at 18,865): first
+# warmup step, end of warmup, start of the cosine, its midpoint, its last step
+SCHEDULE_STEPS = [0, 699, 700, 9782, 18864]
+
+
+@pytest.mark.parametrize("step", SCHEDULE_STEPS)
+def test_adamw_on_identical_fp32_gradients(step):
+    """clip + AdamW + bf16 copy on fp32 state written identically to both sides,
+    with the 124M schedule so that the learning rate is non-zero: the update,
+    the decoupled decay and both moments within 1e-6 relative of the oracle, and
+    the library's learning rate equal to the oracle's."""
+    m, ocfg = pair("tiny", warmup_steps=700, total_steps=18865)
+    assert m.lr(step) == pytest.approx(G.lr_at(ocfg, step), rel=1e-6)
+    assert G.lr_at(ocfg, step) > 0
     (x, y), = batch_for("tiny", ocfg)
     m.fwd_bwd(i32(x), i32(y))      # one micro-step pending
     rng = np.random.default_rng(99)
@@ -154,11 +166,13 @@ def test_adamw_on_identical_fp32_gradients():
         Gd[t.name] = (rng.standard_normal(t.shape) * 0.02).astype(np.float32)
         M[t.name] = (rng.standard_normal(t.shape) * 1e-3).astype(np.float32)
         V[t.name] = (rng.random(t.shape) * 1e-4).astype(np.float32)
+        if t.name == "wte.weight":     # padded rows stay zero, as the model keeps them
+            for a in (P, Gd, M, V):
+                a[t.name][ocfg.V:] = 0.0
         m.write(gs.GPT2_PARAMS, i, P[t.name])
         m.write(gs.GPT2_GRADS, i, Gd[t.name])
         m.write(gs.GPT2_ADAM_M, i, M[t.name])
         m.write(gs.GPT2_ADAM_V, i, V[t.name])
-    step = 1000
     norm = m.clip_adamw(step, want_norm=True)
     # oracle on the same fp32 values, per kind arrays assembled from named tensors
     def kinds(named):
@@ -172,13 +186,27 @@ def test_adamw_on_identical_fp32_gradients():
                 out[kind][layer] = named[name]
         return out
     op, og, om, ov = kinds(P), kinds(Gd), kinds(M), kinds(V)
+    w0 = {k: v.copy() for k, v in op.items()}
     onorm = G.clip_adamw(ocfg, op, og, om, ov, step)
+    assert onorm > 1.0                 # the clip is active
     assert norm == pytest.approx(onorm, rel=ADAM_TOL)
     for what, ref in ((gs.GPT2_PARAMS, op), (gs.GPT2_ADAM_M, om), (gs.GPT2_ADAM_V, ov)):
         got = m.read_all(what)
         refn = oracle_named(ocfg, ref)
         for n in names:
             assert rel_l2(got[n], refn[n]) <= ADAM_TOL, (what, n, rel_l2(got[n], refn[n]))
+    # the update itself (w1 - w0), not only w1, matches. It is lr-sized, far below
+    # |w|, so storing w1 in fp32 alone costs a relative error `floor` (the fp32
+    # rounding of the exact w1); the bar is 1e-4 above twice that floor.
+    got = m.read_all(gs.GPT2_PARAMS)
+    w1 = flat(oracle_named(ocfg, op), names)
+    d_got = flat({n: got[n] - P[n] for n in names}, names)
+    d_ref = w1 - flat(oracle_named(ocfg, w0), names)
+    floor = rel_l2(w1.astype(np.float32).astype(np.float64) - flat(oracle_named(ocfg, w0), names), d_ref)
+    err = rel_l2(d_got, d_ref)
+    print(f"step {step}: lr {G.lr_at(ocfg, step):.3e}, update rel L2 {err:.3e} (fp32 storage floor {floor:.3e})")
+    assert err <= 1e-4 + 2 * floor, (err, floor)
+    assert np.all(got["wte.weight"][ocfg.V:] == 0.0)
 
 
 def test_bad_token_and_nonfinite_are_reported():

@@ -250,3 +250,25 @@ def test_embedding_fwd_bwd():
     bad[1, 5] = V + 3
     gs.embedding_fwd(i32(bad), bf16(wte), bf16(wpe), out, V, err)
     assert int(err[0]) & 1
+
+
+# --- failure handling: the bounded device wait -----------------------------------------------
+
+def test_bounded_wait_times_out_and_the_context_stays_usable():
+    """A wait on a barrier that nothing completes gives up after its limit: the
+    kernel records the timeout flag (4) in the device error word and returns,
+    the call maps it to GPT2_ERR_TIMEOUT (6), and the GPU keeps working."""
+    import time
+    err = err_word()
+    t0 = time.perf_counter()
+    st = gs.wait_selftest(50_000_000, err)       # 50 ms
+    dt = time.perf_counter() - t0
+    assert st == 6, st
+    assert int(err[0]) == 4
+    assert 0.04 <= dt < 5.0, dt
+    # the context is intact: an ordinary op still runs and is correct
+    x, w = rnd((256, 128), 70), rnd((256, 128), 71, 0.05)
+    out = torch.empty(256, 256, dtype=torch.bfloat16, device="cuda")
+    err2 = err_word()
+    gs.linear_fwd(bf16(x), bf16(w), None, None, out, err2)
+    assert rel_l2(host(out), rounded(x) @ rounded(w).T) < BF16_TOL and int(err2.sum()) == 0
