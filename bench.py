@@ -17,10 +17,15 @@ measurement through gpt2_train_step_host with pinned host token buffers (the
 host->device copies and the loss/norm readback inside the timed region).
 With --gpus N the ranks train one model data-parallel (the pages' multi-card
 arrangement, §4.4): each rank takes its own micro-batches from its own token
-stream, the fp32 gradients are averaged across ranks by one NCCL all-reduce
-before every clip + AdamW (gpt_step_b200.dp), and the weights stay identical
-(checked after the timed region). Per-rank work is fixed, so scaling is weak.
---parallel replicas instead trains N independent replicas (no exchange).
+stream and the gradients are averaged across ranks before every update
+(gpt_step_b200.dp). --dp-mode zero1 (default): NCCL reduce-scatter of each
+gradient bucket as soon as the last backward has finished it (overlapping the
+remaining backward), the norm from a scalar all-reduce, each rank's AdamW on
+its shards, NCCL all-gather of the bf16 weights; --dp-mode allreduce: one
+all-reduce of the fp32 gradients and the full update on every rank. The
+weights every rank computes with stay identical (checked after the timed
+region). Per-rank work is fixed, so scaling is weak. --parallel replicas
+instead trains N independent replicas (no exchange).
 
 --impl reference times the CPU oracle (the fp64 numpy definition of the same
 step) on the host cores on a bounded sample of the same workload.
@@ -58,7 +63,7 @@ def load_peaks():
             "source": "fallback"}
 
 
-def workload_desc(w, n_gpus, parallel="dp"):
+def workload_desc(w, n_gpus, parallel="dp", dp_mode="zero1"):
     return {
         "workload": (f"GPT-2 124M training step: L{w['n_layer']} H{w['n_head']} C{w['n_embd']} "
                      f"T{w['seq_len']} V{w['vocab_real']}->50304, micro-batch {w['micro_batch']} x "
@@ -67,7 +72,9 @@ def workload_desc(w, n_gpus, parallel="dp"):
         "seq_len": w["seq_len"],
         "tokens_per_step": w["micro_batch"] * w["grad_accum"] * w["seq_len"] * n_gpus,
         "parallelism": ("single GPU" if n_gpus == 1 else
-                        f"dp{n_gpus} (NCCL all-reduce of the fp32 gradients per optimizer step)"
+                        (f"dp{n_gpus} (ZeRO-1: per-bucket NCCL reduce-scatter overlapped with the last backward, "
+                         "sharded AdamW, bf16 all-gather)" if dp_mode == "zero1" else
+                         f"dp{n_gpus} (NCCL all-reduce of the fp32 gradients per optimizer step)")
                         if parallel == "dp" else f"replicas x{n_gpus}"),
         "l2": "inputs larger than L2 (each micro-step touches ~8 GB of activations and logits)",
         "inputs": "synthetic Zipf(1.1) token stream, geometric(1000) documents, seed 1337+rank",
@@ -196,6 +203,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--parallel", default="dp", choices=["dp", "replicas"])
+    ap.add_argument("--dp-mode", default="zero1", choices=["zero1", "allreduce"])
     args = ap.parse_args()
 
     from gpt_step_b200.replicas import job_throughput, max_over_ranks, rank_env, replica_seed
@@ -226,7 +234,7 @@ def main():
     # data parallel: one model (the same initial weights everywhere), per-rank data
     model = gs.GPT2(cfg, 1337 if dp_mode else replica_seed(1337, rank))
     from gpt_step_b200.dp import DataParallel
-    par = DataParallel(model) if dp_mode else None
+    par = DataParallel(model, mode=args.dp_mode) if dp_mode else None
     n_steps = args.warmup + args.steps
     n_win = n_steps * A * B
     src = synth.TokenSource(B, T, cfg.vocab_real, replica_seed(1337, rank), w["mean_doc_len"], n_win)
@@ -245,8 +253,9 @@ def main():
             j = i * A + a
             model.fwd_bwd(tok[j], tgt[j])
         if par is not None:
-            par.sync_grads()           # no-op on one rank
-        model.clip_adamw(i if sched is None else sched)
+            par.update(i if sched is None else sched)   # exchange + (sharded) update; plain update on one rank
+        else:
+            model.clip_adamw(i if sched is None else sched)
 
     def barrier():
         torch.cuda.synchronize()
@@ -335,7 +344,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 3),
             "higher_is_better": True, "scaling": "weak",
             "vs_baseline": round(value / PAGES_TOKENS_PER_S, 3),
-            "dtype": "bf16", "data": "synthetic", "config": workload_desc(w, world, args.parallel),
+            "dtype": "bf16", "data": "synthetic", "config": workload_desc(w, world, args.parallel, args.dp_mode),
             "mfu": round(mfu, 4), "mfu_peak": f"{peaks['bf16_tflops']} TFLOP/s bf16 dense ({peaks['source']})",
             "loss": round(loss, 4), "grad_norm": round(norm, 4),
             "gpu_launches": int(launches), "clocks": clk, "roofline": roof, "e2e": e2e,

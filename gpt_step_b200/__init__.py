@@ -16,7 +16,7 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgpt2step.so")
 
-GPT2_PARAMS, GPT2_GRADS, GPT2_ADAM_M, GPT2_ADAM_V = 0, 1, 2, 3
+GPT2_PARAMS, GPT2_GRADS, GPT2_ADAM_M, GPT2_ADAM_V, GPT2_WEIGHTS_BF16 = 0, 1, 2, 3, 4
 STATUS = {0: "GPT2_OK", 1: "GPT2_ERR_ARG", 2: "GPT2_ERR_CUDA", 3: "GPT2_ERR_TOKEN_RANGE",
           4: "GPT2_ERR_NONFINITE", 5: "GPT2_ERR_STATE", 6: "GPT2_ERR_TIMEOUT"}
 
@@ -82,6 +82,11 @@ _SIGNATURES = {
     "gpt2_read": (_I, [_P, _I, _I, _FP]),
     "gpt2_write": (_I, [_P, _I, _I, _FP]),
     "gpt2_state_device_ptr": (_I, [_P, _I, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(_I64)]),
+    "gpt2_num_buckets": (_I, [_P]),
+    "gpt2_bucket_range": (_I, [_P, _I, ctypes.POINTER(_I64), ctypes.POINTER(_I64)]),
+    "gpt2_set_bucket_events": (_I, [_P, ctypes.POINTER(_P), _I]),
+    "gpt2_grad_sumsq": (_I, [_P, ctypes.POINTER(_I64), _I, _P]),
+    "gpt2_clip_adamw_ranges": (_I, [_P, _I32, ctypes.POINTER(_I64), _I, _P, _FP]),
     "gpt2op_linear_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "gpt2op_linear_fwd_gelu": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _P, _P]),
     "gpt2op_linear_dgrad": (_I, [_P, _P, _P, _P, _I, _I, _I, _P, _P]),
@@ -295,12 +300,47 @@ class GPT2:
         check(lib().gpt2_write(self.h, what, idx, a.ctypes.data_as(_FP)), "gpt2_write")
 
     def state_tensor(self, what: int):
-        """The flat fp32 state array `what` as a torch view of the arena (no copy)."""
+        """The flat state array `what` (fp32; bf16 for GPT2_WEIGHTS_BF16) as a torch view of the arena."""
         ptr, n = ctypes.c_void_p(), ctypes.c_int64()
         check(lib().gpt2_state_device_ptr(self.h, what, ctypes.byref(ptr), ctypes.byref(n)),
               "gpt2_state_device_ptr")
         off = ptr.value - self.arena.data_ptr()
+        if what == GPT2_WEIGHTS_BF16:
+            return self.arena[off: off + 2 * n.value].view(self.torch.bfloat16)
         return self.arena[off: off + 4 * n.value].view(self.torch.float32)
+
+    # -- sharded optimizer step -------------------------------------------------------------
+    def num_buckets(self) -> int:
+        return lib().gpt2_num_buckets(self.h)
+
+    def bucket_range(self, b: int):
+        """(begin, end) elements of bucket b, or of the 1-D region for b = -1."""
+        lo, hi = ctypes.c_int64(), ctypes.c_int64()
+        check(lib().gpt2_bucket_range(self.h, b, ctypes.byref(lo), ctypes.byref(hi)), "gpt2_bucket_range")
+        return lo.value, hi.value
+
+    def set_bucket_events(self, events):
+        """Register torch.cuda.Event objects (one per bucket); [] clears."""
+        self._bucket_events = list(events)
+        arr = (ctypes.c_void_p * max(1, len(events)))(*[e.cuda_event for e in events])
+        check(lib().gpt2_set_bucket_events(self.h, arr, len(events)), "gpt2_set_bucket_events")
+
+    @staticmethod
+    def _ranges(ranges):
+        flat = [int(v) for r in ranges for v in r]
+        return (ctypes.c_int64 * len(flat))(*flat), len(ranges)
+
+    def grad_sumsq(self, ranges, dev_out):
+        """Enqueue: dev_out (a device float64 tensor of one element) = sum of g^2 over the ranges."""
+        arr, n = self._ranges(ranges)
+        check(lib().gpt2_grad_sumsq(self.h, arr, n, _ptr(dev_out)), "gpt2_grad_sumsq")
+
+    def clip_adamw_ranges(self, step: int, ranges, dev_sumsq, want_norm: bool = False):
+        arr, n = self._ranges(ranges)
+        out = ctypes.c_float()
+        check(lib().gpt2_clip_adamw_ranges(self.h, step, arr, n, _ptr(dev_sumsq),
+                                           ctypes.byref(out) if want_norm else None), "gpt2_clip_adamw_ranges")
+        return out.value if want_norm else None
 
     def read_all(self, what: int) -> dict:
         return {t.name: self.read(what, i) for i, t in enumerate(self.tensors())}

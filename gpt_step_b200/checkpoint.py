@@ -152,9 +152,10 @@ def run(model, source, first_step: int, last_step: int, put, cadence: Cadence,
     pre-clip gradient norm, and the eval loss where one was due).
 
     With ``par`` (a ``dp.DataParallel``) the run is one rank of a data-parallel
-    job: gradients are averaged across ranks before each update, the logged
-    and held-out losses are averaged across ranks, and rank 0 alone writes the
-    checkpoints. Every rank's data cursor advances alike (same micro-batch
+    job: gradients are averaged across ranks before each update (in the
+    sharded form each rank updates its shards and the weights are gathered),
+    the logged and held-out losses are averaged across ranks, and rank 0 alone
+    writes the checkpoints, after the sharded state has been gathered. Every rank's data cursor advances alike (same micro-batch
     count per step), so rank 0's cursor is every rank's.
     """
     records = []
@@ -166,13 +167,16 @@ def run(model, source, first_step: int, last_step: int, put, cadence: Cadence,
             x, y = source.get()
             model.fwd_bwd(put(x), put(y))
         if par is not None:
-            par.sync_grads()
-        model.clip_adamw(step)
+            par.update(step)          # the exchange across ranks and the (sharded) update
+        else:
+            model.clip_adamw(step)
         loss, norm = model.last_step_stats()
         rec = {"step": step, "loss": mean(loss), "grad_norm": norm}
         done = step + 1
         if evaluate is not None and cadence.eval_due(done):
             rec["eval_loss"] = mean(evaluate(model))
+        if ckpt_dir is not None and cadence.ckpt_due(done) and par is not None:
+            par.gather_state()        # collective: sharded masters and moments made whole on every rank
         if ckpt_dir is not None and cadence.ckpt_due(done) and writer:
             os.makedirs(ckpt_dir, exist_ok=True)
             rec["checkpoint"] = save(model, ckpt_path(ckpt_dir, done), done, getattr(source, "next", None))

@@ -68,15 +68,30 @@ bool resolve(const gpt2_config* c, Dims* d) {
 }
 
 struct KindInfo {
-  long off, n;       // element offset in the flat arrays, element count
+  long n;            // element count of the kind (all layers)
   int rows, cols;    // per-layer matrix shape (cols = 0 for vectors)
   bool per_layer, decay;
 };
 
+// Flat parameter layout (the same for params, grads, Adam m, v and the bf16 copy):
+//   region 0  [0, P1)   the 1-D parameters (LayerNorm gains and biases, linear
+//                       biases), kind by kind, layers contiguous;
+//   buckets   [P1, P)   the 2-D weights (decayed), grouped by when the backward
+//                       pass finishes their gradients: one bucket per block from
+//                       the last to the first ({mlp proj, mlp fc, attention proj,
+//                       qkv} of that block), then {wpe, wte}. Each bucket is padded
+//                       with zeros to a multiple of kBucketAlign elements, so that
+//                       it splits into equal 64-element-aligned shards for any
+//                       world size dividing 120.
+constexpr long kBucketAlign = 64 * 120;
+
 struct Layout {
   Dims d;
   KindInfo kind[NUM_KINDS];
-  long P;  // flat length (padded, multiple of 64)
+  std::vector<long> off[NUM_KINDS];   // element offset of each (kind, layer) block
+  std::vector<long> bucket_end;        // end of each bucket; bucket 0 starts at P1
+  long P1;   // end of the 1-D region (multiple of 64)
+  long P;    // flat length
   size_t params, grads, adam_m, adam_v, pbf;
   size_t resid, ln1, ln1_mean, ln1_rstd, qkv, atty, lse, resid_mid, ln2, ln2_mean, ln2_rstd, fch, fchg;
   size_t lnf, lnf_mean, lnf_rstd, logits, lse_part;
@@ -97,13 +112,38 @@ void make_layout(const Dims& d, Layout* lay) {
       {3 * d.C, d.C, true, true}, {3 * d.C, 0, true, false}, {d.C, d.C, true, true},   {d.C, 0, true, false},
       {d.C, 0, true, false},     {d.C, 0, true, false},     {4 * d.C, d.C, true, true}, {4 * d.C, 0, true, false},
       {d.C, 4 * d.C, true, true}, {d.C, 0, true, false},    {d.C, 0, false, false},    {d.C, 0, false, false}};
-  long off = 0;
   for (int k = 0; k < NUM_KINDS; ++k) {
     const Def& f = defs[k];
     const long per = (long)f.rows * (f.cols ? f.cols : 1);
-    lay->kind[k] = {off, per * (f.per_layer ? L : 1), f.rows, f.cols, f.per_layer, f.decay};
-    off += align_up(lay->kind[k].n, 64);
+    lay->kind[k] = {per * (f.per_layer ? L : 1), f.rows, f.cols, f.per_layer, f.decay};
+    lay->off[k].assign(f.per_layer ? (size_t)std::max<long>(L, 1) : 1, 0);
   }
+  auto per = [&](int k) { return (long)lay->kind[k].rows * (lay->kind[k].cols ? lay->kind[k].cols : 1); };
+  long off = 0;
+  // region 0: the 1-D kinds
+  const int vec_kinds[] = {K_LN1W, K_LN1B, K_QKVB, K_ATTPROJB, K_LN2W, K_LN2B, K_FCB, K_FCPROJB, K_LNFW, K_LNFB};
+  for (int k : vec_kinds) {
+    const int nl = lay->kind[k].per_layer ? (int)L : 1;
+    for (int l = 0; l < nl; ++l) lay->off[k][l] = off + (long)l * per(k);
+    off = (long)align_up(off + lay->kind[k].n, 64);
+  }
+  lay->P1 = off;
+  // buckets of 2-D weights in the order the backward pass completes them
+  lay->bucket_end.clear();
+  for (int l = (int)L - 1; l >= 0; --l) {
+    for (int k : {K_FCPROJW, K_FCW, K_ATTPROJW, K_QKVW}) {
+      lay->off[k][l] = off;
+      off += per(k);
+    }
+    off = (long)align_up(off, kBucketAlign);
+    lay->bucket_end.push_back(off);
+  }
+  for (int k : {K_WPE, K_WTE}) {
+    lay->off[k][0] = off;
+    off += per(k);
+  }
+  off = (long)align_up(off, kBucketAlign);
+  lay->bucket_end.push_back(off);
   lay->P = off;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t r = o; o = align_up(o + bytes, 1024); return r; };
@@ -203,6 +243,7 @@ struct gpt2_model {
   bool stepped;  // at least one clip_adamw has run
   int64_t launches = 0;  // kernels this model has launched
   Profiler prof;
+  std::vector<cudaEvent_t> bucket_events;  // caller's events, recorded when each bucket's gradients are final
   std::vector<NamedTensor> tensors;
   ~gpt2_model() {
     for (cudaEvent_t e : prof.ev) cudaEventDestroy(e);
@@ -213,9 +254,10 @@ struct gpt2_model {
   float* params() const { return at<float>(lay.params); }
   float* grads() const { return at<float>(lay.grads); }
   bf16* pbf() const { return at<bf16>(lay.pbf); }
-  float* P(int k, int l = 0) const { return params() + lay.kind[k].off + (long)l * per(k); }
-  float* G(int k, int l = 0) const { return grads() + lay.kind[k].off + (long)l * per(k); }
-  bf16* W(int k, int l = 0) const { return pbf() + lay.kind[k].off + (long)l * per(k); }
+  long off(int k, int l) const { return lay.off[k][lay.kind[k].per_layer ? l : 0]; }
+  float* P(int k, int l = 0) const { return params() + off(k, l); }
+  float* G(int k, int l = 0) const { return grads() + off(k, l); }
+  bf16* W(int k, int l = 0) const { return pbf() + off(k, l); }
   long per(int k) const { return (long)lay.kind[k].rows * (lay.kind[k].cols ? lay.kind[k].cols : 1); }
   int* err() const { return at<int>(lay.err); }
   k::StepScalars* sc() const { return at<k::StepScalars>(lay.scalars); }
@@ -637,6 +679,9 @@ int backward(gpt2_model* m, const int32_t* tok) {
       cd.a = dqkv; cd.lda = 3 * C; cd.b = m->W(K_QKVW, l); cd.ldb = C; cd.out = dln; cd.ldo = C;
       GPT2_TRY(run_gemm_group(m, cd, cw));
     }
+    // every 2-D weight gradient of this block is final for this micro-step
+    if (!m->bucket_events.empty() && cudaEventRecord(m->bucket_events[L - 1 - l], s) != cudaSuccess)
+      return GPT2_ERR_CUDA;
     GPT2_TRY(bias_grad_m(m, dqkv, m->G(K_QKVB, l), N, 3 * C));
     GPT2_TRY(ln_bwd_m(m, dln, x_in, m->at<float>(y.ln1_mean) + l * d.N, m->at<float>(y.ln1_rstd) + l * d.N, K_LN1W,
                       K_LN1B, l, dresid, dresid, l > 0 ? m->G(K_FCPROJB, l - 1) : nullptr));
@@ -649,6 +694,8 @@ int backward(gpt2_model* m, const int32_t* tok) {
                                                                                       d.V);
     prof_end(m, p, PC_EMBED, (double)N * (2.0 * C + 4) + 2.0 * N * C * 4 + 8.0 * T * C, 2);
   }
+  // the last bucket (wpe, wte) and the 1-D region are final now
+  if (!m->bucket_events.empty() && cudaEventRecord(m->bucket_events.back(), s) != cudaSuccess) return GPT2_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -742,7 +789,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, void* dev_arena, size_t a
     t.name = name; t.kind = kind; t.layer = layer;
     const KindInfo& ki = m->lay.kind[kind];
     const long per = (long)ki.rows * (ki.cols ? ki.cols : 1);
-    t.off = ki.off + (layer > 0 ? (long)layer * per : 0);
+    t.off = m->off(kind, layer > 0 ? layer : 0);
     t.n = per;
     t.ndim = ki.cols ? 2 : 1;
     t.shape[0] = ki.rows;
@@ -773,8 +820,15 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, void* dev_arena, size_t a
       default: mode = 2; break;
     }
     if (ki.n == 0) continue;
-    k::init_kind_kernel<<<launch::grid_for((ki.n + 3) / 4, 256), 256, 0, s>>>(
-        m->params() + ki.off, m->pbf() + ki.off, ki.n, mode, sd, (uint32_t)kk, seed, zero_from);
+    // one launch per (kind, layer) block; the generator's counter runs over the
+    // kind's elements in layer order, whatever the block's place in the layout
+    const long per = m->per(kk);
+    const int nl = ki.per_layer ? d.L : 1;
+    for (int l = 0; l < nl; ++l) {
+      const long o = m->off(kk, l);
+      k::init_kind_kernel<<<launch::grid_for((per + 3) / 4, 256), 256, 0, s>>>(
+          m->params() + o, m->pbf() + o, per, mode, sd, (uint32_t)kk, seed, zero_from, (long)l * per / 4);
+    }
   }
   if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) { delete m; return GPT2_ERR_CUDA; }
   *out = m;
@@ -796,33 +850,44 @@ int gpt2_fwd_bwd(gpt2_model* m, const int32_t* tokens, const int32_t* targets, f
   return GPT2_OK;
 }
 
-int gpt2_clip_adamw(gpt2_model* m, int32_t step, float* grad_norm_out) {
-  if (!m || step < 0) return GPT2_ERR_ARG;
-  if (m->n_micro == 0) return GPT2_ERR_STATE;
+// Host-side form of element ranges: float4 ranges, validated against the layout
+// (each 64-element aligned, inside [0, P), at most Ranges4::kMax of them).
+static bool to_ranges4(const gpt2_model* m, const int64_t* ranges, int n, k::Ranges4* out) {
+  if (n < 1 || n > k::Ranges4::kMax || !ranges) return false;
+  out->n = n;
+  for (int r = 0; r < n; ++r) {
+    const int64_t b = ranges[2 * r], e = ranges[2 * r + 1];
+    if (b < 0 || e < b || e > m->lay.P || (b % 64) || (e % 64)) return false;
+    out->begin[r] = b / 4;
+    out->end[r] = e / 4;
+  }
+  return true;
+}
+
+// The update half of the step over the given ranges, with the norm finalised from
+// `sumsq` (one device double: the sum of squares of the accumulated gradients).
+static int clip_adamw_impl(gpt2_model* m, int32_t step, const k::Ranges4& rg, const double* sumsq, int nparts,
+                           bool clear_all_grads, float* grad_norm_out) {
   cudaStream_t s = m->stream;
   const Layout& y = m->lay;
-  const long n4 = y.P / 4;
-  double* part = m->at<double>(y.norm_part);
   const size_t pr = prof_begin(m);
-  k::sumsq_partial_kernel<<<kNormBlocks, 512, 0, s>>>(m->grads(), n4, part);
-  k::norm_finalize_kernel<<<1, 256, 0, s>>>(part, kNormBlocks, m->sc(), m->n_micro, y.d.N, m->cfg.grad_clip,
-                                            m->err());
-  k::KindTable kt{};
-  kt.nk = NUM_KINDS;
-  for (int kk = 0; kk < NUM_KINDS; ++kk) {
-    kt.bound[kk] = y.kind[kk].off;
-    if (y.kind[kk].decay) kt.decay_mask |= 1u << kk;
-  }
-  kt.bound[NUM_KINDS] = y.P;
+  k::norm_finalize_kernel<<<1, 256, 0, s>>>(sumsq, nparts, m->sc(), m->n_micro, y.d.N, m->cfg.grad_clip, m->err());
   const double lr = lr_at(m->cfg, step);
   const double t = (double)step + 1.0;
   const float bc1 = (float)(1.0 - pow((double)m->cfg.beta1, t));
   const float bc2 = (float)(1.0 - pow((double)m->cfg.beta2, t));
+  long n4 = 0;
+  for (int r = 0; r < rg.n; ++r) n4 += rg.end[r] - rg.begin[r];
   k::adamw_kernel<<<launch::grid_for(n4, 256), 256, 0, s>>>(m->params(), m->grads(), m->at<float>(y.adam_m),
-                                                             m->at<float>(y.adam_v), m->pbf(), n4, kt, m->sc(),
-                                                             (float)lr, m->cfg.beta1, m->cfg.beta2, m->cfg.eps,
-                                                             m->cfg.weight_decay, bc1, bc2);
-  prof_end(m, pr, PC_OPT, 38.0 * (double)y.P, 3);
+                                                             m->at<float>(y.adam_v), m->pbf(), rg, y.P1 / 4,
+                                                             m->sc(), (float)lr, m->cfg.beta1, m->cfg.beta2,
+                                                             m->cfg.eps, m->cfg.weight_decay, bc1, bc2);
+  int nl = 2;
+  if (clear_all_grads) {
+    if (cudaMemsetAsync(m->grads(), 0, (size_t)y.P * 4, s) != cudaSuccess) return GPT2_ERR_CUDA;
+    ++nl;
+  }
+  prof_end(m, pr, PC_OPT, 34.0 * 4.0 * (double)n4, nl);
   if (cudaGetLastError() != cudaSuccess) return GPT2_ERR_CUDA;
   m->n_micro = 0;
   m->stepped = true;
@@ -833,6 +898,75 @@ int gpt2_clip_adamw(gpt2_model* m, int32_t step, float* grad_norm_out) {
     return st;
   }
   return GPT2_OK;
+}
+
+int gpt2_clip_adamw(gpt2_model* m, int32_t step, float* grad_norm_out) {
+  if (!m || step < 0) return GPT2_ERR_ARG;
+  if (m->n_micro == 0) return GPT2_ERR_STATE;
+  const Layout& y = m->lay;
+  k::Ranges4 all{};
+  all.n = 1;
+  all.begin[0] = 0;
+  all.end[0] = y.P / 4;
+  double* part = m->at<double>(y.norm_part);
+  const size_t pr = prof_begin(m);
+  k::sumsq_partial_kernel<<<kNormBlocks, 512, 0, m->stream>>>(m->grads(), all, part);
+  prof_end(m, pr, PC_OPT, 4.0 * (double)y.P, 1);
+  return clip_adamw_impl(m, step, all, part, kNormBlocks, false, grad_norm_out);
+}
+
+int gpt2_num_buckets(const gpt2_model* m) { return m ? (int)m->lay.bucket_end.size() : -1; }
+
+int gpt2_bucket_range(const gpt2_model* m, int b, int64_t* begin, int64_t* end) {
+  if (!m || !begin || !end) return GPT2_ERR_ARG;
+  const Layout& y = m->lay;
+  if (b == -1) {
+    *begin = 0;
+    *end = y.P1;
+    return GPT2_OK;
+  }
+  if (b < 0 || b >= (int)y.bucket_end.size()) return GPT2_ERR_ARG;
+  *begin = b == 0 ? y.P1 : y.bucket_end[b - 1];
+  *end = y.bucket_end[b];
+  return GPT2_OK;
+}
+
+int gpt2_set_bucket_events(gpt2_model* m, void* const* events, int n) {
+  if (!m) return GPT2_ERR_ARG;
+  if (n == 0) {
+    m->bucket_events.clear();
+    return GPT2_OK;
+  }
+  if (!events || n != (int)m->lay.bucket_end.size()) return GPT2_ERR_ARG;
+  m->bucket_events.assign(n, nullptr);
+  for (int i = 0; i < n; ++i) {
+    if (!events[i]) { m->bucket_events.clear(); return GPT2_ERR_ARG; }
+    m->bucket_events[i] = static_cast<cudaEvent_t>(events[i]);
+  }
+  return GPT2_OK;
+}
+
+int gpt2_grad_sumsq(gpt2_model* m, const int64_t* ranges, int n_ranges, double* dev_out) {
+  if (!m || !dev_out) return GPT2_ERR_ARG;
+  k::Ranges4 rg{};
+  if (!to_ranges4(m, ranges, n_ranges, &rg)) return GPT2_ERR_ARG;
+  double* part = m->at<double>(m->lay.norm_part);
+  long n4 = 0;
+  for (int r = 0; r < rg.n; ++r) n4 += rg.end[r] - rg.begin[r];
+  const size_t pr = prof_begin(m);
+  k::sumsq_partial_kernel<<<kNormBlocks, 512, 0, m->stream>>>(m->grads(), rg, part);
+  k::sum_partials_kernel<<<1, 256, 0, m->stream>>>(part, kNormBlocks, dev_out);
+  prof_end(m, pr, PC_OPT, 16.0 * (double)n4, 2);
+  return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
+}
+
+int gpt2_clip_adamw_ranges(gpt2_model* m, int32_t step, const int64_t* ranges, int n_ranges, const double* dev_sumsq,
+                           float* grad_norm_out) {
+  if (!m || step < 0 || !dev_sumsq) return GPT2_ERR_ARG;
+  if (m->n_micro == 0) return GPT2_ERR_STATE;
+  k::Ranges4 rg{};
+  if (!to_ranges4(m, ranges, n_ranges, &rg)) return GPT2_ERR_ARG;
+  return clip_adamw_impl(m, step, rg, dev_sumsq, 1, true, grad_norm_out);
 }
 
 int gpt2_last_step_stats(gpt2_model* m, float* mean_loss_out, float* grad_norm_out) {
@@ -952,6 +1086,11 @@ static float* state_array(gpt2_model* m, int what) {
 
 int gpt2_state_device_ptr(gpt2_model* m, int what, void** dev_ptr, int64_t* count) {
   if (!m || !dev_ptr || !count) return GPT2_ERR_ARG;
+  if (what == GPT2_WEIGHTS_BF16) {
+    *dev_ptr = m->pbf();
+    *count = (int64_t)m->lay.P;
+    return GPT2_OK;
+  }
   float* base = state_array(m, what);
   if (!base) return GPT2_ERR_ARG;
   *dev_ptr = base;

@@ -33,13 +33,18 @@ GPT2_DEV float u01(uint32_t x) { return ((float)(x >> 9) + 0.5f) * (1.0f / 83886
 
 // Init one parameter kind: mode 0 = N(0, std) (rows >= zero_row_from are 0),
 // 1 = ones, 2 = zeros. Writes the fp32 master and the bf16 copy.
+// `ctr_base` is the generator counter of the block's first four elements (its
+// element offset within the kind / 4), so that a kind split into per-layer
+// blocks draws the same numbers as the kind in one piece; `zero_from` counts
+// from the block's start.
 __global__ void init_kind_kernel(float* __restrict__ p, bf16* __restrict__ pb, long n, int mode, float stddev,
-                                 uint32_t kind, uint64_t seed, long zero_from) {
+                                 uint32_t kind, uint64_t seed, long zero_from, long ctr_base) {
   const long nblk = (n + 3) / 4;
   for (long c = blockIdx.x * (long)blockDim.x + threadIdx.x; c < nblk; c += (long)gridDim.x * blockDim.x) {
     float z[4];
     if (mode == 0) {
-      uint32_t ctr[4] = {(uint32_t)(c & 0xFFFFFFFFu), (uint32_t)((uint64_t)c >> 32), kind, 0u};
+      const uint64_t cg = (uint64_t)(ctr_base + c);
+      uint32_t ctr[4] = {(uint32_t)(cg & 0xFFFFFFFFu), (uint32_t)(cg >> 32), kind, 0u};
       philox4x32_10(ctr, (uint32_t)(seed & 0xFFFFFFFFu), (uint32_t)(seed >> 32));
       const float r01 = sqrtf(-2.0f * logf(u01(ctr[0])));
       const float r23 = sqrtf(-2.0f * logf(u01(ctr[2])));
@@ -652,14 +657,25 @@ __global__ void loss_reduce_kernel(const float* __restrict__ losses, int n, doub
 // a12  global gradient norm. Pass 1: per-block fp64 partial sums of g^2 over
 // the flat fp32 gradient array (float4 loads).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(512) sumsq_partial_kernel(const float* __restrict__ g, long n4,
+// Half-open ranges of float4 indices into the flat parameter arrays (passed by value).
+struct Ranges4 {
+  static constexpr int kMax = 64;
+  long begin[kMax], end[kMax];
+  int n;
+};
+
+// Partial sums of squares of g over the ranges, one per block.
+__global__ void __launch_bounds__(512) sumsq_partial_kernel(const float* __restrict__ g, const Ranges4 rg,
                                                             double* __restrict__ part) {
   __shared__ double red[16];
   double s = 0.0;
   const float4* g4 = reinterpret_cast<const float4*>(g);
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
-    const float4 v = g4[i];
-    s += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+  for (int r = 0; r < rg.n; ++r) {
+    for (long i = rg.begin[r] + blockIdx.x * (long)blockDim.x + threadIdx.x; i < rg.end[r];
+         i += (long)gridDim.x * blockDim.x) {
+      const float4 v = g4[i];
+      s += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
+    }
   }
   s = warp_sum_d(s);
   if (lane_id() == 0) red[threadIdx.x >> 5] = s;
@@ -710,37 +726,45 @@ __global__ void norm_finalize_kernel(const double* __restrict__ part, int nparts
   }
 }
 
-// ---------------------------------------------------------------------------
-// a13  clipped AdamW over the flat parameter arrays (float4 per thread).
-// Kinds are contiguous and 64-element aligned; `bound[k]` is the first element
-// of kind k (bound[nk] = end) and bit k of `decay_mask` says whether kind k is a
-// 2-D weight that takes decoupled weight decay. Writes p, m, v, the bf16 copy
-// and clears g. If the step is flagged non-finite only g is cleared.
-// ---------------------------------------------------------------------------
-struct KindTable {
-  long bound[17];
-  int nk;
-  unsigned decay_mask;
-};
+// Sum of the partials into one double (the caller's device value).
+__global__ void sum_partials_kernel(const double* __restrict__ part, int nparts, double* __restrict__ out) {
+  __shared__ double red[32];
+  double s = 0.0;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) s += part[i];
+  s = warp_sum_d(s);
+  if (lane_id() == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+    *out = t;
+  }
+}
 
+// ---------------------------------------------------------------------------
+// a13  clipped AdamW over the given float4 ranges of the flat parameter arrays.
+// The 2-D weights (which take decoupled weight decay) are exactly the elements
+// from decay_from4 * 4 on; the zero padding there stays zero. Writes p, m, v,
+// the bf16 copy and clears g in the ranges. If the step is flagged non-finite
+// only g is cleared.
+// ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, float* __restrict__ g,
                                                     float* __restrict__ m, float* __restrict__ v,
-                                                    bf16* __restrict__ pb, long n4, const KindTable kt,
+                                                    bf16* __restrict__ pb, const Ranges4 rg, long decay_from4,
                                                     const StepScalars* __restrict__ sc, float lr, float beta1,
                                                     float beta2, float eps, float wd, float bc1, float bc2) {
   const float gs = sc->gscale;
   const int skip = sc->skip;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n4; i += (long)gridDim.x * blockDim.x) {
+  for (int r = 0; r < rg.n; ++r)
+  for (long i = rg.begin[r] + blockIdx.x * (long)blockDim.x + threadIdx.x; i < rg.end[r];
+       i += (long)gridDim.x * blockDim.x) {
     const long e = i * 4;
     float4* g4 = reinterpret_cast<float4*>(g) + i;
     if (skip) {
       *g4 = make_float4(0.f, 0.f, 0.f, 0.f);
       continue;
     }
-    int kind = 0;
-#pragma unroll 1
-    while (kind + 1 < kt.nk && e >= kt.bound[kind + 1]) ++kind;
-    const float lam = ((kt.decay_mask >> kind) & 1u) ? wd : 0.f;
+    const float lam = i >= decay_from4 ? wd : 0.f;
     float4 gv = *g4;
     float4 pv = reinterpret_cast<float4*>(p)[i];
     float4 mv = reinterpret_cast<float4*>(m)[i];

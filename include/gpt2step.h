@@ -56,8 +56,9 @@ typedef struct gpt2_config {
 
 typedef struct gpt2_model gpt2_model; /* opaque */
 
-/* Which state array gpt2_read / gpt2_write address. */
-enum { GPT2_PARAMS = 0, GPT2_GRADS = 1, GPT2_ADAM_M = 2, GPT2_ADAM_V = 3 };
+/* Which state array gpt2_read / gpt2_write address (GPT2_WEIGHTS_BF16, the
+ * bf16 copy the tensor cores read, only through gpt2_state_device_ptr). */
+enum { GPT2_PARAMS = 0, GPT2_GRADS = 1, GPT2_ADAM_M = 2, GPT2_ADAM_V = 3, GPT2_WEIGHTS_BF16 = 4 };
 
 /* Bytes of device memory the caller must provide to gpt2_create for this
  * configuration (fp32 params, grads, m, v; bf16 weight copy; saved activations;
@@ -162,15 +163,64 @@ int gpt2_tensor_info(const gpt2_model* model, int idx, const char** name, int64_
 int gpt2_read(gpt2_model* model, int what, int idx, float* host_dst);
 int gpt2_write(gpt2_model* model, int what, int idx, const float* host_src);
 
-/* Device address and length (fp32 elements, padded flat layout: every tensor
- * at a 64-element aligned offset, gaps zero) of the whole state array `what`
- * inside the caller's arena, for collectives over it: data-parallel ranks
- * ("Pretraining and adapting a language model on a dependency-free stack",
- * §4.4, three cards) average GPT2_GRADS across ranks between their last
- * gpt2_fwd_bwd and gpt2_clip_adamw, on the model's stream. Valid while the
- * model lives; no copy, no synchronisation. Writing GPT2_PARAMS through it
- * does not refresh the bf16 copy (use gpt2_write). */
+/* Device address and length (elements: fp32, or bf16 for GPT2_WEIGHTS_BF16)
+ * of the whole state array `what` inside the caller's arena, for collectives
+ * over it: data-parallel ranks ("Pretraining and adapting a language model on
+ * a dependency-free stack", §4.4, three cards) average GPT2_GRADS across ranks
+ * between their last gpt2_fwd_bwd and gpt2_clip_adamw, on the model's stream.
+ * Valid while the model lives; no copy, no synchronisation. Writing
+ * GPT2_PARAMS through it does not refresh the bf16 copy (use gpt2_write).
+ *
+ * Flat layout (the same for every array): region 0 = [0, P1) holds the 1-D
+ * parameters (LayerNorm gains and biases, linear biases); [P1, P) holds the
+ * 2-D weights in buckets, in the order the backward pass finishes their
+ * gradients: one bucket per block from the last block to the first, then
+ * {wpe, wte}. Tensors start 64-element aligned; each bucket is zero-padded to
+ * a multiple of 7,680 elements, so it splits into equal shards that are
+ * multiples of 64 elements for any world size dividing 120. Gaps stay zero. */
 int gpt2_state_device_ptr(gpt2_model* model, int what, void** dev_ptr, int64_t* count);
+
+/* ---- sharded optimizer step (data parallelism in the ZeRO-1 form) ----------
+ * §4.4 averages the gradients across cards once per optimizer step. In the
+ * sharded form each rank reduce-scatters (averages) the 2-D buckets so that it
+ * holds the averaged gradient of one shard of every bucket, all-reduces region
+ * 0, updates region 0 and its shards only, and all-gathers the bf16 weights of
+ * every bucket. The fp32 masters and Adam moments outside a rank's shards are
+ * then stale and unused (the forward and backward read the 2-D weights only
+ * through the bf16 copy and region 0 in fp32). */
+
+/* Number of 2-D buckets (n_layer + 1). */
+int gpt2_num_buckets(const gpt2_model* model);
+
+/* Element range [begin, end) of bucket b (0 .. gpt2_num_buckets - 1, in the
+ * order their gradients become final), or of region 0 for b = -1. */
+int gpt2_bucket_range(const gpt2_model* model, int b, int64_t* begin, int64_t* end);
+
+/* Register one cudaEvent_t per bucket (n == gpt2_num_buckets; n == 0 clears).
+ * Every gpt2_fwd_bwd then records event b on the model's stream as soon as
+ * bucket b's gradients are final for that micro-step (the last event also
+ * marks region 0), so that a collective on another stream can start on a
+ * bucket while the backward works on the earlier blocks. The events stay the
+ * caller's; they must outlive the registration. */
+int gpt2_set_bucket_events(gpt2_model* model, void* const* events, int n);
+
+/* Enqueue on the model's stream: *dev_out (a device double) = the sum of
+ * squares of the accumulated gradients over the element ranges
+ * ranges[2i] .. ranges[2i+1] (n_ranges <= 64, bounds multiples of 64 inside
+ * the flat array). */
+int gpt2_grad_sumsq(gpt2_model* model, const int64_t* ranges, int n_ranges, double* dev_out);
+
+/* The update of gpt2_clip_adamw restricted to the given element ranges, with
+ * the global norm taken from *dev_sumsq (device double: the sum of squares of
+ * the accumulated gradients over the whole model, e.g. gpt2_grad_sumsq's
+ * partials summed across ranks): norm = sqrt(*dev_sumsq) / micro-steps, clip
+ * scale min(1, clip / norm), AdamW with the schedule's lr(step) on params, m, v
+ * and the bf16 copy inside the ranges; then ALL gradients are cleared and the
+ * micro-step count restarts. GPT2_ERR_STATE without a micro-step since the
+ * last update; *grad_norm_out (may be NULL) synchronises, as in
+ * gpt2_clip_adamw. */
+int gpt2_clip_adamw_ranges(gpt2_model* model, int32_t step, const int64_t* ranges, int n_ranges,
+                           const double* dev_sumsq, float* grad_norm_out);
 
 /* Total parameter count: real vocabulary rows only (124,439,808 for GPT-2
  * 124M, §4.1) when padded == 0, all stored rows when padded != 0. */

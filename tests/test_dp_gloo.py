@@ -7,15 +7,21 @@ of the micro-batches and average their gradients must end where one process
 that took all of them ends, with bit-identical weights on both ranks; the
 held-out loss is the mean of the ranks' losses.
 """
+import math
 import multiprocessing as mp
 import socket
 
 import numpy as np
+import pytest
 import torch
 
 from gpt_step_b200 import dp
 
-N = 37
+# flat layout of the fake: region 0 (the "1-D parameters") then three buckets
+REGION0 = (0, 64)
+BUCKETS = [(64, 320), (320, 448), (448, 832)]
+N = 832
+LR0, B1, B2, EPS, WD = 0.1, 0.9, 0.95, 1e-8, 0.1
 
 
 def _feat(x, y):
@@ -27,39 +33,75 @@ def _feat(x, y):
 
 
 class FakeModel:
-    def __init__(self, seed=0):
+    """fp64 stand-in with the device model's state interface: fp32-master-like
+    parameters p, the copy w the forward reads outside region 0 (the bf16 copy on
+    the device), gradients accumulated over micro-steps, AdamW moments, the
+    bucket layout, and the range-restricted update with an external norm."""
+
+    def __init__(self, seed=0, dtype=torch.float64):
         g = torch.Generator().manual_seed(seed)
-        self.p = torch.randn(N, generator=g, dtype=torch.float64)
-        self.g = torch.zeros(N, dtype=torch.float64)
+        self.dtype = dtype
+        self.p = torch.randn(N, generator=g, dtype=torch.float64).to(dtype)
+        self.w = self.p.clone()
+        self.g = torch.zeros(N, dtype=dtype)
+        self.m = torch.zeros(N, dtype=dtype)
+        self.v = torch.zeros(N, dtype=dtype)
         self.k = 0
         self.losses = []
         self.stats = (0.0, 0.0)
 
+    def weights(self):
+        """What the forward computes with: region 0 from p, the buckets from the copy."""
+        e = self.w.clone()
+        e[REGION0[0]:REGION0[1]] = self.p[REGION0[0]:REGION0[1]]
+        return e
+
     def state_tensor(self, what):
-        return self.g if what == dp.GRADS else self.p
+        return {dp.PARAMS: self.p, dp.GRADS: self.g, dp.ADAM_M: self.m, dp.ADAM_V: self.v,
+                dp.WEIGHTS_BF16: self.w}[what]
+
+    def num_buckets(self):
+        return len(BUCKETS)
+
+    def bucket_range(self, b):
+        return REGION0 if b == -1 else BUCKETS[b]
 
     def fwd_bwd(self, x, y):
-        f = _feat(x, y)
-        self.g += 0.3 * self.p - f
-        self.losses.append(float(f.sum()))
+        f = _feat(x, y).to(self.dtype)
+        self.g += 0.3 * self.weights() - f
+        self.losses.append(float(f @ self.weights()))
         self.k += 1
 
-    def clip_adamw(self, step):
-        gm = self.g / self.k
-        norm = float(torch.linalg.vector_norm(gm))
-        if norm > 1.0:
-            gm = gm / norm
-        self.p -= 0.1 / (step + 1) * gm
+    def grad_sumsq(self, ranges, out):
+        out[0] = sum(float((self.g[a:b] ** 2).sum()) for a, b in ranges)
+
+    def clip_adamw_ranges(self, step, ranges, sumsq):
+        norm = math.sqrt(float(sumsq[0])) / self.k
+        scale = min(1.0, 1.0 / norm) / self.k
+        lr, t = LR0 / (step + 1), step + 1
+        for a, b in ranges:
+            gg = self.g[a:b] * scale
+            self.m[a:b] = B1 * self.m[a:b] + (1 - B1) * gg
+            self.v[a:b] = B2 * self.v[a:b] + (1 - B2) * gg * gg
+            upd = (self.m[a:b] / (1 - B1 ** t)) / (torch.sqrt(self.v[a:b] / (1 - B2 ** t)) + EPS)
+            lam = torch.where(torch.arange(a, b) >= REGION0[1], WD, 0.0).to(self.dtype)
+            self.p[a:b] = self.p[a:b] - lr * (upd + lam * self.p[a:b])
+            self.w[a:b] = self.p[a:b]
         self.stats = (float(np.mean(self.losses)), norm)
         self.g.zero_()
         self.k = 0
         self.losses = []
 
+    def clip_adamw(self, step):
+        s = torch.zeros(1, dtype=torch.float64)
+        self.grad_sumsq([(0, N)], s)
+        self.clip_adamw_ranges(step, [(0, N)], s)
+
     def last_step_stats(self):
         return self.stats
 
     def eval_loss(self, x, y):
-        return float(_feat(x, y) @ self.p)
+        return float(_feat(x, y).to(self.dtype) @ self.weights())
 
 
 def _batches(step, a, rank, world):
@@ -74,12 +116,12 @@ def _free_port():
         return s.getsockname()[1]
 
 
-def _rank_main(rank, world, port, q, A, steps):
+def _rank_main(rank, world, port, q, A, steps, mode):
     import torch.distributed as dist
     dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
     try:
         m = FakeModel()
-        d = dp.DataParallel(m)
+        d = dp.DataParallel(m, mode=mode)
         norms = []
         for s in range(steps):
             xs, ys = zip(*[_batches(s, a, rank, world) for a in range(A)])
@@ -93,20 +135,28 @@ def _rank_main(rank, world, port, q, A, steps):
         ev_local = m.eval_loss(ex, ey)
         ev = d.eval_loss(ex, ey)
         agree = d.replicas_agree()
+        used = m.weights().tolist()
+        d.gather_state()                  # the sharded masters made whole: every p equals the used weights
+        whole = m.p.tolist()
         if rank == 1:
-            m.p[3] += 1e-9
+            m.p[3] += 1e-9                # region 0: read by the forward in both forms
         disagree = not d.replicas_agree()
-        q.put((rank, m.p.tolist(), norms, ev_local, ev, agree, disagree))
+        q.put((rank, used, norms, ev_local, ev, agree, disagree, whole))
     finally:
         dist.destroy_process_group()
 
 
-def test_two_ranks_average_gradients_like_one_process():
+@pytest.mark.parametrize("mode", ["zero1", "allreduce"])
+def test_two_ranks_average_gradients_like_one_process(mode):
+    """Two ranks with half the micro-batches each end where one process with all
+    of them ends: in the sharded form (reduce-scatter per bucket, norm from the
+    summed shard partials, update of the own shards, gather of the copies) and
+    in the all-reduce form."""
     A, steps, world = 3, 3, 2
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q, A, steps)) for r in range(world)]
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q, A, steps, mode)) for r in range(world)]
     for p in procs:
         p.start()
     out = sorted(q.get(timeout=120) for _ in procs)
@@ -125,8 +175,9 @@ def test_two_ranks_average_gradients_like_one_process():
         ref_norms.append(ref.last_step_stats()[1])
 
     p0, p1 = np.array(out[0][1]), np.array(out[1][1])
-    assert np.array_equal(p0[:3], p1[:3]) and np.array_equal(p0[4:], p1[4:])
+    assert np.array_equal(p0, p1)                      # every rank computes with the same weights
     assert np.allclose(p0, ref.p.numpy(), rtol=0, atol=1e-13)
+    assert np.array_equal(np.array(out[0][7]), p0) and np.array_equal(np.array(out[1][7]), p1)
     assert np.allclose(out[0][2], ref_norms, rtol=1e-12)
     assert out[0][2] == out[1][2]                      # the same norm on every rank
     # held-out loss: the mean of the ranks' own losses
@@ -152,40 +203,26 @@ def test_single_process_is_the_plain_step():
 # --- data parallel with the checkpoint / eval cadence ----------------------------------------
 
 class CkptFake(FakeModel):
-    """FakeModel in fp32 with the state interface a checkpoint needs."""
+    """FakeModel with the state interface a checkpoint needs (one flat tensor)."""
 
     class Cfg(dict):
         grad_accum = 2
 
     def __init__(self, seed=0):
-        super().__init__(seed)
-        self.p = self.p.float()
-        self.g = self.g.float()
-        self.mom = {2: torch.zeros(N), 3: torch.zeros(N)}
+        super().__init__(seed, dtype=torch.float32)     # fp32 state, as the checkpoint stores it
         self.cfg = CkptFake.Cfg(n_embd=N, grad_accum=2)
-
-    def fwd_bwd(self, x, y):
-        f = _feat(x, y).float()
-        self.g += 0.3 * self.p - f
-        self.losses.append(float(f.sum()))
-        self.k += 1
-
-    def eval_loss(self, x, y):
-        return float(_feat(x, y).float() @ self.p)
 
     def tensors(self):
         from types import SimpleNamespace
         return [SimpleNamespace(name="w", shape=(N,))]
 
     def read(self, what, i):
-        return (self.p if what == dp.PARAMS else self.mom[what]).numpy().copy()
+        return self.state_tensor(what).numpy().copy()
 
     def write(self, what, i, a):
-        t = torch.tensor(a)
-        if what == dp.PARAMS:
-            self.p = t
-        else:
-            self.mom[what] = t
+        self.state_tensor(what)[:] = torch.tensor(a, dtype=self.dtype)
+        if what == dp.PARAMS:          # as gpt2_write: the copy follows the masters
+            self.w[:] = self.p
 
 
 class RankSource:
@@ -221,7 +258,7 @@ def _ckpt_rank_main(rank, world, port, q, root):
         s.next = h["data_cursor"]
         rc = ck.run(c, s, h["step"], 4, ident, cad, None, ev, par=dp.DataParallel(c))
         strip = lambda recs: [{k: v for k, v in r.items() if k != "checkpoint"} for r in recs]
-        q.put((rank, a.p.tolist(), c.p.tolist(), strip(ra), strip(ra[:2]) + strip(rc),
+        q.put((rank, a.weights().tolist(), c.weights().tolist(), strip(ra), strip(ra[:2]) + strip(rc),
                sorted(os.listdir(os.path.join(root, "b")))))
     finally:
         dist.destroy_process_group()

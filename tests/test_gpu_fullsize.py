@@ -92,9 +92,12 @@ def sample_rows(n, k=40, seed=0):
 
 
 def assert_bf16_of_exact(got, exact):
-    """bf16 round-to-nearest of an exactly known value: relative error <= 2^-9."""
-    bound = np.abs(exact) * 2.0 ** -9 + 1e-30
-    assert np.all(np.abs(got - exact) <= bound), float(np.max(np.abs(got - exact) - bound))
+    """bf16 round-to-nearest of an exactly known value: within half a unit in the
+    last place (bf16 keeps 8 significant bits: half an ulp is 2^(e - 8) for
+    2^e <= |x| < 2^(e+1)), and exact zeros stay zero."""
+    a = np.abs(exact)
+    half_ulp = np.where(a > 0, np.exp2(np.floor(np.log2(np.where(a > 0, a, 1.0))) - 8), 0.0)
+    assert np.all(np.abs(got - exact) <= half_ulp), float(np.max(np.abs(got - exact) - half_ulp))
 
 
 def test_lm_head_backward_full_size():
