@@ -104,6 +104,7 @@ _SIGNATURES = {
     "gpt2op_attention_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P]),
     "gpt2op_softmax_ce": (_I, [_P, _P, _P, _I, _I, _I, _F, _P, _P]),
     "gpt2op_softmax_ce_masked": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P]),
+    "gpt2op_lm_head_loss": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P]),
     "gpt2op_lm_head_ce_workspace": (_SZ, [_I, _I]),
     "gpt2op_lm_head_ce": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P, _SZ, _P, _P]),
     "gpt2op_embedding_fwd": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _P]),
@@ -479,6 +480,15 @@ def lm_head_ce(h, wte, targets, logits, losses, V, dscale, write_grad, ws, err, 
                                   dscale, 1 if write_grad else 0, _ptr(ws),
                                   0 if ws is None else ws.numel() * ws.element_size(), _ptr(err), _s(stream)),
           "gpt2op_lm_head_ce")
+
+
+def lm_head_loss(h, wte, targets, losses, V, ws, err, stream=None):
+    """Per-row losses of the tied lm_head with the logits never stored."""
+    N, C = h.shape
+    Vp = wte.shape[0]
+    check(lib().gpt2op_lm_head_loss(_ptr(h), _ptr(wte), _ptr(targets), _ptr(losses), N, C, V, Vp, _ptr(ws),
+                                    0 if ws is None else ws.numel() * ws.element_size(), _ptr(err), _s(stream)),
+          "gpt2op_lm_head_loss")
 
 
 def embedding_fwd(tokens, wte, wpe, out, V, err, stream=None):

@@ -39,6 +39,8 @@ enum Epi : int {
   EPI_ACC_F32 = 4,  // outf += acc (fp32; atomic when the reduction is split)
   EPI_LSE = 5,      // pair kernel only: out = bf16(acc), and per row and half tile the
                     // running (max, sum of 2^) of log2(e) * out over columns < lse_V
+  EPI_LSE_ONLY = 6, // pair kernel only: the partials of EPI_LSE and the row's target logit
+                    // bf16(acc)[row, lse_tgt[row]] into lse_tgt_val[row]; nothing else stored
 };
 
 struct Params {
@@ -48,6 +50,8 @@ struct Params {
   float* colsum;  // pair kernel, EPI_DGELU: column sums of the (bf16) output added here, or null
   float2* lse_part;  // pair kernel, EPI_LSE: [M][lse_slots] (max, sum) partials, slot = 2 * n_tile + half
   int lse_V, lse_slots;
+  const int32_t* lse_tgt;  // EPI_LSE_ONLY: target id per row (ids outside [0, lse_V) give no value)
+  float* lse_tgt_val;      // EPI_LSE_ONLY: the target's (bf16-rounded) logit per row
   bf16* out;
   bf16* out2;
   int ldo;
@@ -384,6 +388,8 @@ struct Call {
   float* colsum;     // EPI_DGELU with >= 256 rows: add the output's column sums here (else null)
   float2* lse_part;  // EPI_LSE: [M][2 * ceil(N / 256)] row partials (see Params)
   int lse_V;         // EPI_LSE: columns >= lse_V are stored but left out of the partials
+  const int32_t* lse_tgt;  // EPI_LSE_ONLY (see Params)
+  float* lse_tgt_val;
 };
 
 // Tile width: whole waves of 148 SMs, with 128-wide tiles charged 1.3x because a

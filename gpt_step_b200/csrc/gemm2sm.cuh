@@ -162,7 +162,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       tma_prefetch_desc(&tmA1);
       tma_prefetch_desc(&tmB1);
     }
-    if (EPI != gemm::EPI_ACC_F32) tma_prefetch_desc(&tmO);
+    if (EPI != gemm::EPI_ACC_F32 && EPI != gemm::EPI_LSE_ONLY) tma_prefetch_desc(&tmO);
     if (EPI == gemm::EPI_GELU) tma_prefetch_desc(&tmO2);
   }
   if (warp == 1) {
@@ -313,7 +313,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         // then runs at about the pace of the next tile's main loop.
         constexpr bool kBias = EPI == gemm::EPI_STORE || EPI == gemm::EPI_RESID || EPI == gemm::EPI_GELU ||
                                EPI == gemm::EPI_LSE;
-        constexpr bool kLse = EPI == gemm::EPI_LSE;
+        constexpr bool kLse = EPI == gemm::EPI_LSE || EPI == gemm::EPI_LSE_ONLY;
+        constexpr bool kStore = EPI != gemm::EPI_LSE_ONLY;
+        // EPI_LSE_ONLY: the row's target id, if it falls in this half tile (else -1)
+        int tgt_col = -1;
+        if (EPI == gemm::EPI_LSE_ONLY && row_ok) {
+          const int tg = __ldg(p.lse_tgt + row) - (nb * BN + hv * (BN / 2));
+          if (tg >= 0 && tg < BN / 2 && nb * BN + hv * (BN / 2) + tg < p.lse_V) tgt_col = tg;
+        }
         // EPI_LSE: this row's running max (log2 units) and sum of 2^(y - max) over the half tile
         float lse_m = -INFINITY, lse_s = 0.f;
         constexpr bool kAux = EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU;
@@ -431,7 +438,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
               for (int i = 0; i < 32; ++i) a[i & 3] += ex2_approx(fmaf(f[i], kL2e, -lse_m));
               lse_s += (a[0] + a[1]) + (a[2] + a[3]);
             }
+            if (EPI == gemm::EPI_LSE_ONLY) {
+              const int k = tgt_col - (c - c_beg);
+              if (k >= 0 && k < 32) {
+                float tv = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) tv = (i == k) ? f[i] : tv;
+                p.lse_tgt_val[row] = tv;
+              }
+            }
           }
+          if (!kStore) continue;
           if (EPI == gemm::EPI_DGELU && p.colsum != nullptr) {
             // column sums of the stored (bf16) values over this warp's 32 rows: a
             // transpose-reduce leaves column `lane` of the chunk in cs[0]
@@ -474,7 +491,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(acc ? tempty_leader1 : tempty_leader0);
     }
-    if (EPI != gemm::EPI_ACC_F32 && lane == 0) gemm::bulk_wait_all<0>();
+    if (EPI != gemm::EPI_ACC_F32 && EPI != gemm::EPI_LSE_ONLY && lane == 0) gemm::bulk_wait_all<0>();
   }
 
   tc_fence_before();
@@ -559,11 +576,16 @@ static int prepare(const gemm::Call& c, int splits_forced, Params& p, CUtensorMa
   p.num_tiles = p.num_m * p.num_n * p.splits;
   p.raster_gm = std::min(p.num_m, c.kind == WGRAD ? kRasterRowsWgrad : kRasterRows);
   p.colsum = c.epi == EPI_DGELU ? c.colsum : nullptr;
-  if (c.epi == EPI_LSE) {
+  if (c.epi == EPI_LSE || c.epi == EPI_LSE_ONLY) {
     if (c.kind != FWD || !c.lse_part || c.lse_V <= 0 || c.lse_V > c.N) return GPT2_ERR_ARG;
     p.lse_part = c.lse_part;
     p.lse_V = c.lse_V;
     p.lse_slots = 2 * p.num_n;
+    if (c.epi == EPI_LSE_ONLY) {
+      if (!c.lse_tgt || !c.lse_tgt_val) return GPT2_ERR_ARG;
+      p.lse_tgt = c.lse_tgt;
+      p.lse_tgt_val = c.lse_tgt_val;
+    }
   }
   p.out = c.out; p.out2 = c.out2; p.ldo = c.ldo;
   p.aux = c.aux; p.ld_aux = c.ld_aux; p.bias = c.bias;
@@ -582,7 +604,7 @@ static int prepare(const gemm::Call& c, int splits_forced, Params& p, CUtensorMa
     ok = make_map(&ta, c.a, c.K, c.M, c.lda, 64, 128) && make_map(&tb, c.b, c.K, c.N, c.ldb, 64, BN / 2);
   }
   if (!ok) return GPT2_ERR_ARG;
-  if (c.epi != EPI_ACC_F32) {
+  if (c.epi != EPI_ACC_F32 && c.epi != EPI_LSE_ONLY) {
     if (!make_map(&to, c.out, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return GPT2_ERR_ARG;
     if (c.epi == EPI_GELU && !make_map(&to2, c.out2, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
       return GPT2_ERR_ARG;
@@ -608,6 +630,7 @@ static int run(const gemm::Call& c, cudaStream_t s) {
       case EPI_RESID: e = launch_tc2<256, false, false, EPI_RESID>(ta, tb, to, to2, p, s); break;
       case EPI_GELU: e = launch_tc2<256, false, false, EPI_GELU>(ta, tb, to, to2, p, s); break;
       case EPI_LSE: e = launch_tc2<256, false, false, EPI_LSE>(ta, tb, to, to2, p, s); break;
+      case EPI_LSE_ONLY: e = launch_tc2<256, false, false, EPI_LSE_ONLY>(ta, tb, to, to2, p, s); break;
       default: return GPT2_ERR_ARG;
     }
   } else if (c.kind == DGRAD) {

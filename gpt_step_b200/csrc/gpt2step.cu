@@ -369,12 +369,14 @@ int bias_grad(const bf16* dout, float* db, int M, int N, float* part, size_t par
 // logits GEMM's EPI_LSE row partials ([N][slots]), or null to scan the row.
 int softmax_ce(bf16* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,
                int write_grad, int* err, cudaStream_t s, int ignore_index = INT_MIN,
-               const float2* part = nullptr, int slots = 0) {
+               const float2* part = nullptr, int slots = 0, const float* tgt_val = nullptr) {
   if (Vp % 8 || V > Vp || V <= 0) return GPT2_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(logits) & 15) != 0) return GPT2_ERR_ARG;
   if (part && slots <= 0) return GPT2_ERR_ARG;
+  if (tgt_val && (!part || write_grad)) return GPT2_ERR_ARG;   // logits-free: a loss from the partials only
+  if (!logits && !tgt_val) return GPT2_ERR_ARG;
   k::softmax_ce_kernel<<<N, k::kCeThreads, 0, s>>>(logits, targets, losses, V, Vp, dscale, write_grad, err,
-                                                    ignore_index, part, slots);
+                                                    ignore_index, part, slots, tgt_val);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -541,23 +543,30 @@ int forward(gpt2_model* m, const int32_t* tok, const int32_t* tgt, int b, bool t
   GPT2_TRY(ln_fwd_m(m, resid + L * NC, K_LNFW, K_LNFB, 0, lnf, m->at<float>(y.lnf_mean), m->at<float>(y.lnf_rstd),
                     (int)N));
   bf16* logits = m->at<bf16>(y.logits);
+  float* losses = m->at<float>(y.losses);
   // the pair kernel's epilogue also leaves each row's (max, sum) partials, so the
-  // cross-entropy reads the logits once
+  // cross-entropy reads the logits once; for a loss alone (evaluation) it keeps
+  // only the partials and the target logit, and the logits are never stored
   float2* lse_part = nullptr;
+  bool logits_free = false;
   {
     gemm::Call c = gemm_call(gemm::FWD, gemm::EPI_STORE, (int)N, d.Vp, C, err);
     c.a = lnf; c.lda = C; c.b = m->W(K_WTE); c.ldb = C; c.out = logits; c.ldo = d.Vp;
     if (gemm2::uses_pair(c)) {
       lse_part = m->at<float2>(y.lse_part);
       c.epi = gemm::EPI_LSE; c.lse_part = lse_part; c.lse_V = d.V;
+      if (!train) {
+        c.epi = gemm::EPI_LSE_ONLY; c.lse_tgt = tgt; c.lse_tgt_val = losses;
+        logits_free = true;
+      }
     }
     GPT2_TRY(run_gemm(m, c));
   }
-  float* losses = m->at<float>(y.losses);
   {
     const size_t p = prof_begin(m);
-    GPT2_TRY(launch::softmax_ce(logits, tgt, losses, (int)N, d.V, d.Vp, 1.0f / (float)N, train ? 1 : 0, err, s,
-                                INT_MIN, lse_part, lse_slots(d.Vp)));
+    GPT2_TRY(launch::softmax_ce(logits_free ? nullptr : logits, tgt, losses, (int)N, d.V, d.Vp, 1.0f / (float)N,
+                                train ? 1 : 0, err, s, INT_MIN, lse_part, lse_slots(d.Vp),
+                                logits_free ? losses : nullptr));
     k::loss_reduce_kernel<<<1, 1024, 0, s>>>(losses, (int)N, loss_acc, &m->sc()->micro_loss);
     // algorithmic bytes: the logits read (and overwritten when training), or with
     // the GEMM's partials those plus the partials, and no row scan for a loss alone
@@ -1314,6 +1323,23 @@ int gpt2op_lm_head_ce(const void* h, const void* wte, const int32_t* targets, vo
   if (st != GPT2_OK) return st;
   return launch::softmax_ce(static_cast<bf16*>(logits), targets, losses, N, V, Vp, dscale, write_grad ? 1 : 0,
                             dev_err, s, INT_MIN, part, lse_slots(Vp));
+}
+
+int gpt2op_lm_head_loss(const void* h, const void* wte, const int32_t* targets, float* losses, int N, int C, int V,
+                        int Vp, void* workspace, size_t ws_bytes, int* dev_err, void* stream) {
+  if (!h || !wte || !targets || !losses || !dev_err || N <= 0 || C <= 0 || V <= 0 || V > Vp) return GPT2_ERR_ARG;
+  if (!workspace || ws_bytes < gpt2op_lm_head_ce_workspace(N, Vp) || (reinterpret_cast<uintptr_t>(workspace) & 7) != 0)
+    return GPT2_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  gemm::Call c = gemm_call(gemm::FWD, gemm::EPI_LSE_ONLY, N, Vp, C, dev_err);
+  c.a = static_cast<const bf16*>(h); c.lda = C; c.b = static_cast<const bf16*>(wte); c.ldb = C;
+  if (!gemm2::uses_pair(c)) return GPT2_ERR_ARG;
+  float2* part = static_cast<float2*>(workspace);
+  c.lse_part = part; c.lse_V = V; c.lse_tgt = targets; c.lse_tgt_val = losses;
+  const int st = gemm2::run(c, s);
+  if (st != GPT2_OK) return st;
+  return launch::softmax_ce(nullptr, targets, losses, N, V, Vp, 1.0f, 0, dev_err, s, INT_MIN, part, lse_slots(Vp),
+                            losses);
 }
 
 int gpt2op_softmax_ce_masked(void* logits, const int32_t* targets, float* losses, int N, int V, int Vp,

@@ -533,12 +533,15 @@ GPT2_DEV void ce_combine(float& m, float& s, float om, float os) {
 // overwrites it with dz. With `part` given, pass 1 instead combines the row's
 // `slots` (max, sum) partials that the logits GEMM's epilogue left (the same
 // base-2 quantities over the same stored values), and the row is read once.
+// With `tgt_val` given as well (a loss without gradient), the target logit is
+// taken from tgt_val[row] and the logits are not read at all (may be null);
+// tgt_val may alias `losses`.
 __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict__ logits,
                                                                 const int32_t* __restrict__ targets,
                                                                 float* __restrict__ losses, int V, int Vp,
                                                                 float dscale, int write_grad, int* err,
                                                                 int ignore_index, const float2* __restrict__ part,
-                                                                int slots) {
+                                                                int slots, const float* tgt_val) {
   __shared__ float red_m[kCeThreads / 32], red_s[kCeThreads / 32];
   __shared__ float bc[2];
   const int row = blockIdx.x;
@@ -598,7 +601,7 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
   }
   if (threadIdx.x == 0) {
     // loss = lse - z[t] = (M2 + log2 S2) * ln2 - z[t]
-    const float zt = tok_ok ? __bfloat162float(logits[(size_t)row * Vp + t]) : 0.f;
+    const float zt = !tok_ok ? 0.f : (tgt_val ? tgt_val[row] : __bfloat162float(logits[(size_t)row * Vp + t]));
     losses[row] = tok_ok ? ((M2 + log2f(S2)) * kLn2F - zt) : 0.f;
   }
   if (!write_grad) return;

@@ -16,10 +16,11 @@
       op-level C ABI and prints TFLOP/s (causal FLOPs: the T(T+1)/2 visible pairs).
 
   python -m gpt_step_b200.profile_step head --shape N,C,Vp [--iters n]
-      Times the tied lm_head + softmax-CE both ways: the plain GEMM followed by
-      the two-pass CE, and the GEMM whose epilogue leaves the row partials
-      followed by the one-pass CE (real vocabulary Vp - 47), each alone and
-      together, in milliseconds.
+      Times the tied lm_head + softmax-CE: the plain GEMM followed by the
+      two-pass CE, the GEMM whose epilogue leaves the row partials followed by
+      the one-pass CE (real vocabulary Vp - 47), each alone and together, and
+      the logits-free loss (partials and target logit only, nothing stored),
+      in milliseconds.
 
   python -m gpt_step_b200.profile_step bw --kernel ln_fwd|ln_bwd|ce|colsum|embed_fwd|embed_bwd --shape rows,C [--iters n]
       Times a bandwidth-bound kernel alone and prints GB/s of algorithmic bytes
@@ -246,6 +247,8 @@ def run_head(args):
     out["gemm_store_ms"] = _time(gemm, args.iters)
     out["gemm_lse_plus_loss_only_ms"] = _time(
         lambda: gs.lm_head_ce(h, w, t, logits, losses, V, 1.0 / N, False, ws, err), args.iters)
+    # logits never stored: the GEMM keeps the row partials and the target logit only
+    out["logits_free_loss_ms"] = _time(lambda: gs.lm_head_loss(h, w, t, losses, V, ws, err), args.iters)
     out["ce_two_pass_ms"] = _time(lambda: (gemm(), ce2()), args.iters) - out["gemm_store_ms"]
     out["unfused_total_ms"] = out["gemm_store_ms"] + out["ce_two_pass_ms"]
     out["fused_total_ms"] = _time(lambda: gs.lm_head_ce(h, w, t, logits, losses, V, 1.0 / N, True, ws, err),

@@ -151,6 +151,16 @@ int gpt2op_lm_head_ce(const void* h, const void* wte, const int32_t* targets, vo
                       int C, int V, int Vp, float dscale, int write_grad, void* workspace, size_t ws_bytes,
                       int* dev_err, void* stream);
 
+/* The loss of the tied lm_head without its logits ever being stored (the
+ * evaluation form of gpt2op_lm_head_ce; §4.1 tied head, softmax over the V real
+ * ids): the GEMM's epilogue keeps, per row, only the (max, sum) partials of the
+ * bf16-rounded logits over ids < V and the target's logit, and losses fp32 [N] =
+ * lse - z[target]. No gradient. h bf16 [N,C], wte bf16 [Vp,C]; N >= 256 (the
+ * CTA-pair GEMM; smaller N returns GPT2_ERR_ARG); workspace as
+ * gpt2op_lm_head_ce_workspace. A target outside [0, V) gives loss 0 and flag 1. */
+int gpt2op_lm_head_loss(const void* h, const void* wte, const int32_t* targets, float* losses, int N, int C, int V,
+                        int Vp, void* workspace, size_t ws_bytes, int* dev_err, void* stream);
+
 /* Cross-entropy with an ignore index per target (the loss taken only on chosen
  * positions, e.g. the answers of question/answer text; "Pretraining and
  * adapting a language model on a dependency-free stack" trains its adapter that

@@ -196,6 +196,14 @@ def test_lm_head_ce(N, C, V, Vp):
     lr, dzr = G.softmax_ce(z, t, V)
     l0 = host(losses)
     assert np.max(np.abs(l0 - lr)) < 1e-4
+    # the logits-free evaluation form: the same partials and target logit, no logits stored
+    lf = torch.empty(N, device="cuda")
+    if N >= 256:
+        gs.lm_head_loss(hd, wd, td, lf, V, ws, err)
+        assert np.array_equal(host(lf), l0)
+    else:
+        with pytest.raises(gs.GPT2Error):
+            gs.lm_head_loss(hd, wd, td, lf, V, ws, err)
     gs.lm_head_ce(hd, wd, td, logits, losses, V, 1.0 / N, True, ws, err)
     assert np.array_equal(host(losses), l0)
     dz = host(logits)
