@@ -1,6 +1,7 @@
 """GPT-2 124M training throughput on B200 (fwd + bwd + clip + AdamW), one JSON line.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload gpt2_124m|gpt2_124m_b64|wide]
 
 Workload: GPT-2 124M (12 blocks, 12 heads, 768 channels, context 1,024,
 vocabulary 50,257 padded to 50,304, tied embeddings), micro-batch 19 x 9
@@ -29,6 +30,13 @@ instead trains N independent replicas (no exchange).
 
 --impl reference times the CPU oracle (the fp64 numpy definition of the same
 step) on the host cores on a bounded sample of the same workload.
+
+--workload selects one of the configurations the pages' recipe is run at (the
+headline is gpt2_124m): gpt2_124m_b64 is the same model at micro-batch 64 x 8
+accumulation (524,288 tokens per step), followed by its held-out pass (20
+batches of 64 x 1024 from a separately seeded stream, timed on its own and
+reported under "eval"); wide is 16 blocks, 24 heads, 1,536 channels,
+vocabulary 8,449 padded to 8,576, micro-batch 8 x 8.
 """
 from __future__ import annotations
 
@@ -48,8 +56,12 @@ sys.path.insert(0, ROOT)
 
 WORKLOAD = "gpt2_124m"
 PAGES_TOKENS_PER_S = 43374.0  # the pages' own stack, one card of their 3-card box (numbat §5.4, Table 3)
-N_PARAMS = 124_439_808
-FLOPS_PER_TOKEN = 6 * N_PARAMS + 6 * 12 * 768 * 1024  # 6N + causal attention
+DATASHEET_BF16_TFLOPS = 2250.0   # dense bf16 per GPU, NVIDIA's figure without 2:4 sparsity
+
+
+def flops_per_token(args, n_params):
+    """6 N (N = parameters over the real vocabulary) + causal attention 6 L C T."""
+    return 6.0 * n_params + 6.0 * args["n_layer"] * args["n_embd"] * args["seq_len"]
 
 
 def load_peaks():
@@ -63,11 +75,15 @@ def load_peaks():
             "source": "fallback"}
 
 
-def workload_desc(w, n_gpus, parallel="dp", dp_mode="zero1"):
+def workload_desc(w, n_gpus, parallel="dp", dp_mode="zero1", name=WORKLOAD):
+    vp = (w["vocab_real"] + 127) // 128 * 128
+    title = {"gpt2_124m": "GPT-2 124M", "gpt2_124m_b64": "GPT-2 124M at micro-batch 64",
+             "wide": "Wider GPT-2-style"}.get(name, name)
     return {
-        "workload": (f"GPT-2 124M training step: L{w['n_layer']} H{w['n_head']} C{w['n_embd']} "
-                     f"T{w['seq_len']} V{w['vocab_real']}->50304, micro-batch {w['micro_batch']} x "
+        "workload": (f"{title} training step: L{w['n_layer']} H{w['n_head']} C{w['n_embd']} "
+                     f"T{w['seq_len']} V{w['vocab_real']}->{vp}, micro-batch {w['micro_batch']} x "
                      f"{w['grad_accum']} accumulation"),
+        "name": name,
         "global_batch": w["micro_batch"] * w["grad_accum"] * n_gpus,
         "seq_len": w["seq_len"],
         "tokens_per_step": w["micro_batch"] * w["grad_accum"] * w["seq_len"] * n_gpus,
@@ -77,7 +93,8 @@ def workload_desc(w, n_gpus, parallel="dp", dp_mode="zero1"):
                          f"dp{n_gpus} (NCCL all-reduce of the fp32 gradients per optimizer step)")
                         if parallel == "dp" else f"replicas x{n_gpus}"),
         "l2": "inputs larger than L2 (each micro-step touches ~8 GB of activations and logits)",
-        "inputs": "synthetic Zipf(1.1) token stream, geometric(1000) documents, seed 1337+rank",
+        "inputs": (f"synthetic Zipf(1.1) token stream, geometric({w['mean_doc_len']}) documents, "
+                   "seed 1337+rank"),
     }
 
 
@@ -137,33 +154,41 @@ def run_reference(args, rank, world):
     """Time the CPU oracle on a bounded sample of the workload (rank 0 only)."""
     if rank != 0:
         return
-    res = cpu_baseline(target_seconds=max(10.0, 4.0 * args.steps), steps=args.steps, warmup=args.warmup)
-    w = __import__("gpt_step_b200.workloads", fromlist=["WORKLOADS"]).WORKLOADS[WORKLOAD]
+    from gpt_step_b200 import workloads
+    name = args.workload
+    w = workloads.WORKLOADS[name]
+    res = cpu_baseline(name, target_seconds=max(10.0, 4.0 * args.steps), steps=args.steps, one_core=False)
+    tokens_per_step = w["micro_batch"] * w["grad_accum"] * w["seq_len"]
     line = {
         "metric": "GPT-2 124M train tokens/s on 1 B200 (fwd+bwd+AdamW); MFU vs bf16 dense peak",
         "impl": "reference",
         "value": res["value"], "unit": "tokens/s", "n_gpus": 0, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": 1000.0 * w["micro_batch"] * w["grad_accum"] * 1024 / res["value"],
+        "warmup": args.warmup, "ms_per_step": 1000.0 * tokens_per_step / res["value"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_desc(w, 1),
+        "data": "synthetic", "config": workload_desc(w, 1, name=name),
         "cpu_baseline": res,
         "e2e": {"value": res["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
-def cpu_baseline(target_seconds=15.0, steps=1, warmup=0):
-    """Oracle tokens/s: fwd+bwd of 1 x 1024 tokens plus AdamW amortised over a full step."""
-    from gpt_step_b200 import synth, workloads
-    from oracle import gpt2 as G
+def _oracle_threads():
     try:
         from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
     except Exception:
-        cores = os.cpu_count()
-    args = workloads.model_args(WORKLOAD, micro_batch=1)
+        return os.cpu_count()
+
+
+def cpu_baseline(name=WORKLOAD, target_seconds=15.0, steps=1, one_core=True):
+    """Oracle tokens/s on the host: fwd+bwd of 1 x T tokens plus AdamW amortised over
+    a full step, with all the BLAS threads the process has, and (one_core) once
+    more with one thread."""
+    from gpt_step_b200 import synth, workloads
+    from oracle import gpt2 as G
+    args = workloads.model_args(name, micro_batch=1)
     cfg = G.Config(**args)
-    w = workloads.WORKLOADS[WORKLOAD]
+    w = workloads.WORKLOADS[name]
     p = G.init_params(cfg, 1337)
     src = synth.TokenSource(1, cfg.T, cfg.V, 1337, w["mean_doc_len"], 8)
     t_micro = []
@@ -185,11 +210,31 @@ def cpu_baseline(target_seconds=15.0, steps=1, warmup=0):
     t_adam = time.perf_counter() - a
     seqs_per_step = w["micro_batch"] * w["grad_accum"]
     t_seq = statistics.median(t_micro)
-    sec_per_token = (t_seq + t_adam / seqs_per_step) / cfg.T
-    return {"value": 1.0 / sec_per_token, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": (f"{n} oracle micro-steps of 1 x 1024 tokens (fwd+bwd, fp64 numpy; median "
-                       f"{t_seq:.2f} s) + one clip+AdamW over all 124.5M parameters "
-                       f"({t_adam:.2f} s) amortised over the {seqs_per_step} sequences of a step")}
+    value = 1.0 / ((t_seq + t_adam / seqs_per_step) / cfg.T)
+    cores = _oracle_threads()
+    out = {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "omp_num_threads": os.environ.get("OMP_NUM_THREADS", "unset"),
+           "host_cpus": os.cpu_count(),
+           "sample": (f"{n} oracle micro-steps of 1 x {cfg.T} tokens (fwd+bwd, fp64 numpy, {cores} BLAS threads; "
+                      f"median {t_seq:.2f} s) + one clip+AdamW over all parameters ({t_adam:.2f} s) "
+                      f"amortised over the {seqs_per_step} sequences of a step")}
+    if one_core:
+        try:
+            from threadpoolctl import threadpool_limits
+            x, y = src.get()
+            with threadpool_limits(1):
+                a = time.perf_counter()
+                G.fwd_bwd(cfg, p, x, y)
+                t1 = time.perf_counter() - a
+                a = time.perf_counter()
+                G.clip_adamw(cfg, p, g, m, v, 1)
+                ta1 = time.perf_counter() - a
+            out["one_core"] = {"value": 1.0 / ((t1 + ta1 / seqs_per_step) / cfg.T), "unit": "tokens/s",
+                               "sample": f"one micro-step of 1 x {cfg.T} tokens ({t1:.2f} s) + one AdamW "
+                                         f"({ta1:.2f} s) with the BLAS pool limited to 1 thread"}
+        except Exception as e:  # threadpoolctl missing: report without the one-thread figure
+            out["one_core"] = {"unavailable": str(e)[:100]}
+    return out
 
 
 # --------------------------------------------------------------------------- our arm
@@ -204,6 +249,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--parallel", default="dp", choices=["dp", "replicas"])
     ap.add_argument("--dp-mode", default="zero1", choices=["zero1", "allreduce"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=["gpt2_124m", "gpt2_124m_b64", "wide"])
     args = ap.parse_args()
 
     from gpt_step_b200.replicas import job_throughput, max_over_ranks, rank_env, replica_seed
@@ -227,9 +273,12 @@ def main():
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
 
-    w = workloads.WORKLOADS[WORKLOAD]
+    name = args.workload
+    w = workloads.WORKLOADS[name]
     B, T, A = w["micro_batch"], w["seq_len"], w["grad_accum"]
-    cfg = gs.Config.make(**workloads.model_args(WORKLOAD))
+    margs = workloads.model_args(name)
+    cfg = gs.Config.make(**margs)
+    fpt = flops_per_token(margs, gs.num_params(cfg))
     dp_mode = args.parallel == "dp"
     # data parallel: one model (the same initial weights everywhere), per-rank data
     model = gs.GPT2(cfg, 1337 if dp_mode else replica_seed(1337, rank))
@@ -324,6 +373,29 @@ def main():
                "api": ("DataParallel.step_host (pinned host tokens/targets, NCCL gradient average)" if multi
                        else "gpt2_train_step_host (pinned host tokens/targets)")}
 
+    # the held-out pass of the large-micro-batch workload: 20 batches of 64 x 1024
+    # from a separately seeded stream, losses only (no logits stored), timed alone
+    ev = None
+    if "eval_batches" in w:
+        eb, nb = w["eval_batch"], w["eval_batches"]
+        esrc = synth.TokenSource(eb, T, cfg.vocab_real, w["eval_seed"] + rank, w["mean_doc_len"], eb * nb)
+        etok, etgt = [], []
+        for _ in range(nb):
+            x, y = esrc.get()
+            etok.append(torch.tensor(x, device="cuda"))
+            etgt.append(torch.tensor(y, device="cuda"))
+        model.eval_loss(etok[0], etgt[0])          # warm-up
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        eloss = [model.eval_loss(a, b) for a, b in zip(etok, etgt)]
+        e1.record(stream)
+        barrier()
+        ems = max_over_ranks(e0.elapsed_time(e1), device="cuda")
+        ev = {"batches": nb, "batch": eb, "loss": round(float(np.mean(eloss)), 5),
+              "tokens_per_s": job_throughput(nb * eb * T, world, ems), "ms": round(ems, 3),
+              "seed": w["eval_seed"], "note": "eval_loss per batch includes its host read of the loss"}
+
     peaks = load_peaks()
     roof = None
     if prof and prof.get("gemm", {}).get("ms", 0) > 0:
@@ -337,23 +409,30 @@ def main():
                 "timing": "CUDA events around each launch in a second pass of K steps"}
 
     if rank == 0:
-        mfu = value / world * FLOPS_PER_TOKEN / (peaks["bf16_tflops"] * 1e12)
+        mfu = value / world * fpt / (peaks["bf16_tflops"] * 1e12)
         line = {
             "metric": "GPT-2 124M train tokens/s on 1 B200 (fwd+bwd+AdamW); MFU vs bf16 dense peak",
             "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(t_max / args.steps, 3),
             "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": round(value / PAGES_TOKENS_PER_S, 3),
-            "dtype": "bf16", "data": "synthetic", "config": workload_desc(w, world, args.parallel, args.dp_mode),
+            # the pages' figure is for this model at micro-batch 19 x 9 only
+            "vs_baseline": round(value / PAGES_TOKENS_PER_S, 3) if name == WORKLOAD else None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": workload_desc(w, world, args.parallel, args.dp_mode, name),
             "mfu": round(mfu, 4), "mfu_peak": f"{peaks['bf16_tflops']} TFLOP/s bf16 dense ({peaks['source']})",
+            "mfu_datasheet": round(value / world * fpt / (DATASHEET_BF16_TFLOPS * 1e12), 4),
+            "mfu_datasheet_peak": f"{DATASHEET_BF16_TFLOPS} TFLOP/s bf16 dense (datasheet)",
+            "flops_per_token": fpt,
             "loss": round(loss, 4), "grad_norm": round(norm, 4),
             "gpu_launches": int(launches), "clocks": clk, "roofline": roof, "e2e": e2e,
             "kernels": prof,
         }
+        if ev is not None:
+            line["eval"] = ev
         if agree is not None:
             line["replicas_agree"] = agree
         if not args.no_cpu_baseline and world == 1:
-            line["cpu_baseline"] = cpu_baseline()
+            line["cpu_baseline"] = cpu_baseline(name)
         print(json.dumps(line), flush=True)
     model.close()
     if world > 1:

@@ -407,8 +407,8 @@ def bias_grad_workspace(M, N):
 
 def bias_grad(dout, db, workspace, stream=None):
     M, N = dout.shape
-    check(lib().gpt2op_bias_grad(_ptr(dout), _ptr(db), M, N, _ptr(workspace), workspace.numel(),
-                                 _s(stream)), "gpt2op_bias_grad")
+    check(lib().gpt2op_bias_grad(_ptr(dout), _ptr(db), M, N, _ptr(workspace),
+                                 0 if workspace is None else workspace.numel(), _s(stream)), "gpt2op_bias_grad")
 
 
 def layernorm_fwd(x, w, b, y, mean, rstd, stream=None):
@@ -425,7 +425,8 @@ def layernorm_bwd(dy, x, mean, rstd, w, dresid, dx, dw, db, workspace, stream=No
     rows, C = x.shape
     check(lib().gpt2op_layernorm_bwd(_ptr(dy), _ptr(x), _ptr(mean), _ptr(rstd), _ptr(w), _ptr(dresid),
                                      _ptr(dx), _ptr(dw), _ptr(db), rows, C, _ptr(workspace),
-                                     workspace.numel(), _s(stream)), "gpt2op_layernorm_bwd")
+                                     0 if workspace is None else workspace.numel(), _s(stream)),
+          "gpt2op_layernorm_bwd")
 
 
 def layernorm_bwd_noalloc(dy, x, mean, rstd, w, dresid, dx, dw, db, stream=None):

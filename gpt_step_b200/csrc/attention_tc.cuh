@@ -38,6 +38,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kRescaleThreshold = 8.0f;    // log2(256)
 
+
 GPT2_DEV void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -265,25 +266,37 @@ __global__ void __launch_bounds__(kThreads, 2)
       float spart[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) spart[t] = 0.f;
-      uint32_t pkall[4][16];
+      // P_j as bf16 pairs (keys 2i, 2i+1 of this query row in column P_COL + i),
+      // in two halves of 64 keys: the first half's 32 words are stored (once the
+      // PV product of block j-1 has read the P buffer) before the second half is
+      // formed, so only 32 packed words are live at a time
+      bool waited = false;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i]), sl2, -m_new));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, -m_new));
-          spart[i & 7] += p0 + p1;
-          pkall[c][i] = pack_bf16x2(p0, p1);
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * half + cc;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i]), sl2, -m_new));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, -m_new));
+            spart[i & 7] += p0 + p1;
+            pk[cc * 16 + i] = pack_bf16x2(p0, p1);
+          }
         }
+        if (!waited) {
+          // the P buffer was last read by the PV product of block j-1
+          if (j >= 1 && !mbar_wait(smem_u32(p_empty), (j - 1) & 1, err)) { ok = false; }
+          tc_fence_after();
+          waited = true;
+        }
+        if (ok) tmem_st32_u(tmem + lane_off + P_COL + 32 * half, pk);
+      }
+      if (!ok) break;
       float sum = 0.f;
 #pragma unroll
       for (int t = 0; t < 8; ++t) sum += spart[t];
-      // the P buffer was last read by the PV product of block j-1
-      if (j >= 1 && !mbar_wait(smem_u32(p_empty), (j - 1) & 1, err)) { ok = false; break; }
-      tc_fence_after();
-      // P_j as bf16 pairs: keys 2i, 2i+1 of this query row in column P_COL + i
-      tmem_st32_u(tmem + lane_off + P_COL, *reinterpret_cast<const uint32_t(*)[32]>(&pkall[0][0]));
-      tmem_st32_u(tmem + lane_off + P_COL + 32, *reinterpret_cast<const uint32_t(*)[32]>(&pkall[2][0]));
       l = l * alpha + sum;
       m = m_new;
       // O rescale (rows whose maximum moved) once the PV product of block j-1 is done

@@ -237,6 +237,12 @@ GPT2_DEV void warp_colsum32(float (&cs)[32], int lane) {
   }
 }
 
+// Four fp32 atomic adds to 16-byte aligned global memory in one instruction.
+GPT2_DEV void red_add_f32x4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 GPT2_DEV float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

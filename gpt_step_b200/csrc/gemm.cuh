@@ -50,6 +50,8 @@ struct Params {
   float* colsum;  // pair kernel, EPI_DGELU: column sums of the (bf16) output added here, or null
   float2* lse_part;  // pair kernel, EPI_LSE: [M][lse_slots] (max, sum) partials, slot = 2 * n_tile + half
   int lse_V, lse_slots;
+  const int* sched;        // pair kernel: per-pair tile lists ([pairs + 1] offsets, then tile ids), or
+                           // null for the static stride (tile t on pair t mod pairs)
   const int32_t* lse_tgt;  // EPI_LSE_ONLY: target id per row (ids outside [0, lse_V) give no value)
   float* lse_tgt_val;      // EPI_LSE_ONLY: the target's (bf16-rounded) logit per row
   bf16* out;

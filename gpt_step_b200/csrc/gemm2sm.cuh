@@ -17,6 +17,7 @@
 // No TMA multicast is used: every load reads global memory into its own CTA.
 #pragma once
 #include <algorithm>
+#include <functional>
 #include <vector>
 
 #include "gemm.cuh"
@@ -144,6 +145,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   const bool leader = (rank == 0);
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
   const int total_tiles = p.num_tiles + (GROUP ? p1.num_tiles : 0);
+  // this pair's tiles: a host-built list, or every ncl-th tile from cid
+  const int* sch = p.sched;
+  const int k_beg = sch ? sch[cid] : cid, k_end = sch ? sch[cid + 1] : total_tiles, k_step = sch ? 1 : ncl;
+  const int* sch_tiles = sch ? sch + ncl + 1 : nullptr;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -180,7 +185,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      for (int t = cid; t < total_tiles && ok; t += ncl) {
+      for (int k = k_beg; k < k_end && ok; k += k_step) {
+        const int t = sch ? sch_tiles[k] : k;
         const bool second = GROUP && t >= p.num_tiles;
         const Params& q = second ? p1 : p;
         int mb, nb, sp;
@@ -228,7 +234,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int t = cid; t < total_tiles && ok; t += ncl, ++it) {
+      for (int k = k_beg; k < k_end && ok; k += k_step, ++it) {
+        const int t = sch ? sch_tiles[k] : k;
         const bool second = GROUP && t >= p.num_tiles;
         const Params& q = second ? p1 : p;
         const int tt = second ? t - p.num_tiles : t;
@@ -273,7 +280,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     int it = 0;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
-    for (int t = cid; t < total_tiles; t += ncl, ++it) {
+    for (int k = k_beg; k < k_end; k += k_step, ++it) {
+      const int t = sch ? sch_tiles[k] : k;
       const bool second = GROUP && t >= p.num_tiles;
       int mb, nb, sp;
       tile_coords(second ? p1 : p, second ? t - p.num_tiles : t, mb, nb, sp);
@@ -516,7 +524,8 @@ static cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& tb, cons
   if (GROUP) q1 = *p1;
   const int total = p.num_tiles + q1.num_tiles;
   const int pairs = gemm::num_sms() / 2;
-  const int grid = 2 * (total < pairs ? total : pairs);
+  // a planned schedule has one tile list per pair, some possibly empty
+  const int grid = 2 * ((p.sched != nullptr || total >= pairs) ? pairs : total);
   kern<<<grid, kThreads2, C::SMEM, s>>>(ta, tb, to, to2, p, GROUP ? *ta1 : ta, GROUP ? *tb1 : tb, q1);
   return cudaGetLastError();
 }
@@ -646,16 +655,84 @@ static int run(const gemm::Call& c, cudaStream_t s) {
   return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
+// Tile plan of a grouped launch whose schedule is built once on the host and
+// kept in device memory by the caller: the weight gradient's reduction split
+// and, per SM pair, the list of tiles it runs.
+struct GroupPlan {
+  int splits1 = 0;              // 0: no plan (static stride, split chosen per call)
+  std::vector<int> table;       // [pairs + 1] offsets, then tile ids
+  long makespan = 0;            // estimated k-block units of the busiest pair
+};
+
+// Longest-processing-time-first assignment: tiles in order of decreasing cost
+// (k-blocks plus an epilogue allowance, plus an atomic-pass allowance for split
+// weight-gradient tiles), each to the least loaded pair; each pair then runs its
+// tiles in increasing tile order, so pairs working at the same time stay on
+// nearby raster panels. The split of the weight gradient is the one with the
+// smallest estimated makespan.
+static GroupPlan plan_group(const gemm::Call& c0, const gemm::Call& c1, int pairs) {
+  using namespace gemm;
+  constexpr int kEpi = 2, kAtomic = 8;
+  GroupPlan best;
+  const long tiles0 = (long)((c0.M + BM_PAIR - 1) / BM_PAIR) * ((c0.N + 255) / 256);
+  const int cost0 = c0.K / BK + kEpi;
+  const int nkb1 = c1.K / BK;
+  const long tiles1 = (long)((c1.M + BM_PAIR - 1) / BM_PAIR) * (c1.N / 256);
+  for (int sp = 1; sp <= 32 && nkb1 >= 8 * sp; ++sp) {
+    const int kbps = (nkb1 + sp - 1) / sp;
+    const int nsp = (nkb1 + kbps - 1) / kbps;
+    if (nsp != sp) continue;
+    const int cost1 = kbps + kEpi + (nsp > 1 ? kAtomic : 0);
+    const long n = tiles0 + tiles1 * nsp;
+    // tiles of the costlier product first; within a product in tile order
+    std::vector<std::pair<long, int>> heap;   // (load, pair) min-heap
+    for (int i = 0; i < pairs; ++i) heap.push_back({0L, i});
+    std::vector<std::vector<int>> lists(pairs);
+    auto assign = [&](long first, long count, int cost) {
+      for (long t = first; t < first + count; ++t) {
+        std::pop_heap(heap.begin(), heap.end(), std::greater<>());
+        heap.back().first += cost;
+        lists[heap.back().second].push_back((int)t);
+        std::push_heap(heap.begin(), heap.end(), std::greater<>());
+      }
+    };
+    if (cost0 >= cost1) { assign(0, tiles0, cost0); assign(tiles0, tiles1 * nsp, cost1); }
+    else { assign(tiles0, tiles1 * nsp, cost1); assign(0, tiles0, cost0); }
+    long mk = 0;
+    for (auto& h : heap) mk = std::max(mk, h.first);
+    if (best.splits1 == 0 || mk < best.makespan) {
+      best.splits1 = nsp;
+      best.makespan = mk;
+      best.table.assign(pairs + 1 + n, 0);
+      int o = 0;
+      for (int i = 0; i < pairs; ++i) {
+        std::sort(lists[i].begin(), lists[i].end());
+        best.table[i] = o;
+        for (int t : lists[i]) best.table[pairs + 1 + o++] = t;
+      }
+      best.table[pairs] = o;
+    }
+  }
+  return best;
+}
+
 // A layer's input gradient (dgrad, c0) and weight gradient (wgrad, c1) in one
 // launch: c1's tiles follow c0's in the persistent tile list, its reduction
 // split chosen so that its tiles carry about as many k-blocks as c0's. Falls
 // back to two launches when either product does not take the pair kernel.
-static int run_group(const gemm::Call& c0, const gemm::Call& c1, cudaStream_t s, int* launches,
-                     int* splits_out = nullptr) {
+// With a plan (its split and its per-pair tile lists already in device memory
+// at dev_sched), the pairs run the planned lists.
+// Whether a dgrad (c0) and a wgrad (c1) can share one launch of the pair kernel.
+static bool groupable(const gemm::Call& c0, const gemm::Call& c1) {
   using namespace gemm;
-  const bool ok_shapes = c0.kind == DGRAD && c1.kind == WGRAD && c1.epi == EPI_ACC_F32 && c0.M > 0 &&
-                         c0.N % 32 == 0 && c0.K % BK == 0 && c1.K % BK == 0 && c1.K > 0 && uses_pair(c0) &&
-                         uses_pair(c1) && c1.N % 256 == 0;
+  return c0.kind == DGRAD && c1.kind == WGRAD && c1.epi == EPI_ACC_F32 && c0.M > 0 && c0.N % 32 == 0 &&
+         c0.K % BK == 0 && c1.K % BK == 0 && c1.K > 0 && uses_pair(c0) && uses_pair(c1) && c1.N % 256 == 0;
+}
+
+static int run_group(const gemm::Call& c0, const gemm::Call& c1, cudaStream_t s, int* launches,
+                     int* splits_out = nullptr, int plan_splits = 0, const int* dev_sched = nullptr) {
+  using namespace gemm;
+  const bool ok_shapes = groupable(c0, c1);
   *launches = ok_shapes ? 1 : 2;
   if (splits_out) *splits_out = 0;
   if (!ok_shapes) {
@@ -686,8 +763,14 @@ static int run_group(const gemm::Call& c0, const gemm::Call& c1, cudaStream_t s,
     const long mk = *std::max_element(load.begin(), load.end());
     if (best < 0 || mk < best) { best = mk; splits1 = nsp; }
   }
+  if (dev_sched != nullptr) {
+    if (plan_splits <= 0) return GPT2_ERR_ARG;
+    splits1 = plan_splits;
+  }
   st = prepare(c1, splits1, p1, ta1, tb1, to1, to21);
   if (st != GPT2_OK) return st;
+  if (dev_sched != nullptr && p1.splits != plan_splits) return GPT2_ERR_ARG;
+  p0.sched = dev_sched;
   if (splits_out) *splits_out = p1.splits;
   cudaError_t e = cudaErrorInvalidValue;
   switch (c0.epi) {

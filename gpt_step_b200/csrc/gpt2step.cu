@@ -41,6 +41,10 @@ enum KindId {
 constexpr int kNormBlocks = 2 * 148;
 constexpr int kLnBwdBlocks = 2 * 148;
 constexpr int kMaxStrips = 256;
+// grouped dgrad + wgrad launches of the backward: the four linear layers of a
+// block and the tied lm_head; each gets a tile plan of at most kSchedInts ints
+enum GroupId { G_MLP_PROJ = 0, G_MLP_FC, G_ATTN_PROJ, G_QKV, G_LM_HEAD, kNumGroups };
+constexpr int kSchedInts = 16384;
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -96,7 +100,7 @@ struct Layout {
   size_t resid, ln1, ln1_mean, ln1_rstd, qkv, atty, lse, resid_mid, ln2, ln2_mean, ln2_rstd, fch, fchg;
   size_t lnf, lnf_mean, lnf_rstd, logits, lse_part;
   size_t dresid, dln, d4c, dqkv, datty, dq_acc, attD;
-  size_t ln_part, col_part, norm_part, losses, scalars, eval_acc, err, tok, tgt;
+  size_t norm_part, losses, scalars, eval_acc, err, tok, tgt, sched;
   size_t total;
 };
 
@@ -178,9 +182,8 @@ void make_layout(const Dims& d, Layout* lay) {
   lay->datty = take(N * C * 2);
   lay->dq_acc = take(N * C * 4);
   lay->attD = take(N * d.H * 32);
-  lay->ln_part = take((size_t)kLnBwdBlocks * 3 * C * 4);
-  lay->col_part = take((size_t)kMaxStrips * 4 * C * 4);
   lay->norm_part = take(kNormBlocks * 8);
+  lay->sched = take((size_t)kNumGroups * kSchedInts * 4);
   lay->losses = take(N * 4);
   lay->scalars = take(sizeof(k::StepScalars));
   lay->eval_acc = take(64);
@@ -244,6 +247,7 @@ struct gpt2_model {
   int64_t launches = 0;  // kernels this model has launched
   Profiler prof;
   std::vector<cudaEvent_t> bucket_events;  // caller's events, recorded when each bucket's gradients are final
+  int group_splits[kNumGroups] = {};       // planned wgrad splits (0: no plan for that group)
   std::vector<NamedTensor> tensors;
   ~gpt2_model() {
     for (cudaEvent_t e : prof.ev) cudaEventDestroy(e);
@@ -268,11 +272,29 @@ struct gpt2_model {
 // ---------------------------------------------------------------------------
 namespace launch {
 
+// Resident CTAs of `kern` on the current device (blocks of `threads`, no dynamic shared memory).
+template <typename K>
+int resident_ctas(PerDeviceOnce& once, int (&cache)[PerDeviceOnce::kMaxDevices], K* kern, int threads) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= PerDeviceOnce::kMaxDevices) return 148;
+  once.run([&] {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    cache[dev] = per_sm * device_sm_count();
+    return cudaSuccess;
+  });
+  return cache[dev] > 0 ? cache[dev] : 148;
+}
+
 template <int C>
 void ln_fwd_c(const bf16* x, const float* w, const float* b, bf16* y, float* mean, float* rstd, int rows,
               cudaStream_t s) {
-  constexpr int rows_per_cta = 8 * k::kLnFwdRows;
-  k::layernorm_fwd_kernel<C><<<(rows + rows_per_cta - 1) / rows_per_cta, 256, 0, s>>>(x, w, b, y, mean, rstd, rows);
+  static PerDeviceOnce once;
+  static int cache[PerDeviceOnce::kMaxDevices] = {};
+  const int full = resident_ctas(once, cache, k::layernorm_fwd_kernel<C>, k::kLnFwdWarps * 32);
+  const int need = (rows + k::kLnFwdWarps - 1) / k::kLnFwdWarps;
+  k::layernorm_fwd_kernel<C><<<std::min(need, full), k::kLnFwdWarps * 32, 0, s>>>(x, w, b, y, mean, rstd, rows);
 }
 
 int ln_fwd(const bf16* x, const float* w, const float* b, bf16* y, float* mean, float* rstd, int rows, int C,
@@ -303,39 +325,43 @@ size_t ln_bwd_workspace(int rows, int C, int nq = 2) { return (size_t)ln_bwd_blo
 
 template <int C>
 cudaError_t ln_bwd_c(const bf16* dy, const bf16* x, const float* mean, const float* rstd, const float* w,
-                     const bf16* dresid, bf16* dx, float* part, int rows, int blocks, int with_dxsum, cudaStream_t s) {
+                     const bf16* dresid, bf16* dx, float* part, int rows, int blocks, int with_dxsum, float* dw,
+                     float* db, float* dbias, cudaStream_t s) {
   using Cfg = k::LnBwdCfg<C>;
   static PerDeviceOnce once;
   const cudaError_t e = smem_optin(once, k::layernorm_bwd_kernel<C>, Cfg::SMEM);
   if (e != cudaSuccess) return e;
   k::layernorm_bwd_kernel<C><<<blocks, Cfg::WARPS * 32, Cfg::SMEM, s>>>(dy, x, mean, rstd, w, dresid, dx, part, rows,
-                                                                        with_dxsum);
+                                                                        with_dxsum, dw, db, dbias);
   return cudaGetLastError();
 }
 
 // dbias (may be NULL) receives the column sum of dx: the bias gradient of the
-// projection whose output gradient dx is.
+// projection whose output gradient dx is. With a workspace (`part`) the column
+// sums are combined in a fixed order by a second launch (deterministic); with
+// part == NULL each CTA adds its sums into dw, db, dbias by fp32 vector atomics
+// in the same launch (dw, db, dbias then 16-byte aligned).
 int ln_bwd(const bf16* dy, const bf16* x, const float* mean, const float* rstd, const float* w, const bf16* dresid,
            bf16* dx, float* dw, float* db, float* dbias, int rows, int C, float* part, size_t part_bytes,
            cudaStream_t s) {
   const int nq = dbias ? 3 : 2;
   const int blocks = ln_bwd_blocks(rows, C);
-  if (part_bytes < (size_t)blocks * nq * C * 4) return GPT2_ERR_ARG;
+  if (part && part_bytes < (size_t)blocks * nq * C * 4) return GPT2_ERR_ARG;
+  if (!part && ((reinterpret_cast<uintptr_t>(dw) | reinterpret_cast<uintptr_t>(db) |
+                 reinterpret_cast<uintptr_t>(dbias)) & 15))
+    return GPT2_ERR_ARG;
   const int wd = dbias ? 1 : 0;
   cudaError_t e;
   switch (C) {
-    case 128: e = ln_bwd_c<128>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 256: e = ln_bwd_c<256>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 384: e = ln_bwd_c<384>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 512: e = ln_bwd_c<512>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 768: e = ln_bwd_c<768>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 1024: e = ln_bwd_c<1024>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 1536: e = ln_bwd_c<1536>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
-    case 2048: e = ln_bwd_c<2048>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, s); break;
+#define GPT2_LN_BWD_CASE(CC) \
+    case CC: e = ln_bwd_c<CC>(dy, x, mean, rstd, w, dresid, dx, part, rows, blocks, wd, dw, db, dbias, s); break;
+    GPT2_LN_BWD_CASE(128) GPT2_LN_BWD_CASE(256) GPT2_LN_BWD_CASE(384) GPT2_LN_BWD_CASE(512)
+    GPT2_LN_BWD_CASE(768) GPT2_LN_BWD_CASE(1024) GPT2_LN_BWD_CASE(1536) GPT2_LN_BWD_CASE(2048)
+#undef GPT2_LN_BWD_CASE
     default: return GPT2_ERR_ARG;
   }
   if (e != cudaSuccess) return GPT2_ERR_CUDA;
-  k::partial_rows_reduce_kernel<<<(nq * C + 31) / 32, 256, 0, s>>>(part, blocks, nq * C, dw, db, dbias, C);
+  if (part) k::partial_rows_reduce_kernel<<<(nq * C + 31) / 32, 256, 0, s>>>(part, blocks, nq * C, dw, db, dbias, C);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -354,14 +380,18 @@ size_t bias_grad_workspace(int M, int N) {
   return (size_t)strips * N * 4;
 }
 
+// With a workspace the strips' sums are combined in a fixed order by a second
+// launch (deterministic); with part == NULL they go into db by fp32 atomics in
+// the same launch (db then 16-byte aligned).
 int bias_grad(const bf16* dout, float* db, int M, int N, float* part, size_t part_bytes, cudaStream_t s) {
   if (N % 8) return GPT2_ERR_ARG;
   int strips, rps;
   colsum_geometry(M, N, &strips, &rps);
-  if (part_bytes < (size_t)strips * N * 4) return GPT2_ERR_ARG;
+  if (part && part_bytes < (size_t)strips * N * 4) return GPT2_ERR_ARG;
+  if (!part && (reinterpret_cast<uintptr_t>(db) & 15)) return GPT2_ERR_ARG;
   dim3 grid((N / 8 + 31) / 32, strips);
-  k::colsum_partial_kernel<<<grid, 256, 0, s>>>(dout, part, M, N, rps);
-  k::colsum_final_kernel<<<(N + 255) / 256, 256, 0, s>>>(part, db, strips, N);
+  k::colsum_partial_kernel<<<grid, 256, 0, s>>>(dout, part, M, N, rps, db);
+  if (part) k::colsum_final_kernel<<<(N + 255) / 256, 256, 0, s>>>(part, db, strips, N);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -460,11 +490,14 @@ int run_gemm(gpt2_model* m, const gemm::Call& c) {
   return st;
 }
 
-// A layer's dgrad (c0) and wgrad (c1) as one grouped launch where possible.
-int run_gemm_group(gpt2_model* m, const gemm::Call& c0, const gemm::Call& c1) {
+// A layer's dgrad (c0) and wgrad (c1) as one grouped launch where possible, on
+// the tile plan made at creation for that group.
+int run_gemm_group(gpt2_model* m, const gemm::Call& c0, const gemm::Call& c1, int group) {
   const size_t p = prof_begin(m);
   int nl = 2;
-  const int st = gemm2::run_group(c0, c1, m->stream, &nl);
+  const int sp = m->group_splits[group];
+  const int* sched = sp ? m->at<int>(m->lay.sched) + (size_t)group * kSchedInts : nullptr;
+  const int st = gemm2::run_group(c0, c1, m->stream, &nl, nullptr, sp, sched);
   prof_end(m, p, PC_GEMM, 2.0 * c0.M * c0.N * c0.K + 2.0 * c1.M * c1.N * c1.K, nl);
   return st;
 }
@@ -579,9 +612,8 @@ int forward(gpt2_model* m, const int32_t* tok, const int32_t* tgt, int b, bool t
 
 int bias_grad_m(gpt2_model* m, const bf16* dout, float* db, int M, int N) {
   const size_t p = prof_begin(m);
-  const int st = launch::bias_grad(dout, db, M, N, m->at<float>(m->lay.col_part),
-                                   (size_t)kMaxStrips * 4 * m->lay.d.C * 4, m->stream);
-  prof_end(m, p, PC_BIAS, 2.0 * M * N, 2);
+  const int st = launch::bias_grad(dout, db, M, N, nullptr, 0, m->stream);
+  prof_end(m, p, PC_BIAS, 2.0 * M * N, 1);
   return st;
 }
 
@@ -590,9 +622,8 @@ int ln_bwd_m(gpt2_model* m, const bf16* dy, const bf16* x, const float* mean, co
   const Dims& d = m->lay.d;
   const size_t p = prof_begin(m);
   const int st = launch::ln_bwd(dy, x, mean, rstd, m->P(kw, l), dresid, dx, m->G(kw, l), m->G(kb, l), dbias,
-                                (int)d.N, d.C, m->at<float>(m->lay.ln_part), (size_t)kLnBwdBlocks * 3 * d.C * 4,
-                                m->stream);
-  prof_end(m, p, PC_LN_BWD, (double)d.N * ((dresid ? 8.0 : 6.0) * d.C + 8), 2);
+                                (int)d.N, d.C, nullptr, 0, m->stream);
+  prof_end(m, p, PC_LN_BWD, (double)d.N * ((dresid ? 8.0 : 6.0) * d.C + 8), 1);
   return st;
 }
 
@@ -613,16 +644,13 @@ int backward(gpt2_model* m, const int32_t* tok) {
   bf16* dlogits = m->at<bf16>(y.logits);
   bf16* lnf = m->at<bf16>(y.lnf);
 
-  // tied head: dlnf = dlogits . wte ; dwte += dlogits^T . lnf
+  // tied head: dlnf = dlogits . wte ; dwte += dlogits^T . lnf (one grouped launch)
   {
-    gemm::Call c = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, d.Vp, err);
-    c.a = dlogits; c.lda = d.Vp; c.b = m->W(K_WTE); c.ldb = C; c.out = dln; c.ldo = C;
-    GPT2_TRY(run_gemm(m, c));
-  }
-  {
-    gemm::Call c = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, d.Vp, C, N, err);
-    c.a = dlogits; c.lda = d.Vp; c.b = lnf; c.ldb = C; c.outf = m->G(K_WTE); c.ldf = C;
-    GPT2_TRY(run_gemm(m, c));
+    gemm::Call cd = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, d.Vp, err);
+    cd.a = dlogits; cd.lda = d.Vp; cd.b = m->W(K_WTE); cd.ldb = C; cd.out = dln; cd.ldo = C;
+    gemm::Call cw = gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, d.Vp, C, N, err);
+    cw.a = dlogits; cw.lda = d.Vp; cw.b = lnf; cw.ldb = C; cw.outf = m->G(K_WTE); cw.ldf = C;
+    GPT2_TRY(run_gemm_group(m, cd, cw, G_LM_HEAD));
   }
   // the residual gradient leaving ln_f is the output gradient of the last MLP projection
   GPT2_TRY(ln_bwd_m(m, dln, resid + L * NC, m->at<float>(y.lnf_mean), m->at<float>(y.lnf_rstd), K_LNFW, K_LNFB, 0,
@@ -652,7 +680,7 @@ int backward(gpt2_model* m, const int32_t* tok) {
       cd.colsum = m->G(K_FCB, l);
       fused_fcb = gemm2::uses_pair(cd);
       if (!fused_fcb) cd.colsum = nullptr;
-      GPT2_TRY(run_gemm_group(m, cd, cw));
+      GPT2_TRY(run_gemm_group(m, cd, cw, G_MLP_PROJ));
     }
     // MLP fc
     {
@@ -660,7 +688,7 @@ int backward(gpt2_model* m, const int32_t* tok) {
       cw.a = d4c; cw.lda = 4 * C; cw.b = ln2; cw.ldb = C; cw.outf = m->G(K_FCW, l); cw.ldf = C;
       gemm::Call cd = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, 4 * C, err);
       cd.a = d4c; cd.lda = 4 * C; cd.b = m->W(K_FCW, l); cd.ldb = C; cd.out = dln; cd.ldo = C;
-      GPT2_TRY(run_gemm_group(m, cd, cw));
+      GPT2_TRY(run_gemm_group(m, cd, cw, G_MLP_FC));
     }
     if (!fused_fcb) GPT2_TRY(bias_grad_m(m, d4c, m->G(K_FCB, l), N, 4 * C));
     GPT2_TRY(ln_bwd_m(m, dln, xmid, m->at<float>(y.ln2_mean) + l * d.N, m->at<float>(y.ln2_rstd) + l * d.N, K_LN2W,
@@ -671,7 +699,7 @@ int backward(gpt2_model* m, const int32_t* tok) {
       cw.a = dresid; cw.lda = C; cw.b = atty; cw.ldb = C; cw.outf = m->G(K_ATTPROJW, l); cw.ldf = C;
       gemm::Call cd = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, C, err);
       cd.a = dresid; cd.lda = C; cd.b = m->W(K_ATTPROJW, l); cd.ldb = C; cd.out = datty; cd.ldo = C;
-      GPT2_TRY(run_gemm_group(m, cd, cw));
+      GPT2_TRY(run_gemm_group(m, cd, cw, G_ATTN_PROJ));
     }
     {
       const size_t p = prof_begin(m);
@@ -686,7 +714,7 @@ int backward(gpt2_model* m, const int32_t* tok) {
       cw.a = dqkv; cw.lda = 3 * C; cw.b = ln1; cw.ldb = C; cw.outf = m->G(K_QKVW, l); cw.ldf = C;
       gemm::Call cd = gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, 3 * C, err);
       cd.a = dqkv; cd.lda = 3 * C; cd.b = m->W(K_QKVW, l); cd.ldb = C; cd.out = dln; cd.ldo = C;
-      GPT2_TRY(run_gemm_group(m, cd, cw));
+      GPT2_TRY(run_gemm_group(m, cd, cw, G_QKV));
     }
     // every 2-D weight gradient of this block is final for this micro-step
     if (!m->bucket_events.empty() && cudaEventRecord(m->bucket_events[L - 1 - l], s) != cudaSuccess)
@@ -713,6 +741,40 @@ int status_of_device_word(int h) {
   if (h & DEVERR_TIMEOUT) return GPT2_ERR_TIMEOUT;
   if (h & DEVERR_TOKEN_RANGE) return GPT2_ERR_TOKEN_RANGE;
   if (h & DEVERR_NONFINITE) return GPT2_ERR_NONFINITE;
+  return GPT2_OK;
+}
+
+// Tile plans of the backward's grouped launches (the shapes are fixed by the
+// configuration), built on the host once and copied into the arena.
+int make_group_plans(gpt2_model* m) {
+  const Dims& d = m->lay.d;
+  const int N = (int)d.N, C = d.C;
+  struct Pair { gemm::Call cd, cw; };
+  Pair g[kNumGroups] = {
+      {gemm_call(gemm::DGRAD, gemm::EPI_DGELU, N, 4 * C, C, nullptr),
+       gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, C, 4 * C, N, nullptr)},
+      {gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, 4 * C, nullptr),
+       gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, 4 * C, C, N, nullptr)},
+      {gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, C, nullptr),
+       gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, C, C, N, nullptr)},
+      {gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, 3 * C, nullptr),
+       gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, 3 * C, C, N, nullptr)},
+      {gemm_call(gemm::DGRAD, gemm::EPI_STORE, N, C, d.Vp, nullptr),
+       gemm_call(gemm::WGRAD, gemm::EPI_ACC_F32, d.Vp, C, N, nullptr)}};
+  std::vector<int> host((size_t)kNumGroups * kSchedInts, 0);
+  const int pairs = gemm::num_sms() / 2;
+  for (int gi = 0; gi < kNumGroups; ++gi) {
+    m->group_splits[gi] = 0;
+    if (!gemm2::groupable(g[gi].cd, g[gi].cw)) continue;
+    const gemm2::GroupPlan plan = gemm2::plan_group(g[gi].cd, g[gi].cw, pairs);
+    if (plan.splits1 <= 0 || plan.table.size() > (size_t)kSchedInts) continue;
+    std::copy(plan.table.begin(), plan.table.end(), host.begin() + (size_t)gi * kSchedInts);
+    m->group_splits[gi] = plan.splits1;
+  }
+  if (cudaMemcpyAsync(m->at<int>(m->lay.sched), host.data(), host.size() * sizeof(int), cudaMemcpyHostToDevice,
+                      m->stream) != cudaSuccess ||
+      cudaStreamSynchronize(m->stream) != cudaSuccess)
+    return GPT2_ERR_CUDA;
   return GPT2_OK;
 }
 
@@ -840,6 +902,7 @@ int gpt2_create(const gpt2_config* cfg, uint64_t seed, void* dev_arena, size_t a
     }
   }
   if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) { delete m; return GPT2_ERR_CUDA; }
+  if (make_group_plans(m) != GPT2_OK) { delete m; return GPT2_ERR_CUDA; }
   *out = m;
   return GPT2_OK;
 }
@@ -1195,7 +1258,7 @@ int gpt2op_linear_bwd(const void* dout, const void* w, const void* inp, const vo
 size_t gpt2op_bias_grad_workspace(int M, int N) { return launch::bias_grad_workspace(M, N); }
 
 int gpt2op_bias_grad(const void* dout, float* db, int M, int N, void* workspace, size_t ws_bytes, void* stream) {
-  if (!dout || !db || !workspace) return GPT2_ERR_ARG;
+  if (!dout || !db) return GPT2_ERR_ARG;
   return launch::bias_grad(static_cast<const bf16*>(dout), db, M, N, static_cast<float*>(workspace), ws_bytes,
                            static_cast<cudaStream_t>(stream));
 }
@@ -1212,7 +1275,7 @@ size_t gpt2op_layernorm_bwd_workspace(int rows, int C) { return launch::ln_bwd_w
 int gpt2op_layernorm_bwd(const void* dy, const void* x, const float* mean, const float* rstd, const float* w,
                          const void* dresid, void* dx, float* dw, float* db, int rows, int C, void* workspace,
                          size_t ws_bytes, void* stream) {
-  if (!dy || !x || !mean || !rstd || !w || !dx || !dw || !db || !workspace || rows <= 0) return GPT2_ERR_ARG;
+  if (!dy || !x || !mean || !rstd || !w || !dx || !dw || !db || rows <= 0) return GPT2_ERR_ARG;
   return launch::ln_bwd(static_cast<const bf16*>(dy), static_cast<const bf16*>(x), mean, rstd, w,
                         static_cast<const bf16*>(dresid), static_cast<bf16*>(dx), dw, db, nullptr, rows, C,
                         static_cast<float*>(workspace), ws_bytes, static_cast<cudaStream_t>(stream));

@@ -144,40 +144,44 @@ __global__ void embed_bwd_wte_kernel(const int32_t* __restrict__ tok, const bf16
 }
 
 // ---------------------------------------------------------------------------
-// a2/a6/a9  LayerNorm forward: one warp per LN_ROWS rows (all their loads in
-// flight before any arithmetic), fp32 statistics (eps 1e-5, biased variance),
-// y = (x - mean) * rstd * w + b in bf16.
+// a2/a6/a9  LayerNorm forward: one warp per row in a grid-stride loop over the
+// rows (the next row's loads in flight while one is normalised; the grid is the
+// resident-CTA count, so there is no partial last wave), fp32 statistics (eps
+// 1e-5, biased variance), y = (x - mean) * rstd * w + b in bf16.
 // ---------------------------------------------------------------------------
-constexpr int kLnFwdRows = 2;   // rows per warp
+constexpr int kLnFwdWarps = 8;   // warps per CTA
+// CTAs per SM: as many as the row's registers allow without spilling
+__host__ __device__ constexpr int ln_fwd_minb(int C) { return C <= 512 ? 4 : (C <= 1024 ? 3 : 2); }
 template <int C>
-__global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restrict__ x, const float* __restrict__ w,
-                                                            const float* __restrict__ b, bf16* __restrict__ y,
-                                                            float* __restrict__ mean, float* __restrict__ rstd,
-                                                            int rows) {
+__global__ void __launch_bounds__(kLnFwdWarps * 32, ln_fwd_minb(C)) layernorm_fwd_kernel(const bf16* __restrict__ x,
+                                                                        const float* __restrict__ w,
+                                                                        const float* __restrict__ b,
+                                                                        bf16* __restrict__ y, float* __restrict__ mean,
+                                                                        float* __restrict__ rstd, int rows) {
   constexpr int NV = C / 8;                 // 16-byte vectors per row
   constexpr int VPL = (NV + 31) / 32;       // vectors per lane
-  constexpr int R = kLnFwdRows;
-  const int row0 = (blockIdx.x * 8 + (threadIdx.x >> 5)) * R;
   const int l = lane_id();
-  if (row0 >= rows) return;
-  uint4 u[R][VPL];
-#pragma unroll
-  for (int k = 0; k < R; ++k)
+  const int stride = gridDim.x * kLnFwdWarps;
+  int row = blockIdx.x * kLnFwdWarps + (threadIdx.x >> 5);
+  auto load = [&](int r, uint4 (&u)[VPL]) {
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int vi = l + 32 * i;
-      u[k][i] = (vi < NV && row0 + k < rows) ? __ldcs(reinterpret_cast<const uint4*>(x + (size_t)(row0 + k) * C) + vi)
-                                              : make_uint4(0u, 0u, 0u, 0u);
+      u[i] = (vi < NV && r < rows) ? __ldcs(reinterpret_cast<const uint4*>(x + (size_t)r * C) + vi)
+                                   : make_uint4(0u, 0u, 0u, 0u);
     }
-#pragma unroll
-  for (int k = 0; k < R; ++k) {
-    const int row = row0 + k;
-    if (row >= rows) break;
+  };
+  // grid-stride over rows, one row per warp at a time, the next row's loads in
+  // flight while this one is normalised
+  uint4 cur[VPL], nxt[VPL];
+  load(row, cur);
+  for (; row < rows; row += stride) {
+    load(row + stride, nxt);
     float v[VPL][8];
     float s = 0.f;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      const uint32_t wv[4] = {u[k][i].x, u[k][i].y, u[k][i].z, u[k][i].w};
+      const uint32_t wv[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const float2 f = unpack_bf16x2(wv[j]);
@@ -204,6 +208,7 @@ __global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restri
     for (int i = 0; i < VPL; ++i) {
       const int vi = l + 32 * i;
       if (vi < NV) {
+        // gain and shift: L1-resident after the first row
         const float4 w0 = __ldg(reinterpret_cast<const float4*>(w + vi * 8));
         const float4 w1 = __ldg(reinterpret_cast<const float4*>(w + vi * 8 + 4));
         const float4 b0 = __ldg(reinterpret_cast<const float4*>(b + vi * 8));
@@ -215,6 +220,7 @@ __global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restri
         for (int j = 0; j < 4; ++j)
           o[j] = pack_bf16x2((v[i][2 * j] - mu) * rs * ww[2 * j] + bb[2 * j],
                              (v[i][2 * j + 1] - mu) * rs * ww[2 * j + 1] + bb[2 * j + 1]);
+        // a plain store: the next GEMM reads y while it is still in L2
         *reinterpret_cast<uint4*>(yr + vi * 8) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
@@ -222,6 +228,8 @@ __global__ void __launch_bounds__(256) layernorm_fwd_kernel(const bf16* __restri
       mean[row] = mu;
       rstd[row] = rs;
     }
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) cur[i] = nxt[i];
   }
 }
 
@@ -250,7 +258,7 @@ template <int C>
 __global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, LnBwdCfg<C>::MINB)
     layernorm_bwd_kernel(const bf16* __restrict__ dy, const bf16* __restrict__ x, const float* __restrict__ mean,
                          const float* __restrict__ rstd, const float* __restrict__ w, const bf16* dresid, bf16* dx,
-                         float* __restrict__ part, int rows, int with_dxsum) {
+                         float* __restrict__ part, int rows, int with_dxsum, float* dw, float* db, float* dbias) {
   constexpr int NV = C / 8;
   constexpr int VPL = (NV + 31) / 32;
   constexpr int WARPS = LnBwdCfg<C>::WARPS;
@@ -378,12 +386,28 @@ __global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, LnBwdCfg<C>::MINB)
     }
   }
   __syncthreads();
-  // combine the warps' column sums in a fixed order (deterministic)
-  for (int c = threadIdx.x; c < nq * C; c += WARPS * 32) {
-    float sum = 0.f;
+  if (part != nullptr) {
+    // combine the warps' column sums in a fixed order (deterministic); a second
+    // launch sums the CTAs' partial rows
+    for (int c = threadIdx.x; c < nq * C; c += WARPS * 32) {
+      float sum = 0.f;
 #pragma unroll
-    for (int wi = 0; wi < WARPS; ++wi) sum += ln_acc[wi * 3 * C + c];
-    part[(size_t)blockIdx.x * nq * C + c] = sum;
+      for (int wi = 0; wi < WARPS; ++wi) sum += ln_acc[wi * 3 * C + c];
+      part[(size_t)blockIdx.x * nq * C + c] = sum;
+    }
+  } else {
+    // the CTA's column sums go straight into dw, db (and dbias) by vector atomics:
+    // one launch, summation order across CTAs unspecified
+    for (int c = 4 * threadIdx.x; c < nq * C; c += 4 * WARPS * 32) {
+      float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int wi = 0; wi < WARPS; ++wi) {
+        const float4 a = *reinterpret_cast<const float4*>(ln_acc + wi * 3 * C + c);
+        sum.x += a.x; sum.y += a.y; sum.z += a.z; sum.w += a.w;
+      }
+      float* dst = c < C ? dw + c : (c < 2 * C ? db + (c - C) : dbias + (c - 2 * C));
+      red_add_f32x4(dst, sum.x, sum.y, sum.z, sum.w);
+    }
   }
 }
 
@@ -413,8 +437,10 @@ __global__ void __launch_bounds__(256) partial_rows_reduce_kernel(const float* _
 // bias gradient: db[n] += sum_m dout[m, n] (bf16 input, two deterministic passes)
 // Pass 1: block (32 x 8 threads) covers 256 columns over a strip of rows.
 // ---------------------------------------------------------------------------
+// With part == nullptr the strip's sums are added into db directly (fp32 atomics,
+// no second pass).
 __global__ void __launch_bounds__(256) colsum_partial_kernel(const bf16* __restrict__ a, float* __restrict__ part,
-                                                             int M, int N, int rows_per_strip) {
+                                                             int M, int N, int rows_per_strip, float* db) {
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int c = (blockIdx.x * 32 + tx) * 8;
   const int r0 = blockIdx.y * rows_per_strip;
@@ -455,12 +481,19 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const bf16* __restr
   for (int j = 0; j < 8; ++j) red[ty][tx][j] = acc[j];
   __syncthreads();
   if (ty == 0 && c < N) {
+    float s[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      float s = 0.f;
+      s[j] = 0.f;
 #pragma unroll
-      for (int y = 0; y < 8; ++y) s += red[y][tx][j];
-      part[(size_t)blockIdx.y * N + c + j] = s;
+      for (int y = 0; y < 8; ++y) s[j] += red[y][tx][j];
+    }
+    if (part != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) part[(size_t)blockIdx.y * N + c + j] = s[j];
+    } else {
+      red_add_f32x4(db + c, s[0], s[1], s[2], s[3]);
+      red_add_f32x4(db + c + 4, s[4], s[5], s[6], s[7]);
     }
   }
 }

@@ -66,8 +66,11 @@ int gpt2op_linear_wgrad(const void* dout, const void* inp, float* dw, int M, int
 int gpt2op_linear_bwd(const void* dout, const void* w, const void* inp, const void* gelu_pre, void* din, float* dw,
                       float* colsum, int M, int N, int K, int* splits_out, int* dev_err, void* stream);
 
-/* Bias gradient: db[N] (fp32) += sum over rows of dout[M,N] (bf16),
- * deterministic two-pass column sum. N % 8 == 0. */
+/* Bias gradient: db[N] (fp32) += sum over rows of dout[M,N] (bf16). N % 8 == 0.
+ * With a workspace: a deterministic two-pass column sum. With workspace NULL:
+ * one launch whose strips add into db by fp32 atomics (the form gpt2_fwd_bwd
+ * uses; db 16-byte aligned; the order of the additions, and so the last bits,
+ * may vary between runs). */
 size_t gpt2op_bias_grad_workspace(int M, int N);
 int gpt2op_bias_grad(const void* dout, float* db, int M, int N, void* workspace, size_t ws_bytes, void* stream);
 
@@ -80,7 +83,11 @@ int gpt2op_layernorm_fwd(const void* x, const float* w, const float* b, void* y,
 
 /* LayerNorm backward: dx = LN'(dy) (+ dresid, the residual-stream gradient, may
  * be NULL; dx may alias dresid); dw, db (fp32 [C]) += column sums of dy * xhat
- * and dy (deterministic). */
+ * and dy. With a workspace the column sums are combined in a fixed order by a
+ * second launch (deterministic). With workspace NULL each CTA adds its sums
+ * into dw and db by fp32 vector atomics in the same launch (the form
+ * gpt2_fwd_bwd uses; dw, db 16-byte aligned; the last bits may vary between
+ * runs). */
 size_t gpt2op_layernorm_bwd_workspace(int rows, int C);
 int gpt2op_layernorm_bwd(const void* dy, const void* x, const float* mean, const float* rstd, const float* w,
                          const void* dresid, void* dx, float* dw, float* db, int rows, int C, void* workspace,

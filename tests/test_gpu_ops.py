@@ -81,20 +81,26 @@ def test_linear_wgrad(M, N, K, splits):
     assert rel_l2(host(dw), ref) < 1e-5
 
 
-def test_bias_grad():
+@pytest.mark.parametrize("atomic", [False, True])
+def test_bias_grad(atomic):
+    """Column sums: deterministic two-pass with a workspace, one launch with fp32
+    atomics without (the form the model uses)."""
     M, N = 3000, 2304
     dy = rnd((M, N), 14)
     db0 = rnd(N, 15)
     db = f32(db0)
-    ws = torch.empty(gs.bias_grad_workspace(M, N), dtype=torch.uint8, device="cuda")
+    ws = None if atomic else torch.empty(gs.bias_grad_workspace(M, N), dtype=torch.uint8, device="cuda")
     gs.bias_grad(bf16(dy), db, ws)
     assert rel_l2(host(db), db0.astype(np.float32) + rounded(dy).sum(0)) < 1e-6
 
 
 # --- a2/a6/a9: LayerNorm -------------------------------------------------------------------
 
-@pytest.mark.parametrize("C", [128, 384, 768, 1536])
-def test_layernorm_fwd_bwd(C):
+@pytest.mark.parametrize("C,atomic", [(128, False), (384, False), (768, False), (1536, False), (128, True),
+                                      (768, True), (1536, True)])
+def test_layernorm_fwd_bwd(C, atomic):
+    """LayerNorm forward and backward; the backward's column sums both ways: a
+    fixed-order second pass over a workspace, or fp32 atomics in one launch."""
     rows = 1000
     x = rnd((rows, C), 16, 2.0) + 0.5
     w, b = 1.0 + rnd(C, 17, 0.1), rnd(C, 18, 0.1)
@@ -112,7 +118,7 @@ def test_layernorm_fwd_bwd(C):
     dx = torch.empty_like(y)
     dw0, db0 = rnd(C, 21), rnd(C, 22)
     dw, db = f32(dw0), f32(db0)
-    ws = torch.empty(gs.layernorm_bwd_workspace(rows, C), dtype=torch.uint8, device="cuda")
+    ws = None if atomic else torch.empty(gs.layernorm_bwd_workspace(rows, C), dtype=torch.uint8, device="cuda")
     gs.layernorm_bwd(bf16(dy), xd, mean, rstd, f32(w), bf16(dres), dx, dw, db, ws)
     rdx, rdw, rdb = G.layernorm_bwd(rounded(dy), xr, mr, rr, w32)
     assert rel_l2(host(dx), rdx + rounded(dres)) < BF16_TOL
@@ -172,9 +178,10 @@ def test_softmax_ce(N, V, Vp):
     assert int(err[0]) & 1
 
 
-@pytest.mark.parametrize("N,C,V,Vp", [(700, 256, 50257, 50304), (512, 768, 50257, 50304), (1024, 384, 4353, 4480),
-                                       (300, 256, 1000, 1024), (128, 128, 4353, 4480)])
-def test_lm_head_ce(N, C, V, Vp):
+@pytest.mark.parametrize("N,C,V,Vp,pair", [(700, 256, 50257, 50304, True), (512, 768, 50257, 50304, True),
+                                            (1024, 384, 4353, 4480, True), (300, 256, 1000, 1024, False),
+                                            (128, 128, 4353, 4480, False)])
+def test_lm_head_ce(N, C, V, Vp, pair):
     """Tied lm_head GEMM + softmax-CE. The first three shapes run the GEMM on CTA
     pairs, whose epilogue leaves per-row (max, sum) partials so that the CE reads
     the logits once (700 rows: a ragged last row tile); the last two take the
@@ -198,7 +205,7 @@ def test_lm_head_ce(N, C, V, Vp):
     assert np.max(np.abs(l0 - lr)) < 1e-4
     # the logits-free evaluation form: the same partials and target logit, no logits stored
     lf = torch.empty(N, device="cuda")
-    if N >= 256:
+    if pair:
         gs.lm_head_loss(hd, wd, td, lf, V, ws, err)
         assert np.array_equal(host(lf), l0)
     else:
