@@ -23,15 +23,35 @@
 
 namespace attn_tc {
 
-constexpr int BQ = 128, BKV = 128, HD = 64;
+constexpr int BQ = 128, BKV = 128, HD = 64;   // HD: the backward's head size (the forward is templated)
 constexpr int kThreads = 192;
-constexpr int Q_BYTES = BQ * HD * 2;         // 16 KB
-constexpr int KV_BYTES = BKV * HD * 2;       // 16 KB each for K and V
 constexpr int STAGES = 2;
-// No alignment slack: without static shared memory the dynamic block starts on a
-// 1 KB boundary (checked at run time). 82,944 bytes and 256 TMEM columns a CTA:
-// two CTAs share an SM.
-constexpr int SMEM_BYTES = Q_BYTES + STAGES * 2 * KV_BYTES + 1024 /*barriers*/;
+// Forward geometry for head size D (64 or 32): Q, K, V tiles of 128 rows of D
+// bf16 (rows of 128 or 64 bytes, in the tensor core's 128- or 64-byte swizzled
+// layout, which the TMA's swizzle of the same width writes). No alignment
+// slack: without static shared memory the dynamic block starts on a 1 KB
+// boundary (checked at run time). At most 82,944 bytes and 256 TMEM columns a
+// CTA: two CTAs share an SM.
+template <int D>
+struct FwdGeom {
+  static_assert(D == 64 || D == 32, "head size");
+  static constexpr int ROW = D * 2;                       // bytes per tile row
+  static constexpr int Q_BYTES = BQ * ROW;
+  static constexpr int KV_BYTES = BKV * ROW;
+  static constexpr int SMEM_BYTES = Q_BYTES + STAGES * 2 * KV_BYTES + 1024 /*barriers*/;
+  static constexpr uint64_t kSwizzle = D == 64 ? 2 : 4;  // descriptor layout: 128- / 64-byte swizzle
+};
+// Shared-memory matrix descriptor for a swizzled tile (layout 2: 128-byte rows,
+// 4: 64-byte rows); strides in bytes.
+GPT2_DEV uint64_t smem_desc_swz(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes, uint64_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  d |= layout << 61;
+  return d;
+}
 constexpr int TMEM_COLS = 256;               // S [0,128), O [128,192), P [192,256); two CTAs share an SM
 constexpr uint32_t S_COL0 = 0, O_COL = 128, P_COL = 192;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -73,9 +93,13 @@ GPT2_DEV void tmem_st32_u(uint32_t taddr, const uint32_t (&v)[32]) {
 }
 GPT2_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
                        int T, int H, float scale, int* err) {
+  using G = FwdGeom<D>;
+  constexpr int HD = D;
+  constexpr int Q_BYTES = G::Q_BYTES, KV_BYTES = G::KV_BYTES;
   extern __shared__ __align__(1024) uint8_t smem_raw_af[];
   uint8_t* smem = smem_raw_af;
   if (smem_u32(smem) & 1023u) {  // the swizzled tiles need a 1 KB-aligned base
@@ -182,9 +206,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t k_addr = smem_u32(sK + st * KV_BYTES);
         const uint32_t d = tmem + S_COL0;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk)
-          tc_mma_bf16(d, smem_desc_sw128(q_addr + kk * 32, 16, 1024), smem_desc_sw128(k_addr + kk * 32, 16, 1024),
-                      idesc_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < HD / 16; ++kk)   // K-major Q, K: 16 head-dim columns (32 bytes) a step
+          tc_mma_bf16(d, smem_desc_swz(q_addr + kk * 32, 16, 8 * G::ROW, G::kSwizzle),
+                      smem_desc_swz(k_addr + kk * 32, 16, 8 * G::ROW, G::kSwizzle), idesc_s, kk > 0 ? 1u : 0u);
         tc_commit(smem_u32(s_full));
         tc_commit(smem_u32(&k_empty[st]));
       };
@@ -209,10 +233,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!mbar_wait(smem_u32(&v_full[st]), (j >> 1) & 1, err)) { ok = false; break; }
         tc_fence_after();
         const uint32_t v_addr = smem_u32(sV + st * KV_BYTES);
-        const uint64_t vd = smem_desc_sw128(v_addr, 8192, 1024);
+        // V as stored ([key][head dim]): an MN-major B operand whose 8-key groups are
+        // 8 rows apart; its head dimension is one swizzle atom wide
+        const uint64_t vd = smem_desc_swz(v_addr, D == 64 ? 8192 : 8 * G::ROW, 8 * G::ROW, G::kSwizzle);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)   // A = P from tensor memory, 16 keys = 8 columns a step
-          tc_mma_bf16_ts(tmem + O_COL, tmem + P_COL + kk * 8, vd + kk * 128, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_bf16_ts(tmem + O_COL, tmem + P_COL + kk * 8, vd + kk * ((16 * G::ROW) >> 4), idesc_o,
+                         (j > 0 || kk > 0) ? 1u : 0u);
         tc_commit(smem_u32(p_empty));
         tc_commit(smem_u32(&v_empty[st]));
         tc_commit(smem_u32(o_done));
@@ -342,23 +369,28 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-// qkv bf16 [B*T, 3C] (q | k | v, heads contiguous), out bf16 [B*T, C], lse fp32 [B, H, T].
+// qkv bf16 [B*T, 3C] (q | k | v, heads contiguous), out bf16 [B*T, C], lse fp32 [B, H, T];
+// head size D = 64 or 32, T a multiple of 128.
+template <int D>
 static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, int* err, cudaStream_t s) {
+  using G = FwdGeom<D>;
   static PerDeviceOnce once;
   cudaError_t e0 = once.run([] {
-    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    cudaError_t e = cudaFuncSetAttribute(attn_fwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         G::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     // ask for the whole shared-memory carveout so that two CTAs share an SM
-    return cudaFuncSetAttribute(attn_fwd_tc_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return cudaFuncSetAttribute(attn_fwd_tc_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   });
   if (e0 != cudaSuccess) return e0;
-  const int C = H * HD;
+  if (T % BQ) return cudaErrorInvalidValue;
+  const int C = H * D;
   CUtensorMap tm;
   if (!encode_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qkv, 3 * (uint64_t)C, (uint64_t)B * T, 3 * (uint64_t)C,
-                     64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+                     D, 128, D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   dim3 grid(T / BQ, B * H);
-  attn_fwd_tc_kernel<<<grid, kThreads, SMEM_BYTES, s>>>(tm, out, lse, T, H, 1.0f / sqrtf((float)HD), err);
+  attn_fwd_tc_kernel<D><<<grid, kThreads, G::SMEM_BYTES, s>>>(tm, out, lse, T, H, 1.0f / sqrtf((float)D), err);
   return cudaGetLastError();
 }
 

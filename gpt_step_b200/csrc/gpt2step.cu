@@ -415,7 +415,8 @@ int softmax_ce(bf16* logits, const int32_t* targets, float* losses, int N, int V
 int attention_fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, int hd, int* err, cudaStream_t s) {
   if (T % 64) return GPT2_ERR_ARG;
   cudaError_t e;
-  if (hd == 64 && T % attn_tc::BQ == 0 && err != nullptr) e = attn_tc::fwd(qkv, out, lse, B, T, H, err, s);
+  if (hd == 64 && T % attn_tc::BQ == 0 && err != nullptr) e = attn_tc::fwd<64>(qkv, out, lse, B, T, H, err, s);
+  else if (hd == 32 && T % attn_tc::BQ == 0 && err != nullptr) e = attn_tc::fwd<32>(qkv, out, lse, B, T, H, err, s);
   else if (hd == 64) e = attn::fwd<64>(qkv, out, lse, B, T, H, s);
   else if (hd == 32) e = attn::fwd<32>(qkv, out, lse, B, T, H, s);
   else return GPT2_ERR_ARG;
@@ -727,8 +728,8 @@ int backward(gpt2_model* m, const int32_t* tok) {
   {
     const size_t p = prof_begin(m);
     k::embed_bwd_wpe_kernel<<<(T * C / 8 + 255) / 256, 256, 0, s>>>(dresid, m->G(K_WPE), d.B, T, C);
-    k::embed_bwd_wte_kernel<<<launch::grid_for((long)N * C / 8, 256), 256, 0, s>>>(tok, dresid, m->G(K_WTE), N, C,
-                                                                                      d.V);
+    k::embed_bwd_wte_kernel<<<(N + k::kEmbRows - 1) / k::kEmbRows, 256, 0, s>>>(tok, dresid, m->G(K_WTE), N, C,
+                                                                                d.V);
     prof_end(m, p, PC_EMBED, (double)N * (2.0 * C + 4) + 2.0 * N * C * 4 + 8.0 * T * C, 2);
   }
   // the last bucket (wpe, wte) and the 1-D region are final now
@@ -1438,8 +1439,8 @@ int gpt2op_embedding_bwd(const int32_t* tokens, const void* dx, float* dwte, flo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long N = (long)B * T;
   k::embed_bwd_wpe_kernel<<<(T * C / 8 + 255) / 256, 256, 0, s>>>(static_cast<const bf16*>(dx), dwpe, B, T, C);
-  k::embed_bwd_wte_kernel<<<launch::grid_for(N * C / 8, 256), 256, 0, s>>>(tokens, static_cast<const bf16*>(dx), dwte,
-                                                                           (int)N, C, V);
+  k::embed_bwd_wte_kernel<<<(int)((N + k::kEmbRows - 1) / k::kEmbRows), 256, 0, s>>>(
+      tokens, static_cast<const bf16*>(dx), dwte, (int)N, C, V);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 

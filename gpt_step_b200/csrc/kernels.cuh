@@ -123,23 +123,56 @@ __global__ void embed_bwd_wpe_kernel(const bf16* __restrict__ dx, float* __restr
   d[1] = d1;
 }
 
-// a1 backward, token part: dwte[tok[n], :] += dx[n, :]   (fp32 vector atomics)
-__global__ void embed_bwd_wte_kernel(const int32_t* __restrict__ tok, const bf16* __restrict__ dx,
-                                     float* __restrict__ dwte, int N, int C, int V) {
+// a1 backward, token part: dwte[tok[n], :] += dx[n, :]. A CTA takes kEmbRows
+// consecutive positions; rows with the same token id are summed inside the CTA
+// (in position order) and added into dwte once per id by fp32 vector atomics, so
+// a frequent id (the Zipf head of the stream) sees one atomic per CTA instead
+// of one per occurrence.
+constexpr int kEmbRows = 64;
+__global__ void __launch_bounds__(256) embed_bwd_wte_kernel(const int32_t* __restrict__ tok,
+                                                            const bf16* __restrict__ dx, float* __restrict__ dwte,
+                                                            int N, int C, int V) {
+  __shared__ int st[kEmbRows];
+  __shared__ unsigned char lead[kEmbRows];
+  const int r0 = blockIdx.x * kEmbRows;
+  if (threadIdx.x < kEmbRows) {
+    const int n = r0 + threadIdx.x;
+    const int t = n < N ? tok[n] : -1;
+    st[threadIdx.x] = (t >= 0 && t < V) ? t : -1;
+  }
+  __syncthreads();
+  if (threadIdx.x < kEmbRows) {
+    const int t = st[threadIdx.x];
+    bool first = t >= 0;
+    for (int j = 0; j < (int)threadIdx.x && first; ++j) first = st[j] != t;
+    lead[threadIdx.x] = first ? 1 : 0;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   const int vpr = C / 8;
-  const long total = (long)N * vpr;
-  for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
-    const int n = (int)(i / vpr), c = (int)(i % vpr) * 8;
-    const int t = tok[n];
-    if (t < 0 || t >= V) continue;
-    const uint4 u = *reinterpret_cast<const uint4*>(dx + (size_t)n * C + c);
-    const float2 f0 = unpack_bf16x2(u.x), f1 = unpack_bf16x2(u.y), f2 = unpack_bf16x2(u.z), f3 = unpack_bf16x2(u.w);
-    float* d = dwte + (size_t)t * C + c;
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(d), "f"(f0.x), "f"(f0.y), "f"(f1.x), "f"(f1.y)
-                 : "memory");
-    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(d + 4), "f"(f2.x), "f"(f2.y), "f"(f3.x),
-                 "f"(f3.y)
-                 : "memory");
+  // leaders in round robin over the warps; a lane owns the 16-byte chunks lane, lane + 32, ..
+  int k = 0;
+  for (int i = 0; i < kEmbRows; ++i) {
+    if (!lead[i]) continue;
+    if ((k++ % nw) != warp) continue;
+    const int t = st[i];
+    for (int v = lane; v < vpr; v += 32) {
+      float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      for (int j = i; j < kEmbRows; ++j) {
+        if (st[j] != t) continue;
+        const uint4 u = *reinterpret_cast<const uint4*>(dx + (size_t)(r0 + j) * C + v * 8);
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = unpack_bf16x2(w[q]);
+          acc[2 * q] += f.x;
+          acc[2 * q + 1] += f.y;
+        }
+      }
+      float* d = dwte + (size_t)t * C + v * 8;
+      red_add_f32x4(d, acc[0], acc[1], acc[2], acc[3]);
+      red_add_f32x4(d + 4, acc[4], acc[5], acc[6], acc[7]);
+    }
   }
 }
 
@@ -706,9 +739,19 @@ __global__ void __launch_bounds__(512) sumsq_partial_kernel(const float* __restr
   __shared__ double red[16];
   double s = 0.0;
   const float4* g4 = reinterpret_cast<const float4*>(g);
+  const long stride = (long)gridDim.x * blockDim.x;
   for (int r = 0; r < rg.n; ++r) {
-    for (long i = rg.begin[r] + blockIdx.x * (long)blockDim.x + threadIdx.x; i < rg.end[r];
-         i += (long)gridDim.x * blockDim.x) {
+    long i = rg.begin[r] + blockIdx.x * (long)blockDim.x + threadIdx.x;
+    // four loads in flight per thread
+    for (; i + 3 * stride < rg.end[r]; i += 4 * stride) {
+      float4 v[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[q] = __ldcs(g4 + i + q * stride);
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        s += (double)v[q].x * v[q].x + (double)v[q].y * v[q].y + (double)v[q].z * v[q].z + (double)v[q].w * v[q].w;
+    }
+    for (; i < rg.end[r]; i += stride) {
       const float4 v = g4[i];
       s += (double)v.x * v.x + (double)v.y * v.y + (double)v.z * v.z + (double)v.w * v.w;
     }

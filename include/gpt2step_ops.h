@@ -183,7 +183,10 @@ int gpt2op_softmax_ce_masked(void* logits, const int32_t* targets, float* losses
 int gpt2op_embedding_fwd(const int32_t* tokens, const void* wte, const void* wpe, void* out, int B, int T, int C,
                          int V, int* dev_err, void* stream);
 
-/* Embedding backward: dwte[tok,:] += dx (fp32 atomics), dwpe[t,:] += sum_b dx. */
+/* Embedding backward: dwte[tok,:] += dx, dwpe[t,:] += sum_b dx (fp32). Rows with
+ * the same id within a block of 64 positions are summed in position order and
+ * added into dwte once by fp32 vector atomics (dwte 16-byte aligned; the last
+ * bits may vary between runs); ids outside [0, V) are skipped. */
 int gpt2op_embedding_bwd(const int32_t* tokens, const void* dx, float* dwte, float* dwpe, int B, int T, int C, int V,
                          void* stream);
 

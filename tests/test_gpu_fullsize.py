@@ -40,11 +40,15 @@ def _gpu():
 
 # --- a4: attention with many work items per persistent CTA -------------------------------------
 
-@pytest.mark.parametrize("Bt", [4, 19])
-def test_attention_many_items_per_cta(Bt):
+@pytest.mark.parametrize("Bt,HDt", [(4, 64), (19, 64), (16, 32)])
+def test_attention_many_items_per_cta(Bt, HDt):
     """(Bt, 1024, 12, 64): 384 and 1,824 backward work items against 148 SMs,
-    so most CTAs run the cross-item K/V prefetch and accumulator hand-over.
-    Every dQ, dK, dV element, the output and the lse are compared."""
+    so most CTAs run the cross-item K/V prefetch and accumulator hand-over; and
+    head size 32 at (16, 1024, 12) (the small configuration's attention, the
+    forward on the tensor cores with 64-byte rows). Every dQ, dK, dV element,
+    the output and the lse are compared."""
+    HD = HDt
+    C = H * HD
     rng = np.random.default_rng(40 + Bt)
     qkv = rng.standard_normal((Bt, T, 3 * C)).astype(np.float32)
     do = rng.standard_normal((Bt, T, C)).astype(np.float32)
