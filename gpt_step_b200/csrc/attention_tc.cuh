@@ -93,6 +93,19 @@ GPT2_DEV void tmem_st32_u(uint32_t taddr, const uint32_t (&v)[32]) {
 }
 GPT2_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Load 16 consecutive fp32 columns of this warp's 32 TMEM lanes.
+GPT2_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
@@ -433,7 +446,6 @@ static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int
 namespace bwd {
 constexpr int BKEY = 128, BQRY = 128;
 constexpr int NQS = 3;                              // Q / dO ring depth
-constexpr int T_BYTES = 128 * HD * 2;               // 16 KB: a 128-row tile of K, V, Q or dO
 constexpr int DST_BYTES = BKEY * BQRY * 2;          // 32 KB: dS^T
 constexpr int DQW_BYTES = 32 * 32 * 4;              // 4 KB: one warp's dQ staging box
 constexpr int kSoftmaxWarps = 8;
@@ -444,9 +456,18 @@ constexpr int kThreads = 128 + 32 * kSoftmaxWarps;
 constexpr int kLaunchRegs = 168, kCtlRegs = 152, kSoftmaxRegs = 176;
 static_assert(128 * kCtlRegs + 32 * kSoftmaxWarps * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int XT_BYTES = 128 * 16 * 2;              // 4 KB: a 128 x 16 extra-K operand tile
-constexpr int SMEM_BYTES = 2 * T_BYTES /*K,V*/ + NQS * 2 * T_BYTES /*Q,dO*/ + DST_BYTES +
-                           kSoftmaxWarps * DQW_BYTES + NQS * XT_BYTES /*X_i*/ + 2 * XT_BYTES /*K', V' columns*/ +
-                           256 /*barriers*/ + 1024 /*align*/;
+// Per head size D (64 or 32): a 128-row tile of K, V, Q or dO has rows of 2 D
+// bytes in the 128- or 64-byte swizzled layout.
+template <int D>
+struct Geom {
+  static constexpr int ROW = D * 2;
+  static constexpr int T_BYTES = 128 * ROW;
+  static constexpr int SMEM_BYTES = 2 * T_BYTES /*K,V*/ + NQS * 2 * T_BYTES /*Q,dO*/ + DST_BYTES +
+                                    kSoftmaxWarps * DQW_BYTES + NQS * XT_BYTES /*X_i*/ +
+                                    2 * XT_BYTES /*K', V' columns*/ + 256 /*barriers*/ + 1024 /*align*/;
+  static constexpr uint64_t kSwizzle = D == 64 ? 2 : 4;
+  static constexpr uint32_t kMnLbo = D == 64 ? 8192 : 8 * ROW;   // MN-major: one swizzle atom wide, unused
+};
 constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 320, C_DQ = 384, C_P = 448;
 constexpr int TMEM_COLS_BWD = 512;
 constexpr int kPrepRows = 32;                       // query rows per prep block
@@ -507,13 +528,15 @@ GPT2_DEV void bwd_softmax_row(const uint32_t (&sv)[2][32], const uint32_t (&dv)[
 }
 
 // Block: 32 consecutive query rows of one sequence, all heads. Each warp takes
-// four rows; lanes hold 16-byte chunks of O and dO, eight chunks per head.
+// four rows; lanes hold 16-byte chunks of O and dO, D / 8 chunks per head.
+template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
                                                        const float* __restrict__ lse, uint8_t* __restrict__ xtiles,
                                                        float* __restrict__ dq_acc, int T, int H, float scale) {
   using namespace bwd;
+  constexpr int CPH = D / 8;                 // 16-byte chunks per head
   __shared__ float sDot[kMaxHeads][kPrepRows];
-  const int C = H * HD;
+  const int C = H * D;
   const int NV = C / 8;                      // 16-byte chunks per row
   const int row0 = blockIdx.x * kPrepRows;   // global row (b*T + t) of the first query
   const int b = row0 / T, t0 = row0 % T;
@@ -534,10 +557,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ 
           acc = fmaf(fa.x, fc.x, fmaf(fa.y, fc.y, acc));
         }
       }
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-      if ((lane & 7) == 0 && vi < NV) sDot[vi >> 3][rl] = acc;
+#pragma unroll
+      for (int o = 1; o < CPH; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if ((lane & (CPH - 1)) == 0 && vi < NV) sDot[vi / CPH][rl] = acc;
     }
   }
   __syncthreads();
@@ -574,11 +596,16 @@ __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__
   }
 }
 
+template <int D>
 __global__ void __launch_bounds__(bwd::kThreads, 1)
     attn_bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, const __grid_constant__ CUtensorMap tm_do,
                        const __grid_constant__ CUtensorMap tm_dq, const uint8_t* __restrict__ xtiles,
                        bf16* __restrict__ dqkv, int T, int H, int BH, float scale, int* err) {
   using namespace bwd;
+  using G = Geom<D>;
+  constexpr int HD = D;
+  constexpr int T_BYTES = G::T_BYTES;
+  constexpr int NO = D / 2;                       // head-dim columns of dQ, dK, dV per softmax warp
   extern __shared__ __align__(1024) uint8_t smem_raw_ab[];
   uint8_t* smem =
       reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_ab) + 1023) & ~uintptr_t(1023));
@@ -694,15 +721,17 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         constexpr uint32_t id_q = idesc_bf16_f32(BQRY, HD, true, true);       // dQ
         // Descriptors are formed once; a shared-memory offset is added in 16-byte
         // units to the start-address field (addresses stay below 2^18, no carry).
-        const uint64_t dK_k = smem_desc_sw128(smem_u32(sK), 16, 1024);        // K, K-major
-        const uint64_t dV_k = smem_desc_sw128(smem_u32(sV), 16, 1024);        // V, K-major
-        const uint64_t dK_mn = smem_desc_sw128(smem_u32(sK), 8192, 1024);     // K, MN-major
+        constexpr uint32_t kSbo = 8 * G::ROW;                                 // 8-row groups
+        const uint64_t dK_k = smem_desc_swz(smem_u32(sK), 16, kSbo, G::kSwizzle);        // K, K-major
+        const uint64_t dV_k = smem_desc_swz(smem_u32(sV), 16, kSbo, G::kSwizzle);        // V, K-major
+        const uint64_t dK_mn = smem_desc_swz(smem_u32(sK), G::kMnLbo, kSbo, G::kSwizzle);  // K, MN-major
         const uint64_t dDS_k = smem_desc_sw128(smem_u32(sDST), 16, 1024);     // dS^T, K-major
         const uint64_t dDS_mn = smem_desc_sw128(smem_u32(sDST), BKEY * 128, 1024);  // dS, MN-major
-        const uint64_t dQ0_k = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-        const uint64_t dQ0_mn = smem_desc_sw128(smem_u32(sQ), 8192, 1024);
-        const uint64_t dO0_k = smem_desc_sw128(smem_u32(sDO), 16, 1024);
-        const uint64_t dO0_mn = smem_desc_sw128(smem_u32(sDO), 8192, 1024);
+        const uint64_t dQ0_k = smem_desc_swz(smem_u32(sQ), 16, kSbo, G::kSwizzle);
+        const uint64_t dQ0_mn = smem_desc_swz(smem_u32(sQ), G::kMnLbo, kSbo, G::kSwizzle);
+        const uint64_t dO0_k = smem_desc_swz(smem_u32(sDO), 16, kSbo, G::kSwizzle);
+        const uint64_t dO0_mn = smem_desc_swz(smem_u32(sDO), G::kMnLbo, kSbo, G::kSwizzle);
+        constexpr uint64_t kMnStep = (16 * G::ROW) >> 4;   // 16 rows of an MN-major operand, descriptor units
         const uint64_t dXK = smem_desc_interleave(smem_u32(sXK), 128, 256);
         const uint64_t dXV = smem_desc_interleave(smem_u32(sXV), 128, 256);
         const uint64_t dXQ0 = smem_desc_interleave(smem_u32(sXQ), 128, 256);
@@ -750,15 +779,16 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < BQRY / 16; ++kk) {
               const uint32_t aoff = ((kk >> 2) * (BKEY * 128) + (kk & 3) * 32) >> 4;
-              tc_mma_bf16_ts(tmem + C_DV, tmem + C_P + kk * 8, dO0_mn + so + kk * 128, id_kv, kk > 0 ? 1u : acc0);
-              tc_mma_bf16(tmem + C_DK, dDS_k + aoff, dQ0_mn + so + kk * 128, id_kv, kk > 0 ? 1u : acc0);
+              tc_mma_bf16_ts(tmem + C_DV, tmem + C_P + kk * 8, dO0_mn + so + kk * kMnStep, id_kv,
+                             kk > 0 ? 1u : acc0);
+              tc_mma_bf16(tmem + C_DK, dDS_k + aoff, dQ0_mn + so + kk * kMnStep, id_kv, kk > 0 ? 1u : acc0);
             }
             // dQ of this block once the previous block's dQ has left tensor memory
             if (gc > 0 && !mbar_wait(smem_u32(dq_empty), (gc - 1) & 1, err)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < BKEY / 16; ++kk)
-              tc_mma_bf16(tmem + C_DQ, dDS_mn + kk * 128, dK_mn + kk * 128, id_q, kk > 0 ? 1u : 0u);
+              tc_mma_bf16(tmem + C_DQ, dDS_mn + kk * 128, dK_mn + kk * kMnStep, id_q, kk > 0 ? 1u : 0u);
             tc_commit(smem_u32(dq_full));
             tc_commit(smem_u32(ds_empty));
             tc_commit(smem_u32(&qdo_empty[gc % NQS]));
@@ -786,8 +816,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     auto drain_dq = [&](int gq, int hc, int qrow0) -> bool {
       if (!mbar_wait(smem_u32(dq_full), gq & 1, err)) return false;
       tc_fence_after();
-      float v[32];
-      tmem_ld32(tmem + lane_off + C_DQ + hf * 32, v);
+      float v[NO];
+      if (NO == 32) tmem_ld32(tmem + lane_off + C_DQ + hf * NO, *reinterpret_cast<float(*)[32]>(v));
+      else tmem_ld16(tmem + lane_off + C_DQ + hf * NO, *reinterpret_cast<float(*)[16]>(v));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
@@ -795,14 +826,18 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         bulk_wait_group_read<0>();   // this warp's previous reduce has read the box
       }
       __syncwarp();
+      // the staging box: 32 rows of NO floats in the reduce map's swizzled layout
+      // (128-byte rows: chunk ^ (row & 7); 64-byte rows: chunk ^ ((row >> 1) & 3))
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<float4*>(stage + lane * 128 + ((ch ^ (lane & 7)) << 4)) =
+      for (int ch = 0; ch < NO / 4; ++ch) {
+        const int pc = NO == 32 ? (ch ^ (lane & 7)) : (ch ^ ((lane >> 1) & 3));
+        *reinterpret_cast<float4*>(stage + lane * (NO * 4) + (pc << 4)) =
             make_float4(v[4 * ch], v[4 * ch + 1], v[4 * ch + 2], v[4 * ch + 3]);
+      }
       fence_async_smem();
       __syncwarp();
       if (lane == 0) {
-        tma_reduce_add_2d(&tm_dq, smem_u32(stage), hc + hf * 32, qrow0 + q4 * 32);
+        tma_reduce_add_2d(&tm_dq, smem_u32(stage), hc + hf * NO, qrow0 + q4 * 32);
         bulk_commit_group();
       }
       return true;
@@ -855,18 +890,20 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
       // dK, dV of this item for key row r, head-dim columns 32 hf ..
       if (!mbar_wait(smem_u32(dkdv_full), j & 1, err)) { ok = false; break; }
       tc_fence_after();
-      bf16* krow = dqkv + ((size_t)(row_base + kb * BKEY + r)) * 3 * C + C + h * HD + hf * 32;
+      bf16* krow = dqkv + ((size_t)(row_base + kb * BKEY + r)) * 3 * C + C + h * HD + hf * NO;
       bf16* vrow = krow + C;
-      float v[32];
-      tmem_ld32(tmem + lane_off + C_DK + hf * 32, v);
+      float v[NO];
+      if (NO == 32) tmem_ld32(tmem + lane_off + C_DK + hf * NO, *reinterpret_cast<float(*)[32]>(v));
+      else tmem_ld16(tmem + lane_off + C_DK + hf * NO, *reinterpret_cast<float(*)[16]>(v));
 #pragma unroll
-      for (int i2 = 0; i2 < 32; i2 += 8)
+      for (int i2 = 0; i2 < NO; i2 += 8)
         *reinterpret_cast<uint4*>(krow + i2) =
             make_uint4(pack_bf16x2(v[i2], v[i2 + 1]), pack_bf16x2(v[i2 + 2], v[i2 + 3]),
                        pack_bf16x2(v[i2 + 4], v[i2 + 5]), pack_bf16x2(v[i2 + 6], v[i2 + 7]));
-      tmem_ld32(tmem + lane_off + C_DV + hf * 32, v);
+      if (NO == 32) tmem_ld32(tmem + lane_off + C_DV + hf * NO, *reinterpret_cast<float(*)[32]>(v));
+      else tmem_ld16(tmem + lane_off + C_DV + hf * NO, *reinterpret_cast<float(*)[16]>(v));
 #pragma unroll
-      for (int i2 = 0; i2 < 32; i2 += 8)
+      for (int i2 = 0; i2 < NO; i2 += 8)
         *reinterpret_cast<uint4*>(vrow + i2) =
             make_uint4(pack_bf16x2(v[i2], v[i2 + 1]), pack_bf16x2(v[i2 + 2], v[i2 + 3]),
                        pack_bf16x2(v[i2 + 4], v[i2 + 5]), pack_bf16x2(v[i2 + 6], v[i2 + 7]));
@@ -888,36 +925,40 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 
 // The whole backward. xtiles (B*H*T*32 bytes) and dq_acc fp32 [B*T, C] are
 // scratch (contents on entry do not matter); dqkv receives dQ | dK | dV.
+template <int D>
 static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, uint8_t* xtiles,
-                       float* dq_acc, bf16* dqkv, int B, int T, int H, int* err, cudaStream_t s) {
+                           float* dq_acc, bf16* dqkv, int B, int T, int H, int* err, cudaStream_t s) {
+  using G = bwd::Geom<D>;
   static PerDeviceOnce once;
   cudaError_t e0 = once.run([] {
     // The register hand-over inside the kernel needs the block to be launched
     // with kLaunchRegs registers a thread; anything less would stall it.
     cudaFuncAttributes fa;
-    cudaError_t e = cudaFuncGetAttributes(&fa, attn_bwd_tc_kernel);
+    cudaError_t e = cudaFuncGetAttributes(&fa, attn_bwd_tc_kernel<D>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != bwd::kLaunchRegs) return cudaErrorInvalidConfiguration;
-    return cudaFuncSetAttribute(attn_bwd_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bwd::SMEM_BYTES);
+    return cudaFuncSetAttribute(attn_bwd_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM_BYTES);
   });
   if (e0 != cudaSuccess) return e0;
-  if (H > bwd::kMaxHeads || T % bwd::kPrepRows) return cudaErrorInvalidValue;
-  const int C = H * HD;
-  const float scale = 1.0f / sqrtf((float)HD);
+  if (H > bwd::kMaxHeads || T % bwd::kPrepRows || T % bwd::BKEY) return cudaErrorInvalidValue;
+  const int C = H * D;
+  const float scale = 1.0f / sqrtf((float)D);
+  const CUtensorMapSwizzle swz = D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
   CUtensorMap tm_qkv, tm_do, tm_dq;
+  // dQ boxes: 32 query rows x D/2 fp32 columns (128- or 64-byte rows)
   if (!encode_map_2d(&tm_qkv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qkv, 3 * (uint64_t)C, (uint64_t)B * T,
-                     3 * (uint64_t)C, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_map_2d(&tm_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dout, (uint64_t)C, (uint64_t)B * T, (uint64_t)C, 64,
-                     128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+                     3 * (uint64_t)C, D, 128, swz) ||
+      !encode_map_2d(&tm_do, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, dout, (uint64_t)C, (uint64_t)B * T, (uint64_t)C, D,
+                     128, swz) ||
       !encode_map_2d(&tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, (uint64_t)C, (uint64_t)B * T, (uint64_t)C,
-                     32, 32, CU_TENSOR_MAP_SWIZZLE_128B))
+                     D / 2, 32, swz))
     return cudaErrorInvalidValue;
-  bwd_prep_kernel<<<B * T / bwd::kPrepRows, 256, 0, s>>>(out, dout, lse, xtiles, dq_acc, T, H, scale);
+  bwd_prep_kernel<D><<<B * T / bwd::kPrepRows, 256, 0, s>>>(out, dout, lse, xtiles, dq_acc, T, H, scale);
   const int n_items = (T / bwd::BKEY) * B * H;
   const int sms = device_sm_count();   // one persistent CTA per SM
   const int grid = n_items < sms ? n_items : sms;
-  attn_bwd_tc_kernel<<<grid, bwd::kThreads, bwd::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, xtiles, dqkv, T, H, B * H, scale,
-                                                                  err);
+  attn_bwd_tc_kernel<D><<<grid, bwd::kThreads, G::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, xtiles, dqkv, T, H, B * H,
+                                                                   scale, err);
   const int n = B * T * (C / 8);
   int blocks = (n + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;

@@ -272,6 +272,13 @@ GPT2_DEV float gelu_f(float u) {
   const float k = 0.7978845608028654f;  // sqrt(2/pi)
   return 0.5f * u * (1.0f + tanh_hw(k * (u + 0.044715f * u * u * u)));
 }
+// GELU(u) and GELU'(u) from one tanh.
+GPT2_DEV void gelu_and_grad_f(float u, float& g, float& d) {
+  const float k = 0.7978845608028654f;
+  const float t = tanh_hw(k * (u + 0.044715f * u * u * u));
+  g = 0.5f * u * (1.0f + t);
+  d = 0.5f * (1.0f + t) + 0.5f * u * (1.0f - t * t) * k * (1.0f + 3.0f * 0.044715f * u * u);
+}
 GPT2_DEV float gelu_grad_f(float u) {
   const float k = 0.7978845608028654f;
   const float t = tanh_hw(k * (u + 0.044715f * u * u * u));

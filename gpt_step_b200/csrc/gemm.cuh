@@ -41,13 +41,15 @@ enum Epi : int {
                     // running (max, sum of 2^) of log2(e) * out over columns < lse_V
   EPI_LSE_ONLY = 6, // pair kernel only: the partials of EPI_LSE and the row's target logit
                     // bf16(acc)[row, lse_tgt[row]] into lse_tgt_val[row]; nothing else stored
+  EPI_GELU_D = 7,   // pair kernel only: x = acc + bias; out = bf16(GELU'(x)); out2 = bf16(GELU(x))
+  EPI_DMUL = 8,     // pair kernel only: out = bf16(acc * aux) (aux: the saved GELU'(x))
 };
 
 struct Params {
   int M, N, K;
   int num_m, num_n, splits, kb_per_split, nkb, num_tiles;
   int raster_gm;  // row tiles per raster panel (pair kernel); num_m = plain row-major order
-  float* colsum;  // pair kernel, EPI_DGELU: column sums of the (bf16) output added here, or null
+  float* colsum;  // pair kernel, EPI_DGELU / EPI_DMUL: column sums of the (bf16) output added here, or null
   float2* lse_part;  // pair kernel, EPI_LSE: [M][lse_slots] (max, sum) partials, slot = 2 * n_tile + half
   int lse_V, lse_slots;
   const int* sched;        // pair kernel: per-pair tile lists ([pairs + 1] offsets, then tile ids), or

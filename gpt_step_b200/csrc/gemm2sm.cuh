@@ -168,7 +168,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
       tma_prefetch_desc(&tmB1);
     }
     if (EPI != gemm::EPI_ACC_F32 && EPI != gemm::EPI_LSE_ONLY) tma_prefetch_desc(&tmO);
-    if (EPI == gemm::EPI_GELU) tma_prefetch_desc(&tmO2);
+    if (EPI == gemm::EPI_GELU || EPI == gemm::EPI_GELU_D) tma_prefetch_desc(&tmO2);
   }
   if (warp == 1) {
     tmem_alloc2(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -320,7 +320,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         // from global memory, while chunk c is processed: the epilogue of a tile
         // then runs at about the pace of the next tile's main loop.
         constexpr bool kBias = EPI == gemm::EPI_STORE || EPI == gemm::EPI_RESID || EPI == gemm::EPI_GELU ||
-                               EPI == gemm::EPI_LSE;
+                               EPI == gemm::EPI_LSE || EPI == gemm::EPI_GELU_D;
+        constexpr bool kTwoOut = EPI == gemm::EPI_GELU || EPI == gemm::EPI_GELU_D;
         constexpr bool kLse = EPI == gemm::EPI_LSE || EPI == gemm::EPI_LSE_ONLY;
         constexpr bool kStore = EPI != gemm::EPI_LSE_ONLY;
         // EPI_LSE_ONLY: the row's target id, if it falls in this half tile (else -1)
@@ -331,7 +332,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
         }
         // EPI_LSE: this row's running max (log2 units) and sum of 2^(y - max) over the half tile
         float lse_m = -INFINITY, lse_s = 0.f;
-        constexpr bool kAux = EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU;
+        constexpr bool kAux = EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU || EPI == gemm::EPI_DMUL;
         const bool has_bias = kBias && p.bias != nullptr;
         const int c_beg = hv * (BN / 2), c_end = (hv + 1) * (BN / 2);
         uint32_t vr[32];
@@ -377,6 +378,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                 const int i = j * 8 + h * 2;
                 if (EPI == gemm::EPI_RESID) {
                   v[i] += f.x; v[i + 1] += f.y;
+                } else if (EPI == gemm::EPI_DMUL) {
+                  v[i] *= f.x; v[i + 1] *= f.y;
                 } else {
                   v[i] *= gelu_grad_f(f.x); v[i + 1] *= gelu_grad_f(f.y);
                 }
@@ -402,8 +405,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             continue;
           }
           uint32_t pk[16];
+          if (EPI == gemm::EPI_GELU_D) {
+            // first output GELU'(x) (what the backward multiplies by), then GELU(x) into v
 #pragma unroll
-          for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            for (int i = 0; i < 16; ++i) {
+              float g0, d0, g1, d1;
+              gelu_and_grad_f(v[2 * i], g0, d0);
+              gelu_and_grad_f(v[2 * i + 1], g1, d1);
+              pk[i] = pack_bf16x2(d0, d1);
+              v[2 * i] = g0;
+              v[2 * i + 1] = g1;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          }
           if (kLse) {
             // over the stored bf16 values f: chunk max by a bf16x2 tree (exact, and
             // max(f) * log2(e) rounds to the max of the scaled values), then the sum
@@ -457,37 +473,58 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             }
           }
           if (!kStore) continue;
-          if (EPI == gemm::EPI_DGELU && p.colsum != nullptr) {
-            // column sums of the stored (bf16) values over this warp's 32 rows: a
-            // transpose-reduce leaves column `lane` of the chunk in cs[0]
-            float cs[32];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float2 f = unpack_bf16x2(pk[i]);
-              cs[2 * i] = row_ok ? f.x : 0.f;
-              cs[2 * i + 1] = row_ok ? f.y : 0.f;
-            }
-            warp_colsum32(cs, lane);
-            atomicAdd(p.colsum + n + lane, cs[0]);
-          }
           // single-output epilogues alternate two buffers; GELU has one per output
-          const uint32_t b = EPI == gemm::EPI_GELU ? 0u : (nstore & 1);
+          const uint32_t b = kTwoOut ? 0u : (nstore & 1);
           if (lane == 0) {
-            if (EPI == gemm::EPI_GELU) gemm::bulk_wait_read<0>();
+            if (kTwoOut) gemm::bulk_wait_read<0>();
             else gemm::bulk_wait_read<1>();
           }
           __syncwarp();
-          gemm::stage_row(wbuf + b * 2048, lane, pk);
-          if (EPI == gemm::EPI_GELU) {
+          if (!row_ok) {   // rows past M: the store leaves them out; the column sums must see 0
 #pragma unroll
-            for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(gelu_f(v[2 * i]), gelu_f(v[2 * i + 1]));
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+          }
+          gemm::stage_row(wbuf + b * 2048, lane, pk);
+          if ((EPI == gemm::EPI_DGELU || EPI == gemm::EPI_DMUL) && p.colsum != nullptr) {
+            // column sums of the stored (bf16) values over this warp's 32 rows, read
+            // back from the staged box (rows of 64 bytes, 16-byte chunks swizzled by
+            // (row >> 1) & 3; rows past M staged as zeros): lane l adds column pair
+            // l & 15 over rows 16 (l >> 4) .. +15, then the two row halves combine
+            __syncwarp();
+            const uint8_t* box = wbuf + b * 2048;
+            const int cp = lane & 15, r0h = (lane >> 4) * 16;
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+              const int r = r0h + rr;
+              const uint32_t w = *reinterpret_cast<const uint32_t*>(
+                  box + r * 64 + (((cp >> 2) ^ ((r >> 1) & 3)) << 4) + (cp & 3) * 4);
+              const float2 f = unpack_bf16x2(w);
+              s0 += f.x;
+              s1 += f.y;
+            }
+            s0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+            s1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+            if (lane < 16) {
+              atomicAdd(p.colsum + n + 2 * cp, s0);
+              atomicAdd(p.colsum + n + 2 * cp + 1, s1);
+            }
+          }
+          if (kTwoOut) {
+            if (EPI == gemm::EPI_GELU_D) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);   // GELU(x), formed above
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(gelu_f(v[2 * i]), gelu_f(v[2 * i + 1]));
+            }
             gemm::stage_row(wbuf + 2048, lane, pk);
           }
           gemm::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
             gemm::tma_store_2d(&tmO, smem_u32(wbuf + b * 2048), n, row0);
-            if (EPI == gemm::EPI_GELU) gemm::tma_store_2d(&tmO2, smem_u32(wbuf + 2048), n, row0);
+            if (kTwoOut) gemm::tma_store_2d(&tmO2, smem_u32(wbuf + 2048), n, row0);
             gemm::bulk_commit();
           }
           ++nstore;
@@ -584,7 +621,7 @@ static int prepare(const gemm::Call& c, int splits_forced, Params& p, CUtensorMa
   p.splits = (p.nkb + p.kb_per_split - 1) / p.kb_per_split;
   p.num_tiles = p.num_m * p.num_n * p.splits;
   p.raster_gm = std::min(p.num_m, c.kind == WGRAD ? kRasterRowsWgrad : kRasterRows);
-  p.colsum = c.epi == EPI_DGELU ? c.colsum : nullptr;
+  p.colsum = (c.epi == EPI_DGELU || c.epi == EPI_DMUL) ? c.colsum : nullptr;
   if (c.epi == EPI_LSE || c.epi == EPI_LSE_ONLY) {
     if (c.kind != FWD || !c.lse_part || c.lse_V <= 0 || c.lse_V > c.N) return GPT2_ERR_ARG;
     p.lse_part = c.lse_part;
@@ -615,7 +652,8 @@ static int prepare(const gemm::Call& c, int splits_forced, Params& p, CUtensorMa
   if (!ok) return GPT2_ERR_ARG;
   if (c.epi != EPI_ACC_F32 && c.epi != EPI_LSE_ONLY) {
     if (!make_map(&to, c.out, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B)) return GPT2_ERR_ARG;
-    if (c.epi == EPI_GELU && !make_map(&to2, c.out2, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    if ((c.epi == EPI_GELU || c.epi == EPI_GELU_D) &&
+        !make_map(&to2, c.out2, c.N, c.M, c.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
       return GPT2_ERR_ARG;
   }
   return GPT2_OK;
@@ -627,6 +665,7 @@ static int run(const gemm::Call& c, cudaStream_t s) {
   if (c.N % 32 || c.K % BK) return GPT2_ERR_ARG;
   const bool pair = uses_pair(c);
   if (!pair && c.colsum) return GPT2_ERR_ARG;   // fused column sums need the pair kernel
+  if (!pair && (c.epi == EPI_GELU_D || c.epi == EPI_DMUL)) return GPT2_ERR_ARG;
   if (!pair) return gemm::run(c, s);   // refuses EPI_LSE
   Params p;
   CUtensorMap ta, tb, to, to2;
@@ -638,6 +677,7 @@ static int run(const gemm::Call& c, cudaStream_t s) {
       case EPI_STORE: e = launch_tc2<256, false, false, EPI_STORE>(ta, tb, to, to2, p, s); break;
       case EPI_RESID: e = launch_tc2<256, false, false, EPI_RESID>(ta, tb, to, to2, p, s); break;
       case EPI_GELU: e = launch_tc2<256, false, false, EPI_GELU>(ta, tb, to, to2, p, s); break;
+      case EPI_GELU_D: e = launch_tc2<256, false, false, EPI_GELU_D>(ta, tb, to, to2, p, s); break;
       case EPI_LSE: e = launch_tc2<256, false, false, EPI_LSE>(ta, tb, to, to2, p, s); break;
       case EPI_LSE_ONLY: e = launch_tc2<256, false, false, EPI_LSE_ONLY>(ta, tb, to, to2, p, s); break;
       default: return GPT2_ERR_ARG;
@@ -646,6 +686,7 @@ static int run(const gemm::Call& c, cudaStream_t s) {
     switch (c.epi) {
       case EPI_STORE: e = launch_tc2<256, false, true, EPI_STORE>(ta, tb, to, to2, p, s); break;
       case EPI_DGELU: e = launch_tc2<256, false, true, EPI_DGELU>(ta, tb, to, to2, p, s); break;
+      case EPI_DMUL: e = launch_tc2<256, false, true, EPI_DMUL>(ta, tb, to, to2, p, s); break;
       default: return GPT2_ERR_ARG;
     }
   } else {
@@ -776,6 +817,7 @@ static int run_group(const gemm::Call& c0, const gemm::Call& c1, cudaStream_t s,
   switch (c0.epi) {
     case EPI_STORE: e = launch_tc2<256, false, true, EPI_STORE, true>(ta0, tb0, to0, to20, p0, s, &ta1, &tb1, &p1); break;
     case EPI_DGELU: e = launch_tc2<256, false, true, EPI_DGELU, true>(ta0, tb0, to0, to20, p0, s, &ta1, &tb1, &p1); break;
+    case EPI_DMUL: e = launch_tc2<256, false, true, EPI_DMUL, true>(ta0, tb0, to0, to20, p0, s, &ta1, &tb1, &p1); break;
     default: return GPT2_ERR_ARG;
   }
   return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;

@@ -427,9 +427,11 @@ int attention_bwd(const bf16* qkv, const bf16* out, const bf16* dout, const floa
                   bf16* dqkv, int B, int T, int H, int hd, int* err, cudaStream_t s) {
   if (T % 64) return GPT2_ERR_ARG;
   cudaError_t e;
-  if (hd == 64 && T % attn_tc::bwd::BKEY == 0 && H <= attn_tc::bwd::kMaxHeads && err != nullptr) {
+  if ((hd == 64 || hd == 32) && T % attn_tc::bwd::BKEY == 0 && H <= attn_tc::bwd::kMaxHeads && err != nullptr) {
     // Dv holds the 16-column per-query operand tiles here (32 bytes per query and head)
-    e = attn_tc::bwd_run(qkv, out, dout, lse, reinterpret_cast<uint8_t*>(Dv), dq_acc, dqkv, B, T, H, err, s);
+    uint8_t* xt = reinterpret_cast<uint8_t*>(Dv);
+    e = hd == 64 ? attn_tc::bwd_run<64>(qkv, out, dout, lse, xt, dq_acc, dqkv, B, T, H, err, s)
+                 : attn_tc::bwd_run<32>(qkv, out, dout, lse, xt, dq_acc, dqkv, B, T, H, err, s);
   } else if (hd == 64) e = attn::bwd<64>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
   else if (hd == 32) e = attn::bwd<32>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
   else return GPT2_ERR_ARG;
@@ -561,9 +563,12 @@ int forward(gpt2_model* m, const int32_t* tok, const int32_t* tgt, int b, bool t
     GPT2_TRY(ln_fwd_m(m, xmid, K_LN2W, K_LN2B, l, ln2, m->at<float>(y.ln2_mean) + l * d.N,
                       m->at<float>(y.ln2_rstd) + l * d.N, (int)N));
     {
+      // on CTA pairs the fc epilogue saves GELU'(x) for the backward instead of x
+      // (one tanh for both outputs; the backward's epilogue is then one multiply)
       gemm::Call c = gemm_call(gemm::FWD, gemm::EPI_GELU, (int)N, 4 * C, C, err);
       c.a = ln2; c.lda = C; c.b = m->W(K_FCW, l); c.ldb = C; c.out = fch; c.out2 = fchg; c.ldo = 4 * C;
       c.bias = m->P(K_FCB, l);
+      if (gemm2::uses_pair(c)) c.epi = gemm::EPI_GELU_D;
       GPT2_TRY(run_gemm(m, c));
     }
     {
@@ -681,6 +686,9 @@ int backward(gpt2_model* m, const int32_t* tok) {
       cd.colsum = m->G(K_FCB, l);
       fused_fcb = gemm2::uses_pair(cd);
       if (!fused_fcb) cd.colsum = nullptr;
+      // the forward's fc epilogue saved GELU'(x) exactly when it ran on CTA pairs
+      // (the same [N, 4C] output shape decides both)
+      if (fused_fcb) cd.epi = gemm::EPI_DMUL;
       GPT2_TRY(run_gemm_group(m, cd, cw, G_MLP_PROJ));
     }
     // MLP fc
@@ -766,6 +774,11 @@ int make_group_plans(gpt2_model* m) {
   const int pairs = gemm::num_sms() / 2;
   for (int gi = 0; gi < kNumGroups; ++gi) {
     m->group_splits[gi] = 0;
+    // The MLP projection's dgrad tiles carry the GELU' epilogue (the saved
+    // pre-activation read, GELU', the fc bias column sums), which outlasts their
+    // 12 k-blocks; the k-block cost model does not see that, and its plan measured
+    // 11% slower than the static stride with the split the stride simulation picks.
+    if (gi == G_MLP_PROJ) continue;
     if (!gemm2::groupable(g[gi].cd, g[gi].cw)) continue;
     const gemm2::GroupPlan plan = gemm2::plan_group(g[gi].cd, g[gi].cw, pairs);
     if (plan.splits1 <= 0 || plan.table.size() > (size_t)kSchedInts) continue;
