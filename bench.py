@@ -75,6 +75,32 @@ def load_peaks():
             "source": "fallback"}
 
 
+def gemm_traffic_per_launch(name):
+    """DRAM bytes (read + written) per GEMM launch, from the committed ncu launch
+    list of one micro-step of this workload (profiles/launches_<name>_microstep.md),
+    or None when there is none or when the kernel sources have changed since it
+    was captured (the summary records their sha256)."""
+    import re
+    path = os.path.join(ROOT, "profiles", f"launches_{name}_microstep.md")
+    if not os.path.exists(path):
+        return None, "no launch list committed for this workload"
+    from gpt_step_b200.profile_step import kernel_sources_sha256
+    text = open(path).read()
+    m = re.search(r"kernel_sources_sha256: ([0-9a-f]{64})", text)
+    if not m or m.group(1) != kernel_sources_sha256():
+        return None, "the kernels changed since the committed launch list was captured"
+    n, b = 0, 0.0
+    for line in text.splitlines():
+        if line.startswith(("| `gemm2::gemm_tc2_kernel", "| `gemm::gemm_tc_kernel")):
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            n += int(cells[1])
+            b += (float(cells[4]) + float(cells[5])) * 1e6
+    if n == 0:
+        return None, "no GEMM launches in the committed launch list"
+    return b / n, (f"ncu dram__bytes_read.sum + dram__bytes_write.sum, mean over the {n} GEMM launches of "
+                   f"one micro-step + optimizer step ({os.path.relpath(path, ROOT)})")
+
+
 def workload_desc(w, n_gpus, parallel="dp", dp_mode="zero1", name=WORKLOAD):
     vp = (w["vocab_real"] + 127) // 128 * 128
     title = {"gpt2_124m": "GPT-2 124M", "gpt2_124m_b64": "GPT-2 124M at micro-batch 64",
@@ -402,10 +428,12 @@ def main():
         g = prof["gemm"]
         ach = g["flops"] / (g["ms"] / 1000.0) / 1e12
         pk = peaks["bf16_tflops_sustained"]
+        traffic, tsrc = gemm_traffic_per_launch(name)
         roof = {"bound": "tensor", "kernel": "gemm_tc2_kernel / gemm_tc_kernel (every tcgen05 GEMM launch)",
                 "achieved": round(ach, 1), "peak": pk, "unit": "TFLOP/s", "frac": round(ach / pk, 4),
                 "peak_kind": f"bf16 dense, sustained, {peaks['source']}",
-                "traffic": None, "launches": g["launches"], "share_of_step": round(g["ms"] / ms, 4),
+                "traffic": None if traffic is None else round(traffic), "traffic_source": tsrc,
+                "launches": g["launches"], "share_of_step": round(g["ms"] / ms, 4),
                 "timing": "CUDA events around each launch in a second pass of K steps"}
 
     if rank == 0:

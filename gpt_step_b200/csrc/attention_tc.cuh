@@ -288,24 +288,30 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int i = 0; i < 32; ++i)
             if (c * 32 + i > r) sr[c][i] = __float_as_uint(-INFINITY);
       }
-      // row maximum with eight independent partial maxima (short dependency chains)
+      // row maximum with eight independent partial maxima (short dependency
+      // chains), two scores per three-input max
       float mpart[8];
 #pragma unroll
       for (int t = 0; t < 8; ++t) mpart[t] = -INFINITY;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mpart[i & 7] = fmaxf(mpart[i & 7], __uint_as_float(sr[c][i]));
-#pragma unroll
-      for (int t = 1; t < 8; ++t) mpart[0] = fmaxf(mpart[0], mpart[t]);
-      const float mx = mpart[0] * sl2;  // scale > 0: max commutes with it
+        for (int i = 0; i < 32; i += 2)
+          mpart[(i >> 1) & 7] =
+              max3f(mpart[(i >> 1) & 7], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+      const float mx = max3f(max3f(mpart[0], mpart[1], mpart[2]), max3f(mpart[3], mpart[4], mpart[5]),
+                             fmaxf(mpart[6], mpart[7])) *
+                       sl2;  // scale > 0: max commutes with it
       // lazy rescale: keep the stale maximum unless the new one exceeds it by > 2^8
       const bool grow = (mx > m + kRescaleThreshold) || (m == -INFINITY);
       const float m_new = grow ? mx : m;
       const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
-      float spart[8];
+      // four paired partial sums; the scale-and-shift and the sums run as paired
+      // fp32 operations (two scores per instruction)
+      float2 spart[4];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) spart[t] = 0.f;
+      for (int t = 0; t < 4; ++t) spart[t] = make_float2(0.f, 0.f);
+      const float2 sl2x2 = make_float2(sl2, sl2), negm2 = make_float2(-m_new, -m_new);
       // P_j as bf16 pairs (keys 2i, 2i+1 of this query row in column P_COL + i),
       // in two halves of 64 keys: the first half's 32 words are stored (once the
       // PV product of block j-1 has read the P buffer) before the second half is
@@ -319,10 +325,11 @@ __global__ void __launch_bounds__(kThreads, 2)
           const int c = 2 * half + cc;
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i]), sl2, -m_new));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][2 * i + 1]), sl2, -m_new));
-            spart[i & 7] += p0 + p1;
-            pk[cc * 16 + i] = pack_bf16x2(p0, p1);
+            const float2 y =
+                f2_fma(make_float2(__uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1])), sl2x2, negm2);
+            const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+            spart[i & 3] = f2_add(spart[i & 3], pp);
+            pk[cc * 16 + i] = pack_bf16x2(pp.x, pp.y);
           }
         }
         if (!waited) {
@@ -334,9 +341,9 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (ok) tmem_st32_u(tmem + lane_off + P_COL + 32 * half, pk);
       }
       if (!ok) break;
-      float sum = 0.f;
-#pragma unroll
-      for (int t = 0; t < 8; ++t) sum += spart[t];
+      const float2 s01 = f2_add(spart[0], spart[1]), s23 = f2_add(spart[2], spart[3]);
+      const float2 s4 = f2_add(s01, s23);
+      const float sum = s4.x + s4.y;
       l = l * alpha + sum;
       m = m_new;
       // O rescale (rows whose maximum moved) once the PV product of block j-1 is done
@@ -507,22 +514,24 @@ GPT2_DEV void regs_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::
 template <bool DIAG>
 GPT2_DEV void bwd_softmax_row(const uint32_t (&sv)[2][32], const uint32_t (&dv)[2][32], float sl2, float scale,
                               int r, int col0, uint32_t (&pp)[32], uint32_t (&pd)[32]) {
+  // two columns per paired fp32 instruction
+  const float2 sl2x2 = make_float2(sl2, sl2), sc2 = make_float2(scale, scale);
 #pragma unroll
   for (int c = 0; c < 2; ++c) {
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      float p[4], ds[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int j = g * 4 + e;   // column within this 32-column chunk
-        p[e] = ex2_approx(__uint_as_float(sv[c][j]) * sl2);          // S' already holds -lse/scale
-        if (DIAG && r > col0 + c * 32 + j) p[e] = 0.f;   // key after query: masked
-        ds[e] = p[e] * (__uint_as_float(dv[c][j]) * scale);          // dP' already holds -D
+    for (int g = 0; g < 16; ++g) {
+      const int j = 2 * g;   // column pair within this 32-column chunk
+      // S' already holds -lse/scale, dP' already holds -D
+      const float2 y = f2_mul(make_float2(__uint_as_float(sv[c][j]), __uint_as_float(sv[c][j + 1])), sl2x2);
+      float2 p = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+      if (DIAG) {   // key after query: masked
+        if (r > col0 + c * 32 + j) p.x = 0.f;
+        if (r > col0 + c * 32 + j + 1) p.y = 0.f;
       }
-      pp[c * 16 + g * 2] = pack_bf16x2(p[0], p[1]);
-      pp[c * 16 + g * 2 + 1] = pack_bf16x2(p[2], p[3]);
-      pd[c * 16 + g * 2] = pack_bf16x2(ds[0], ds[1]);
-      pd[c * 16 + g * 2 + 1] = pack_bf16x2(ds[2], ds[3]);
+      const float2 ds =
+          f2_mul(p, f2_mul(make_float2(__uint_as_float(dv[c][j]), __uint_as_float(dv[c][j + 1])), sc2));
+      pp[c * 16 + g] = pack_bf16x2(p.x, p.y);
+      pd[c * 16 + g] = pack_bf16x2(ds.x, ds.y);
     }
   }
 }

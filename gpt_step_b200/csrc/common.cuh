@@ -189,6 +189,43 @@ GPT2_DEV float ex2_approx(float x) {
   return y;
 }
 
+// Paired fp32 arithmetic: sm_100 executes two independent round-to-nearest
+// fp32 operations as one instruction (.f32x2); each lane of the result is
+// bit-identical to the scalar fmaf / multiply / add.
+GPT2_DEV float2 f2_fma(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+GPT2_DEV float2 f2_mul(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+GPT2_DEV float2 f2_add(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// max(a, b, c) in one instruction (sm_100 three-input max).
+GPT2_DEV float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // Shared-memory matrix descriptor for a tile stored in the canonical
 // 128-byte-swizzled layout (TMA SWIZZLE_128B). Strides are in bytes.
 GPT2_DEV uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
@@ -278,6 +315,24 @@ GPT2_DEV void gelu_and_grad_f(float u, float& g, float& d) {
   const float t = tanh_hw(k * (u + 0.044715f * u * u * u));
   g = 0.5f * u * (1.0f + t);
   d = 0.5f * (1.0f + t) + 0.5f * u * (1.0f - t * t) * k * (1.0f + 3.0f * 0.044715f * u * u);
+}
+// The same for two values in paired fp32 arithmetic, with the polynomial
+// regrouped around s = u^2:
+//   w  = u (k + 0.044715 k s)                 (the tanh argument)
+//   h  = 0.5 + 0.5 tanh(w),  GELU  = u h
+//   GELU' = h + u (0.5 k + 1.5 * 0.044715 k s) (1 - t^2)
+GPT2_DEV void gelu_and_grad_f2(float2 u, float2& g, float2& d) {
+  const float k = 0.7978845608028654f;
+  const float kc = k * 0.044715f;
+  const float2 s = f2_mul(u, u);
+  const float2 w = f2_mul(u, f2_fma(s, make_float2(kc, kc), make_float2(k, k)));
+  const float2 t = make_float2(tanh_hw(w.x), tanh_hw(w.y));
+  const float2 h = f2_fma(t, make_float2(0.5f, 0.5f), make_float2(0.5f, 0.5f));
+  g = f2_mul(u, h);
+  // -(u q) and (t^2 - 1), so that GELU' = h + (-(u q)) (t^2 - 1) is one fused step
+  const float2 nuq = f2_mul(u, f2_fma(s, make_float2(-1.5f * kc, -1.5f * kc), make_float2(-0.5f * k, -0.5f * k)));
+  const float2 t2m1 = f2_fma(t, t, make_float2(-1.f, -1.f));
+  d = f2_fma(nuq, t2m1, h);
 }
 GPT2_DEV float gelu_grad_f(float u) {
   const float k = 0.7978845608028654f;

@@ -44,6 +44,8 @@ enum Epi : int {
   EPI_GELU_D = 7,   // pair kernel only: x = acc + bias; out = bf16(GELU'(x)); out2 = bf16(GELU(x))
   EPI_DMUL = 8,     // pair kernel only: out = bf16(acc * aux) (aux: the saved GELU'(x))
 };
+// Epilogues that store a second output (through tmO2).
+constexpr bool two_outputs(int epi) { return epi == EPI_GELU || epi == EPI_GELU_D; }
 
 struct Params {
   int M, N, K;

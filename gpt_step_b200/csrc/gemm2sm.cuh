@@ -33,12 +33,16 @@ constexpr int BM_PAIR = 256;  // rows per cluster tile (128 per CTA)
 
 constexpr int kThreads2 = 320;  // TMA, MMA, 8 epilogue warps (two per TMEM lane quarter)
 
-template <int BN>
+// TWO_OUT: the epilogue stores two outputs (GELU(x) and its pre-activation or
+// GELU'(x)); it gets two 2 KB store buffers per output and warp, paid for with
+// one operand stage.
+template <int BN, bool TWO_OUT = false>
 struct Cfg {
-  static constexpr int STAGES = 6;
-  // epilogue staging: 4 KB per epilogue warp (two 2 KB store buffers, or one per
-  // output for the two-output GELU epilogue)
-  static constexpr int EPI_BYTES = 8 * 4096;
+  static constexpr int STAGES = TWO_OUT ? 5 : 6;
+  // epilogue staging per epilogue warp: two 2 KB store buffers per output, so
+  // that a chunk is staged while the previous chunk's TMA store still reads
+  static constexpr int WARP_EPI_BYTES = TWO_OUT ? 8192 : 4096;
+  static constexpr int EPI_BYTES = 8 * WARP_EPI_BYTES;
   static constexpr int A_BYTES = 128 * BK * 2;          // own 128 rows
   static constexpr int B_BYTES = (BN / 2) * BK * 2;     // own half of B
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -126,7 +130,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                     const __grid_constant__ Params p, const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ Params p1) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, gemm::two_outputs(EPI)>;
   constexpr int S = C::STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw2[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
@@ -275,7 +279,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;              // TMEM lane quarter
     const int hv = (warp - 2) >> 2;      // column half of the tile this warp drains
-    uint8_t* wbuf = epi_smem + (warp - 2) * 4096;
+    uint8_t* wbuf = epi_smem + (warp - 2) * C::WARP_EPI_BYTES;
     uint32_t nstore = 0;
     int it = 0;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
@@ -362,10 +366,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(vr[i]);
           // consume this chunk's bias / aux registers, then start the next chunk's loads
+          // (paired fp32 operations: two columns per instruction)
           if (n < p.N && has_bias) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              v[4 * i] += bn4[i].x; v[4 * i + 1] += bn4[i].y; v[4 * i + 2] += bn4[i].z; v[4 * i + 3] += bn4[i].w;
+              const float2 lo = f2_add(make_float2(v[4 * i], v[4 * i + 1]), make_float2(bn4[i].x, bn4[i].y));
+              const float2 hi = f2_add(make_float2(v[4 * i + 2], v[4 * i + 3]), make_float2(bn4[i].z, bn4[i].w));
+              v[4 * i] = lo.x; v[4 * i + 1] = lo.y; v[4 * i + 2] = hi.x; v[4 * i + 3] = hi.y;
             }
           }
           if (kAux && n < p.N && row_ok) {
@@ -376,13 +383,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
               for (int h = 0; h < 4; ++h) {
                 const float2 f = unpack_bf16x2(w[h]);
                 const int i = j * 8 + h * 2;
+                float2 r = make_float2(v[i], v[i + 1]);
                 if (EPI == gemm::EPI_RESID) {
-                  v[i] += f.x; v[i + 1] += f.y;
+                  r = f2_add(r, f);
                 } else if (EPI == gemm::EPI_DMUL) {
-                  v[i] *= f.x; v[i + 1] *= f.y;
+                  r = f2_mul(r, f);
                 } else {
-                  v[i] *= gelu_grad_f(f.x); v[i + 1] *= gelu_grad_f(f.y);
+                  r = f2_mul(r, make_float2(gelu_grad_f(f.x), gelu_grad_f(f.y)));
                 }
+                v[i] = r.x; v[i + 1] = r.y;
               }
             }
           }
@@ -409,12 +418,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             // first output GELU'(x) (what the backward multiplies by), then GELU(x) into v
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              float g0, d0, g1, d1;
-              gelu_and_grad_f(v[2 * i], g0, d0);
-              gelu_and_grad_f(v[2 * i + 1], g1, d1);
-              pk[i] = pack_bf16x2(d0, d1);
-              v[2 * i] = g0;
-              v[2 * i + 1] = g1;
+              float2 g, d;
+              gelu_and_grad_f2(make_float2(v[2 * i], v[2 * i + 1]), g, d);
+              pk[i] = pack_bf16x2(d.x, d.y);
+              v[2 * i] = g.x;
+              v[2 * i + 1] = g.y;
             }
           } else {
 #pragma unroll
@@ -473,12 +481,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
             }
           }
           if (!kStore) continue;
-          // single-output epilogues alternate two buffers; GELU has one per output
-          const uint32_t b = kTwoOut ? 0u : (nstore & 1);
-          if (lane == 0) {
-            if (kTwoOut) gemm::bulk_wait_read<0>();
-            else gemm::bulk_wait_read<1>();
-          }
+          // alternate two buffers per output: the stores of the chunk before the
+          // previous one (one commit group per chunk) must have read theirs
+          const uint32_t b = nstore & 1;
+          if (lane == 0) gemm::bulk_wait_read<1>();
           __syncwarp();
           if (!row_ok) {   // rows past M: the store leaves them out; the column sums must see 0
 #pragma unroll
@@ -518,13 +524,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
 #pragma unroll
               for (int i = 0; i < 16; ++i) pk[i] = pack_bf16x2(gelu_f(v[2 * i]), gelu_f(v[2 * i + 1]));
             }
-            gemm::stage_row(wbuf + 2048, lane, pk);
+            gemm::stage_row(wbuf + 4096 + b * 2048, lane, pk);
           }
           gemm::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
             gemm::tma_store_2d(&tmO, smem_u32(wbuf + b * 2048), n, row0);
-            if (kTwoOut) gemm::tma_store_2d(&tmO2, smem_u32(wbuf + 2048), n, row0);
+            if (kTwoOut) gemm::tma_store_2d(&tmO2, smem_u32(wbuf + 4096 + b * 2048), n, row0);
             gemm::bulk_commit();
           }
           ++nstore;
@@ -552,7 +558,7 @@ static cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& tb, cons
                               const CUtensorMap& to2, const Params& p, cudaStream_t s,
                               const CUtensorMap* ta1 = nullptr, const CUtensorMap* tb1 = nullptr,
                               const Params* p1 = nullptr) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, gemm::two_outputs(EPI)>;
   auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EPI, GROUP>;
   static PerDeviceOnce once;  // per template instance
   const cudaError_t e = smem_optin(once, kern, C::SMEM);

@@ -26,6 +26,14 @@
       Times a bandwidth-bound kernel alone and prints GB/s of algorithmic bytes
       (for ce, C is the padded vocabulary and the real one is C - 47; for the
       embeddings, rows is B * 1024 tokens over a 50,257-id vocabulary).
+
+  python -m gpt_step_b200.profile_step launches --csv LIST.csv
+      Summarises an ncu launch list (the --csv log of a capture with the metrics
+      gpu__time_duration.sum, dram__bytes_read.sum and dram__bytes_write.sum) as
+      a markdown table per kernel: launches, total time, share, DRAM MB read and
+      written. It also prints the hash of the kernel sources as they are now
+      (`kernel_sources_sha256`), so that a summary records which kernels it
+      describes; needs no GPU.
 """
 from __future__ import annotations
 
@@ -65,6 +73,61 @@ def run_step(args):
     prof = m.profile_read()
     print(json.dumps({"workload": args.workload, "micro_batch": B,
                       "launches_in_range": m.kernel_launches() - n0, "classes": prof}))
+
+
+def kernel_sources_sha256() -> str:
+    """sha256 over the CUDA sources of the library (file names and bytes, sorted)."""
+    import hashlib
+    import os
+    d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(f.read())
+    return h.hexdigest()
+
+
+def launch_table(csv_path):
+    """Per-kernel (launches, microseconds, DRAM MB read, DRAM MB written) of an ncu launch list."""
+    import collections
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    hi = next(i for i, r in enumerate(rows) if r and r[0] == "ID")
+    hdr, data = rows[hi], rows[hi + 1:]
+    ki, mi, vi, ui, ii = (hdr.index(k) for k in ("Kernel Name", "Metric Name", "Metric Value", "Metric Unit", "ID"))
+    scale_t = {"ns": 1e-3, "nsecond": 1e-3, "us": 1.0, "usecond": 1.0, "ms": 1e3, "msecond": 1e3}
+    scale_b = {"byte": 1e-6, "Kbyte": 1e-3, "Mbyte": 1.0, "Gbyte": 1e3}
+    per = collections.OrderedDict()
+    for r in data:
+        if len(r) > vi:
+            per.setdefault((int(r[ii]), r[ki]), {})[r[mi]] = (float(r[vi].replace(",", "")), r[ui])
+    agg = collections.OrderedDict()
+    for (_, k), m in sorted(per.items()):
+        name = k.split("(")[0].replace("void ", "")
+        a = agg.setdefault(name, [0, 0.0, 0.0, 0.0])
+        t, u = m["gpu__time_duration.sum"]
+        a[0] += 1
+        a[1] += t * scale_t[u]
+        if "dram__bytes_read.sum" in m:
+            v, u = m["dram__bytes_read.sum"]
+            a[2] += v * scale_b[u]
+            v, u = m["dram__bytes_write.sum"]
+            a[3] += v * scale_b[u]
+    return agg
+
+
+def run_launches(args):
+    agg = launch_table(args.csv)
+    tot = sum(v[1] for v in agg.values())
+    print(f"kernel_sources_sha256: {kernel_sources_sha256()}\n")
+    print("| kernel | launches | total us | share | DRAM read MB | DRAM write MB |")
+    print("|---|---:|---:|---:|---:|---:|")
+    for n, v in sorted(agg.items(), key=lambda kv: -kv[1][1]):
+        print(f"| `{n}` | {v[0]} | {v[1]:.0f} | {100 * v[1] / tot:.1f}% | {v[2]:.1f} | {v[3]:.1f} |")
+    print(f"| total | {sum(v[0] for v in agg.values())} | {tot:.0f} | | "
+          f"{sum(v[2] for v in agg.values()):.0f} | {sum(v[3] for v in agg.values()):.0f} |")
 
 
 def run_gemm(args):
@@ -279,8 +342,11 @@ def main():
                    default="ln_fwd")
     w.add_argument("--shape", default="19456,768")
     w.add_argument("--iters", type=int, default=20)
+    ls = sub.add_parser("launches")
+    ls.add_argument("--csv", required=True)
     args = ap.parse_args()
-    {"step": run_step, "gemm": run_gemm, "attn": run_attn, "bw": run_bw, "head": run_head}[args.mode](args)
+    {"step": run_step, "gemm": run_gemm, "attn": run_attn, "bw": run_bw, "head": run_head,
+     "launches": run_launches}[args.mode](args)
 
 
 if __name__ == "__main__":
