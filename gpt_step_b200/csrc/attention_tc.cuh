@@ -170,6 +170,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_begin();   // set-up above overlaps the previous kernel's drain
 
   if (warp == 0) {
     // -------------------------------------------------------------- TMA producer
@@ -410,7 +411,7 @@ static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int
                      D, 128, D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   dim3 grid(T / BQ, B * H);
-  attn_fwd_tc_kernel<D><<<grid, kThreads, G::SMEM_BYTES, s>>>(tm, out, lse, T, H, 1.0f / sqrtf((float)D), err);
+  launch_pdl(attn_fwd_tc_kernel<D>, dim3(grid), dim3(kThreads), G::SMEM_BYTES, s, tm, out, lse, T, H, 1.0f / sqrtf((float)D), err);
   return cudaGetLastError();
 }
 
@@ -542,6 +543,7 @@ template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
                                                        const float* __restrict__ lse, uint8_t* __restrict__ xtiles,
                                                        float* __restrict__ dq_acc, int T, int H, float scale) {
+  pdl_begin();
   using namespace bwd;
   constexpr int CPH = D / 8;                 // 16-byte chunks per head
   __shared__ float sDot[kMaxHeads][kPrepRows];
@@ -594,6 +596,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ 
 // dq_acc fp32 [rows, C] -> dqkv[:, 0:C] bf16 (row stride 3C); eight columns per thread.
 __global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ dq_acc, bf16* __restrict__ dqkv,
                                                        int rows, int C) {
+  pdl_begin();
   const int per_row = C / 8;
   const int n = rows * per_row;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
@@ -689,6 +692,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_begin();   // set-up above overlaps the previous kernel's drain
 
   if (warp < 4) {
     regs_dec<kCtlRegs>();
@@ -962,16 +966,16 @@ static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, c
       !encode_map_2d(&tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, (uint64_t)C, (uint64_t)B * T, (uint64_t)C,
                      D / 2, 32, swz))
     return cudaErrorInvalidValue;
-  bwd_prep_kernel<D><<<B * T / bwd::kPrepRows, 256, 0, s>>>(out, dout, lse, xtiles, dq_acc, T, H, scale);
+  launch_pdl(bwd_prep_kernel<D>, dim3(B * T / bwd::kPrepRows), dim3(256), 0, s, out, dout, lse, xtiles, dq_acc, T, H, scale);
   const int n_items = (T / bwd::BKEY) * B * H;
   const int sms = device_sm_count();   // one persistent CTA per SM
   const int grid = n_items < sms ? n_items : sms;
-  attn_bwd_tc_kernel<D><<<grid, bwd::kThreads, G::SMEM_BYTES, s>>>(tm_qkv, tm_do, tm_dq, xtiles, dqkv, T, H, B * H,
+  launch_pdl(attn_bwd_tc_kernel<D>, dim3(grid), dim3(bwd::kThreads), G::SMEM_BYTES, s, tm_qkv, tm_do, tm_dq, xtiles, dqkv, T, H, B * H,
                                                                    scale, err);
   const int n = B * T * (C / 8);
   int blocks = (n + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;
-  bwd_post_kernel<<<blocks, 256, 0, s>>>(dq_acc, dqkv, B * T, C);
+  launch_pdl(bwd_post_kernel, dim3(blocks), dim3(256), 0, s, dq_acc, dqkv, B * T, C);
   return cudaGetLastError();
 }
 

@@ -12,6 +12,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <utility>
 
 #include "../../include/gpt2step.h"
 
@@ -100,6 +101,43 @@ GPT2_DEV bool mbar_wait(uint32_t bar, uint32_t parity, int* err) {
 // ---------------------------------------------------------------------------
 // TMA (no cluster multicast anywhere in this library)
 // ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
+// programmatic dependent launch
+// ---------------------------------------------------------------------------
+// A kernel launched by launch_pdl may be scheduled while the kernel before it
+// in the stream is still draining. It calls griddep_wait() before its first
+// access to global memory that earlier work writes or reads (the wait returns
+// once the previous grid has completed and its writes are visible), and
+// griddep_trigger() to let the next kernel launch ahead of its own end. In a
+// kernel launched without the attribute both are no-ops.
+GPT2_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+GPT2_DEV void griddep_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Both, at the start of a kernel (after any set-up that touches no global memory).
+GPT2_DEV void pdl_begin() {
+  griddep_wait();
+  griddep_trigger();
+}
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// Bring the 128-byte line holding `ptr` (a valid global address) into L2.
+GPT2_DEV void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(reinterpret_cast<uint64_t>(ptr)));
+}
 GPT2_DEV void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }

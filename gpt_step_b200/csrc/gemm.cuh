@@ -159,6 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_begin();   // set-up above overlaps the previous kernel's drain
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -360,7 +361,7 @@ static cudaError_t launch_tc(const CUtensorMap& ta, const CUtensorMap& tb, const
   const cudaError_t e = smem_optin(once, kern, C::SMEM);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
-  kern<<<grid, kThreads, C::SMEM, s>>>(ta, tb, to, to2, p);
+  launch_pdl(kern, dim3(grid), dim3(kThreads), C::SMEM, s, ta, tb, to, to2, p);
   return cudaGetLastError();
 }
 

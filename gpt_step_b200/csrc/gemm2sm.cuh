@@ -182,6 +182,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
   cluster_sync();  // both CTAs' barriers exist before anyone signals them
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // set-up above overlaps the previous kernel's drain; operands and outputs only after it
+  pdl_begin();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -284,12 +286,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
     int it = 0;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
+    // The residual / GELU' operand of a tile (this lane's row, this warp's half
+    // of the columns) is prefetched into L2 one tile ahead, while the tensor
+    // cores still work on the tile before it: the epilogue's operand loads then
+    // wait on L2, not DRAM (with a DRAM wait per 32-column chunk the epilogue
+    // outlasted the main loop of the 768 x 768 projection).
+    constexpr bool kAuxPf = EPI == gemm::EPI_RESID || EPI == gemm::EPI_DGELU || EPI == gemm::EPI_DMUL;
+    auto prefetch_aux = [&](int kk) {
+      if (kk >= k_end) return;
+      const int tn = sch ? sch_tiles[kk] : kk;
+      if (GROUP && tn >= p.num_tiles) return;   // weight-gradient tiles read no operand here
+      int mb, nb, sp;
+      tile_coords(p, tn, mb, nb, sp);
+      (void)sp;
+      const int row = mb * BM_PAIR + 128 * rank + q * 32 + lane;
+      const int n0 = nb * BN + hv * (BN / 2);
+      if (row >= p.M || n0 >= p.N) return;
+      const bf16* a = p.aux + (size_t)row * p.ld_aux + n0;
+      const int ncols = min(BN / 2, p.N - n0);
+      for (int c = 0; c < ncols; c += 64) prefetch_l2(a + c);    // 128-byte lines
+      prefetch_l2(a + ncols - 1);
+    };
+    if (kAuxPf && p.aux != nullptr) prefetch_aux(k_beg);
     for (int k = k_beg; k < k_end; k += k_step, ++it) {
       const int t = sch ? sch_tiles[k] : k;
       const bool second = GROUP && t >= p.num_tiles;
       int mb, nb, sp;
       tile_coords(second ? p1 : p, second ? t - p.num_tiles : t, mb, nb, sp);
       (void)sp;
+      if (kAuxPf && p.aux != nullptr) prefetch_aux(k + k_step);
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, p.err)) break;
@@ -569,8 +594,8 @@ static cudaError_t launch_tc2(const CUtensorMap& ta, const CUtensorMap& tb, cons
   const int pairs = gemm::num_sms() / 2;
   // a planned schedule has one tile list per pair, some possibly empty
   const int grid = 2 * ((p.sched != nullptr || total >= pairs) ? pairs : total);
-  kern<<<grid, kThreads2, C::SMEM, s>>>(ta, tb, to, to2, p, GROUP ? *ta1 : ta, GROUP ? *tb1 : tb, q1);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads2), C::SMEM, s, ta, tb, to, to2, p, GROUP ? *ta1 : ta,
+                    GROUP ? *tb1 : tb, q1);
 }
 
 }  // namespace gemm2

@@ -294,7 +294,7 @@ void ln_fwd_c(const bf16* x, const float* w, const float* b, bf16* y, float* mea
   static int cache[PerDeviceOnce::kMaxDevices] = {};
   const int full = resident_ctas(once, cache, k::layernorm_fwd_kernel<C>, k::kLnFwdWarps * 32);
   const int need = (rows + k::kLnFwdWarps - 1) / k::kLnFwdWarps;
-  k::layernorm_fwd_kernel<C><<<std::min(need, full), k::kLnFwdWarps * 32, 0, s>>>(x, w, b, y, mean, rstd, rows);
+  launch_pdl(k::layernorm_fwd_kernel<C>, dim3(std::min(need, full)), dim3(k::kLnFwdWarps * 32), 0, s, x, w, b, y, mean, rstd, rows);
 }
 
 int ln_fwd(const bf16* x, const float* w, const float* b, bf16* y, float* mean, float* rstd, int rows, int C,
@@ -331,7 +331,7 @@ cudaError_t ln_bwd_c(const bf16* dy, const bf16* x, const float* mean, const flo
   static PerDeviceOnce once;
   const cudaError_t e = smem_optin(once, k::layernorm_bwd_kernel<C>, Cfg::SMEM);
   if (e != cudaSuccess) return e;
-  k::layernorm_bwd_kernel<C><<<blocks, Cfg::WARPS * 32, Cfg::SMEM, s>>>(dy, x, mean, rstd, w, dresid, dx, part, rows,
+  launch_pdl(k::layernorm_bwd_kernel<C>, dim3(blocks), dim3(Cfg::WARPS * 32), Cfg::SMEM, s, dy, x, mean, rstd, w, dresid, dx, part, rows,
                                                                         with_dxsum, dw, db, dbias);
   return cudaGetLastError();
 }
@@ -361,7 +361,7 @@ int ln_bwd(const bf16* dy, const bf16* x, const float* mean, const float* rstd, 
     default: return GPT2_ERR_ARG;
   }
   if (e != cudaSuccess) return GPT2_ERR_CUDA;
-  if (part) k::partial_rows_reduce_kernel<<<(nq * C + 31) / 32, 256, 0, s>>>(part, blocks, nq * C, dw, db, dbias, C);
+  if (part) launch_pdl(k::partial_rows_reduce_kernel, dim3((nq * C + 31) / 32), dim3(256), 0, s, part, blocks, nq * C, dw, db, dbias, C);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -390,8 +390,8 @@ int bias_grad(const bf16* dout, float* db, int M, int N, float* part, size_t par
   if (part && part_bytes < (size_t)strips * N * 4) return GPT2_ERR_ARG;
   if (!part && (reinterpret_cast<uintptr_t>(db) & 15)) return GPT2_ERR_ARG;
   dim3 grid((N / 8 + 31) / 32, strips);
-  k::colsum_partial_kernel<<<grid, 256, 0, s>>>(dout, part, M, N, rps, db);
-  if (part) k::colsum_final_kernel<<<(N + 255) / 256, 256, 0, s>>>(part, db, strips, N);
+  launch_pdl(k::colsum_partial_kernel, dim3(grid), dim3(256), 0, s, dout, part, M, N, rps, db);
+  if (part) launch_pdl(k::colsum_final_kernel, dim3((N + 255) / 256), dim3(256), 0, s, part, db, strips, N);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -405,7 +405,7 @@ int softmax_ce(bf16* logits, const int32_t* targets, float* losses, int N, int V
   if (part && slots <= 0) return GPT2_ERR_ARG;
   if (tgt_val && (!part || write_grad)) return GPT2_ERR_ARG;   // logits-free: a loss from the partials only
   if (!logits && !tgt_val) return GPT2_ERR_ARG;
-  k::softmax_ce_kernel<<<N, k::kCeThreads, 0, s>>>(logits, targets, losses, V, Vp, dscale, write_grad, err,
+  launch_pdl(k::softmax_ce_kernel, dim3(N), dim3(k::kCeThreads), 0, s, logits, targets, losses, V, Vp, dscale, write_grad, err,
                                                     ignore_index, part, slots, tgt_val);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
@@ -527,7 +527,7 @@ int forward(gpt2_model* m, const int32_t* tok, const int32_t* tgt, int b, bool t
 
   {
     const size_t p = prof_begin(m);
-    k::embed_fwd_kernel<<<launch::grid_for(N * C / 8, 256), 256, 0, s>>>(tok, m->W(K_WTE), m->W(K_WPE), resid,
+    launch_pdl(k::embed_fwd_kernel, dim3(launch::grid_for(N * C / 8, 256)), dim3(256), 0, s, tok, m->W(K_WTE), m->W(K_WPE), resid,
                                                                           (int)N, T, C, d.V, err);
     prof_end(m, p, PC_EMBED, (double)N * (6.0 * C + 4), 1);
   }
@@ -606,7 +606,7 @@ int forward(gpt2_model* m, const int32_t* tok, const int32_t* tgt, int b, bool t
     GPT2_TRY(launch::softmax_ce(logits_free ? nullptr : logits, tgt, losses, (int)N, d.V, d.Vp, 1.0f / (float)N,
                                 train ? 1 : 0, err, s, INT_MIN, lse_part, lse_slots(d.Vp),
                                 logits_free ? losses : nullptr));
-    k::loss_reduce_kernel<<<1, 1024, 0, s>>>(losses, (int)N, loss_acc, &m->sc()->micro_loss);
+    launch_pdl(k::loss_reduce_kernel, dim3(1), dim3(1024), 0, s, losses, (int)N, loss_acc, &m->sc()->micro_loss);
     // algorithmic bytes: the logits read (and overwritten when training), or with
     // the GEMM's partials those plus the partials, and no row scan for a loss alone
     const double part_bytes = lse_part ? (double)N * lse_slots(d.Vp) * 8.0 : 0.0;
@@ -735,8 +735,8 @@ int backward(gpt2_model* m, const int32_t* tok) {
   // embeddings
   {
     const size_t p = prof_begin(m);
-    k::embed_bwd_wpe_kernel<<<(T * C / 8 + 255) / 256, 256, 0, s>>>(dresid, m->G(K_WPE), d.B, T, C);
-    k::embed_bwd_wte_kernel<<<(N + k::kEmbRows - 1) / k::kEmbRows, 256, 0, s>>>(tok, dresid, m->G(K_WTE), N, C,
+    launch_pdl(k::embed_bwd_wpe_kernel, dim3((T * C / 8 + 255) / 256), dim3(256), 0, s, dresid, m->G(K_WPE), d.B, T, C);
+    launch_pdl(k::embed_bwd_wte_kernel, dim3((N + k::kEmbRows - 1) / k::kEmbRows), dim3(256), 0, s, tok, dresid, m->G(K_WTE), N, C,
                                                                                 d.V);
     prof_end(m, p, PC_EMBED, (double)N * (2.0 * C + 4) + 2.0 * N * C * 4 + 8.0 * T * C, 2);
   }
@@ -957,14 +957,14 @@ static int clip_adamw_impl(gpt2_model* m, int32_t step, const k::Ranges4& rg, co
   cudaStream_t s = m->stream;
   const Layout& y = m->lay;
   const size_t pr = prof_begin(m);
-  k::norm_finalize_kernel<<<1, 256, 0, s>>>(sumsq, nparts, m->sc(), m->n_micro, y.d.N, m->cfg.grad_clip, m->err());
+  launch_pdl(k::norm_finalize_kernel, dim3(1), dim3(256), 0, s, sumsq, nparts, m->sc(), m->n_micro, y.d.N, m->cfg.grad_clip, m->err());
   const double lr = lr_at(m->cfg, step);
   const double t = (double)step + 1.0;
   const float bc1 = (float)(1.0 - pow((double)m->cfg.beta1, t));
   const float bc2 = (float)(1.0 - pow((double)m->cfg.beta2, t));
   long n4 = 0;
   for (int r = 0; r < rg.n; ++r) n4 += rg.end[r] - rg.begin[r];
-  k::adamw_kernel<<<launch::grid_for(n4, 256), 256, 0, s>>>(m->params(), m->grads(), m->at<float>(y.adam_m),
+  launch_pdl(k::adamw_kernel, dim3(launch::grid_for(n4, 256)), dim3(256), 0, s, m->params(), m->grads(), m->at<float>(y.adam_m),
                                                              m->at<float>(y.adam_v), m->pbf(), rg, y.P1 / 4,
                                                              m->sc(), (float)lr, m->cfg.beta1, m->cfg.beta2,
                                                              m->cfg.eps, m->cfg.weight_decay, bc1, bc2);
@@ -996,7 +996,7 @@ int gpt2_clip_adamw(gpt2_model* m, int32_t step, float* grad_norm_out) {
   all.end[0] = y.P / 4;
   double* part = m->at<double>(y.norm_part);
   const size_t pr = prof_begin(m);
-  k::sumsq_partial_kernel<<<kNormBlocks, 512, 0, m->stream>>>(m->grads(), all, part);
+  launch_pdl(k::sumsq_partial_kernel, dim3(kNormBlocks), dim3(512), 0, m->stream, m->grads(), all, part);
   prof_end(m, pr, PC_OPT, 4.0 * (double)y.P, 1);
   return clip_adamw_impl(m, step, all, part, kNormBlocks, false, grad_norm_out);
 }
@@ -1040,8 +1040,8 @@ int gpt2_grad_sumsq(gpt2_model* m, const int64_t* ranges, int n_ranges, double* 
   long n4 = 0;
   for (int r = 0; r < rg.n; ++r) n4 += rg.end[r] - rg.begin[r];
   const size_t pr = prof_begin(m);
-  k::sumsq_partial_kernel<<<kNormBlocks, 512, 0, m->stream>>>(m->grads(), rg, part);
-  k::sum_partials_kernel<<<1, 256, 0, m->stream>>>(part, kNormBlocks, dev_out);
+  launch_pdl(k::sumsq_partial_kernel, dim3(kNormBlocks), dim3(512), 0, m->stream, m->grads(), rg, part);
+  launch_pdl(k::sum_partials_kernel, dim3(1), dim3(256), 0, m->stream, part, kNormBlocks, dev_out);
   prof_end(m, pr, PC_OPT, 16.0 * (double)n4, 2);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
@@ -1202,7 +1202,7 @@ int gpt2_write(gpt2_model* m, int what, int idx, const float* host_src) {
   if (cudaStreamSynchronize(m->stream) != cudaSuccess) return GPT2_ERR_CUDA;
   if (cudaMemcpy(base + t.off, host_src, (size_t)t.n * 4, cudaMemcpyHostToDevice) != cudaSuccess) return GPT2_ERR_CUDA;
   if (what == GPT2_PARAMS) {
-    k::to_bf16_kernel<<<launch::grid_for(t.n, 256), 256, 0, m->stream>>>(base + t.off, m->pbf() + t.off, t.n);
+    launch_pdl(k::to_bf16_kernel, dim3(launch::grid_for(t.n, 256)), dim3(256), 0, m->stream, base + t.off, m->pbf() + t.off, t.n);
     if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(m->stream) != cudaSuccess) return GPT2_ERR_CUDA;
   }
   return GPT2_OK;
@@ -1440,7 +1440,7 @@ int gpt2op_embedding_fwd(const int32_t* tokens, const void* wte, const void* wpe
                          int* dev_err, void* stream) {
   if (!tokens || !wte || !wpe || !out || !dev_err || C % 8) return GPT2_ERR_ARG;
   const long N = (long)B * T;
-  k::embed_fwd_kernel<<<launch::grid_for(N * C / 8, 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+  launch_pdl(k::embed_fwd_kernel, dim3(launch::grid_for(N * C / 8, 256)), dim3(256), 0, static_cast<cudaStream_t>(stream), 
       tokens, static_cast<const bf16*>(wte), static_cast<const bf16*>(wpe), static_cast<bf16*>(out), (int)N, T, C, V,
       dev_err);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
@@ -1451,8 +1451,8 @@ int gpt2op_embedding_bwd(const int32_t* tokens, const void* dx, float* dwte, flo
   if (!tokens || !dx || !dwte || !dwpe || C % 8) return GPT2_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long N = (long)B * T;
-  k::embed_bwd_wpe_kernel<<<(T * C / 8 + 255) / 256, 256, 0, s>>>(static_cast<const bf16*>(dx), dwpe, B, T, C);
-  k::embed_bwd_wte_kernel<<<(int)((N + k::kEmbRows - 1) / k::kEmbRows), 256, 0, s>>>(
+  launch_pdl(k::embed_bwd_wpe_kernel, dim3((T * C / 8 + 255) / 256), dim3(256), 0, s, static_cast<const bf16*>(dx), dwpe, B, T, C);
+  launch_pdl(k::embed_bwd_wte_kernel, dim3((int)((N + k::kEmbRows - 1) / k::kEmbRows)), dim3(256), 0, s, 
       tokens, static_cast<const bf16*>(dx), dwte, (int)N, C, V);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }

@@ -76,6 +76,7 @@ __global__ void init_kind_kernel(float* __restrict__ p, bf16* __restrict__ pb, l
 __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const bf16* __restrict__ wte,
                                  const bf16* __restrict__ wpe, bf16* __restrict__ x, int N, int T, int C, int V,
                                  int* err) {
+  pdl_begin();
   const int vpr = C / 8;
   const long total = (long)N * vpr;
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < total; i += (long)gridDim.x * blockDim.x) {
@@ -100,6 +101,7 @@ __global__ void embed_fwd_kernel(const int32_t* __restrict__ tok, const bf16* __
 
 // a1 backward, position part: dwpe[t, :] += sum_b dx[b, t, :]   (deterministic)
 __global__ void embed_bwd_wpe_kernel(const bf16* __restrict__ dx, float* __restrict__ dwpe, int B, int T, int C) {
+  pdl_begin();
   const int vpr = C / 8;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= T * vpr) return;
@@ -132,6 +134,7 @@ constexpr int kEmbRows = 64;
 __global__ void __launch_bounds__(256) embed_bwd_wte_kernel(const int32_t* __restrict__ tok,
                                                             const bf16* __restrict__ dx, float* __restrict__ dwte,
                                                             int N, int C, int V) {
+  pdl_begin();
   __shared__ int st[kEmbRows];
   __shared__ unsigned char lead[kEmbRows];
   const int r0 = blockIdx.x * kEmbRows;
@@ -191,6 +194,7 @@ __global__ void __launch_bounds__(kLnFwdWarps * 32, ln_fwd_minb(C)) layernorm_fw
                                                                         const float* __restrict__ b,
                                                                         bf16* __restrict__ y, float* __restrict__ mean,
                                                                         float* __restrict__ rstd, int rows) {
+  pdl_begin();
   constexpr int NV = C / 8;                 // 16-byte vectors per row
   constexpr int VPL = (NV + 31) / 32;       // vectors per lane
   const int l = lane_id();
@@ -292,6 +296,7 @@ __global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, LnBwdCfg<C>::MINB)
     layernorm_bwd_kernel(const bf16* __restrict__ dy, const bf16* __restrict__ x, const float* __restrict__ mean,
                          const float* __restrict__ rstd, const float* __restrict__ w, const bf16* dresid, bf16* dx,
                          float* __restrict__ part, int rows, int with_dxsum, float* dw, float* db, float* dbias) {
+  pdl_begin();
   constexpr int NV = C / 8;
   constexpr int VPL = (NV + 31) / 32;
   constexpr int WARPS = LnBwdCfg<C>::WARPS;
@@ -449,6 +454,7 @@ __global__ void __launch_bounds__(LnBwdCfg<C>::WARPS * 32, LnBwdCfg<C>::MINB)
 // grad, when nq == 3). Block (32 x 8): 32 columns, 8 row-lanes, then a fold.
 __global__ void __launch_bounds__(256) partial_rows_reduce_kernel(const float* __restrict__ part, int nblk, int width,
                                                                  float* out0, float* out1, float* out2, int C) {
+  pdl_begin();
   __shared__ float red[8][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int col = blockIdx.x * 32 + tx;
@@ -474,6 +480,7 @@ __global__ void __launch_bounds__(256) partial_rows_reduce_kernel(const float* _
 // no second pass).
 __global__ void __launch_bounds__(256) colsum_partial_kernel(const bf16* __restrict__ a, float* __restrict__ part,
                                                              int M, int N, int rows_per_strip, float* db) {
+  pdl_begin();
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
   const int c = (blockIdx.x * 32 + tx) * 8;
   const int r0 = blockIdx.y * rows_per_strip;
@@ -532,6 +539,7 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const bf16* __restr
 }
 
 __global__ void colsum_final_kernel(const float* __restrict__ part, float* __restrict__ db, int strips, int N) {
+  pdl_begin();
   const int c = blockIdx.x * blockDim.x + threadIdx.x;
   if (c >= N) return;
   float s = 0.f;
@@ -608,6 +616,7 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
                                                                 float dscale, int write_grad, int* err,
                                                                 int ignore_index, const float2* __restrict__ part,
                                                                 int slots, const float* tgt_val) {
+  pdl_begin();
   __shared__ float red_m[kCeThreads / 32], red_s[kCeThreads / 32];
   __shared__ float bc[2];
   const int row = blockIdx.x;
@@ -706,6 +715,7 @@ __global__ void __launch_bounds__(kCeThreads) softmax_ce_kernel(bf16* __restrict
 // mean in *mean_out.
 __global__ void loss_reduce_kernel(const float* __restrict__ losses, int n, double* __restrict__ acc,
                                    float* __restrict__ mean_out) {
+  pdl_begin();
   __shared__ double red[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < n; i += blockDim.x) s += (double)losses[i];
@@ -736,6 +746,7 @@ struct Ranges4 {
 // Partial sums of squares of g over the ranges, one per block.
 __global__ void __launch_bounds__(512) sumsq_partial_kernel(const float* __restrict__ g, const Ranges4 rg,
                                                             double* __restrict__ part) {
+  pdl_begin();
   __shared__ double red[16];
   double s = 0.0;
   const float4* g4 = reinterpret_cast<const float4*>(g);
@@ -782,6 +793,7 @@ struct StepScalars {
 // Pass 2: combine partials; derive the clip multiplier; flag non-finite steps.
 __global__ void norm_finalize_kernel(const double* __restrict__ part, int nparts, StepScalars* sc, int n_micro,
                                      long rows_per_micro, float clip, int* err) {
+  pdl_begin();
   __shared__ double red[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) s += part[i];
@@ -807,6 +819,7 @@ __global__ void norm_finalize_kernel(const double* __restrict__ part, int nparts
 
 // Sum of the partials into one double (the caller's device value).
 __global__ void sum_partials_kernel(const double* __restrict__ part, int nparts, double* __restrict__ out) {
+  pdl_begin();
   __shared__ double red[32];
   double s = 0.0;
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) s += part[i];
@@ -832,6 +845,7 @@ __global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, float
                                                     bf16* __restrict__ pb, const Ranges4 rg, long decay_from4,
                                                     const StepScalars* __restrict__ sc, float lr, float beta1,
                                                     float beta2, float eps, float wd, float bc1, float bc2) {
+  pdl_begin();
   const float gs = sc->gscale;
   const int skip = sc->skip;
   for (int r = 0; r < rg.n; ++r)
@@ -874,6 +888,7 @@ __global__ void __launch_bounds__(256) adamw_kernel(float* __restrict__ p, float
 
 // fp32 -> bf16 copy (used after host writes of parameters).
 __global__ void to_bf16_kernel(const float* __restrict__ src, bf16* __restrict__ dst, long n) {
+  pdl_begin();
   for (long i = blockIdx.x * (long)blockDim.x + threadIdx.x; i < n; i += (long)gridDim.x * blockDim.x)
     dst[i] = __float2bfloat16_rn(src[i]);
 }
