@@ -375,10 +375,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
 #pragma unroll
               for (int i = 0; i < 8; ++i) bn4[i] = __ldg(reinterpret_cast<const float4*>(p.bias + n) + i);
             }
-            if (kAux && row_ok) {
-              const uint4* src = reinterpret_cast<const uint4*>(p.aux + (size_t)row * p.ld_aux + n);
+            if (kAux) {
+              // coalesced: lane l loads 16-byte chunk l & 3 of the warp's rows
+              // (l >> 2) + 8 i, eight 64-byte row segments per instruction; the
+              // staging box turns them into one row per lane when consumed
+              const int j = lane & 3;
 #pragma unroll
-              for (int j = 0; j < 4; ++j) an4[j] = __ldcs(src + j);
+              for (int i = 0; i < 4; ++i) {
+                const int rr = row0 + (lane >> 2) + 8 * i;
+                an4[i] = rr < p.M ? __ldcs(reinterpret_cast<const uint4*>(p.aux + (size_t)rr * p.ld_aux + n + 8 * j))
+                                  : make_uint4(0u, 0u, 0u, 0u);
+              }
             }
           }
         };
@@ -399,6 +406,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
               const float2 hi = f2_add(make_float2(v[4 * i + 2], v[4 * i + 3]), make_float2(bn4[i].z, bn4[i].w));
               v[4 * i] = lo.x; v[4 * i + 1] = lo.y; v[4 * i + 2] = hi.x; v[4 * i + 3] = hi.y;
             }
+          }
+          if (kAux && n < p.N) {
+            // through this chunk's staging box (once the TMA store from it two
+            // chunks ago has read it): written as loaded, read back one row per lane
+            uint8_t* box = wbuf + (nstore & 1) * 2048;
+            if (lane == 0) gemm::bulk_wait_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int r = (lane >> 2) + 8 * i, j = lane & 3;
+              *reinterpret_cast<uint4*>(box + r * 64 + ((j ^ ((r >> 1) & 3)) << 4)) = an4[i];
+            }
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              an4[j] = *reinterpret_cast<const uint4*>(box + lane * 64 + ((j ^ ((lane >> 1) & 3)) << 4));
+            __syncwarp();
           }
           if (kAux && n < p.N && row_ok) {
 #pragma unroll
