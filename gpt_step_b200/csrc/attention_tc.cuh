@@ -464,15 +464,23 @@ constexpr int kThreads = 128 + 32 * kSoftmaxWarps;
 constexpr int kLaunchRegs = 168, kCtlRegs = 152, kSoftmaxRegs = 176;
 static_assert(128 * kCtlRegs + 32 * kSoftmaxWarps * kSoftmaxRegs <= kThreads * kLaunchRegs, "register split");
 constexpr int XT_BYTES = 128 * 16 * 2;              // 4 KB: a 128 x 16 extra-K operand tile
+// The constant extra-K tiles of K' and V' have 128 identical rows: one 8-row
+// group (two core matrices, 256 bytes) serves every row group through a
+// descriptor whose row-group stride is 0.
+constexpr int XC_BYTES = 256;
 // Per head size D (64 or 32): a 128-row tile of K, V, Q or dO has rows of 2 D
 // bytes in the 128- or 64-byte swizzled layout.
 template <int D>
 struct Geom {
   static constexpr int ROW = D * 2;
   static constexpr int T_BYTES = 128 * ROW;
-  static constexpr int SMEM_BYTES = 2 * T_BYTES /*K,V*/ + NQS * 2 * T_BYTES /*Q,dO*/ + DST_BYTES +
+  // K has two buffers (the next item's K loads while this item runs), V one
+  // (it is released once an item's last scores are computed). No alignment
+  // slack: without static shared memory the dynamic block starts on a 1 KB
+  // boundary (checked at run time).
+  static constexpr int SMEM_BYTES = 3 * T_BYTES /*K x2, V*/ + NQS * 2 * T_BYTES /*Q,dO*/ + DST_BYTES +
                                     kSoftmaxWarps * DQW_BYTES + NQS * XT_BYTES /*X_i*/ +
-                                    2 * XT_BYTES /*K', V' columns*/ + 256 /*barriers*/ + 1024 /*align*/;
+                                    2 * XC_BYTES /*K', V' columns*/ + 256 /*barriers*/;
   static constexpr uint64_t kSwizzle = D == 64 ? 2 : 4;
   static constexpr uint32_t kMnLbo = D == 64 ? 8192 : 8 * ROW;   // MN-major: one swizzle atom wide, unused
 };
@@ -619,23 +627,28 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   constexpr int T_BYTES = G::T_BYTES;
   constexpr int NO = D / 2;                       // head-dim columns of dQ, dK, dV per softmax warp
   extern __shared__ __align__(1024) uint8_t smem_raw_ab[];
-  uint8_t* smem =
-      reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_ab) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK = smem;
-  uint8_t* sV = sK + T_BYTES;
+  uint8_t* smem = smem_raw_ab;
+  if (smem_u32(smem) & 1023u) {  // the swizzled tiles need a 1 KB-aligned base
+    if (threadIdx.x == 0) atomicOr(err, DEVERR_TIMEOUT);
+    return;
+  }
+  uint8_t* sK = smem;                             // [2]
+  uint8_t* sV = sK + 2 * T_BYTES;
   uint8_t* sQ = sV + T_BYTES;                     // [NQS]
   uint8_t* sDO = sQ + NQS * T_BYTES;              // [NQS]
   uint8_t* sDST = sDO + NQS * T_BYTES;
   uint8_t* sDQW = sDST + DST_BYTES;               // [kSoftmaxWarps][DQW_BYTES]
   uint8_t* sXQ = sDQW + kSoftmaxWarps * DQW_BYTES;  // [NQS] X_i tiles
   uint8_t* sXK = sXQ + NQS * XT_BYTES;              // K' extra columns: 1 1 0 ..
-  uint8_t* sXV = sXK + XT_BYTES;                    // V' extra columns: 0 0 1 1 0 ..
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sXV + XT_BYTES);
-  uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + 1;
-  uint64_t* qdo_full = bars + 2;          // [NQS]
-  uint64_t* qdo_empty = bars + 2 + NQS;   // [NQS]
-  uint64_t* st_full = bars + 2 + 2 * NQS;
+  uint8_t* sXV = sXK + XC_BYTES;                    // V' extra columns: 0 0 1 1 0 ..
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sXV + XC_BYTES);
+  uint64_t* k_full = bars;                // [2]
+  uint64_t* k_empty = bars + 2;           // [2]
+  uint64_t* v_full = bars + 4;
+  uint64_t* v_empty = bars + 5;
+  uint64_t* qdo_full = bars + 6;          // [NQS]
+  uint64_t* qdo_empty = bars + 6 + NQS;   // [NQS]
+  uint64_t* st_full = bars + 6 + 2 * NQS;
   uint64_t* st_empty = st_full + 1;
   uint64_t* ds_full = st_full + 2;
   uint64_t* ds_empty = st_full + 3;
@@ -656,8 +669,12 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const int n_items = nb * BH;
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(kv_full), 1);
-    mbar_init(smem_u32(kv_empty), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&k_full[i]), 1);
+      mbar_init(smem_u32(&k_empty[i]), 1);
+    }
+    mbar_init(smem_u32(v_full), 1);
+    mbar_init(smem_u32(v_empty), 1);
     for (int i = 0; i < NQS; ++i) {
       mbar_init(smem_u32(&qdo_full[i]), 1);
       mbar_init(smem_u32(&qdo_empty[i]), 1);
@@ -676,8 +693,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     tma_prefetch_desc(&tm_do);
     tma_prefetch_desc(&tm_dq);
   }
-  // constant extra-K columns of K' and V' (1.0 in bf16 is 0x3F80)
-  for (int i = threadIdx.x; i < BKEY * 2; i += blockDim.x) {
+  // constant extra-K columns of K' and V' (1.0 in bf16 is 0x3F80): one row group
+  for (int i = threadIdx.x; i < 8 * 2; i += blockDim.x) {
     const int row = i >> 1, half = i & 1;
     const uint32_t one2 = 0x3F803F80u;
     *reinterpret_cast<uint4*>(sXK + xt_offset(row, 8 * half)) = make_uint4(half ? 0u : one2, 0u, 0u, 0u);
@@ -716,14 +733,28 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           const int row_base = b * T, nit = nb - kb;
           // the first query block of this item may land before its keys
           ok = load_qdo(g, bh, row_base, h, kb);
-          // K, V once the previous item's products no longer read them
-          if (ok && j > 0 && !mbar_wait(smem_u32(kv_empty), (j - 1) & 1, err)) ok = false;
+          // V once the previous item's last scores have been computed
+          if (ok && j > 0 && !mbar_wait(smem_u32(v_empty), (j - 1) & 1, err)) ok = false;
           if (!ok) break;
-          mbar_arrive_expect_tx(smem_u32(kv_full), 2 * T_BYTES);
-          tma_load_2d(smem_u32(sK), &tm_qkv, smem_u32(kv_full), C + h * HD, row_base + kb * BKEY);
-          tma_load_2d(smem_u32(sV), &tm_qkv, smem_u32(kv_full), 2 * C + h * HD, row_base + kb * BKEY);
+          mbar_arrive_expect_tx(smem_u32(v_full), T_BYTES);
+          tma_load_2d(smem_u32(sV), &tm_qkv, smem_u32(v_full), 2 * C + h * HD, row_base + kb * BKEY);
+          if (j == 0) {   // later items' K is loaded one item ahead (below)
+            mbar_arrive_expect_tx(smem_u32(&k_full[0]), T_BYTES);
+            tma_load_2d(smem_u32(sK), &tm_qkv, smem_u32(&k_full[0]), C + h * HD, row_base + kb * BKEY);
+          }
           for (int it = 1; it < nit && ok; ++it) ok = load_qdo(g + it, bh, row_base, h, kb + it);
           g += nit;
+          // the next item's K into the other buffer, once the item before this
+          // one has released it
+          const int i2 = i + gridDim.x;
+          if (ok && i2 < n_items) {
+            const int kb2 = i2 / BH, bh2 = i2 % BH, b2 = bh2 / H, h2 = bh2 % H;
+            const int nbuf = (j + 1) & 1;
+            if (j >= 1 && !mbar_wait(smem_u32(&k_empty[nbuf]), ((j - 1) >> 1) & 1, err)) { ok = false; break; }
+            mbar_arrive_expect_tx(smem_u32(&k_full[nbuf]), T_BYTES);
+            tma_load_2d(smem_u32(sK + nbuf * T_BYTES), &tm_qkv, smem_u32(&k_full[nbuf]), C + h2 * HD,
+                        b2 * T + kb2 * BKEY);
+          }
         }
       }
     } else if (warp == 1) {
@@ -745,17 +776,18 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         const uint64_t dO0_k = smem_desc_swz(smem_u32(sDO), 16, kSbo, G::kSwizzle);
         const uint64_t dO0_mn = smem_desc_swz(smem_u32(sDO), G::kMnLbo, kSbo, G::kSwizzle);
         constexpr uint64_t kMnStep = (16 * G::ROW) >> 4;   // 16 rows of an MN-major operand, descriptor units
-        const uint64_t dXK = smem_desc_interleave(smem_u32(sXK), 128, 256);
-        const uint64_t dXV = smem_desc_interleave(smem_u32(sXV), 128, 256);
+        const uint64_t dXK = smem_desc_interleave(smem_u32(sXK), 128, 0);   // one row group for all
+        const uint64_t dXV = smem_desc_interleave(smem_u32(sXV), 128, 0);
+        constexpr uint64_t kKBuf = T_BYTES >> 4;   // the second K buffer, in descriptor units
         const uint64_t dXQ0 = smem_desc_interleave(smem_u32(sXQ), 128, 256);
         constexpr uint64_t kXStage = XT_BYTES >> 4;
         constexpr uint64_t kStage = T_BYTES >> 4;   // one Q/dO stage, in descriptor units
-        auto issue_st = [&](int gq) {
+        auto issue_st = [&](int gq, uint64_t ko) {
           const uint64_t so = (uint64_t)(gq % NQS) * kStage;
           const uint64_t sx = (uint64_t)(gq % NQS) * kXStage;
 #pragma unroll
           for (int kk = 0; kk < HD / 16; ++kk) {
-            tc_mma_bf16(tmem + C_S, dK_k + kk * 2, dQ0_k + so + kk * 2, id_st, kk > 0 ? 1u : 0u);
+            tc_mma_bf16(tmem + C_S, dK_k + ko + kk * 2, dQ0_k + so + kk * 2, id_st, kk > 0 ? 1u : 0u);
             tc_mma_bf16(tmem + C_DP, dV_k + kk * 2, dO0_k + so + kk * 2, id_st, kk > 0 ? 1u : 0u);
           }
           // the per-query terms: S^T - lse/scale, dP^T - D
@@ -767,12 +799,15 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         int g = 0;
         for (int i = blockIdx.x, j = 0; i < n_items && ok; i += gridDim.x, ++j) {
           const int nit = nb - i / BH;
+          const uint64_t ko = (j & 1) ? kKBuf : 0;
           // this item's keys, its first query block, and the previous scores out of TMEM
-          if (!mbar_wait(smem_u32(kv_full), j & 1, err)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&k_full[j & 1]), (j >> 1) & 1, err)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(v_full), j & 1, err)) { ok = false; break; }
           if (!mbar_wait(smem_u32(&qdo_full[g % NQS]), (g / NQS) & 1, err)) { ok = false; break; }
           if (g > 0 && !mbar_wait(smem_u32(st_empty), (g - 1) & 1, err)) { ok = false; break; }
           tc_fence_after();
-          issue_st(g);
+          issue_st(g, ko);
+          if (nit == 1) tc_commit(smem_u32(v_empty));   // the item's last scores read V
           for (int it = 0; it < nit && ok; ++it) {
             const int gc = g + it;
             const uint64_t so = (uint64_t)(gc % NQS) * kStage;
@@ -781,7 +816,8 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
               if (!mbar_wait(smem_u32(&qdo_full[(gc + 1) % NQS]), ((gc + 1) / NQS) & 1, err)) { ok = false; break; }
               if (!mbar_wait(smem_u32(st_empty), gc & 1, err)) { ok = false; break; }
               tc_fence_after();
-              issue_st(gc + 1);
+              issue_st(gc + 1, ko);
+              if (it + 2 == nit) tc_commit(smem_u32(v_empty));   // the item's last scores read V
             }
             // P^T (tensor memory) and dS^T (shared memory) of block it are written
             if (!mbar_wait(smem_u32(ds_full), gc & 1, err)) { ok = false; break; }
@@ -801,13 +837,13 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < BKEY / 16; ++kk)
-              tc_mma_bf16(tmem + C_DQ, dDS_mn + kk * 128, dK_mn + kk * kMnStep, id_q, kk > 0 ? 1u : 0u);
+              tc_mma_bf16(tmem + C_DQ, dDS_mn + kk * 128, dK_mn + ko + kk * kMnStep, id_q, kk > 0 ? 1u : 0u);
             tc_commit(smem_u32(dq_full));
             tc_commit(smem_u32(ds_empty));
             tc_commit(smem_u32(&qdo_empty[gc % NQS]));
           }
           tc_commit(smem_u32(dkdv_full));   // this item's dK, dV are complete
-          tc_commit(smem_u32(kv_empty));    // and its K, V are no longer read
+          tc_commit(smem_u32(&k_empty[j & 1]));   // and its K buffer is no longer read
           g += nit;
         }
         // every product has completed before the block releases tensor memory
