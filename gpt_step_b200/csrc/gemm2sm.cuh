@@ -514,10 +514,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads2, 1)
               lse_m = cm;
             }
             if (cm != -INFINITY) {
-              float a[4] = {0.f, 0.f, 0.f, 0.f};
+              // two columns per paired fp32 instruction, four independent sums
+              const float2 l2e2 = make_float2(kL2e, kL2e), nm2 = make_float2(-lse_m, -lse_m);
+              float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) a[i & 3] += ex2_approx(fmaf(f[i], kL2e, -lse_m));
-              lse_s += (a[0] + a[1]) + (a[2] + a[3]);
+              for (int i = 0; i < 16; ++i) {
+                const float2 y = f2_fma(make_float2(f[2 * i], f[2 * i + 1]), l2e2, nm2);
+                const float2 e = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+                if (i & 1) a1 = f2_add(a1, e);
+                else a0 = f2_add(a0, e);
+              }
+              lse_s += (a0.x + a0.y) + (a1.x + a1.y);
             }
             if (EPI == gemm::EPI_LSE_ONLY) {
               const int k = tgt_col - (c - c_beg);
