@@ -411,7 +411,8 @@ static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int
                      D, 128, D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
   dim3 grid(T / BQ, B * H);
-  launch_pdl(attn_fwd_tc_kernel<D>, dim3(grid), dim3(kThreads), G::SMEM_BYTES, s, tm, out, lse, T, H, 1.0f / sqrtf((float)D), err);
+  launch_pdl(attn_fwd_tc_kernel<D>, dim3(grid), dim3(kThreads), G::SMEM_BYTES, s, tm, out, lse, T, H,
+             1.0f / sqrtf((float)D), err);
   return cudaGetLastError();
 }
 
@@ -1002,12 +1003,13 @@ static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, c
       !encode_map_2d(&tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, (uint64_t)C, (uint64_t)B * T, (uint64_t)C,
                      D / 2, 32, swz))
     return cudaErrorInvalidValue;
-  launch_pdl(bwd_prep_kernel<D>, dim3(B * T / bwd::kPrepRows), dim3(256), 0, s, out, dout, lse, xtiles, dq_acc, T, H, scale);
+  launch_pdl(bwd_prep_kernel<D>, dim3(B * T / bwd::kPrepRows), dim3(256), 0, s, out, dout, lse, xtiles, dq_acc, T, H,
+             scale);
   const int n_items = (T / bwd::BKEY) * B * H;
   const int sms = device_sm_count();   // one persistent CTA per SM
   const int grid = n_items < sms ? n_items : sms;
-  launch_pdl(attn_bwd_tc_kernel<D>, dim3(grid), dim3(bwd::kThreads), G::SMEM_BYTES, s, tm_qkv, tm_do, tm_dq, xtiles, dqkv, T, H, B * H,
-                                                                   scale, err);
+  launch_pdl(attn_bwd_tc_kernel<D>, dim3(grid), dim3(bwd::kThreads), G::SMEM_BYTES, s, tm_qkv, tm_do, tm_dq, xtiles,
+             dqkv, T, H, B * H, scale, err);
   const int n = B * T * (C / 8);
   int blocks = (n + 255) / 256;
   if (blocks > 148 * 8) blocks = 148 * 8;

@@ -294,7 +294,8 @@ void ln_fwd_c(const bf16* x, const float* w, const float* b, bf16* y, float* mea
   static int cache[PerDeviceOnce::kMaxDevices] = {};
   const int full = resident_ctas(once, cache, k::layernorm_fwd_kernel<C>, k::kLnFwdWarps * 32);
   const int need = (rows + k::kLnFwdWarps - 1) / k::kLnFwdWarps;
-  launch_pdl(k::layernorm_fwd_kernel<C>, dim3(std::min(need, full)), dim3(k::kLnFwdWarps * 32), 0, s, x, w, b, y, mean, rstd, rows);
+  launch_pdl(k::layernorm_fwd_kernel<C>, dim3(std::min(need, full)), dim3(k::kLnFwdWarps * 32), 0, s, x, w, b, y,
+             mean, rstd, rows);
 }
 
 int ln_fwd(const bf16* x, const float* w, const float* b, bf16* y, float* mean, float* rstd, int rows, int C,
@@ -331,8 +332,8 @@ cudaError_t ln_bwd_c(const bf16* dy, const bf16* x, const float* mean, const flo
   static PerDeviceOnce once;
   const cudaError_t e = smem_optin(once, k::layernorm_bwd_kernel<C>, Cfg::SMEM);
   if (e != cudaSuccess) return e;
-  launch_pdl(k::layernorm_bwd_kernel<C>, dim3(blocks), dim3(Cfg::WARPS * 32), Cfg::SMEM, s, dy, x, mean, rstd, w, dresid, dx, part, rows,
-                                                                        with_dxsum, dw, db, dbias);
+  launch_pdl(k::layernorm_bwd_kernel<C>, dim3(blocks), dim3(Cfg::WARPS * 32), Cfg::SMEM, s, dy, x, mean, rstd, w,
+             dresid, dx, part, rows, with_dxsum, dw, db, dbias);
   return cudaGetLastError();
 }
 
@@ -361,7 +362,9 @@ int ln_bwd(const bf16* dy, const bf16* x, const float* mean, const float* rstd, 
     default: return GPT2_ERR_ARG;
   }
   if (e != cudaSuccess) return GPT2_ERR_CUDA;
-  if (part) launch_pdl(k::partial_rows_reduce_kernel, dim3((nq * C + 31) / 32), dim3(256), 0, s, part, blocks, nq * C, dw, db, dbias, C);
+  if (part)
+    launch_pdl(k::partial_rows_reduce_kernel, dim3((nq * C + 31) / 32), dim3(256), 0, s, part, blocks, nq * C, dw, db,
+               dbias, C);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -405,8 +408,8 @@ int softmax_ce(bf16* logits, const int32_t* targets, float* losses, int N, int V
   if (part && slots <= 0) return GPT2_ERR_ARG;
   if (tgt_val && (!part || write_grad)) return GPT2_ERR_ARG;   // logits-free: a loss from the partials only
   if (!logits && !tgt_val) return GPT2_ERR_ARG;
-  launch_pdl(k::softmax_ce_kernel, dim3(N), dim3(k::kCeThreads), 0, s, logits, targets, losses, V, Vp, dscale, write_grad, err,
-                                                    ignore_index, part, slots, tgt_val);
+  launch_pdl(k::softmax_ce_kernel, dim3(N), dim3(k::kCeThreads), 0, s, logits, targets, losses, V, Vp, dscale,
+             write_grad, err, ignore_index, part, slots, tgt_val);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -527,8 +530,8 @@ int forward(gpt2_model* m, const int32_t* tok, const int32_t* tgt, int b, bool t
 
   {
     const size_t p = prof_begin(m);
-    launch_pdl(k::embed_fwd_kernel, dim3(launch::grid_for(N * C / 8, 256)), dim3(256), 0, s, tok, m->W(K_WTE), m->W(K_WPE), resid,
-                                                                          (int)N, T, C, d.V, err);
+    launch_pdl(k::embed_fwd_kernel, dim3(launch::grid_for(N * C / 8, 256)), dim3(256), 0, s, tok, m->W(K_WTE),
+               m->W(K_WPE), resid, (int)N, T, C, d.V, err);
     prof_end(m, p, PC_EMBED, (double)N * (6.0 * C + 4), 1);
   }
   for (int l = 0; l < L; ++l) {
@@ -736,8 +739,8 @@ int backward(gpt2_model* m, const int32_t* tok) {
   {
     const size_t p = prof_begin(m);
     launch_pdl(k::embed_bwd_wpe_kernel, dim3((T * C / 8 + 255) / 256), dim3(256), 0, s, dresid, m->G(K_WPE), d.B, T, C);
-    launch_pdl(k::embed_bwd_wte_kernel, dim3((N + k::kEmbRows - 1) / k::kEmbRows), dim3(256), 0, s, tok, dresid, m->G(K_WTE), N, C,
-                                                                                d.V);
+    launch_pdl(k::embed_bwd_wte_kernel, dim3((N + k::kEmbRows - 1) / k::kEmbRows), dim3(256), 0, s, tok, dresid,
+               m->G(K_WTE), N, C, d.V);
     prof_end(m, p, PC_EMBED, (double)N * (2.0 * C + 4) + 2.0 * N * C * 4 + 8.0 * T * C, 2);
   }
   // the last bucket (wpe, wte) and the 1-D region are final now
@@ -957,17 +960,17 @@ static int clip_adamw_impl(gpt2_model* m, int32_t step, const k::Ranges4& rg, co
   cudaStream_t s = m->stream;
   const Layout& y = m->lay;
   const size_t pr = prof_begin(m);
-  launch_pdl(k::norm_finalize_kernel, dim3(1), dim3(256), 0, s, sumsq, nparts, m->sc(), m->n_micro, y.d.N, m->cfg.grad_clip, m->err());
+  launch_pdl(k::norm_finalize_kernel, dim3(1), dim3(256), 0, s, sumsq, nparts, m->sc(), m->n_micro, y.d.N,
+             m->cfg.grad_clip, m->err());
   const double lr = lr_at(m->cfg, step);
   const double t = (double)step + 1.0;
   const float bc1 = (float)(1.0 - pow((double)m->cfg.beta1, t));
   const float bc2 = (float)(1.0 - pow((double)m->cfg.beta2, t));
   long n4 = 0;
   for (int r = 0; r < rg.n; ++r) n4 += rg.end[r] - rg.begin[r];
-  launch_pdl(k::adamw_kernel, dim3(launch::grid_for(n4, 256)), dim3(256), 0, s, m->params(), m->grads(), m->at<float>(y.adam_m),
-                                                             m->at<float>(y.adam_v), m->pbf(), rg, y.P1 / 4,
-                                                             m->sc(), (float)lr, m->cfg.beta1, m->cfg.beta2,
-                                                             m->cfg.eps, m->cfg.weight_decay, bc1, bc2);
+  launch_pdl(k::adamw_kernel, dim3(launch::grid_for(n4, 256)), dim3(256), 0, s, m->params(), m->grads(),
+             m->at<float>(y.adam_m), m->at<float>(y.adam_v), m->pbf(), rg, y.P1 / 4, m->sc(), (float)lr, m->cfg.beta1,
+             m->cfg.beta2, m->cfg.eps, m->cfg.weight_decay, bc1, bc2);
   int nl = 2;
   if (clear_all_grads) {
     if (cudaMemsetAsync(m->grads(), 0, (size_t)y.P * 4, s) != cudaSuccess) return GPT2_ERR_CUDA;
@@ -1202,7 +1205,8 @@ int gpt2_write(gpt2_model* m, int what, int idx, const float* host_src) {
   if (cudaStreamSynchronize(m->stream) != cudaSuccess) return GPT2_ERR_CUDA;
   if (cudaMemcpy(base + t.off, host_src, (size_t)t.n * 4, cudaMemcpyHostToDevice) != cudaSuccess) return GPT2_ERR_CUDA;
   if (what == GPT2_PARAMS) {
-    launch_pdl(k::to_bf16_kernel, dim3(launch::grid_for(t.n, 256)), dim3(256), 0, m->stream, base + t.off, m->pbf() + t.off, t.n);
+    launch_pdl(k::to_bf16_kernel, dim3(launch::grid_for(t.n, 256)), dim3(256), 0, m->stream, base + t.off,
+               m->pbf() + t.off, t.n);
     if (cudaGetLastError() != cudaSuccess || cudaStreamSynchronize(m->stream) != cudaSuccess) return GPT2_ERR_CUDA;
   }
   return GPT2_OK;
@@ -1440,9 +1444,9 @@ int gpt2op_embedding_fwd(const int32_t* tokens, const void* wte, const void* wpe
                          int* dev_err, void* stream) {
   if (!tokens || !wte || !wpe || !out || !dev_err || C % 8) return GPT2_ERR_ARG;
   const long N = (long)B * T;
-  launch_pdl(k::embed_fwd_kernel, dim3(launch::grid_for(N * C / 8, 256)), dim3(256), 0, static_cast<cudaStream_t>(stream), 
-      tokens, static_cast<const bf16*>(wte), static_cast<const bf16*>(wpe), static_cast<bf16*>(out), (int)N, T, C, V,
-      dev_err);
+  launch_pdl(k::embed_fwd_kernel, dim3(launch::grid_for(N * C / 8, 256)), dim3(256), 0,
+             static_cast<cudaStream_t>(stream), tokens, static_cast<const bf16*>(wte), static_cast<const bf16*>(wpe),
+             static_cast<bf16*>(out), (int)N, T, C, V, dev_err);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
@@ -1451,9 +1455,10 @@ int gpt2op_embedding_bwd(const int32_t* tokens, const void* dx, float* dwte, flo
   if (!tokens || !dx || !dwte || !dwpe || C % 8) return GPT2_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long N = (long)B * T;
-  launch_pdl(k::embed_bwd_wpe_kernel, dim3((T * C / 8 + 255) / 256), dim3(256), 0, s, static_cast<const bf16*>(dx), dwpe, B, T, C);
-  launch_pdl(k::embed_bwd_wte_kernel, dim3((int)((N + k::kEmbRows - 1) / k::kEmbRows)), dim3(256), 0, s, 
-      tokens, static_cast<const bf16*>(dx), dwte, (int)N, C, V);
+  launch_pdl(k::embed_bwd_wpe_kernel, dim3((T * C / 8 + 255) / 256), dim3(256), 0, s, static_cast<const bf16*>(dx),
+             dwpe, B, T, C);
+  launch_pdl(k::embed_bwd_wte_kernel, dim3((int)((N + k::kEmbRows - 1) / k::kEmbRows)), dim3(256), 0, s, tokens,
+             static_cast<const bf16*>(dx), dwte, (int)N, C, V);
   return cudaGetLastError() == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 

@@ -76,16 +76,19 @@ def run_step(args):
 
 
 def kernel_sources_sha256() -> str:
-    """sha256 over the CUDA sources of the library (file names and bytes, sorted)."""
+    """sha256 over the CUDA sources of the library: file names in sorted order and
+    their contents with every run of whitespace collapsed to one space, so that a
+    change of layout alone keeps the hash."""
     import hashlib
     import os
+    import re
     d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(d)):
         if name.endswith((".cu", ".cuh", ".h")):
             h.update(name.encode())
             with open(os.path.join(d, name), "rb") as f:
-                h.update(f.read())
+                h.update(re.sub(rb"\s+", b" ", f.read()).strip())
     return h.hexdigest()
 
 
