@@ -96,8 +96,9 @@ def test_bias_grad(atomic):
 
 # --- a2/a6/a9: LayerNorm -------------------------------------------------------------------
 
-@pytest.mark.parametrize("C,atomic", [(128, False), (384, False), (768, False), (1536, False), (128, True),
-                                      (768, True), (1536, True)])
+@pytest.mark.parametrize("C,atomic", [(128, False), (256, False), (384, False), (512, False), (768, False),
+                                      (1024, False), (1536, False), (2048, False), (128, True), (512, True),
+                                      (768, True), (1024, True), (1536, True), (2048, True)])
 def test_layernorm_fwd_bwd(C, atomic):
     """LayerNorm forward and backward; the backward's column sums both ways: a
     fixed-order second pass over a workspace, or fp32 atomics in one launch."""
