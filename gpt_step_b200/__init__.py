@@ -101,7 +101,7 @@ _SIGNATURES = {
     "gpt2op_layernorm_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P]),
     "gpt2op_attention_fwd": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P]),
     "gpt2op_attention_bwd_workspace": (_SZ, [_I, _I, _I, _I]),
-    "gpt2op_attention_bwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P]),
+    "gpt2op_attention_bwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P]),
     "gpt2op_softmax_ce": (_I, [_P, _P, _P, _I, _I, _I, _F, _P, _P]),
     "gpt2op_softmax_ce_masked": (_I, [_P, _P, _P, _I, _I, _I, _I, _F, _P, _P]),
     "gpt2op_lm_head_loss": (_I, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P, _P]),
@@ -448,11 +448,12 @@ def attention_bwd_workspace(B, T, H, hd):
     return lib().gpt2op_attention_bwd_workspace(B, T, H, hd)
 
 
-def attention_bwd(qkv, out, dout, lse, dqkv, n_head, workspace, err, stream=None):
+def attention_bwd(qkv, out, dout, lse, dqkv, n_head, workspace, err, stream=None, dbias=None):
+    """dbias (fp32 [3C]) or None: += the qkv bias gradient (column sums of dqkv)."""
     B, T, C3 = qkv.shape
     hd = C3 // 3 // n_head
-    check(lib().gpt2op_attention_bwd(_ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dqkv), B, T,
-                                     n_head, hd, _ptr(workspace), workspace.numel(), _ptr(err),
+    check(lib().gpt2op_attention_bwd(_ptr(qkv), _ptr(out), _ptr(dout), _ptr(lse), _ptr(dqkv), _ptr(dbias),
+                                     B, T, n_head, hd, _ptr(workspace), workspace.numel(), _ptr(err),
                                      _s(stream)), "gpt2op_attention_bwd")
 
 

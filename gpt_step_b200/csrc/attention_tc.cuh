@@ -487,7 +487,7 @@ struct Geom {
 };
 constexpr uint32_t C_S = 0, C_DP = 128, C_DV = 256, C_DK = 320, C_DQ = 384, C_P = 448;
 constexpr int TMEM_COLS_BWD = 512;
-constexpr int kPrepRows = 32;                       // query rows per prep block
+constexpr int kPrepRows = 64;                       // query rows per prep block
 constexpr int kMaxHeads = 64;
 }  // namespace bwd
 
@@ -546,26 +546,42 @@ GPT2_DEV void bwd_softmax_row(const uint32_t (&sv)[2][32], const uint32_t (&dv)[
   }
 }
 
-// Block: 32 consecutive query rows of one sequence, all heads. Each warp takes
-// four rows; lanes hold 16-byte chunks of O and dO, D / 8 chunks per head.
+// Block: 64 consecutive query rows of one sequence, all heads, in
+// 32 * ceil(C/256) * RW threads, RW = max(1, 12 / ceil(C/256)). Warp w takes
+// the 32 16-byte chunks of group g = w % ceil(C/256) (lanes hold chunks of O
+// and dO, D / 8 chunks per head) in the rows rl = w / ceil(C/256) + RW i.
+// With dbias_v the block also adds the column sums of its 64 rows of dO into
+// dbias_v (fp32 [C], 16-byte aligned): the gradient of the value bias, since
+// every row of causal softmax weights sums to one (an output row is a convex
+// combination of value rows, so a bias added to every value row passes through
+// unchanged). A lane keeps its chunk's sums over its rows in registers; the RW
+// row warps of a chunk group are added once through shared memory.
 template <int D>
-__global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
+__global__ void __launch_bounds__(512) bwd_prep_kernel(const bf16* __restrict__ out, const bf16* __restrict__ dout,
                                                        const float* __restrict__ lse, uint8_t* __restrict__ xtiles,
-                                                       float* __restrict__ dq_acc, int T, int H, float scale) {
+                                                       float* __restrict__ dq_acc, float* __restrict__ dbias_v, int T,
+                                                       int H, float scale) {
   pdl_begin();
   using namespace bwd;
   constexpr int CPH = D / 8;                 // 16-byte chunks per head
   __shared__ float sDot[kMaxHeads][kPrepRows];
+  __shared__ __align__(16) float sPart[512 * 8];
   const int C = H * D;
   const int NV = C / 8;                      // 16-byte chunks per row
+  const int NG = (NV + 31) / 32;             // chunk groups of 32
+  const int RW = (blockDim.x >> 5) / NG;     // row warps per chunk group (the host makes this >= 1)
   const int row0 = blockIdx.x * kPrepRows;   // global row (b*T + t) of the first query
   const int b = row0 / T, t0 = row0 % T;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int rr = 0; rr < kPrepRows / 8; ++rr) {
-    const int rl = warp * (kPrepRows / 8) + rr;
-    const size_t base = (size_t)(row0 + rl) * C;
-    for (int v0 = 0; v0 < NV; v0 += 32) {
-      const int vi = v0 + lane;
+  const int g = warp % NG, rw = warp / NG;
+  const int vi = g * 32 + lane;
+  float cs[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) cs[k] = 0.f;
+  if (rw < RW) {
+#pragma unroll 4
+    for (int rl = rw; rl < kPrepRows; rl += RW) {
+      const size_t base = (size_t)(row0 + rl) * C;
       float acc = 0.f;
       if (vi < NV) {
         const uint4 a = __ldg(reinterpret_cast<const uint4*>(out + base) + vi);
@@ -575,6 +591,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ 
         for (int k = 0; k < 4; ++k) {
           const float2 fa = unpack_bf16x2(aw[k]), fc = unpack_bf16x2(cw[k]);
           acc = fmaf(fa.x, fc.x, fmaf(fa.y, fc.y, acc));
+          cs[2 * k] += fc.x;
+          cs[2 * k + 1] += fc.y;
         }
       }
 #pragma unroll
@@ -582,7 +600,22 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ 
       if ((lane & (CPH - 1)) == 0 && vi < NV) sDot[vi / CPH][rl] = acc;
     }
   }
+  const bool colsum = dbias_v != nullptr;
+  if (colsum && rw < RW && vi < NV) {
+    float4* sp = reinterpret_cast<float4*>(sPart + (rw * NG * 32 + vi) * 8);
+    sp[0] = make_float4(cs[0], cs[1], cs[2], cs[3]);
+    sp[1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
+  }
   __syncthreads();
+  if (colsum)
+    for (int i = threadIdx.x; i < C / 4; i += blockDim.x) {   // i: a group of four columns
+      float4 s4 = reinterpret_cast<const float4*>(sPart)[i];
+      for (int r = 1; r < RW; ++r) {
+        const float4 u = reinterpret_cast<const float4*>(sPart)[r * NG * 64 + i];
+        s4.x += u.x; s4.y += u.y; s4.z += u.z; s4.w += u.w;
+      }
+      red_add_f32x4(dbias_v + 4 * i, s4.x, s4.y, s4.z, s4.w);
+    }
   // X tile of query block (b, h, t / 128), row t % 128: columns 0,1 = (hi, lo) of
   // -lse/scale, columns 2,3 = (hi, lo) of -D, the rest 0
   for (int i = threadIdx.x; i < H * kPrepRows; i += blockDim.x) {
@@ -602,18 +635,50 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const bf16* __restrict__ 
   for (int i = threadIdx.x; i < n4; i += blockDim.x) z[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dq_acc fp32 [rows, C] -> dqkv[:, 0:C] bf16 (row stride 3C); eight columns per thread.
-__global__ void __launch_bounds__(256) bwd_post_kernel(const float* __restrict__ dq_acc, bf16* __restrict__ dqkv,
-                                                       int rows, int C) {
+// dq_acc fp32 [rows, C] -> dqkv[:, 0:C] bf16 (row stride 3C), in blocks of
+// (C/8) * RL threads: thread t of block b converts the eight columns of chunk
+// t % (C/8) in rows (b RL + t / (C/8)) + k gridDim.x RL, so that the grid
+// sweeps the matrix as one contiguous band. With dbias_q the block adds the
+// column sums of its rows of dQ (fp32, before rounding) into dbias_q (fp32
+// [C], 16-byte aligned): the query bias gradient.
+__global__ void __launch_bounds__(1024) bwd_post_kernel(const float* __restrict__ dq_acc, bf16* __restrict__ dqkv,
+                                                        float* __restrict__ dbias_q, int rows, int C) {
   pdl_begin();
-  const int per_row = C / 8;
-  const int n = rows * per_row;
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
-    const int row = i / per_row, c8 = i - row * per_row;
-    const float4* src = reinterpret_cast<const float4*>(dq_acc + (size_t)row * C + c8 * 8);
-    const float4 a = __ldcs(src), c = __ldcs(src + 1);
-    *reinterpret_cast<uint4*>(dqkv + (size_t)row * 3 * C + c8 * 8) =
-        make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
+  __shared__ __align__(16) float sPart[1024 * 8];
+  const int NV = C / 8;
+  const int RL = blockDim.x / NV;             // row lanes (the host makes this >= 1)
+  const int c8 = threadIdx.x % NV, rl = threadIdx.x / NV;
+  const int band = gridDim.x * RL;
+  float cs[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) cs[k] = 0.f;
+  if (rl < RL) {
+#pragma unroll 4
+    for (int row = blockIdx.x * RL + rl; row < rows; row += band) {
+      const float4* src = reinterpret_cast<const float4*>(dq_acc + (size_t)row * C + c8 * 8);
+      const float4 a = __ldcs(src), c = __ldcs(src + 1);
+      *reinterpret_cast<uint4*>(dqkv + (size_t)row * 3 * C + c8 * 8) =
+          make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(c.x, c.y), pack_bf16x2(c.z, c.w));
+      cs[0] += a.x; cs[1] += a.y; cs[2] += a.z; cs[3] += a.w;
+      cs[4] += c.x; cs[5] += c.y; cs[6] += c.z; cs[7] += c.w;
+    }
+  }
+  if (dbias_q == nullptr) return;
+  // the RL row lanes' sums of each chunk, added in a fixed order, then one
+  // vector atomic per four columns
+  float4* sp = reinterpret_cast<float4*>(sPart);
+  if (rl < RL) {
+    sp[2 * threadIdx.x] = make_float4(cs[0], cs[1], cs[2], cs[3]);
+    sp[2 * threadIdx.x + 1] = make_float4(cs[4], cs[5], cs[6], cs[7]);
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 2 * NV; i += blockDim.x) {   // i: a group of four columns
+    float4 s4 = sp[i];
+    for (int r = 1; r < RL; ++r) {
+      const float4 u = sp[r * 2 * NV + i];
+      s4.x += u.x; s4.y += u.y; s4.z += u.z; s4.w += u.w;
+    }
+    red_add_f32x4(dbias_q + 4 * i, s4.x, s4.y, s4.z, s4.w);
   }
 }
 
@@ -974,10 +1039,16 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
 }
 
 // The whole backward. xtiles (B*H*T*32 bytes) and dq_acc fp32 [B*T, C] are
-// scratch (contents on entry do not matter); dqkv receives dQ | dK | dV.
+// scratch (contents on entry do not matter); dqkv receives dQ | dK | dV. With
+// dbias (fp32 [3C], 16-byte aligned) the gradient of the qkv bias is added
+// there: column sums of dQ (post pass) and of dO (prep pass, the value third);
+// the key third gets nothing, its gradient being exactly zero (adding one
+// vector to every key shifts each query's scores by a constant, which the
+// softmax removes).
 template <int D>
 static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, uint8_t* xtiles,
-                           float* dq_acc, bf16* dqkv, int B, int T, int H, int* err, cudaStream_t s) {
+                           float* dq_acc, bf16* dqkv, float* dbias, int B, int T, int H, int* err,
+                           cudaStream_t s) {
   using G = bwd::Geom<D>;
   static PerDeviceOnce once;
   cudaError_t e0 = once.run([] {
@@ -1003,17 +1074,24 @@ static cudaError_t bwd_run(const bf16* qkv, const bf16* out, const bf16* dout, c
       !encode_map_2d(&tm_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dq_acc, (uint64_t)C, (uint64_t)B * T, (uint64_t)C,
                      D / 2, 32, swz))
     return cudaErrorInvalidValue;
-  launch_pdl(bwd_prep_kernel<D>, dim3(B * T / bwd::kPrepRows), dim3(256), 0, s, out, dout, lse, xtiles, dq_acc, T, H,
-             scale);
+  if (dbias && (reinterpret_cast<uintptr_t>(dbias) & 15)) return cudaErrorInvalidValue;
+  // prep pass: ceil(C/256) warps per row group, as many row groups as fit 384 threads
+  const int ng = (C / 8 + 31) / 32;
+  const int prep_threads = 32 * ng * std::max(1, 12 / ng);
+  launch_pdl(bwd_prep_kernel<D>, dim3(B * T / bwd::kPrepRows), dim3(prep_threads), 0, s, out, dout, lse, xtiles,
+             dq_acc, dbias ? dbias + 2 * C : nullptr, T, H, scale);
   const int n_items = (T / bwd::BKEY) * B * H;
   const int sms = device_sm_count();   // one persistent CTA per SM
   const int grid = n_items < sms ? n_items : sms;
   launch_pdl(attn_bwd_tc_kernel<D>, dim3(grid), dim3(bwd::kThreads), G::SMEM_BYTES, s, tm_qkv, tm_do, tm_dq, xtiles,
              dqkv, T, H, B * H, scale, err);
-  const int n = B * T * (C / 8);
-  int blocks = (n + 255) / 256;
-  if (blocks > 148 * 8) blocks = 148 * 8;
-  launch_pdl(bwd_post_kernel, dim3(blocks), dim3(256), 0, s, dq_acc, dqkv, B * T, C);
+  // post pass: C/8 chunk columns times as many row lanes as fit 1024 threads
+  // (C/8 <= 512); one wave of blocks
+  const int nv = C / 8, rows = B * T;
+  const int rl = 1024 / nv;
+  const int bps = std::max(1, 2048 / (nv * rl));
+  const int post_blocks = std::max(1, std::min(sms * bps, (rows + rl - 1) / rl));
+  launch_pdl(bwd_post_kernel, dim3(post_blocks), dim3(nv * rl), 0, s, dq_acc, dqkv, dbias, rows, C);
   return cudaGetLastError();
 }
 

@@ -426,19 +426,26 @@ int attention_fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int H, i
   return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
 }
 
+// dbias (fp32 [3C], or null): += the gradient of the qkv bias. On tcgen05 the
+// attention backward's own passes add it (the key third exactly zero); on the
+// mma.sync path the column sums of the stored dqkv are added afterwards.
 int attention_bwd(const bf16* qkv, const bf16* out, const bf16* dout, const float* lse, float* Dv, float* dq_acc,
-                  bf16* dqkv, int B, int T, int H, int hd, int* err, cudaStream_t s) {
+                  bf16* dqkv, float* dbias, int B, int T, int H, int hd, int* err, cudaStream_t s) {
   if (T % 64) return GPT2_ERR_ARG;
+  if (dbias && (reinterpret_cast<uintptr_t>(dbias) & 15)) return GPT2_ERR_ARG;
   cudaError_t e;
   if ((hd == 64 || hd == 32) && T % attn_tc::bwd::BKEY == 0 && H <= attn_tc::bwd::kMaxHeads && err != nullptr) {
     // Dv holds the 16-column per-query operand tiles here (32 bytes per query and head)
     uint8_t* xt = reinterpret_cast<uint8_t*>(Dv);
-    e = hd == 64 ? attn_tc::bwd_run<64>(qkv, out, dout, lse, xt, dq_acc, dqkv, B, T, H, err, s)
-                 : attn_tc::bwd_run<32>(qkv, out, dout, lse, xt, dq_acc, dqkv, B, T, H, err, s);
-  } else if (hd == 64) e = attn::bwd<64>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
+    e = hd == 64 ? attn_tc::bwd_run<64>(qkv, out, dout, lse, xt, dq_acc, dqkv, dbias, B, T, H, err, s)
+                 : attn_tc::bwd_run<32>(qkv, out, dout, lse, xt, dq_acc, dqkv, dbias, B, T, H, err, s);
+    return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
+  }
+  if (hd == 64) e = attn::bwd<64>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
   else if (hd == 32) e = attn::bwd<32>(qkv, out, dout, lse, Dv, dq_acc, dqkv, B, T, H, s);
   else return GPT2_ERR_ARG;
-  return e == cudaSuccess ? GPT2_OK : GPT2_ERR_CUDA;
+  if (e != cudaSuccess) return GPT2_ERR_CUDA;
+  return dbias ? bias_grad(dqkv, dbias, B * T, 3 * H * hd, nullptr, 0, s) : GPT2_OK;
 }
 
 int grid_for(long work, int threads) {
@@ -715,8 +722,9 @@ int backward(gpt2_model* m, const int32_t* tok) {
     }
     {
       const size_t p = prof_begin(m);
-      GPT2_TRY(launch::attention_bwd(qkv, atty, datty, lse, m->at<float>(y.attD), m->at<float>(y.dq_acc), dqkv, d.B,
-                                     T, d.H, d.hd, err, s));
+      // the qkv bias gradient comes out of the attention backward's own passes
+      GPT2_TRY(launch::attention_bwd(qkv, atty, datty, lse, m->at<float>(y.attD), m->at<float>(y.dq_acc), dqkv,
+                                     m->G(K_QKVB, l), d.B, T, d.H, d.hd, err, s));
       // causal FLOPs: QK^T, dO V^T, dV, dK and dQ over the visible pairs
       prof_end(m, p, PC_ATTN_BWD, 5.0 * d.B * d.H * (double)T * (T + 1) * d.hd, 3);
     }
@@ -731,7 +739,6 @@ int backward(gpt2_model* m, const int32_t* tok) {
     // every 2-D weight gradient of this block is final for this micro-step
     if (!m->bucket_events.empty() && cudaEventRecord(m->bucket_events[L - 1 - l], s) != cudaSuccess)
       return GPT2_ERR_CUDA;
-    GPT2_TRY(bias_grad_m(m, dqkv, m->G(K_QKVB, l), N, 3 * C));
     GPT2_TRY(ln_bwd_m(m, dln, x_in, m->at<float>(y.ln1_mean) + l * d.N, m->at<float>(y.ln1_rstd) + l * d.N, K_LN1W,
                       K_LN1B, l, dresid, dresid, l > 0 ? m->G(K_FCPROJB, l - 1) : nullptr));
   }
@@ -1359,8 +1366,9 @@ size_t gpt2op_attention_bwd_workspace(int B, int T, int H, int hd) {
   return (size_t)B * T * H * hd * 4 + (size_t)B * H * T * 32;
 }
 
-int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv, int B,
-                         int T, int H, int hd, void* workspace, size_t ws_bytes, int* dev_err, void* stream) {
+int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv,
+                         float* dbias, int B, int T, int H, int hd, void* workspace, size_t ws_bytes, int* dev_err,
+                         void* stream) {
   if (!qkv || !out || !dout || !lse || !dqkv || !workspace || !dev_err) return GPT2_ERR_ARG;
   if (ws_bytes < gpt2op_attention_bwd_workspace(B, T, H, hd)) return GPT2_ERR_ARG;
   float* dq_acc = static_cast<float*>(workspace);
@@ -1368,8 +1376,8 @@ int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, con
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaMemsetAsync(dq_acc, 0, (size_t)B * T * H * hd * 4, s) != cudaSuccess) return GPT2_ERR_CUDA;
   return launch::attention_bwd(static_cast<const bf16*>(qkv), static_cast<const bf16*>(out),
-                               static_cast<const bf16*>(dout), lse, Dv, dq_acc, static_cast<bf16*>(dqkv), B, T, H, hd,
-                               dev_err, s);
+                               static_cast<const bf16*>(dout), lse, Dv, dq_acc, static_cast<bf16*>(dqkv), dbias, B, T,
+                               H, hd, dev_err, s);
 }
 
 int gpt2op_softmax_ce(void* logits, const int32_t* targets, float* losses, int N, int V, int Vp, float dscale,

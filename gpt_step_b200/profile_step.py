@@ -192,7 +192,8 @@ def run_attn(args):
         dout = torch.tensor(rng.standard_normal((B, T, C)).astype(np.float32)).to(torch.bfloat16).cuda()
         dqkv = torch.empty_like(qkv)
         ws = torch.empty(gs.attention_bwd_workspace(B, T, H, hd), dtype=torch.uint8, device="cuda")
-        fn = lambda: gs.attention_bwd(qkv, out, dout, lse, dqkv, H, ws, err)
+        dbias = torch.zeros(3 * C, device="cuda")   # the model's form: the qkv bias gradient added too
+        fn = lambda: gs.attention_bwd(qkv, out, dout, lse, dqkv, H, ws, err, dbias=dbias)
         flops = 5.0 * B * H * T * (T + 1) * hd
     for _ in range(3):
         fn()

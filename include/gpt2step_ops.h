@@ -116,20 +116,29 @@ int gpt2op_layernorm_bwd_noalloc(const void* dy, const void* x, const float* mea
 /* Causal multi-head attention forward (grow_a_language_model_intro, activities
  * 5-6: softmax(Q K^T / sqrt(hd)) V with a causal mask). qkv bf16 [B,T,3C]
  * (q | k | v, heads contiguous), out bf16 [B,T,C], lse fp32 [B,H,T] (natural
- * log-sum-exp of the scaled scores). hd in {32, 64}, T % 64 == 0. Head size 64
- * with T % 128 == 0 runs on tcgen05 (scores and output accumulated in tensor
- * memory); other shapes on mma.sync. */
+ * log-sum-exp of the scaled scores). hd in {32, 64}, T % 64 == 0. T % 128 == 0
+ * runs on tcgen05 (scores and output accumulated in tensor memory); other
+ * shapes on mma.sync. */
 int gpt2op_attention_fwd(const void* qkv, void* out, float* lse, int B, int T, int H, int hd, int* dev_err,
                          void* stream);
 
-/* Attention backward from the saved output and lse: dqkv bf16 [B,T,3C]. Head
- * size 64 with T % 128 == 0 (and H <= 64) runs on tcgen05, other shapes on
- * mma.sync. The workspace (fp32 dQ accumulator [B*T, C] followed by 32 bytes
- * per query and head of per-query terms) must be 16-byte aligned; its contents
- * on entry do not matter. Concurrent calls must not share a workspace. */
+/* Attention backward from the saved output and lse: dqkv bf16 [B,T,3C].
+ * T % 128 == 0 (and H <= 64) runs on tcgen05, other shapes on mma.sync. The
+ * workspace (fp32 dQ accumulator [B*T, C] followed by 32 bytes per query and
+ * head of per-query terms) must be 16-byte aligned; its contents on entry do
+ * not matter. Concurrent calls must not share a workspace.
+ * dbias, if not NULL (fp32 [3C], 16-byte aligned, else GPT2_ERR_ARG): += the
+ * gradient of a bias added to qkv, i.e. the column sums of dqkv over the B*T
+ * rows. On tcgen05 they are formed from exact identities: the q third sums dQ
+ * in fp32 before rounding, the v third sums dO (each causal softmax row sums
+ * to one, so dV's column sums equal dO's), the k third gets nothing (its
+ * gradient is exactly zero: a shift shared by a query's scores cancels in the
+ * softmax). On mma.sync the column sums of the stored bf16 dqkv are added
+ * (fp32 atomics; the k third then holds rounding-level values). */
 size_t gpt2op_attention_bwd_workspace(int B, int T, int H, int hd);
-int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv, int B,
-                         int T, int H, int hd, void* workspace, size_t ws_bytes, int* dev_err, void* stream);
+int gpt2op_attention_bwd(const void* qkv, const void* out, const void* dout, const float* lse, void* dqkv,
+                         float* dbias, int B, int T, int H, int hd, void* workspace, size_t ws_bytes, int* dev_err,
+                         void* stream);
 
 /* Vocabulary-masked softmax cross-entropy, forward and backward fused (§4.1:
  * softmax over the V real ids only). logits bf16 [N,Vp] are overwritten in

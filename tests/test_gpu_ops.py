@@ -147,12 +147,26 @@ def test_attention_fwd_bwd(B, T, H, hd):
     do = rnd((B, T, C), 24)
     dqkv = torch.empty_like(qd)
     ws = torch.empty(gs.attention_bwd_workspace(B, T, H, hd), dtype=torch.uint8, device="cuda")
-    gs.attention_bwd(qd, out, bf16(do), lse, dqkv, H, ws, err)
+    db0 = rnd(3 * C, 27).astype(np.float32)
+    dbias = f32(db0)
+    gs.attention_bwd(qd, out, bf16(do), lse, dqkv, H, ws, err, dbias=dbias)
     dor = rounded(do).reshape(B, T, H, hd).transpose(0, 2, 1, 3)
     dq, dk, dv = G.attention_bwd(dor, q, k, v)
     got = host(dqkv)
     for i, ref in enumerate((dq, dk, dv)):
         assert rel_l2(got[..., i * C:(i + 1) * C], ref.transpose(0, 2, 1, 3).reshape(B, T, C)) < 2e-2, "qkv"[i]
+    # the qkv bias gradient: column sums of dq | dk | dv over the B*T rows
+    sq, sk, sv = (r.transpose(0, 2, 1, 3).reshape(B * T, C).sum(0) for r in (dq, dk, dv))
+    assert np.max(np.abs(sk)) < 1e-9 * np.max(np.abs(sq))      # the oracle: the key bias has no gradient
+    gb = host(dbias).astype(np.float64) - db0
+    tc = T % 128 == 0
+    assert rel_l2(gb[:C], sq) < 2e-2
+    if tc:
+        assert np.all(host(dbias)[C:2 * C] == db0[C:2 * C])      # nothing added to the key third
+        assert rel_l2(gb[2 * C:], sv) < 1e-5                     # dV's column sums are dO's
+    else:                                                        # column sums of the stored bf16 dqkv
+        assert np.max(np.abs(gb[C:2 * C])) < 2e-2 * np.max(np.abs(sq))
+        assert rel_l2(gb[2 * C:], sv) < 2e-2
     assert int(err.sum()) == 0
 
 

@@ -208,6 +208,26 @@ def test_attention_backward_matches_torch():
         np.testing.assert_allclose(a, b.grad.numpy(), rtol=1e-10, atol=1e-13)
 
 
+def test_attention_bias_gradient_identities():
+    """The column sums that the fused QKV bias gradient uses: over all queries,
+    dk sums to zero (a shift shared by a query's scores cancels in its softmax)
+    and dv sums to do (every causal softmax row sums to one); checked against
+    the oracle's gradients and against finite differences of the loss in a bias
+    added to every key or value row."""
+    rng = np.random.default_rng(16)
+    q, k, v, do = (rng.standard_normal((2, 3, 11, 4)) for _ in range(4))
+    dq, dk, dv = G.attention_bwd(do, q, k, v)
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+    np.testing.assert_allclose(dv.sum(axis=2), do.sum(axis=2), rtol=1e-12, atol=1e-12)
+    loss = lambda kk, vv: float((G.attention_fwd(q, kk, vv)[0] * do).sum())
+    e = 1e-6
+    bk = rng.standard_normal(4)
+    assert abs(loss(k + e * bk, v) - loss(k - e * bk, v)) / (2 * e) < 1e-7
+    bv = rng.standard_normal(4)
+    fd = (loss(k, v + e * bv) - loss(k, v - e * bv)) / (2 * e)
+    assert fd == pytest.approx(float((do.sum(axis=(0, 2)) * bv).sum()), rel=1e-6)
+
+
 def test_layernorm_brute_force_and_invariants():
     rng = np.random.default_rng(7)
     x = rng.standard_normal((3, 10)) * 2 + 1
