@@ -1,11 +1,13 @@
-// Causal flash attention forward on the 5th-generation tensor cores (head size 64).
+// Causal flash attention forward on the 5th-generation tensor cores (head size 64 or 32).
 //
 // Same operation as attn::attn_fwd_kernel (grow_a_language_model_intro,
 // activities 5-6: softmax(Q K^T / sqrt(d)) V with a causal mask, per head),
 // organised for tcgen05:
 //
-//   CTA     one (batch, head) and 128 query rows; walks key blocks of 128
-//   warp 0  TMA: Q once, then K_j and V_j (double-buffered ring)
+//   CTA     persistent, two an SM; a tile is one (batch, head) and 128 query
+//           rows, which walks key blocks of 128; the CTA takes tiles in a
+//           stride over a heaviest-first order
+//   warp 0  TMA: Q per tile (double-buffered), K_j and V_j (double-buffered rings)
 //   warp 1  tensor-memory allocation; lane 0 issues
 //             S_j = Q K_j^T   (M=128, N=128, K=64)  into S[j % 2] (TMEM)
 //             O  += P_j V_j   (M=128, N=64,  K=128) into O (TMEM)
@@ -30,7 +32,7 @@ constexpr int STAGES = 2;
 // bf16 (rows of 128 or 64 bytes, in the tensor core's 128- or 64-byte swizzled
 // layout, which the TMA's swizzle of the same width writes). No alignment
 // slack: without static shared memory the dynamic block starts on a 1 KB
-// boundary (checked at run time). At most 82,944 bytes and 256 TMEM columns a
+// boundary (checked at run time). At most 99,328 bytes and 256 TMEM columns a
 // CTA: two CTAs share an SM.
 template <int D>
 struct FwdGeom {
@@ -38,7 +40,7 @@ struct FwdGeom {
   static constexpr int ROW = D * 2;                       // bytes per tile row
   static constexpr int Q_BYTES = BQ * ROW;
   static constexpr int KV_BYTES = BKV * ROW;
-  static constexpr int SMEM_BYTES = Q_BYTES + STAGES * 2 * KV_BYTES + 1024 /*barriers*/;
+  static constexpr int SMEM_BYTES = 2 * Q_BYTES + STAGES * 2 * KV_BYTES + 1024 /*barriers*/;
   static constexpr uint64_t kSwizzle = D == 64 ? 2 : 4;  // descriptor layout: 128- / 64-byte swizzle
 };
 // Shared-memory matrix descriptor for a swizzled tile (layout 2: 128-byte rows,
@@ -109,7 +111,7 @@ GPT2_DEV void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_qkv, bf16* __restrict__ out, float* __restrict__ lse,
-                       int T, int H, float scale, int* err) {
+                       int T, int H, int BH, float scale, int* err) {
   using G = FwdGeom<D>;
   constexpr int HD = D;
   constexpr int Q_BYTES = G::Q_BYTES, KV_BYTES = G::KV_BYTES;
@@ -119,35 +121,45 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (threadIdx.x == 0) atomicOr(err, DEVERR_TIMEOUT);
     return;
   }
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + Q_BYTES;                  // [STAGES][KV_BYTES]
+  uint8_t* sQ = smem;                          // [2][Q_BYTES]
+  uint8_t* sK = sQ + 2 * Q_BYTES;              // [STAGES][KV_BYTES]
   uint8_t* sV = sK + STAGES * KV_BYTES;        // [STAGES][KV_BYTES]
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + STAGES * KV_BYTES);
-  uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;     // [2]  K_j landed
-  uint64_t* k_empty = bars + 3;    // [2]  S_j computed: K stage free
-  uint64_t* v_full = bars + 5;     // [2]
-  uint64_t* v_empty = bars + 7;    // [2]  P_j V_j computed: V stage free
-  uint64_t* s_full = bars + 9;
-  uint64_t* s_empty = bars + 10;
-  uint64_t* p_full = bars + 11;
-  uint64_t* p_empty = bars + 12;
-  uint64_t* o_done = bars + 13;
-  uint64_t* done = bars + 14;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 15);
+  uint64_t* q_full = bars;         // [2]  Q of a tile landed
+  uint64_t* q_empty = bars + 2;    // [2]  the tile's last S computed: Q buffer free
+  uint64_t* k_full = bars + 4;     // [2]  K_j landed
+  uint64_t* k_empty = bars + 6;    // [2]  S_j computed: K stage free
+  uint64_t* v_full = bars + 8;     // [2]
+  uint64_t* v_empty = bars + 10;   // [2]  P_j V_j computed: V stage free
+  uint64_t* s_full = bars + 12;
+  uint64_t* s_empty = bars + 13;
+  uint64_t* p_full = bars + 14;
+  uint64_t* p_empty = bars + 15;
+  uint64_t* o_done = bars + 16;
+  uint64_t* done = bars + 17;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 18);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nqb = T / BQ;
-  const int qb = nqb - 1 - blockIdx.x;  // heaviest query tiles first
-  const int bh = blockIdx.y;
-  const int b = bh / H, h = bh % H;
+  const int n_tiles = nqb * BH;
   const int C = H * HD;
-  const int row_base = b * T;           // row of token (b, 0) in the [B*T, 3C] view
-  const int nkv = qb + 1;               // causal: key blocks 0..qb
+  // Persistent: tile t is query block nqb - 1 - t / BH (the heaviest first) of
+  // (batch, head) t % BH. In round r the CTAs take tiles r G .. r G + G - 1
+  // (G CTAs), in reversed order in odd rounds, so that a CTA that drew a heavy
+  // tile draws a light one next (over 8 query blocks the busiest CTA gets ~29
+  // key blocks against a mean of 27.7; a plain stride gives it 32). Key blocks
+  // are counted across the CTA's tiles (gb), so the K/V rings and the S, P and
+  // O barriers run on without a reset between tiles.
+  // the CTA's tile after tile t (the one it takes in the next round)
+  auto next_tile = [](int t) {
+    const int r = t / (int)gridDim.x + 1;
+    return r * (int)gridDim.x + ((r & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
+  };
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(q_full), 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&q_full[i]), 1);
+      mbar_init(smem_u32(&q_empty[i]), 1);
       mbar_init(smem_u32(&k_full[i]), 1);
       mbar_init(smem_u32(&k_empty[i]), 1);
       mbar_init(smem_u32(&v_full[i]), 1);
@@ -175,37 +187,54 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) {
     // -------------------------------------------------------------- TMA producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(smem_u32(q_full), Q_BYTES);
-      tma_load_2d(smem_u32(sQ), &tm_qkv, smem_u32(q_full), h * HD, row_base + qb * BQ);
       // K and V run as separate two-deep rings: K_j is released once S_j is
-      // computed, V_j once P_j V_j is, so K runs further ahead than V.
-      int nk = 0, nv = 0;
-      const unsigned long long t0 = globaltimer_ns();
-      while (nk < nkv || nv < nkv) {
-        bool progressed = false;
-        if (nk < nkv && (nk < 2 || mbar_try_wait(smem_u32(&k_empty[nk & 1]), ((nk >> 1) & 1) ^ 1))) {
-          const int st = nk & 1;
-          mbar_arrive_expect_tx(smem_u32(&k_full[st]), KV_BYTES);
-          tma_load_2d(smem_u32(sK + st * KV_BYTES), &tm_qkv, smem_u32(&k_full[st]), C + h * HD,
-                      row_base + nk * BKV);
-          ++nk;
-          progressed = true;
-        }
-        if (nv < nkv && nv < nk && (nv < 2 || mbar_try_wait(smem_u32(&v_empty[nv & 1]), ((nv >> 1) & 1) ^ 1))) {
-          const int st = nv & 1;
-          mbar_arrive_expect_tx(smem_u32(&v_full[st]), KV_BYTES);
-          tma_load_2d(smem_u32(sV + st * KV_BYTES), &tm_qkv, smem_u32(&v_full[st]), 2 * C + h * HD,
-                      row_base + nv * BKV);
-          ++nv;
-          progressed = true;
-        }
-        if (!progressed) {
-          if (*(volatile int*)err & DEVERR_TIMEOUT) break;
-          if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            atomicOr(err, DEVERR_TIMEOUT);
-            break;
+      // computed, V_j once P_j V_j is, so K runs further ahead than V. Q is
+      // double-buffered: the next tile's Q loads while this tile still runs.
+      int gk = 0;   // key blocks of earlier tiles (ring positions)
+      bool ok = true;
+      for (int t = blockIdx.x, it = 0; t < n_tiles && ok; t = next_tile(t)) {
+        const int qb = nqb - 1 - t / BH, bh = t % BH;
+        const int b = bh / H, h = bh % H;
+        const int row_base = b * T, nkv = qb + 1;
+        const int qs = it & 1;
+        if (it >= 2 && !mbar_wait(smem_u32(&q_empty[qs]), ((it >> 1) & 1) ^ 1, err)) break;
+        mbar_arrive_expect_tx(smem_u32(&q_full[qs]), Q_BYTES);
+        tma_load_2d(smem_u32(sQ + qs * Q_BYTES), &tm_qkv, smem_u32(&q_full[qs]), h * HD, row_base + qb * BQ);
+        int nk = 0, nv = 0;
+        unsigned long long t0 = globaltimer_ns();
+        while (nk < nkv || nv < nkv) {
+          bool progressed = false;
+          const int uk = gk + nk;
+          if (nk < nkv && (uk < 2 || mbar_try_wait(smem_u32(&k_empty[uk & 1]), ((uk >> 1) & 1) ^ 1))) {
+            const int st = uk & 1;
+            mbar_arrive_expect_tx(smem_u32(&k_full[st]), KV_BYTES);
+            tma_load_2d(smem_u32(sK + st * KV_BYTES), &tm_qkv, smem_u32(&k_full[st]), C + h * HD,
+                        row_base + nk * BKV);
+            ++nk;
+            progressed = true;
+          }
+          const int uv = gk + nv;
+          if (nv < nkv && nv < nk && (uv < 2 || mbar_try_wait(smem_u32(&v_empty[uv & 1]), ((uv >> 1) & 1) ^ 1))) {
+            const int st = uv & 1;
+            mbar_arrive_expect_tx(smem_u32(&v_full[st]), KV_BYTES);
+            tma_load_2d(smem_u32(sV + st * KV_BYTES), &tm_qkv, smem_u32(&v_full[st]), 2 * C + h * HD,
+                        row_base + nv * BKV);
+            ++nv;
+            progressed = true;
+          }
+          if (progressed) {
+            t0 = globaltimer_ns();
+          } else {
+            if (*(volatile int*)err & DEVERR_TIMEOUT) { ok = false; break; }
+            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+              atomicOr(err, DEVERR_TIMEOUT);
+              ok = false;
+              break;
+            }
           }
         }
+        gk += nkv;
+        ++it;
       }
     }
   } else if (warp == 1) {
@@ -213,10 +242,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(BQ, BKV, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(BQ, HD, false, true);
-      bool ok = mbar_wait(smem_u32(q_full), 0, err);
-      const uint32_t q_addr = smem_u32(sQ);
-      auto issue_s = [&](int j) {
-        const int st = j & 1;
+      // S_g = Q K_g^T for key block g (K ring position g) with Q buffer qs
+      auto issue_s = [&](int g, int qs) {
+        const int st = g & 1;
+        const uint32_t q_addr = smem_u32(sQ + qs * Q_BYTES);
         const uint32_t k_addr = smem_u32(sK + st * KV_BYTES);
         const uint32_t d = tmem + S_COL0;
 #pragma unroll
@@ -226,37 +255,53 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_commit(smem_u32(s_full));
         tc_commit(smem_u32(&k_empty[st]));
       };
-      if (ok && mbar_wait(smem_u32(&k_full[0]), 0, err)) {
-        tc_fence_after();
-        issue_s(0);
-      } else {
-        ok = false;
-      }
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j & 1;
-        if (j + 1 < nkv) {
-          const int sn = (j + 1) & 1;
-          // K_{j+1} landed, and the softmax has taken S_j out of tensor memory
-          if (!mbar_wait(smem_u32(&k_full[sn]), ((j + 1) >> 1) & 1, err)) { ok = false; break; }
-          if (!mbar_wait(smem_u32(s_empty), j & 1, err)) { ok = false; break; }
+      bool ok = true;
+      if (blockIdx.x < n_tiles) {   // round 0 gives every CTA a tile
+        ok = mbar_wait(smem_u32(&q_full[0]), 0, err) && mbar_wait(smem_u32(&k_full[0]), 0, err);
+        if (ok) {
           tc_fence_after();
-          issue_s(j + 1);
+          issue_s(0, 0);
         }
-        // P_j written (and O rescaled if needed)
-        if (!mbar_wait(smem_u32(p_full), j & 1, err)) { ok = false; break; }
-        if (!mbar_wait(smem_u32(&v_full[st]), (j >> 1) & 1, err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sV + st * KV_BYTES);
-        // V as stored ([key][head dim]): an MN-major B operand whose 8-key groups are
-        // 8 rows apart; its head dimension is one swizzle atom wide
-        const uint64_t vd = smem_desc_swz(v_addr, D == 64 ? 8192 : 8 * G::ROW, 8 * G::ROW, G::kSwizzle);
+      }
+      int gb = 0;   // key blocks issued in earlier iterations
+      for (int t = blockIdx.x, it = 0; t < n_tiles && ok; t = next_tile(t)) {
+        const int nkv = nqb - t / BH;   // causal: key blocks 0..qb
+        const bool more = next_tile(t) < n_tiles;
+        for (int j = 0; j < nkv; ++j, ++gb) {
+          // S of the next key block: this tile's next one, or the next tile's first,
+          // once its K landed and the softmax has taken S_gb out of tensor memory
+          const bool last = (j + 1 == nkv);
+          if (last) tc_commit(smem_u32(&q_empty[it & 1]));   // this tile's last S read Q
+          if (!last || more) {
+            const int gn = gb + 1;
+            int qs = it & 1;
+            if (!mbar_wait(smem_u32(&k_full[gn & 1]), (gn >> 1) & 1, err)) { ok = false; break; }
+            if (!mbar_wait(smem_u32(s_empty), gb & 1, err)) { ok = false; break; }
+            if (last) {
+              qs = (it + 1) & 1;
+              if (!mbar_wait(smem_u32(&q_full[qs]), ((it + 1) >> 1) & 1, err)) { ok = false; break; }
+            }
+            tc_fence_after();
+            issue_s(gn, qs);
+          }
+          // P_gb written (and O rescaled if needed)
+          const int st = gb & 1;
+          if (!mbar_wait(smem_u32(p_full), gb & 1, err)) { ok = false; break; }
+          if (!mbar_wait(smem_u32(&v_full[st]), (gb >> 1) & 1, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(sV + st * KV_BYTES);
+          // V as stored ([key][head dim]): an MN-major B operand whose 8-key groups are
+          // 8 rows apart; its head dimension is one swizzle atom wide
+          const uint64_t vd = smem_desc_swz(v_addr, D == 64 ? 8192 : 8 * G::ROW, 8 * G::ROW, G::kSwizzle);
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)   // A = P from tensor memory, 16 keys = 8 columns a step
-          tc_mma_bf16_ts(tmem + O_COL, tmem + P_COL + kk * 8, vd + kk * ((16 * G::ROW) >> 4), idesc_o,
-                         (j > 0 || kk > 0) ? 1u : 0u);
-        tc_commit(smem_u32(p_empty));
-        tc_commit(smem_u32(&v_empty[st]));
-        tc_commit(smem_u32(o_done));
+          for (int kk = 0; kk < BKV / 16; ++kk)   // A = P from tensor memory, 16 keys = 8 columns a step
+            tc_mma_bf16_ts(tmem + O_COL, tmem + P_COL + kk * 8, vd + kk * ((16 * G::ROW) >> 4), idesc_o,
+                           (j > 0 || kk > 0) ? 1u : 0u);
+          tc_commit(smem_u32(p_empty));
+          tc_commit(smem_u32(&v_empty[st]));
+          tc_commit(smem_u32(o_done));
+        }
+        ++it;
       }
       tc_commit(smem_u32(done));
       mbar_wait(smem_u32(done), 0, err);
@@ -265,110 +310,118 @@ __global__ void __launch_bounds__(kThreads, 2)
     // -------------------------------------------------------------- softmax / epilogue
     const int q4 = warp & 3;                        // TMEM lane quarter
     const int r = q4 * 32 + lane;                   // query row within the tile
-    const int qrow = qb * BQ + r;                   // query position
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     const float sl2 = scale * kLog2e;
-    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
-      if (!mbar_wait(smem_u32(s_full), j & 1, err)) { ok = false; break; }
-      tc_fence_after();
-      const bool diag = (j == qb);
-      const uint32_t s_tm = tmem + lane_off + S_COL0;
-      // the whole score row (128 fp32) in four loads, one wait; S is free again at once
-      uint32_t sr[4][32];
+    int gb = 0;   // key blocks of earlier tiles and of this one so far
+    for (int t = blockIdx.x; t < n_tiles && ok; t = next_tile(t)) {
+      const int qb = nqb - 1 - t / BH;
+      const int nkv = qb + 1;
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < nkv; ++j, ++gb) {
+        if (!mbar_wait(smem_u32(s_full), gb & 1, err)) { ok = false; break; }
+        tc_fence_after();
+        const bool diag = (j == qb);
+        const uint32_t s_tm = tmem + lane_off + S_COL0;
+        // the whole score row (128 fp32) in four loads, one wait; S is free again at once
+        uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32_async(s_tm + c * 32, sr[c]);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(smem_u32(s_empty));
-      if (diag) {
+        for (int c = 0; c < 4; ++c) tmem_ld32_async(s_tm + c * 32, sr[c]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(smem_u32(s_empty));
+        if (diag) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (c * 32 + i > r) sr[c][i] = __float_as_uint(-INFINITY);
+        }
+        // row maximum with eight independent partial maxima (short dependency
+        // chains), two scores per three-input max
+        float mpart[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mpart[u] = -INFINITY;
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (c * 32 + i > r) sr[c][i] = __float_as_uint(-INFINITY);
-      }
-      // row maximum with eight independent partial maxima (short dependency
-      // chains), two scores per three-input max
-      float mpart[8];
+          for (int i = 0; i < 32; i += 2)
+            mpart[(i >> 1) & 7] =
+                max3f(mpart[(i >> 1) & 7], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
+        const float mx = max3f(max3f(mpart[0], mpart[1], mpart[2]), max3f(mpart[3], mpart[4], mpart[5]),
+                               fmaxf(mpart[6], mpart[7])) *
+                         sl2;  // scale > 0: max commutes with it
+        // lazy rescale: keep the stale maximum unless the new one exceeds it by > 2^8
+        const bool grow = (mx > m + kRescaleThreshold) || (m == -INFINITY);
+        const float m_new = grow ? mx : m;
+        const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
+        // four paired partial sums; the scale-and-shift and the sums run as paired
+        // fp32 operations (two scores per instruction)
+        float2 spart[4];
 #pragma unroll
-      for (int t = 0; t < 8; ++t) mpart[t] = -INFINITY;
+        for (int u = 0; u < 4; ++u) spart[u] = make_float2(0.f, 0.f);
+        const float2 sl2x2 = make_float2(sl2, sl2), negm2 = make_float2(-m_new, -m_new);
+        // P as bf16 pairs (keys 2i, 2i+1 of this query row in column P_COL + i),
+        // in two halves of 64 keys: the first half's 32 words are stored (once the
+        // PV product of the previous key block has read the P buffer) before the
+        // second half is formed, so only 32 packed words are live at a time
+        bool waited = false;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2)
-          mpart[(i >> 1) & 7] =
-              max3f(mpart[(i >> 1) & 7], __uint_as_float(sr[c][i]), __uint_as_float(sr[c][i + 1]));
-      const float mx = max3f(max3f(mpart[0], mpart[1], mpart[2]), max3f(mpart[3], mpart[4], mpart[5]),
-                             fmaxf(mpart[6], mpart[7])) *
-                       sl2;  // scale > 0: max commutes with it
-      // lazy rescale: keep the stale maximum unless the new one exceeds it by > 2^8
-      const bool grow = (mx > m + kRescaleThreshold) || (m == -INFINITY);
-      const float m_new = grow ? mx : m;
-      const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
-      // four paired partial sums; the scale-and-shift and the sums run as paired
-      // fp32 operations (two scores per instruction)
-      float2 spart[4];
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * half + cc;
 #pragma unroll
-      for (int t = 0; t < 4; ++t) spart[t] = make_float2(0.f, 0.f);
-      const float2 sl2x2 = make_float2(sl2, sl2), negm2 = make_float2(-m_new, -m_new);
-      // P_j as bf16 pairs (keys 2i, 2i+1 of this query row in column P_COL + i),
-      // in two halves of 64 keys: the first half's 32 words are stored (once the
-      // PV product of block j-1 has read the P buffer) before the second half is
-      // formed, so only 32 packed words are live at a time
-      bool waited = false;
+            for (int i = 0; i < 16; ++i) {
+              const float2 y = f2_fma(make_float2(__uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1])),
+                                      sl2x2, negm2);
+              const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
+              spart[i & 3] = f2_add(spart[i & 3], pp);
+              pk[cc * 16 + i] = pack_bf16x2(pp.x, pp.y);
+            }
+          }
+          if (!waited) {
+            // the P buffer was last read by the PV product of key block gb - 1
+            if (gb >= 1 && !mbar_wait(smem_u32(p_empty), (gb - 1) & 1, err)) { ok = false; }
+            tc_fence_after();
+            waited = true;
+          }
+          if (ok) tmem_st32_u(tmem + lane_off + P_COL + 32 * half, pk);
+        }
+        if (!ok) break;
+        const float2 s01 = f2_add(spart[0], spart[1]), s23 = f2_add(spart[2], spart[3]);
+        const float2 s4 = f2_add(s01, s23);
+        const float sum = s4.x + s4.y;
+        l = l * alpha + sum;
+        m = m_new;
+        // O rescale (rows whose maximum moved) once the PV product of key block gb - 1 is done
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          if (!mbar_wait(smem_u32(o_done), (gb - 1) & 1, err)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+          for (int c = 0; c < HD / 32; ++c) {
+            float v[32];
+            tmem_ld32(tmem + lane_off + O_COL + c * 32, v);
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = 2 * half + cc;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float2 y =
-                f2_fma(make_float2(__uint_as_float(sr[c][2 * i]), __uint_as_float(sr[c][2 * i + 1])), sl2x2, negm2);
-            const float2 pp = make_float2(ex2_approx(y.x), ex2_approx(y.y));
-            spart[i & 3] = f2_add(spart[i & 3], pp);
-            pk[cc * 16 + i] = pack_bf16x2(pp.x, pp.y);
+            for (int i = 0; i < 32; ++i) v[i] *= alpha;
+            tmem_st32(tmem + lane_off + O_COL + c * 32, v);
           }
         }
-        if (!waited) {
-          // the P buffer was last read by the PV product of block j-1
-          if (j >= 1 && !mbar_wait(smem_u32(p_empty), (j - 1) & 1, err)) { ok = false; }
-          tc_fence_after();
-          waited = true;
-        }
-        if (ok) tmem_st32_u(tmem + lane_off + P_COL + 32 * half, pk);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(smem_u32(p_full));
       }
       if (!ok) break;
-      const float2 s01 = f2_add(spart[0], spart[1]), s23 = f2_add(spart[2], spart[3]);
-      const float2 s4 = f2_add(s01, s23);
-      const float sum = s4.x + s4.y;
-      l = l * alpha + sum;
-      m = m_new;
-      // O rescale (rows whose maximum moved) once the PV product of block j-1 is done
-      if (j > 0 && __any_sync(0xffffffffu, grow)) {
-        if (!mbar_wait(smem_u32(o_done), (j - 1) & 1, err)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          float v[32];
-          tmem_ld32(tmem + lane_off + O_COL + c * 32, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= alpha;
-          tmem_st32(tmem + lane_off + O_COL + c * 32, v);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(smem_u32(p_full));
-    }
-    // epilogue: O / l, log-sum-exp
-    if (ok && mbar_wait(smem_u32(o_done), (nkv - 1) & 1, err)) {
+      // epilogue: O / l, log-sum-exp, once the tile's last PV product is done; O is
+      // read out before this warp's next P is posted, so the next tile's first PV
+      // product (which overwrites O) cannot start earlier
+      if (!mbar_wait(smem_u32(o_done), (gb - 1) & 1, err)) break;
       tc_fence_after();
+      const int bh = t % BH;
+      const int qrow = qb * BQ + r;                 // query position
       const float inv = 1.0f / l;
-      bf16* orow = out + ((size_t)(row_base + qrow)) * C + h * HD;
+      bf16* orow = out + ((size_t)((bh / H) * T + qrow)) * C + (bh % H) * HD;
 #pragma unroll
       for (int c = 0; c < HD / 32; ++c) {
         float v[32];
@@ -380,6 +433,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                          pack_bf16x2(v[i + 4] * inv, v[i + 5] * inv), pack_bf16x2(v[i + 6] * inv, v[i + 7] * inv));
       }
       lse[(size_t)bh * T + qrow] = (m + log2f(l)) * kLn2;
+      tc_fence_before();
     }
   }
   tc_fence_before();
@@ -410,8 +464,10 @@ static cudaError_t fwd(const bf16* qkv, bf16* out, float* lse, int B, int T, int
   if (!encode_map_2d(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, qkv, 3 * (uint64_t)C, (uint64_t)B * T, 3 * (uint64_t)C,
                      D, 128, D == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
-  dim3 grid(T / BQ, B * H);
-  launch_pdl(attn_fwd_tc_kernel<D>, dim3(grid), dim3(kThreads), G::SMEM_BYTES, s, tm, out, lse, T, H,
+  // persistent: two CTAs an SM, or one per tile if there are fewer tiles
+  const int n_tiles = (T / BQ) * B * H;
+  const int grid = std::min(n_tiles, 2 * device_sm_count());
+  launch_pdl(attn_fwd_tc_kernel<D>, dim3(grid), dim3(kThreads), G::SMEM_BYTES, s, tm, out, lse, T, H, B * H,
              1.0f / sqrtf((float)D), err);
   return cudaGetLastError();
 }

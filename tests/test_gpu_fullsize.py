@@ -45,8 +45,9 @@ def test_attention_many_items_per_cta(Bt, HDt):
     """(Bt, 1024, 12, 64): 384 and 1,824 backward work items against 148 SMs,
     so most CTAs run the cross-item K/V prefetch and accumulator hand-over; and
     head size 32 at (16, 1024, 12) (the small configuration's attention, the
-    forward on the tensor cores with 64-byte rows). Every dQ, dK, dV element,
-    the output and the lse are compared."""
+    forward on the tensor cores with 64-byte rows). The forward's persistent
+    CTAs take 2 to 7 query tiles each. Every dQ, dK, dV element, the output,
+    the lse and the qkv bias gradient are compared."""
     HD = HDt
     C = H * HD
     rng = np.random.default_rng(40 + Bt)
@@ -59,11 +60,13 @@ def test_attention_many_items_per_cta(Bt, HDt):
     gs.attention_fwd(qd, out, lse, H, err)
     dqkv = torch.empty_like(qd)
     ws = torch.empty(gs.attention_bwd_workspace(Bt, T, H, HD), dtype=torch.uint8, device="cuda")
-    gs.attention_bwd(qd, out, bf16(do), lse, dqkv, H, ws, err)
-    got_o, got_l, got_d = host(out), host(lse), host(dqkv)
+    dbias = torch.zeros(3 * C, device="cuda")
+    gs.attention_bwd(qd, out, bf16(do), lse, dqkv, H, ws, err, dbias=dbias)
+    got_o, got_l, got_d, got_b = host(out), host(lse), host(dqkv), host(dbias)
     assert int(err.sum()) == 0
     qr, dr = rounded(qkv), rounded(do)
     worst = {"o": 0.0, "dq": 0.0, "dk": 0.0, "dv": 0.0, "lse": 0.0}
+    sums = np.zeros(3 * C)   # the qkv bias gradient: column sums of dq | dk | dv over all rows
     for b in range(Bt):     # the oracle one sequence at a time (its score matrices are T x T per head)
         q, k, v = (qr[b, :, i * C:(i + 1) * C].reshape(T, H, HD).transpose(1, 0, 2) for i in range(3))
         o, l = G.attention_fwd(q, k, v)
@@ -71,11 +74,16 @@ def test_attention_many_items_per_cta(Bt, HDt):
         worst["o"] = max(worst["o"], rel_l2(got_o[b], o.transpose(1, 0, 2).reshape(T, C)))
         worst["lse"] = max(worst["lse"], float(np.max(np.abs(got_l[b] - l))))
         for i, (name, ref) in enumerate((("dq", dq), ("dk", dk), ("dv", dv))):
-            e = rel_l2(got_d[b, :, i * C:(i + 1) * C], ref.transpose(1, 0, 2).reshape(T, C))
+            ref = ref.transpose(1, 0, 2).reshape(T, C)
+            e = rel_l2(got_d[b, :, i * C:(i + 1) * C], ref)
             worst[name] = max(worst[name], e)
+            sums[i * C:(i + 1) * C] += ref.sum(axis=0)
     print("attention worst per-sequence errors:", worst)
     assert worst["o"] < 1e-2 and worst["lse"] < 2e-3
     assert worst["dq"] < 2e-2 and worst["dk"] < 2e-2 and worst["dv"] < 2e-2
+    assert rel_l2(got_b[:C], sums[:C]) < 2e-2
+    assert np.all(got_b[C:2 * C] == 0.0) and np.max(np.abs(sums[C:2 * C])) < 1e-9 * np.max(np.abs(sums[:C]))
+    assert rel_l2(got_b[2 * C:], sums[2 * C:]) < 1e-5
 
 
 # --- a10, a3/a5/a7/a8 backward: full-size GEMMs on exact inputs -----------------------------------
