@@ -784,11 +784,18 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nb = T / BKEY;
   const int C = H * HD;
-  // Persistent: this CTA takes work items blockIdx.x, blockIdx.x + gridDim.x, ..
-  // of the nb * BH (key block, batch-head) items; heaviest key blocks (kb = 0:
-  // every query block) come first. Barrier phases run over g, the CTA's count of
-  // query blocks processed, and over j, its count of items.
+  // Persistent: item i is key block i / BH of (batch, head) i % BH, so the
+  // heaviest key blocks (kb = 0: every query block) come first; in round r the
+  // CTAs take items r G .. r G + G - 1 (G CTAs), in reversed order in odd
+  // rounds, so that a CTA that drew a heavy item draws a light one next (the
+  // busiest CTA gets ~56 query blocks against a mean of 55.5 at 8 key blocks,
+  // 148 CTAs; a plain stride gives it 60). Barrier phases run over g, the CTA's
+  // count of query blocks processed, and over j, its count of items.
   const int n_items = nb * BH;
+  auto next_item = [](int i) {   // the CTA's item after item i
+    const int r = i / (int)gridDim.x + 1;
+    return r * (int)gridDim.x + ((r & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -850,7 +857,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           bulk_load_1d(smem_u32(sXQ + s * XT_BYTES), xtiles + ((size_t)bh * nb + qi) * XT_BYTES, XT_BYTES, fb);
           return true;
         };
-        for (int i = blockIdx.x, j = 0; i < n_items && ok; i += gridDim.x, ++j) {
+        for (int i = blockIdx.x, j = 0; i < n_items && ok; i = next_item(i), ++j) {
           const int kb = i / BH, bh = i % BH, b = bh / H, h = bh % H;
           const int row_base = b * T, nit = nb - kb;
           // the first query block of this item may land before its keys
@@ -868,7 +875,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
           g += nit;
           // the next item's K into the other buffer, once the item before this
           // one has released it
-          const int i2 = i + gridDim.x;
+          const int i2 = next_item(i);
           if (ok && i2 < n_items) {
             const int kb2 = i2 / BH, bh2 = i2 % BH, b2 = bh2 / H, h2 = bh2 % H;
             const int nbuf = (j + 1) & 1;
@@ -919,7 +926,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
         };
         bool ok = true;
         int g = 0;
-        for (int i = blockIdx.x, j = 0; i < n_items && ok; i += gridDim.x, ++j) {
+        for (int i = blockIdx.x, j = 0; i < n_items && ok; i = next_item(i), ++j) {
           const int nit = nb - i / BH;
           const uint64_t ko = (j & 1) ? kKBuf : 0;
           // this item's keys, its first query block, and the previous scores out of TMEM
@@ -1016,7 +1023,7 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
     bool ok = true;
     int g = 0;
     int prev_hc = 0, prev_qrow0 = 0;   // where the previous block's dQ goes
-    for (int i = blockIdx.x, j = 0; i < n_items && ok; i += gridDim.x, ++j) {
+    for (int i = blockIdx.x, j = 0; i < n_items && ok; i = next_item(i), ++j) {
       const int kb = i / BH, bh = i % BH, b = bh / H, h = bh % H;
       const int row_base = b * T, nit = nb - kb;
       for (int it = 0; it < nit && ok; ++it) {
