@@ -293,7 +293,8 @@ void ln_fwd_c(const bf16* x, const float* w, const float* b, bf16* y, float* mea
   static PerDeviceOnce once;
   static int cache[PerDeviceOnce::kMaxDevices] = {};
   const int full = resident_ctas(once, cache, k::layernorm_fwd_kernel<C>, k::kLnFwdWarps * 32);
-  const int need = (rows + k::kLnFwdWarps - 1) / k::kLnFwdWarps;
+  const int per_cta = k::kLnFwdWarps * k::ln_fwd_rows(C);   // rows a CTA takes per pass
+  const int need = (rows + per_cta - 1) / per_cta;
   launch_pdl(k::layernorm_fwd_kernel<C>, dim3(std::min(need, full)), dim3(k::kLnFwdWarps * 32), 0, s, x, w, b, y,
              mean, rstd, rows);
 }

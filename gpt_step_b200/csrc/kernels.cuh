@@ -180,14 +180,17 @@ __global__ void __launch_bounds__(256) embed_bwd_wte_kernel(const int32_t* __res
 }
 
 // ---------------------------------------------------------------------------
-// a2/a6/a9  LayerNorm forward: one warp per row in a grid-stride loop over the
-// rows (the next row's loads in flight while one is normalised; the grid is the
-// resident-CTA count, so there is no partial last wave), fp32 statistics (eps
+// a2/a6/a9  LayerNorm forward: a warp normalises RP rows at a time (RP = 2 for
+// C <= 768, else 1) in a grid-stride loop over the rows, the next RP rows'
+// loads in flight while these are normalised; the RP rows' warp reductions
+// are interleaved, so their shuffle latencies overlap (the grid is the
+// resident-CTA count, so there is no partial last wave). fp32 statistics (eps
 // 1e-5, biased variance), y = (x - mean) * rstd * w + b in bf16.
 // ---------------------------------------------------------------------------
 constexpr int kLnFwdWarps = 8;   // warps per CTA
-// CTAs per SM: as many as the row's registers allow without spilling
-__host__ __device__ constexpr int ln_fwd_minb(int C) { return C <= 512 ? 4 : (C <= 1024 ? 3 : 2); }
+__host__ __device__ constexpr int ln_fwd_rows(int C) { return C <= 768 ? 2 : 1; }
+// CTAs per SM: as many as the rows' registers allow without spilling
+__host__ __device__ constexpr int ln_fwd_minb(int C) { return C <= 768 ? 2 : (C <= 1024 ? 3 : 2); }
 template <int C>
 __global__ void __launch_bounds__(kLnFwdWarps * 32, ln_fwd_minb(C)) layernorm_fwd_kernel(const bf16* __restrict__ x,
                                                                         const float* __restrict__ w,
@@ -197,50 +200,66 @@ __global__ void __launch_bounds__(kLnFwdWarps * 32, ln_fwd_minb(C)) layernorm_fw
   pdl_begin();
   constexpr int NV = C / 8;                 // 16-byte vectors per row
   constexpr int VPL = (NV + 31) / 32;       // vectors per lane
+  constexpr int RP = ln_fwd_rows(C);        // rows a warp normalises together
   const int l = lane_id();
-  const int stride = gridDim.x * kLnFwdWarps;
-  int row = blockIdx.x * kLnFwdWarps + (threadIdx.x >> 5);
-  auto load = [&](int r, uint4 (&u)[VPL]) {
+  const int stride = gridDim.x * kLnFwdWarps * RP;
+  int row = (blockIdx.x * kLnFwdWarps + (threadIdx.x >> 5)) * RP;
+  auto load = [&](int r, uint4 (&u)[RP][VPL]) {
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const int vi = l + 32 * i;
-      u[i] = (vi < NV && r < rows) ? __ldcs(reinterpret_cast<const uint4*>(x + (size_t)r * C) + vi)
-                                   : make_uint4(0u, 0u, 0u, 0u);
-    }
+    for (int p = 0; p < RP; ++p)
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int vi = l + 32 * i;
+        u[p][i] = (vi < NV && r + p < rows) ? __ldcs(reinterpret_cast<const uint4*>(x + (size_t)(r + p) * C) + vi)
+                                            : make_uint4(0u, 0u, 0u, 0u);
+      }
   };
-  // grid-stride over rows, one row per warp at a time, the next row's loads in
-  // flight while this one is normalised
-  uint4 cur[VPL], nxt[VPL];
+  uint4 cur[RP][VPL], nxt[RP][VPL];
   load(row, cur);
   for (; row < rows; row += stride) {
     load(row + stride, nxt);
-    float v[VPL][8];
-    float s = 0.f;
+    float v[RP][VPL][8];
+    float s[RP];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      const uint32_t wv[4] = {cur[i].x, cur[i].y, cur[i].z, cur[i].w};
+    for (int p = 0; p < RP; ++p) {
+      s[p] = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float2 f = unpack_bf16x2(wv[j]);
-        v[i][2 * j] = f.x;
-        v[i][2 * j + 1] = f.y;
-        s += f.x + f.y;
-      }
-    }
-    const float mu = warp_sum(s) * (1.0f / C);
-    float ss = 0.f;
+      for (int i = 0; i < VPL; ++i) {
+        const uint32_t wv[4] = {cur[p][i].x, cur[p][i].y, cur[p][i].z, cur[p][i].w};
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      if (l + 32 * i < NV) {
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float d = v[i][j] - mu;
-          ss += d * d;
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = unpack_bf16x2(wv[j]);
+          v[p][i][2 * j] = f.x;
+          v[p][i][2 * j + 1] = f.y;
+          s[p] += f.x + f.y;
         }
       }
     }
-    const float rs = rsqrtf(warp_sum(ss) * (1.0f / C) + 1e-5f);
-    bf16* yr = y + (size_t)row * C;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int p = 0; p < RP; ++p) s[p] += __shfl_xor_sync(0xffffffffu, s[p], o);
+    float mu[RP], ss[RP];
+#pragma unroll
+    for (int p = 0; p < RP; ++p) {
+      mu[p] = s[p] * (1.0f / C);
+      ss[p] = 0.f;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (l + 32 * i < NV)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float d = v[p][i][j] - mu[p];
+            ss[p] += d * d;
+          }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int p = 0; p < RP; ++p) ss[p] += __shfl_xor_sync(0xffffffffu, ss[p], o);
+    float rs[RP];
+#pragma unroll
+    for (int p = 0; p < RP; ++p) rs[p] = rsqrtf(ss[p] * (1.0f / C) + 1e-5f);
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int vi = l + 32 * i;
@@ -252,21 +271,30 @@ __global__ void __launch_bounds__(kLnFwdWarps * 32, ln_fwd_minb(C)) layernorm_fw
         const float4 b1 = __ldg(reinterpret_cast<const float4*>(b + vi * 8 + 4));
         const float ww[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
         const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        uint32_t o[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          o[j] = pack_bf16x2((v[i][2 * j] - mu) * rs * ww[2 * j] + bb[2 * j],
-                             (v[i][2 * j + 1] - mu) * rs * ww[2 * j + 1] + bb[2 * j + 1]);
-        // a plain store: the next GEMM reads y while it is still in L2
-        *reinterpret_cast<uint4*>(yr + vi * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+        for (int p = 0; p < RP; ++p) {
+          if (row + p >= rows) continue;
+          uint32_t o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            o[j] = pack_bf16x2((v[p][i][2 * j] - mu[p]) * rs[p] * ww[2 * j] + bb[2 * j],
+                               (v[p][i][2 * j + 1] - mu[p]) * rs[p] * ww[2 * j + 1] + bb[2 * j + 1]);
+          // a plain store: the next GEMM reads y while it is still in L2
+          *reinterpret_cast<uint4*>(y + (size_t)(row + p) * C + vi * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
       }
     }
-    if (l == 0) {
-      mean[row] = mu;
-      rstd[row] = rs;
-    }
+    // lane p writes the statistics of row p
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) cur[i] = nxt[i];
+    for (int p = 0; p < RP; ++p)
+      if (l == p && row + p < rows) {
+        mean[row + p] = mu[p];
+        rstd[row + p] = rs[p];
+      }
+#pragma unroll
+    for (int p = 0; p < RP; ++p)
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) cur[p][i] = nxt[p][i];
   }
 }
 
