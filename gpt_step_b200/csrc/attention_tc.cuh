@@ -144,13 +144,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int n_tiles = nqb * BH;
   const int C = H * HD;
   // Persistent: tile t is query block nqb - 1 - t / BH (the heaviest first) of
-  // (batch, head) t % BH. In round r the CTAs take tiles r G .. r G + G - 1
-  // (G CTAs), in reversed order in odd rounds, so that a CTA that drew a heavy
+  // (batch, head) t % BH. In pass r the CTAs take tiles r G .. r G + G - 1
+  // (G CTAs), in reversed order in odd passes, so that a CTA that drew a heavy
   // tile draws a light one next (over 8 query blocks the busiest CTA gets ~29
   // key blocks against a mean of 27.7; a plain stride gives it 32). Key blocks
   // are counted across the CTA's tiles (gb), so the K/V rings and the S, P and
   // O barriers run on without a reset between tiles.
-  // the CTA's tile after tile t (the one it takes in the next round)
+  // the CTA's tile after tile t (the one it takes in the next pass)
   auto next_tile = [](int t) {
     const int r = t / (int)gridDim.x + 1;
     return r * (int)gridDim.x + ((r & 1) ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x);
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         tc_commit(smem_u32(&k_empty[st]));
       };
       bool ok = true;
-      if (blockIdx.x < n_tiles) {   // round 0 gives every CTA a tile
+      if (blockIdx.x < n_tiles) {   // the first pass gives every CTA a tile
         ok = mbar_wait(smem_u32(&q_full[0]), 0, err) && mbar_wait(smem_u32(&k_full[0]), 0, err);
         if (ok) {
           tc_fence_after();
@@ -785,9 +785,9 @@ __global__ void __launch_bounds__(bwd::kThreads, 1)
   const int nb = T / BKEY;
   const int C = H * HD;
   // Persistent: item i is key block i / BH of (batch, head) i % BH, so the
-  // heaviest key blocks (kb = 0: every query block) come first; in round r the
+  // heaviest key blocks (kb = 0: every query block) come first; in pass r the
   // CTAs take items r G .. r G + G - 1 (G CTAs), in reversed order in odd
-  // rounds, so that a CTA that drew a heavy item draws a light one next (the
+  // passes, so that a CTA that drew a heavy item draws a light one next (the
   // busiest CTA gets ~56 query blocks against a mean of 55.5 at 8 key blocks,
   // 148 CTAs; a plain stride gives it 60). Barrier phases run over g, the CTA's
   // count of query blocks processed, and over j, its count of items.

@@ -77,8 +77,8 @@ def run_step(args):
 
 def kernel_sources_sha256() -> str:
     """sha256 over the CUDA sources of the library: file names in sorted order and
-    their contents with every run of whitespace collapsed to one space, so that a
-    change of layout alone keeps the hash."""
+    their contents with comments removed and every run of whitespace collapsed
+    to one space, so that a change of comments or layout alone keeps the hash."""
     import hashlib
     import os
     import re
@@ -88,7 +88,9 @@ def kernel_sources_sha256() -> str:
         if name.endswith((".cu", ".cuh", ".h")):
             h.update(name.encode())
             with open(os.path.join(d, name), "rb") as f:
-                h.update(re.sub(rb"\s+", b" ", f.read()).strip())
+                text = re.sub(rb"/\*.*?\*/", b" ", f.read(), flags=re.S)
+                text = re.sub(rb"//[^\n]*", b" ", text)
+                h.update(re.sub(rb"\s+", b" ", text).strip())
     return h.hexdigest()
 
 
