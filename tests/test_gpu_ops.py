@@ -127,6 +127,27 @@ def test_layernorm_fwd_bwd(C, atomic):
     assert rel_l2(host(db), db0.astype(np.float32) + rdb) < 1e-5
 
 
+@pytest.mark.parametrize("rows,C", [(1, 768), (999, 768), (4737, 768), (999, 128), (333, 1024)])
+def test_layernorm_fwd_row_counts(rows, C):
+    """The forward takes rows in pairs for C <= 768, so an odd count leaves the
+    last pair with one row: a single row, 999 rows, and 4,737 rows (one more
+    than a whole pass of the resident grid on 148 SMs). Wider rows go one at a
+    time. Every output row and statistic is compared; rows past the end are
+    never written."""
+    x = rnd((rows, C), 30, 1.5) - 0.25
+    w, b = 1.0 + rnd(C, 31, 0.1), rnd(C, 32, 0.1)
+    y = torch.full((rows + 2, C), 7.0, dtype=torch.bfloat16, device="cuda")
+    mean = torch.full((rows + 2,), 7.0, device="cuda")
+    rstd = torch.full((rows + 2,), 7.0, device="cuda")
+    gs.layernorm_fwd(bf16(x), f32(w), f32(b), y[:rows], mean[:rows], rstd[:rows])
+    w32, b32 = w.astype(np.float32).astype(np.float64), b.astype(np.float32).astype(np.float64)
+    yr, mr, rr = G.layernorm_fwd(rounded(x), w32, b32)
+    got = host(y)
+    assert rel_l2(got[:rows], yr) < BF16_TOL
+    assert rel_l2(host(mean)[:rows], mr) < 1e-6 and rel_l2(host(rstd)[:rows], rr) < 1e-5
+    assert np.all(got[rows:] == 7.0) and np.all(host(mean)[rows:] == 7.0) and np.all(host(rstd)[rows:] == 7.0)
+
+
 # --- a4: causal attention ------------------------------------------------------------------
 
 @pytest.mark.parametrize("B,T,H,hd", [(2, 64, 2, 32), (2, 192, 3, 64), (1, 1024, 2, 64), (2, 256, 4, 32),
