@@ -40,10 +40,11 @@ def _gpu():
 
 # --- a4: attention with many work items per persistent CTA -------------------------------------
 
-@pytest.mark.parametrize("Bt,HDt", [(4, 64), (19, 64), (16, 32)])
+@pytest.mark.parametrize("Bt,HDt", [(3, 64), (4, 64), (19, 64), (16, 32)])
 def test_attention_many_items_per_cta(Bt, HDt):
-    """(Bt, 1024, 12, 64): 384 and 1,824 backward work items against 148 SMs,
-    so most CTAs run the cross-item K/V prefetch and accumulator hand-over; and
+    """(Bt, 1024, 12, 64): 288, 384 and 1,824 backward work items against 148
+    SMs, so most CTAs run the cross-item K/V prefetch and accumulator hand-over
+    (288 = 148 + 140 ends on a partial pass taken in reversed order); and
     head size 32 at (16, 1024, 12) (the small configuration's attention, the
     forward on the tensor cores with 64-byte rows). The forward's persistent
     CTAs take 2 to 7 query tiles each. Every dQ, dK, dV element, the output,
